@@ -1,0 +1,326 @@
+"""OWQ oracle: a plain, slow, obviously-correct CPU implementation of the mixed-precision
+weight-only matmul and of the quantiser that produces its operands.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this module. The CUDA library never calls it, and it shares
+no code with the CUDA library: it imports numpy and nothing else of this repository.
+
+Sources (five web pages about the OWQ paper, Lee et al., arXiv:2306.02272):
+  [SUM]  "OWQ -- paper by Lee et al. (2023) -- summary and ideas" (research.elamur.ai):
+         sections "Key points" and "Interesting ideas".
+  [PL]   "OWQ: Outlier-Aware Weight Quantization for Efficient Fine-Tuning and Inference of
+         Large Language Models" (paperlayer.ai), whose items name the paper's sections:
+         "Problem Definition and Motivation" (p.3), "Layer-wise Quantization and Hessian"
+         (p.3), "OWQ: Outlier-aware Weight Quantization" (p.4), "Acceleration on Real
+         Device" (p.6), appendix "§1" (p.10, Eq. (10)) and "§2 Storage Methods" (pp.10-11).
+
+Every floating-point reduction is fp64 in a fixed order (index ascending). Every decision
+that turns a float into an integer (a quantised code, the zero point, the top-k order) is
+taken in the precision stated at that step, with IEEE round-to-nearest-even.
+
+Readings of the pages where they are silent (each is listed with its reason in the design
+notes): the sensitivity uses the perturbation of an all-column RTN pre-quantisation; the
+quantisation range always contains 0; a degenerate range becomes [-1, 1]; rounding is
+half-to-even; the dequantised weight is fp16_rn(s * (q - z)); weak positions carry the code
+q = z (so they dequantise to exactly 0); groups are contiguous blocks of the original column
+order; top-k ties go to the lower column index and the index list is stored ascending.
+
+Parity status of each function (what pins it, in tests/test_oracle_pins.py):
+  hessian_diag, sensitivity   pinned: brute-force output error of a one-column perturbation.
+  select_weak                 pinned: exhaustive subset search; planted outlier channel.
+  quantize_rtn                pinned: hand-worked rows (tests/golden/rtn_rows.txt), RTN error
+                              bound, range/zero-point invariants.  The exact choice of
+                              scale/zero among valid min-max RTN variants is a reading, not a
+                              page value (the pages print no quantised example).
+  pack / unpack               pinned: hand-derived packed words (tests/golden/pack_words.txt).
+  dequant                     pinned: exact small-integer cases and the RTN error bound.
+  matmul                      pinned: k = K reproduces W x exactly; k = 0 is the plain quantised
+                              product; the RTN error bound; brute force on tiny shapes.
+  bits_per_weight             pinned: the pages' 3.01 -> 3.012 and 0.21% figures.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "hessian_diag",
+    "quantize_rtn",
+    "dequant",
+    "sensitivity",
+    "select_weak",
+    "owq_quantize",
+    "pack",
+    "unpack",
+    "matmul",
+    "matmul_rows",
+    "bits_per_weight",
+    "layer_bytes",
+]
+
+F16 = np.float16
+F32 = np.float32
+F64 = np.float64
+
+
+# ----------------------------------------------------------------------------------------
+# Calibration statistics and sensitivity
+# ----------------------------------------------------------------------------------------
+def hessian_diag(X: np.ndarray) -> np.ndarray:
+    """lambda_j = sum_t X[t, j]^2, the diagonal of X^T X (fp64, t ascending).
+
+    [PL] "Error Analysis" / appendix §1 Eq. (10): the per-output-channel error is
+    dW_i H dW_i^T with H built from the calibration inputs; [PL] "Error Decomposition":
+    one C_in x C_in Hessian is shared by all output rows. OPTQ's H = 2 X^T X differs from
+    X^T X by a constant factor, which does not change any ranking, so the oracle keeps
+    X^T X.  Only the diagonal enters the weak-column score ([PL] "Weak-column selection").
+    """
+    X64 = np.asarray(X, dtype=F16).astype(F64)
+    lam = np.zeros(X64.shape[1], dtype=F64)
+    for t in range(X64.shape[0]):
+        lam += X64[t] * X64[t]
+    return lam
+
+
+def sensitivity(W: np.ndarray, W_hat0: np.ndarray, lam: np.ndarray) -> np.ndarray:
+    """sens_j = lambda_j * sum_i (W_ij - W_hat0_ij)^2 (fp64, i ascending).
+
+    [PL] "Weak-column selection" (paper p.4): the score of a column combines its
+    perturbation norm with the matching Hessian diagonal element; with a diagonal H the
+    second-order error of appendix Eq. (10) summed over rows is exactly this product.
+    [SUM] "Interesting ideas": the metric multiplies Hessian sensitivity by the weight
+    perturbation.
+    """
+    d = np.asarray(W, dtype=F16).astype(F64) - np.asarray(W_hat0, dtype=F16).astype(F64)
+    col = np.zeros(d.shape[1], dtype=F64)
+    for i in range(d.shape[0]):
+        col += d[i] * d[i]
+    return np.asarray(lam, dtype=F64) * col
+
+
+def select_weak(sens: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k most sensitive columns, returned in ascending order (int32).
+
+    [PL] "Weak-column selection": OWQ keeps the top-k columns by sensitivity in fp16 and
+    excludes them from quantisation. Order: sensitivity descending, ties to the lower
+    column index; the stored list is ascending.
+    """
+    sens = np.asarray(sens, dtype=F64)
+    K = sens.size
+    if not 0 <= k <= K:
+        raise ValueError("k out of range")
+    order = np.lexsort((np.arange(K), -sens))      # primary: -sens ascending; then index
+    return np.sort(order[:k]).astype(np.int32)
+
+
+# ----------------------------------------------------------------------------------------
+# Min-max round-to-nearest quantiser
+# ----------------------------------------------------------------------------------------
+def quantize_rtn(W: np.ndarray, bits: int, group: int, weak_idx=None):
+    """Asymmetric min-max RTN, per output row and per group of `group` contiguous columns.
+
+    Returns (codes uint8 N x K, scales fp16 N x G, zeros fp16 N x G), G = K / group.
+    [SUM] "Key points" names min-max RTN as the simple quantiser OWQ is compared with;
+    [PL] "Weak-column selection": weak columns are excluded from quantisation, so they are
+    left out of their group's min/max and get the code q = z ([PL] "Storage Methods": the
+    latency-favoured matrix is zero-filled at the weak columns).
+
+    For each (row, group), over the group's dense (non-weak) columns, in fp32:
+        mn = min(0, min w), mx = max(0, max w)
+        if mn == mx: mn, mx = -1, 1
+        s  = fp16_rn((mx - mn) / (2^b - 1))         (fp32 subtract and divide, then fp16)
+        if s == 0:  mn, mx = -1, 1 and s recomputed (a range below fp16 resolution)
+        z  = clamp(rint(-mn / s), 0, 2^b - 1)       (stored as an exactly-integral fp16)
+        q  = clamp(rint(w / s) + z, 0, 2^b - 1)     (rint = round half to even)
+    """
+    W = np.asarray(W, dtype=F16)
+    N, K = W.shape
+    if K % group:
+        raise ValueError("K must be a multiple of the group size")
+    G = K // group
+    qmax = (1 << bits) - 1
+    dense = np.ones(K, dtype=bool)
+    if weak_idx is not None and len(weak_idx):
+        dense[np.asarray(weak_idx, dtype=np.int64)] = False
+
+    W32 = W.astype(F32).reshape(N, G, group)
+    # 0 is always inside the range, so a weak column replaced by 0 leaves min/max unchanged.
+    Wm = np.where(dense.reshape(1, G, group), W32, F32(0))
+    mn = np.minimum(Wm.min(axis=2), F32(0))
+    mx = np.maximum(Wm.max(axis=2), F32(0))
+    deg = mn == mx
+    mn = np.where(deg, F32(-1), mn).astype(F32)
+    mx = np.where(deg, F32(1), mx).astype(F32)
+    s16 = ((mx - mn) / F32(qmax)).astype(F16)
+    tiny = s16 == 0
+    if tiny.any():
+        mn = np.where(tiny, F32(-1), mn).astype(F32)
+        mx = np.where(tiny, F32(1), mx).astype(F32)
+        s16 = ((mx - mn) / F32(qmax)).astype(F16)
+    s32 = s16.astype(F32)
+    z32 = np.clip(np.rint(-mn / s32), F32(0), F32(qmax)).astype(F32)
+    q32 = np.clip(np.rint(W32 / s32[:, :, None]) + z32[:, :, None], F32(0), F32(qmax))
+    q32 = np.where(dense.reshape(1, G, group), q32, z32[:, :, None])
+    codes = q32.reshape(N, K).astype(np.uint8)
+    return codes, s16, z32.astype(F16)
+
+
+def dequant(codes: np.ndarray, scales: np.ndarray, zeros: np.ndarray) -> np.ndarray:
+    """W_hat = fp16_rn(s * (q - z)) with the (row, group) scale and zero of each entry.
+
+    q - z is an exact small integer and s * (q - z) is exact in fp32 (an 11-bit times a
+    5-bit significand), so the only rounding is the final one to fp16.
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    G = np.asarray(scales).shape[1]
+    group = K // G
+    s = np.repeat(np.asarray(scales, dtype=F16).astype(F32), group, axis=1)
+    z = np.repeat(np.asarray(zeros, dtype=F16).astype(F32), group, axis=1)
+    return (s * (codes.astype(F32) - z)).astype(F16)
+
+
+def owq_quantize(W: np.ndarray, X: np.ndarray, bits: int, group: int, k: int) -> dict:
+    """The OWQ quantiser used by the oracle: selection, then RTN of the dense part.
+
+    1. lambda = diag(X^T X)                                   (hessian_diag)
+    2. W_hat0 = RTN of W over all columns                      (quantize_rtn, no exclusion)
+    3. sens_j = lambda_j * ||W[:, j] - W_hat0[:, j]||^2        (sensitivity)
+    4. idx = top-k of sens, ascending                          (select_weak)
+    5. codes/scales/zeros = RTN with idx excluded, q = z there (quantize_rtn)
+    6. W_weak = W[:, idx], bit-exact fp16                      ([PL] "Storage Methods")
+    The selection precedes the exclusion, so the score has to come from a quantisation
+    that still includes every column; [PL] "Weak-column selection" then "Low-precision
+    quantization" give that order.
+    """
+    W = np.asarray(W, dtype=F16)
+    lam = hessian_diag(X)
+    c0, s0, z0 = quantize_rtn(W, bits, group, None)
+    sens = sensitivity(W, dequant(c0, s0, z0), lam)
+    idx = select_weak(sens, k)
+    codes, scales, zeros = quantize_rtn(W, bits, group, idx)
+    w_weak = np.ascontiguousarray(W[:, idx])
+    return {"codes": codes, "scales": scales, "zeros": zeros, "idx": idx, "w_weak": w_weak,
+            "lam": lam, "sens": sens}
+
+
+# ----------------------------------------------------------------------------------------
+# Packed layout (latency-favoured, zero-filled; the format of this library)
+# ----------------------------------------------------------------------------------------
+# A row of K codes is cut into chunks of 32 consecutive codes; chunk c of row i is stored
+# as `bits` little-endian 32-bit words at word offset (i * K/32 + c) * bits.  Codes 2t and
+# 2t+1 of a chunk form pair t; the even code sits in the low 16 bits of a word and the odd
+# code in the high 16 bits, at the same offset.
+#   bits = 4: pair t is in word t // 4 at offset 4 * (t % 4) (and 16 + that).
+#   bits = 3: pair t < 15 is in word t // 5 at offset 3 * (t % 5) (and 16 + that);
+#             pair 15: bit e of code 30 is bit 15 of word e, bit e of code 31 is bit 31
+#             of word e (e = 0, 1, 2).
+def pack(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Pack N x K codes into N x (K * bits / 32) uint32 words (format above)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    N, K = codes.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    C = K // 32
+    c = codes.reshape(N, C, 32).astype(np.uint32)
+    words = np.zeros((N, C, bits), dtype=np.uint32)
+    if bits == 4:
+        for t in range(16):
+            j, off = t // 4, 4 * (t % 4)
+            words[:, :, j] |= (c[:, :, 2 * t] << off) | (c[:, :, 2 * t + 1] << (16 + off))
+    elif bits == 3:
+        for t in range(15):
+            j, off = t // 5, 3 * (t % 5)
+            words[:, :, j] |= (c[:, :, 2 * t] << off) | (c[:, :, 2 * t + 1] << (16 + off))
+        for e in range(3):
+            words[:, :, e] |= (((c[:, :, 30] >> e) & 1) << 15) | (((c[:, :, 31] >> e) & 1) << 31)
+    else:
+        raise ValueError("bits must be 3 or 4")
+    return words.reshape(N, C * bits)
+
+
+def unpack(words: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """Inverse of pack: N x (K * bits / 32) uint32 words -> N x K uint8 codes."""
+    words = np.asarray(words, dtype=np.uint32)
+    N = words.shape[0]
+    C = K // 32
+    w = words.reshape(N, C, bits)
+    c = np.zeros((N, C, 32), dtype=np.uint32)
+    if bits == 4:
+        for t in range(16):
+            j, off = t // 4, 4 * (t % 4)
+            c[:, :, 2 * t] = (w[:, :, j] >> off) & 0xF
+            c[:, :, 2 * t + 1] = (w[:, :, j] >> (16 + off)) & 0xF
+    elif bits == 3:
+        for t in range(15):
+            j, off = t // 5, 3 * (t % 5)
+            c[:, :, 2 * t] = (w[:, :, j] >> off) & 0x7
+            c[:, :, 2 * t + 1] = (w[:, :, j] >> (16 + off)) & 0x7
+        for e in range(3):
+            c[:, :, 30] |= ((w[:, :, e] >> 15) & 1) << e
+            c[:, :, 31] |= ((w[:, :, e] >> 31) & 1) << e
+    else:
+        raise ValueError("bits must be 3 or 4")
+    return c.reshape(N, K).astype(np.uint8)
+
+
+# ----------------------------------------------------------------------------------------
+# The product
+# ----------------------------------------------------------------------------------------
+def matmul(W_hat: np.ndarray, w_weak: np.ndarray, idx: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """y64[m, i] = sum_j W_hat[i, j] x[m, j] + sum_t W_weak[i, t] x[m, idx[t]]   (fp64).
+
+    [PL] "Real-device acceleration" (paper "Acceleration on Real Device", p.6): a low-bit
+    dense product plus an fp16 product over the weak-column activation channels gathered
+    on the fly.  W_hat is zero at the weak columns, so the two terms together are the
+    full-precision weak columns times their activations plus the quantised rest.
+    Every fp16 value converts to fp64 exactly; the library matmul accumulates in fp64.
+    """
+    x64 = np.asarray(x, dtype=F16).astype(F64)
+    y = np.asarray(W_hat, dtype=F16).astype(F64) @ x64.T
+    idx = np.asarray(idx, dtype=np.int64)
+    if idx.size:
+        y += np.asarray(w_weak, dtype=F16).astype(F64) @ x64[:, idx].T
+    return np.ascontiguousarray(y.T)
+
+
+def matmul_rows(codes, scales, zeros, w_weak, idx, x, rows) -> np.ndarray:
+    """y64 restricted to the output rows `rows` (for sampled checks of large layers).
+
+    Returns an M x len(rows) array; the same arithmetic as ``matmul`` on those rows.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    W_hat = dequant(np.asarray(codes)[rows], np.asarray(scales)[rows], np.asarray(zeros)[rows])
+    return matmul(W_hat, np.asarray(w_weak)[rows], idx, x)
+
+
+# ----------------------------------------------------------------------------------------
+# Storage accounting
+# ----------------------------------------------------------------------------------------
+def layer_bytes(N: int, K: int, bits: int, group: int, k: int) -> dict:
+    """Bytes of the latency-favoured layout: packed codes, fp16 scale + zero per (row,
+    group), fp16 weak block N x k, int32 index list."""
+    G = K // group
+    return {"packed": N * K * bits // 8, "scales_zeros": N * G * 4, "weak": N * k * 2, "idx": 4 * k}
+
+
+def bits_per_weight(K: int, bits: int, k: float, layout: str = "latency",
+                    group: int | None = None, N: int | None = None) -> float:
+    """Effective bits per weight.
+
+    [PL] "Storage Methods" (appendix §2, pp.10-11): the storage-favoured form keeps only
+    the dense codes plus the fp16 weak columns, b + (16 - b) k / K; the latency-favoured
+    form also keeps the zero-filled codes of the weak columns, b + 16 k / K.  With
+    `group` given, the fp16 scale and zero (32 bits per group) are added; with N also
+    given, the int32 index list (32 k bits over N K weights).
+    """
+    if layout == "storage":
+        b = bits + (16 - bits) * k / K
+    elif layout == "latency":
+        b = bits + 16.0 * k / K
+    else:
+        raise ValueError(layout)
+    if group is not None:
+        b += 32.0 / group
+        if N is not None:
+            b += 32.0 * k / (N * K)
+    return b

@@ -1,0 +1,113 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin catches each one.
+
+Every mutant replaces one oracle function for the duration of a test; the pins of
+test_oracle_pins.py must then fail.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.owq_oracle as oo
+import tests.test_oracle_pins as pins
+
+F16, F32, F64 = np.float16, np.float32, np.float64
+
+
+def _patch(monkeypatch, name, fn):
+    monkeypatch.setattr(oo, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def test_mutant_select_ascending_is_caught(monkeypatch):
+    def bad(sens, k):
+        return np.sort(np.argsort(np.asarray(sens), kind="stable")[:k]).astype(np.int32)
+    _patch(monkeypatch, "select_weak", bad)
+    with pytest.raises(AssertionError):
+        pins.test_planted_outlier_channels_are_selected()
+
+
+def test_mutant_sensitivity_without_hessian_is_caught(monkeypatch):
+    orig = oo.sensitivity
+
+    def bad(W, W_hat0, lam):
+        return orig(W, W_hat0, np.ones_like(np.asarray(lam)))
+    _patch(monkeypatch, "sensitivity", bad)
+    with pytest.raises(AssertionError):
+        pins.test_sensitivity_is_output_error_of_one_column()
+
+
+def test_mutant_sensitivity_on_weights_not_perturbation_is_caught(monkeypatch):
+    def bad(W, W_hat0, lam):
+        d = np.asarray(W, dtype=F16).astype(F64)
+        return np.asarray(lam) * (d * d).sum(axis=0)
+    _patch(monkeypatch, "sensitivity", bad)
+    with pytest.raises(AssertionError):
+        pins.test_sensitivity_is_output_error_of_one_column()
+
+
+def test_mutant_round_half_up_is_caught(monkeypatch, golden_dir):
+    orig_rint = np.rint
+
+    def half_up(v):
+        return np.floor(np.asarray(v) + F32(0.5)).astype(np.asarray(v).dtype)
+    monkeypatch.setattr(oo.np, "rint", half_up)
+    try:
+        with pytest.raises(AssertionError):
+            pins.test_rtn_hand_worked_rows(golden_dir)
+    finally:
+        monkeypatch.setattr(oo.np, "rint", orig_rint)
+
+
+def test_mutant_weak_code_zero_is_caught(monkeypatch):
+    orig = oo.quantize_rtn
+
+    def bad(W, bits, group, weak_idx=None):
+        c, s, z = orig(W, bits, group, weak_idx)
+        if weak_idx is not None and len(weak_idx):
+            c = c.copy()
+            c[:, np.asarray(weak_idx)] = 0
+        return c, s, z
+    _patch(monkeypatch, "quantize_rtn", bad)
+    with pytest.raises(AssertionError):
+        pins.test_rtn_invariants_and_error_bound(3, 64)
+
+
+def test_mutant_dropped_weak_term_is_caught(monkeypatch):
+    def bad(W_hat, w_weak, idx, x):
+        return np.ascontiguousarray((np.asarray(W_hat, F16).astype(F64) @ np.asarray(x, F16).astype(F64).T).T)
+    _patch(monkeypatch, "matmul", bad)
+    with pytest.raises(AssertionError):
+        pins.test_all_columns_weak_is_exact_full_precision_product()
+
+
+def test_mutant_transposed_weak_block_is_caught(monkeypatch):
+    orig = oo.matmul
+
+    def bad(W_hat, w_weak, idx, x):
+        ww = np.asarray(w_weak)
+        return orig(W_hat, ww[::-1] if ww.shape[0] > 1 else ww, idx, x)
+    _patch(monkeypatch, "matmul", bad)
+    with pytest.raises(AssertionError):
+        pins.test_split_product_equals_patched_matrix_brute_force(3, 16, 2)
+
+
+def test_mutant_swapped_pair_halves_is_caught(monkeypatch, golden_dir):
+    orig = oo.pack
+
+    def bad(codes, bits):
+        c = np.asarray(codes).copy()
+        c[:, 0::2], c[:, 1::2] = np.asarray(codes)[:, 1::2], np.asarray(codes)[:, 0::2]
+        return orig(c, bits)
+    _patch(monkeypatch, "pack", bad)
+    with pytest.raises(AssertionError):
+        pins.test_pack_hand_derived_words(golden_dir)
+
+
+def test_mutant_latency_bits_without_zero_fill_is_caught(monkeypatch):
+    orig = oo.bits_per_weight
+
+    def bad(K, bits, k, layout="latency", group=None, N=None):
+        return orig(K, bits, k, "storage" if layout == "latency" else layout, group, N)
+    _patch(monkeypatch, "bits_per_weight", bad)
+    with pytest.raises(AssertionError):
+        pins.test_bits_per_weight_reproduces_page_numbers()
