@@ -1,0 +1,170 @@
+/*
+ * owq.h -- C ABI of the OWQ mixed-precision weight-only matmul for NVIDIA B200 (sm_100a).
+ *
+ * The operation (OWQ, Lee et al., arXiv:2306.02272; pages: "OWQ: Outlier-Aware Weight
+ * Quantization for Efficient Fine-Tuning and Inference of Large Language Models",
+ * paperlayer.ai, items "Weak-column selection" (paper p.4), "Real-device acceleration"
+ * (paper "Acceleration on Real Device", p.6) and "Storage Methods" (appendix §2,
+ * pp.10-11)):
+ *
+ *     y[m, i] = sum_j W_hat[i, j] x[m, j]  +  sum_t W_weak[i, t] x[m, idx[t]]
+ *
+ * W is N x K (N output channels, K input channels; y = x W^T as in a PyTorch Linear).
+ * The dense part W_hat is stored as 3- or 4-bit codes q with an fp16 scale s and an fp16
+ * integral zero point z per (output row, group of `group` consecutive input columns):
+ * W_hat = fp16_rn(s * (q - z)).  The k "weak" columns listed in idx stay in fp16 (W_weak,
+ * N x k) and their codes in the dense matrix are q = z, so the dense part is exactly 0
+ * there (the latency-favoured, zero-filled layout).
+ *
+ * Conventions for every call:
+ *   - fp16 values are passed as their IEEE binary16 bit patterns (uint16_t).
+ *   - Every data pointer is a DEVICE pointer on the current CUDA device, owned by the
+ *     caller, unless the comment says "host".  The library never frees caller memory.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default stream) unless
+ *     its comment says it synchronises.
+ *   - On any error nothing is launched and no output is written; the return value says
+ *     why.  Arguments are validated on the host before any launch.
+ *   - Shapes: K is a multiple of 128 (the packed block), 128 <= K <= 65536, 1 <= N <= 2^20.
+ *     group is K (per output channel) or 128.  bits is 3 or 4.  0 <= k <= K, k <= 1024.
+ *   - Alignment: every device pointer is 16-byte aligned (OWQ_ERR_ALIGN otherwise).
+ */
+#ifndef OWQ_H_
+#define OWQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int owq_status_t;
+#define OWQ_OK            0
+#define OWQ_ERR_NULL      1   /* a required pointer is NULL                                 */
+#define OWQ_ERR_SHAPE     2   /* N, K, M, T or k outside the ranges above                    */
+#define OWQ_ERR_BITS      3   /* bits not 3 or 4                                             */
+#define OWQ_ERR_GROUP     4   /* group neither K nor 128                                     */
+#define OWQ_ERR_INDEX     5   /* idx not strictly ascending or outside [0, K)                */
+#define OWQ_ERR_ALIGN     6   /* a device pointer is not 16-byte aligned                      */
+#define OWQ_ERR_CUDA      7   /* a CUDA runtime call or a launch failed                       */
+#define OWQ_ERR_TIMEOUT   8   /* a bounded device-side wait gave up (see owq_device_status)    */
+#define OWQ_ERR_NOMEM     9   /* a device or host allocation failed                           */
+#define OWQ_ERR_HANDLE    10  /* the layer handle is NULL or not one this library made         */
+#define OWQ_ERR_DEVICE    11  /* no CUDA device, or the device is not sm_100                   */
+
+/* Opaque handle of one packed layer; owns the device buffers owq_pack allocated. */
+typedef struct owq_layer_s* owq_layer_t;
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* owq_stream_t;
+
+/*
+ * owq_quantize -- the OWQ quantiser on the GPU: weak-column selection, then min-max RTN
+ * of the dense columns.  Pages: "Weak-column selection" (paper p.4; the score combines
+ * a column's perturbation norm with its Hessian diagonal) and the min-max RTN quantiser
+ * named in "OWQ -- paper by Lee et al. (2023) -- summary and ideas", Key points.
+ *   lambda_j = sum_t X[t, j]^2                        (fp64, t ascending)
+ *   W_hat0   = min-max RTN of W over all columns
+ *   sens_j   = lambda_j * sum_i (W[i,j] - W_hat0[i,j])^2   (fp64, i ascending)
+ *   idx      = the k largest sens_j (ties: lower j), stored ascending
+ *   codes/scales/zeros = min-max RTN with the idx columns excluded from each range and
+ *              coded q = z;  w_weak[i, t] = W[i, idx[t]] (bit copy).
+ * RTN per (row, group), fp32, round-half-to-even: mn = min(0, min w), mx = max(0, max w)
+ * over the dense columns ([-1, 1] if mn == mx or if the fp16 scale would be 0);
+ * s = fp16(fp32(mx - mn) / (2^bits - 1)); z = clamp(rint(-mn / s)); q = clamp(rint(w / s) + z).
+ * In:  W  fp16 N x K row-major; X fp16 T x K row-major (calibration tokens), 1 <= T <= 2^20.
+ * Out: codes uint8 N x K; scales, zeros fp16 N x (K / group); idx int32 k; w_weak fp16 N x k.
+ * Allocates and frees its own device scratch (stream-ordered; about 20 K + 8 N K / group
+ * bytes).  Deterministic: the same inputs give bit-identical outputs.
+ */
+owq_status_t owq_quantize(const uint16_t* W, const uint16_t* X, int N, int K, int T,
+                          int bits, int group, int k,
+                          uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                          int32_t* idx, uint16_t* w_weak, owq_stream_t stream);
+
+/*
+ * owq_pack -- build a layer handle in the packed, latency-favoured layout ("Storage
+ * Methods", appendix §2: a full low-precision matrix, zero-filled at the weak columns,
+ * plus a separate fp16 block of the weak columns).
+ * In:  codes uint8 N x K (values < 2^bits; the codes of the idx columns are ignored and
+ *      stored as z); scales, zeros fp16 N x (K / group) (zeros integral in [0, 2^bits-1]);
+ *      idx int32 k (device; strictly ascending in [0, K)); w_weak fp16 N x k row-major.
+ *      idx and w_weak may be NULL when k == 0.
+ * Out: *out = a new handle.  The handle owns copies of everything; the inputs may be
+ *      freed once this call returns.
+ * Packed format (per row, 32-code chunks of `bits` uint32 words, little-endian):
+ *   pair t = codes (2t, 2t+1) of a chunk; even code in bits [o, o+bits) and odd code in
+ *   bits [16+o, 16+o+bits) of the same word.  bits=4: word t/4, o = 4 (t%4).  bits=3:
+ *   t < 15 -> word t/5, o = 3 (t%5); bit e of code 30 (31) is bit 15 (31) of word e.
+ * Synchronises `stream` once (idx is copied to the host and validated: OWQ_ERR_INDEX).
+ */
+owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group,
+                      const uint16_t* scales, const uint16_t* zeros,
+                      const int32_t* idx, int k, const uint16_t* w_weak,
+                      owq_stream_t stream, owq_layer_t* out);
+
+/*
+ * owq_gemv -- decode product for 1 <= M <= 16 tokens ("Real-device acceleration",
+ * paper p.6: low-bit dense product plus fp16 weak columns on the activation channels
+ * selected on the fly).  One kernel: 128-bit loads of the packed words, in-register
+ * unpack, fp32 accumulation of exact fp16 products, the weak-column gather and product in
+ * the same pass, warp-shuffle reduction, one fp16 rounding of each output.
+ * In:  x fp16 M x K row-major.   Out: y fp16 M x N row-major (fully overwritten).
+ * Calls on the same handle may run concurrently (the handle is read-only here).
+ */
+owq_status_t owq_gemv(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
+                      owq_stream_t stream);
+
+/*
+ * owq_gemv_multi -- `count` independent decode products in ONE launch (layers that
+ * read their inputs before any of them writes, e.g. q/k/v of one attention block).
+ * layers, xs, ys are HOST arrays of `count` entries; xs[i] is M x K_i and ys[i] is
+ * M x N_i (device).  All layers must share bits; 1 <= count <= 16.  Output buffers must
+ * not overlap inputs of another entry.
+ */
+owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs,
+                            uint16_t* const* ys, int count, int M, owq_stream_t stream);
+
+/*
+ * owq_gemm -- prefill product for any M >= 1 (tuned for M >= 64): TMA-staged packed tiles,
+ * dequantised into shared memory (weak columns patched in as their fp16 values) and fed
+ * to tcgen05 MMA with fp32 accumulators in tensor memory.  Same semantics and layouts as
+ * owq_gemv; M <= 65536.  Bounded device waits: on a timeout the kernel abandons its tile,
+ * sets the device status word and this call's later owq_device_status returns
+ * OWQ_ERR_TIMEOUT (y is then undefined).
+ */
+owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
+                      owq_stream_t stream);
+
+/*
+ * owq_dequant -- test hook: write W_hat = fp16_rn(s * (q - z)) (N x K fp16, 0 at the weak
+ * columns) and, if codes is not NULL, the unpacked codes (N x K uint8).
+ */
+owq_status_t owq_dequant(owq_layer_t layer, uint16_t* w_hat, uint8_t* codes,
+                         owq_stream_t stream);
+
+/* Shape of a layer (host outputs; any may be NULL). */
+owq_status_t owq_layer_info(owq_layer_t layer, int* N, int* K, int* bits, int* group, int* k);
+
+/* Bytes the layer stores, per part (host outputs; any may be NULL): packed codes
+ * N*K*bits/8, scales+zeros 4*N*K/group, weak block 2*N*k, index list 4*k. */
+owq_status_t owq_layer_bytes(owq_layer_t layer, size_t* packed, size_t* scales_zeros,
+                             size_t* weak, size_t* index);
+
+/* Release a layer (stream-ordered on the stream given to owq_pack). NULL is a no-op. */
+owq_status_t owq_layer_free(owq_layer_t layer);
+
+/* Synchronises the device, then returns and clears the device status word that bounded
+ * waits set (OWQ_OK, or OWQ_ERR_TIMEOUT). */
+owq_status_t owq_device_status(void);
+
+/* Static, human-readable name of a status code. */
+const char* owq_status_string(owq_status_t status);
+
+/* Library version as "major.minor.patch" (static string). */
+const char* owq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OWQ_H_ */

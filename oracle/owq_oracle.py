@@ -129,7 +129,7 @@ def quantize_rtn(W: np.ndarray, bits: int, group: int, weak_idx=None):
         if mn == mx: mn, mx = -1, 1
         s  = fp16_rn((mx - mn) / (2^b - 1))         (fp32 subtract and divide, then fp16)
         if s == 0:  mn, mx = -1, 1 and s recomputed (a range below fp16 resolution)
-        z  = clamp(rint(-mn / s), 0, 2^b - 1)       (stored as an exactly-integral fp16)
+        z  = clamp(rint(-mn / s), 0, 2^b - 1)       (an exactly-integral fp16, +0 for zero)
         q  = clamp(rint(w / s) + z, 0, 2^b - 1)     (rint = round half to even)
     """
     W = np.asarray(W, dtype=F16)
@@ -157,7 +157,8 @@ def quantize_rtn(W: np.ndarray, bits: int, group: int, weak_idx=None):
         mx = np.where(tiny, F32(1), mx).astype(F32)
         s16 = ((mx - mn) / F32(qmax)).astype(F16)
     s32 = s16.astype(F32)
-    z32 = np.clip(np.rint(-mn / s32), F32(0), F32(qmax)).astype(F32)
+    # the zero point is an integer: "+ 0" maps a -0.0 (from mn == 0) to the canonical +0
+    z32 = (np.clip(np.rint(-mn / s32), F32(0), F32(qmax)) + F32(0)).astype(F32)
     q32 = np.clip(np.rint(W32 / s32[:, :, None]) + z32[:, :, None], F32(0), F32(qmax))
     q32 = np.where(dense.reshape(1, G, group), q32, z32[:, :, None])
     codes = q32.reshape(N, K).astype(np.uint8)

@@ -1,0 +1,84 @@
+"""The C-ABI library loads, exports every symbol include/owq.h declares, and rejects bad
+arguments on the host (no GPU needed for any of these)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+
+def _gpu_present():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.fixture(scope="module")
+def owq():
+    from weight_only_mixed_owq_b200 import build
+    build.build()
+    import weight_only_mixed_owq_b200 as m
+    return m
+
+
+def _declared_functions():
+    txt = open(os.path.join(ROOT, "include", "owq.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(owq_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for must in ("owq_pack", "owq_gemv", "owq_gemm", "owq_quantize", "owq_dequant"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(owq):
+    lib = ctypes.CDLL(owq.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert {p[0] for p in owq.PROTOTYPES} == set(_declared_functions())
+
+
+def test_status_strings_and_version(owq):
+    for code, name in owq.STATUS_NAMES.items():
+        assert owq.owq_status_string(code).startswith(name)
+    assert re.match(r"^\d+\.\d+\.\d+$", owq.owq_version())
+
+
+def test_host_validation_rejects_bad_arguments(owq):
+    A = 0x10000  # never dereferenced: every call below fails validation first
+    # NULL pointers
+    assert owq.owq_quantize(None, A, 16, 128, 8, 3, 128, 1, A, A, A, A, A) == 1
+    st, h = owq.owq_pack(None, 16, 128, 3, 128, A, A, A, 1, A)
+    assert st == 1 and h is None
+    # bits, group, shape
+    assert owq.owq_quantize(A, A, 16, 128, 8, 5, 128, 1, A, A, A, A, A) == 3
+    assert owq.owq_quantize(A, A, 16, 256, 8, 3, 64, 1, A, A, A, A, A) == 4
+    assert owq.owq_quantize(A, A, 16, 100, 8, 3, 100, 1, A, A, A, A, A) == 2
+    assert owq.owq_quantize(A, A, 0, 128, 8, 3, 128, 1, A, A, A, A, A) == 2
+    assert owq.owq_quantize(A, A, 16, 128, 0, 3, 128, 1, A, A, A, A, A) == 2
+    assert owq.owq_quantize(A, A, 16, 128, 8, 3, 128, 129, A, A, A, A, A) == 2
+    # alignment
+    assert owq.owq_quantize(A + 2, A, 16, 128, 8, 3, 128, 1, A, A, A, A, A) == 6
+    # handles
+    assert owq.owq_gemv(None, A, A, 1) == 10
+    assert owq.owq_gemv(A, A, A, 1) == 10
+    assert owq.owq_gemm(A, A, A, 64) == 10
+    assert owq.owq_dequant(A, A) == 10
+    assert owq.owq_layer_free(A) == 10
+    assert owq.owq_layer_free(None) == 0
+    assert owq.owq_layer_info(A)[0] == 10
+    assert owq.owq_layer_bytes(A)[0] == 10
+
+
+@pytest.mark.skipif(_gpu_present(), reason="checks the no-device path; needs a machine without a GPU")
+def test_valid_arguments_without_device_report_device_error(owq):
+    A = 0x10000
+    assert owq.owq_quantize(A, A, 16, 128, 8, 3, 128, 1, A, A, A, A, A) == 11
+    st, _ = owq.owq_pack(A, 16, 128, 3, 128, A, A, A, 1, A)
+    assert st == 11

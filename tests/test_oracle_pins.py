@@ -81,6 +81,14 @@ def test_rtn_invariants_and_error_bound(bits, group):
     assert G == s.shape[1]
 
 
+def test_rtn_zero_point_is_canonical_integer():
+    # a row with no negative entry has mn = 0, so z = 0: stored as +0 (bits 0x0000)
+    W = np.array([[0.0, 0.25, 0.5, 1.0, -0.0, 0.125, 0.75, 0.0]], dtype=F16)
+    c, s, z = oracle.quantize_rtn(W, 3, 8)
+    assert z.view(np.uint16)[0, 0] == 0
+    assert c[0].tolist() == [0, 2, 4, 7, 0, 1, 5, 0]
+
+
 def test_rtn_k_equal_bits_reaches_extremes():
     # a row whose min and max are both non-zero uses code 0 and code 2^b - 1 exactly
     W = np.array([[-0.5, 0.25, 0.1, 1.25, 0.0, -0.3, 0.7, 0.9]], dtype=F16)

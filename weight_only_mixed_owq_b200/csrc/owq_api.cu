@@ -1,0 +1,313 @@
+// C ABI of the library (declared in include/owq.h): argument validation, layer handles,
+// launches.  Every argument is validated on the host before anything is launched.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <unordered_set>
+#include <vector>
+
+#include "owq_internal.cuh"
+
+namespace owq {
+
+__device__ int g_device_status;
+
+int* device_status_ptr() {
+  int* p = nullptr;
+  if (cudaGetSymbolAddress((void**)&p, g_device_status) != cudaSuccess) return nullptr;
+  return p;
+}
+
+namespace {
+
+std::mutex g_mu;
+std::unordered_set<Layer*>& registry() {
+  static std::unordered_set<Layer*> s;
+  return s;
+}
+
+Layer* lookup(owq_layer_t h) {
+  Layer* L = reinterpret_cast<Layer*>(h);
+  if (!L) return nullptr;
+  std::lock_guard<std::mutex> g(g_mu);
+  return registry().count(L) ? L : nullptr;
+}
+
+owq_status_t check_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_DEVICE; }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return OWQ_ERR_DEVICE;
+  }
+  return major == 10 ? OWQ_OK : OWQ_ERR_DEVICE;
+}
+
+owq_status_t check_shape(int N, int K, int bits, int group, int k) {
+  if (bits != 3 && bits != 4) return OWQ_ERR_BITS;
+  if (N < 1 || N > (1 << 20) || K < kBlockCodes || K > 65536 || K % kBlockCodes) return OWQ_ERR_SHAPE;
+  if (group != K && group != 128) return OWQ_ERR_GROUP;
+  if (k < 0 || k > K || k > kMaxWeak) return OWQ_ERR_SHAPE;
+  return OWQ_OK;
+}
+
+owq_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return OWQ_OK;
+  cudaGetLastError();
+  return e == cudaErrorMemoryAllocation ? OWQ_ERR_NOMEM : OWQ_ERR_CUDA;
+}
+
+void release(Layer* L) {
+  if (!L) return;
+  cudaFree(L->packed);
+  cudaFree(L->scales);
+  cudaFree(L->zeros);
+  cudaFree(L->w_weak);
+  cudaFree(L->idx);
+  cudaFree(L->blk_weak);
+  delete[] L->idx_host;
+  L->magic = 0;
+  delete L;
+}
+
+}  // namespace
+}  // namespace owq
+
+using namespace owq;
+
+extern "C" {
+
+const char* owq_status_string(owq_status_t s) {
+  switch (s) {
+    case OWQ_OK: return "OWQ_OK";
+    case OWQ_ERR_NULL: return "OWQ_ERR_NULL: a required pointer is NULL";
+    case OWQ_ERR_SHAPE: return "OWQ_ERR_SHAPE: N, K, M, T or k out of range";
+    case OWQ_ERR_BITS: return "OWQ_ERR_BITS: bits must be 3 or 4";
+    case OWQ_ERR_GROUP: return "OWQ_ERR_GROUP: group must be K or 128";
+    case OWQ_ERR_INDEX: return "OWQ_ERR_INDEX: idx must be strictly ascending in [0, K)";
+    case OWQ_ERR_ALIGN: return "OWQ_ERR_ALIGN: device pointers must be 16-byte aligned";
+    case OWQ_ERR_CUDA: return "OWQ_ERR_CUDA: a CUDA call or launch failed";
+    case OWQ_ERR_TIMEOUT: return "OWQ_ERR_TIMEOUT: a bounded device wait gave up";
+    case OWQ_ERR_NOMEM: return "OWQ_ERR_NOMEM: allocation failed";
+    case OWQ_ERR_HANDLE: return "OWQ_ERR_HANDLE: not a live layer handle";
+    case OWQ_ERR_DEVICE: return "OWQ_ERR_DEVICE: no sm_100 CUDA device";
+    default: return "OWQ: unknown status";
+  }
+}
+
+const char* owq_version(void) { return "0.1.0"; }
+
+owq_status_t owq_quantize(const uint16_t* W, const uint16_t* X, int N, int K, int T, int bits,
+                          int group, int k, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                          int32_t* idx, uint16_t* w_weak, owq_stream_t stream) {
+  if (!W || !X || !codes || !scales || !zeros) return OWQ_ERR_NULL;
+  if (k > 0 && (!idx || !w_weak)) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, group, k);
+  if (st) return st;
+  if (T < 1 || T > (1 << 20)) return OWQ_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros) ||
+      (k > 0 && (!aligned16(idx) || !aligned16(w_weak))))
+    return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  return cuda_status(launch_quantize(reinterpret_cast<const __half*>(W), reinterpret_cast<const __half*>(X),
+                                     N, K, T, bits, group, k, codes, reinterpret_cast<__half*>(scales),
+                                     reinterpret_cast<__half*>(zeros), idx, reinterpret_cast<__half*>(w_weak),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, const uint16_t* scales,
+                      const uint16_t* zeros, const int32_t* idx, int k, const uint16_t* w_weak,
+                      owq_stream_t stream, owq_layer_t* out) {
+  if (!out) return OWQ_ERR_NULL;
+  *out = nullptr;
+  if (!codes || !scales || !zeros) return OWQ_ERR_NULL;
+  if (k > 0 && (!idx || !w_weak)) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, group, k);
+  if (st) return st;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(zeros) ||
+      (k > 0 && (!aligned16(idx) || !aligned16(w_weak))))
+    return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // idx: copy to the host and validate before anything is allocated or launched
+  std::vector<int32_t> hidx(k);
+  if (k > 0) {
+    if (cudaMemcpyAsync(hidx.data(), idx, sizeof(int32_t) * k, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return OWQ_ERR_CUDA;
+    }
+    for (int t = 0; t < k; ++t) {
+      if (hidx[t] < 0 || hidx[t] >= K) return OWQ_ERR_INDEX;
+      if (t > 0 && hidx[t] <= hidx[t - 1]) return OWQ_ERR_INDEX;
+    }
+  }
+
+  Layer* L = new (std::nothrow) Layer();
+  if (!L) return OWQ_ERR_NOMEM;
+  L->magic = kLayerMagic;
+  cudaGetDevice(&L->device);
+  L->N = N; L->K = K; L->bits = bits; L->group = group; L->G = K / group; L->k = k;
+  L->k_ld = std::max(8, (k + 7) & ~7);
+  L->stream = s;
+  L->maps_ready = false;
+  const size_t packed_bytes = (size_t)N * K * bits / 8;
+  const size_t sz_bytes = (size_t)N * L->G * sizeof(__half);
+  const size_t weak_bytes = (size_t)N * L->k_ld * sizeof(__half);
+  const int Kb = K / kBlockCodes;
+  L->idx_host = new (std::nothrow) int32_t[std::max(k, 1)];
+  if (!L->idx_host) { release(L); return OWQ_ERR_NOMEM; }
+  std::copy(hidx.begin(), hidx.end(), L->idx_host);
+
+  cudaError_t e = cudaSuccess;
+  auto alloc = [&](void** p, size_t n) { if (e == cudaSuccess) e = cudaMalloc(p, std::max<size_t>(n, 16)); };
+  alloc((void**)&L->packed, packed_bytes);
+  alloc((void**)&L->scales, sz_bytes);
+  alloc((void**)&L->zeros, sz_bytes);
+  alloc((void**)&L->w_weak, weak_bytes);
+  alloc((void**)&L->idx, sizeof(int32_t) * std::max(k, 1));
+  alloc((void**)&L->blk_weak, sizeof(int32_t) * (Kb + 1));
+  uint32_t* mask_dev = nullptr;
+  alloc((void**)&mask_dev, sizeof(uint32_t) * (K / 32));
+  if (e != cudaSuccess) { cudaFree(mask_dev); release(L); return cuda_status(e); }
+
+  // host-side tables: weak bitmask per 32-code chunk, weak range per 128-code block
+  std::vector<uint32_t> mask(K / 32, 0u);
+  std::vector<int32_t> blk(Kb + 1, 0);
+  for (int t = 0; t < k; ++t) mask[hidx[t] / 32] |= 1u << (hidx[t] % 32);
+  for (int b = 0, t = 0; b <= Kb; ++b) {
+    while (t < k && hidx[t] < b * kBlockCodes) ++t;
+    blk[b] = t;
+  }
+
+  if (e == cudaSuccess) e = cudaMemcpyAsync(L->scales, scales, sz_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(L->zeros, zeros, sz_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(L->w_weak, 0, weak_bytes, s);
+  if (e == cudaSuccess && k > 0)
+    e = cudaMemcpy2DAsync(L->w_weak, (size_t)L->k_ld * sizeof(__half), w_weak, (size_t)k * sizeof(__half),
+                          (size_t)k * sizeof(__half), N, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && k > 0) e = cudaMemcpyAsync(L->idx, idx, sizeof(int32_t) * k, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(L->blk_weak, blk.data(), sizeof(int32_t) * (Kb + 1), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(mask_dev, mask.data(), sizeof(uint32_t) * (K / 32), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = launch_pack(codes, reinterpret_cast<const __half*>(zeros), mask_dev, N, K, bits, group, L->packed, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // host tables above must outlive the copies
+  cudaFree(mask_dev);
+  if (e != cudaSuccess) { release(L); return cuda_status(e); }
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    registry().insert(L);
+  }
+  *out = reinterpret_cast<owq_layer_t>(L);
+  return OWQ_OK;
+}
+
+static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvProblem* P) {
+  if (!x || !y) return OWQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(y)) return OWQ_ERR_ALIGN;
+  P->packed = L->packed;
+  P->scales = L->scales;
+  P->zeros = L->zeros;
+  P->w_weak = L->w_weak;
+  P->idx = L->idx;
+  P->x = reinterpret_cast<const __half*>(x);
+  P->y = reinterpret_cast<__half*>(y);
+  P->N = L->N; P->K = L->K; P->G = L->G; P->k = L->k; P->k_ld = L->k_ld;
+  P->row_groups = 0; P->group_base = 0;
+  return OWQ_OK;
+}
+
+owq_status_t owq_gemv(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, owq_stream_t stream) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (M < 1 || M > kMaxGemvM) return OWQ_ERR_SHAPE;
+  GemvProblem P;
+  owq_status_t st = make_problem(L, x, y, &P);
+  if (st) return st;
+  return cuda_status(launch_gemv(&P, 1, L->bits, M, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs, uint16_t* const* ys,
+                            int count, int M, owq_stream_t stream) {
+  if (!layers || !xs || !ys) return OWQ_ERR_NULL;
+  if (count < 1 || count > 16 || M < 1 || M > kMaxGemvM) return OWQ_ERR_SHAPE;
+  GemvProblem P[16];
+  int bits = 0;
+  for (int q = 0; q < count; ++q) {
+    Layer* L = lookup(layers[q]);
+    if (!L) return OWQ_ERR_HANDLE;
+    if (q == 0) bits = L->bits;
+    else if (L->bits != bits) return OWQ_ERR_BITS;
+    owq_status_t st = make_problem(L, xs[q], ys[q], &P[q]);
+    if (st) return st;
+  }
+  return cuda_status(launch_gemv(P, count, bits, M, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, owq_stream_t stream) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (M < 1 || M > 65536) return OWQ_ERR_SHAPE;
+  if (!x || !y) return OWQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(y)) return OWQ_ERR_ALIGN;
+  return gemm_sm100(*L, reinterpret_cast<const __half*>(x), reinterpret_cast<__half*>(y), M,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+owq_status_t owq_dequant(owq_layer_t layer, uint16_t* w_hat, uint8_t* codes, owq_stream_t stream) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (!w_hat) return OWQ_ERR_NULL;
+  if (!aligned16(w_hat) || (codes && !aligned16(codes))) return OWQ_ERR_ALIGN;
+  return cuda_status(launch_dequant(*L, reinterpret_cast<__half*>(w_hat), codes,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+owq_status_t owq_layer_info(owq_layer_t layer, int* N, int* K, int* bits, int* group, int* k) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (N) *N = L->N;
+  if (K) *K = L->K;
+  if (bits) *bits = L->bits;
+  if (group) *group = L->group;
+  if (k) *k = L->k;
+  return OWQ_OK;
+}
+
+owq_status_t owq_layer_bytes(owq_layer_t layer, size_t* packed, size_t* scales_zeros, size_t* weak,
+                             size_t* index) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (packed) *packed = (size_t)L->N * L->K * L->bits / 8;
+  if (scales_zeros) *scales_zeros = (size_t)L->N * L->G * 4;
+  if (weak) *weak = (size_t)L->N * L->k * 2;
+  if (index) *index = (size_t)L->k * 4;
+  return OWQ_OK;
+}
+
+owq_status_t owq_layer_free(owq_layer_t layer) {
+  if (!layer) return OWQ_OK;
+  Layer* L = reinterpret_cast<Layer*>(layer);
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!registry().erase(L)) return OWQ_ERR_HANDLE;
+  }
+  release(L);
+  return OWQ_OK;
+}
+
+owq_status_t owq_device_status(void) {
+  owq_status_t st = check_device();
+  if (st) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_CUDA; }
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_CUDA; }
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_CUDA; }
+  return v ? OWQ_ERR_TIMEOUT : OWQ_OK;
+}
+
+}  // extern "C"

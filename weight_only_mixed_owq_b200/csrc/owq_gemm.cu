@@ -1,0 +1,351 @@
+// Prefill product y = W_tilde x^T for many tokens on the 5th-generation tensor cores.
+//
+// Pages: "Real-device acceleration" (OWQ paper "Acceleration on Real Device", p.6, as
+// summarised on paperlayer.ai: a 3-bit weight x fp16 activation product with the weak-
+// column activations picked on the fly) and "Storage Methods" (appendix §2: the dense
+// low-precision matrix is zero-filled at the weak columns, the weak columns are a separate
+// fp16 block).  W_tilde is the dequantised dense matrix with its weak columns replaced by
+// their fp16 values, so y = W_hat x + W_weak x[idx] exactly as the method defines it.
+//
+// One CTA computes a 128-weight-row x BN-token tile of y^T (MMA M = weight rows,
+// MMA N = tokens), looping over K in 128-code steps through an S-stage ring:
+//   warp 0      TMA producer: the packed 128 x (16*bits) byte tile (no swizzle) and two
+//               128B-swizzled BN x 64 fp16 activation boxes per step.
+//   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16,
+//               fp32 accumulator BN columns wide in tensor memory).
+//   warps 2-9   dequantisation: each thread owns one weight row and one 64-code half of a
+//               step, unpacks the codes in registers, forms fp16_rn(s (q - z)) with exact
+//               fp16x2 arithmetic, stores the 16-byte chunks into the K-major 128B-swizzled
+//               A tile, then overwrites the weak columns of that slab with their fp16
+//               values (no activation gather is needed).  The same warps run the epilogue
+//               (tcgen05.ld of their TMEM lane quarter, fp16 rounding, coalesced stores).
+// Every mbarrier wait is bounded (clock64 limit): on expiry the thread records the device
+// status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
+#include <cstring>
+
+#include "owq_internal.cuh"
+#include "owq_sm100.cuh"
+
+namespace owq {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;               // weight rows per tile (MMA M)
+constexpr int kStepCodes = 128;        // K per pipeline step
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = 32 * (2 + kDequantWarps);
+constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
+
+template <int BITS, int BN>
+struct Smem {
+  static constexpr int kX = 2 * BN * 128;           // two 64-column swizzled boxes
+  static constexpr int kA = 2 * kBM * 128;          // two 64-column swizzled slabs
+  static constexpr int kP = kBM * 16 * BITS;        // packed tile
+  static constexpr int kStage = ((kX + kA + kP) + 1023) & ~1023;
+};
+
+template <int BITS, int BN, int S>
+constexpr int smem_bytes() { return S * Smem<BITS, BN>::kStage + 1024 /*barriers*/ + 1024 /*align slack*/; }
+
+struct GemmParams {
+  const __half* scales;
+  const __half* zeros;
+  const __half* w_weak;
+  const int32_t* idx;
+  const int32_t* blk_weak;
+  __half* y;
+  int* status;
+  int N, K, M, G, k_ld;
+};
+
+// fp16x2 helpers (exact integer arithmetic on small values)
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_splat(float v) {
+  __half h = __float2half_rn(v);
+  uint32_t u = __half_as_ushort(h);
+  return u | (u << 16);
+}
+
+// Dequantise one 32-code chunk into 16 fp16x2 values (k = 2t, 2t+1 in pair t).
+// A pair at bit offset o is lifted as (v & mask) | 0x6400 per half = 1024 + q 2^o, then
+// (1024 + q 2^o) * 2^-o - (1024 2^-o + z) = q - z exactly, then * s: fp16_rn(s (q - z)).
+template <int BITS>
+__device__ __forceinline__ void dequant_chunk(const uint32_t* w, uint32_t s2, const uint32_t* scl,
+                                              const uint32_t* nz, uint32_t* out) {
+  constexpr uint32_t kMagic = 0x64006400u;
+  if constexpr (BITS == 3) {
+    #pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const uint32_t v = w[j], u = v >> 9;
+      out[5 * j + 0] = h2_mul(h2_fma((v & 0x00070007u) | kMagic, scl[0], nz[0]), s2);
+      out[5 * j + 1] = h2_mul(h2_fma((v & 0x00380038u) | kMagic, scl[1], nz[1]), s2);
+      out[5 * j + 2] = h2_mul(h2_fma((v & 0x01C001C0u) | kMagic, scl[2], nz[2]), s2);
+      out[5 * j + 3] = h2_mul(h2_fma((u & 0x00070007u) | kMagic, scl[0], nz[0]), s2);
+      out[5 * j + 4] = h2_mul(h2_fma((u & 0x00380038u) | kMagic, scl[1], nz[1]), s2);
+    }
+    const uint32_t p15 = ((w[0] >> 15) & 0x00010001u) | ((w[1] >> 14) & 0x00020002u) |
+                         ((w[2] >> 13) & 0x00040004u);
+    out[15] = h2_mul(h2_fma(p15 | kMagic, scl[0], nz[0]), s2);
+  } else {
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t v = w[j], u = v >> 8;
+      out[4 * j + 0] = h2_mul(h2_fma((v & 0x000F000Fu) | kMagic, scl[0], nz[0]), s2);
+      out[4 * j + 1] = h2_mul(h2_fma((v & 0x00F000F0u) | kMagic, scl[1], nz[1]), s2);
+      out[4 * j + 2] = h2_mul(h2_fma((u & 0x000F000Fu) | kMagic, scl[0], nz[0]), s2);
+      out[4 * j + 3] = h2_mul(h2_fma((u & 0x00F000F0u) | kMagic, scl[1], nz[1]), s2);
+    }
+  }
+}
+
+// byte offset of (row r, 16-byte chunk c) inside a 128-row, 128B-swizzled K-major slab
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+template <int BITS, int BN, int S>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_p,
+             const __grid_constant__ GemmParams p) {
+  using L = Smem<BITS, BN>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage);
+  uint64_t* full = bars;            // [S] TMA landed
+  uint64_t* empty = bars + S;       // [S] MMAs of the stage done
+  uint64_t* afull = bars + 2 * S;   // [S] A tile written
+  uint64_t* accf = bars + 3 * S;    // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBM;      // first weight row
+  const int m0 = blockIdx.y * BN;       // first token
+  const int nK = p.K / kStepCodes;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&afull[s], 32 * kDequantWarps);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+    prefetch_tmap(&map_x);
+    prefetch_tmap(&map_p);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      constexpr uint32_t kBytes = L::kX + L::kP;
+      bool ok = true;
+      for (int kb = 0; kb < nK && ok; ++kb) {
+        const int s = kb % S, u = kb / S;
+        if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, p.status, kWaitLimit);
+        if (!ok) break;
+        unsigned char* st = smem + s * L::kStage;
+        mbar_arrive_expect_tx(&full[s], kBytes);
+        tma_load_2d(st + L::kX + L::kA, &map_p, &full[s], kb * 16 * BITS, n0);
+        tma_load_2d(st, &map_x, &full[s], kb * kStepCodes, m0);
+        tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
+      }
+      // never leave with copies in flight: wait for the last use of every stage
+      for (int kb = (nK > S ? nK - S : 0); kb < nK; ++kb)
+        mbar_wait(&full[kb % S], (kb / S) & 1, p.status, kWaitLimit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_f16_f32(kBM, BN);
+      bool ok = true;
+      for (int kb = 0; kb < nK && ok; ++kb) {
+        const int s = kb % S, u = kb / S;
+        ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit) &&
+             mbar_wait(&afull[s], u & 1, p.status, kWaitLimit);
+        if (!ok) break;
+        tc_fence_after();
+        unsigned char* st = smem + s * L::kStage;
+        const uint32_t xa = smem_u32(st), aa = smem_u32(st + L::kX);
+        #pragma unroll
+        for (int a = 0; a < 2; ++a)
+          #pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = desc_sw128_kmajor(aa + a * kBM * 128 + kk * 32);
+            const uint64_t bd = desc_sw128_kmajor(xa + a * BN * 128 + kk * 32);
+            mma_f16(tmem, ad, bd, idesc, (kb | a | kk) != 0);
+          }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accf);
+    }
+  } else {
+    // ---------------- dequantisation ----------------
+    const int td = threadIdx.x - 64;          // 0..255
+    const int r = td & (kBM - 1), h = td >> 7;
+    const int row = min(n0 + r, p.N - 1);
+    const bool per_channel = p.G == 1;
+    uint32_t s2 = 0, scl[3], nz[3];
+    constexpr float kOff[3] = {1.f, BITS == 3 ? 8.f : 16.f, 64.f};
+    scl[0] = h2_splat(1.f);
+    scl[1] = h2_splat(1.f / kOff[1]);
+    scl[2] = h2_splat(1.f / kOff[2]);
+    auto load_sz = [&](int g) {
+      const __half sh = p.scales[(size_t)row * p.G + g];
+      const float z = __half2float(p.zeros[(size_t)row * p.G + g]);
+      const uint32_t su = __half_as_ushort(sh);
+      s2 = su | (su << 16);
+      #pragma unroll
+      for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
+    };
+    if (per_channel) load_sz(0);
+    bool ok = true;
+    for (int kb = 0; kb < nK && ok; ++kb) {
+      const int s = kb % S, u = kb / S;
+      if (!per_channel) load_sz(kb);
+      ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit);
+      if (!ok) break;
+      unsigned char* st = smem + s * L::kStage;
+      const uint32_t* pw = reinterpret_cast<const uint32_t*>(st + L::kX + L::kA + r * 16 * BITS) + h * 2 * BITS;
+      unsigned char* slab = st + L::kX + h * kBM * 128;
+      #pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t w[BITS];
+        #pragma unroll
+        for (int j = 0; j < BITS; ++j) w[j] = pw[cc * BITS + j];
+        uint32_t o[16];
+        dequant_chunk<BITS>(w, s2, scl, nz, o);
+        #pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(slab + sw128_off(r, cc * 4 + j)) =
+              make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      }
+      // weak columns of this 64-code slab: their fp16 values replace the zero-filled codes
+      const int t0 = p.blk_weak[kb], t1 = p.blk_weak[kb + 1];
+      for (int t = t0; t < t1; ++t) {
+        const int col = p.idx[t] - kb * kStepCodes;
+        if ((col >> 6) != h) continue;
+        const int c = col & 63;
+        __half* dst = reinterpret_cast<__half*>(slab + sw128_off(r, c >> 3)) + (c & 7);
+        *dst = p.w_weak[(size_t)row * p.k_ld + t];
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&afull[s]);
+    }
+
+    // ---------------- epilogue ----------------
+    const int wd = warp - 2, q = warp & 3, chalf = wd >> 2;
+    const bool acc_ok = mbar_wait(accf, 0, p.status, kWaitLimit);
+    tc_fence_after();
+    const int orow = n0 + 32 * q + lane;
+    #pragma unroll 1
+    for (int c0 = chalf * (BN / 2); c0 < (chalf + 1) * (BN / 2); c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+      tmem_ld_wait();
+      if (acc_ok && orow < p.N) {
+        #pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = m0 + c0 + j;
+          if (t < p.M) p.y[(size_t)t * p.N + orow] = __float2half_rn(__uint_as_float(v[j]));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+    tmem_relinquish();
+  }
+}
+
+// ---- host side ----
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encoder() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(f);
+  }
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiled enc = get_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BITS, int BN, int S>
+owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
+  if (!L.maps_ready) {
+    const uint64_t rb = (uint64_t)L.K * BITS / 8;
+    if (!encode_2d(&L.map_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.packed, rb, (uint64_t)L.N, rb,
+                   16 * BITS, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return OWQ_ERR_CUDA;
+    L.maps_ready = true;
+  }
+  CUtensorMap mx;
+  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, 64, BN,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return OWQ_ERR_CUDA;
+  GemmParams prm;
+  prm.scales = L.scales; prm.zeros = L.zeros; prm.w_weak = L.w_weak; prm.idx = L.idx;
+  prm.blk_weak = L.blk_weak; prm.y = y; prm.status = device_status_ptr();
+  prm.N = L.N; prm.K = L.K; prm.M = M; prm.G = L.G; prm.k_ld = L.k_ld;
+  if (!prm.status) return OWQ_ERR_CUDA;
+  auto kern = k_gemm_sm100<BITS, BN, S>;
+  constexpr int smem = smem_bytes<BITS, BN, S>();
+  static_assert(smem <= 232448, "shared memory budget");
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return OWQ_ERR_CUDA;
+  }
+  dim3 grid((L.N + kBM - 1) / kBM, (M + BN - 1) / BN);
+  kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, prm);
+  if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
+  return OWQ_OK;
+}
+
+template <int BITS>
+owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
+  if (M <= 64) return run<BITS, 64, 4>(L, x, y, M, s);
+  return run<BITS, 128, 3>(L, x, y, M, s);
+}
+
+}  // namespace
+
+owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
+  return L.bits == 3 ? dispatch<3>(L, x, y, M, s) : dispatch<4>(L, x, y, M, s);
+}
+
+}  // namespace owq

@@ -1,0 +1,69 @@
+// Internal declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda.h>
+
+#include "../../include/owq.h"
+
+namespace owq {
+
+constexpr uint32_t kLayerMagic = 0x4f575131u;  // "OWQ1"
+constexpr int kBlockCodes = 128;               // codes per packed block (16 * bits bytes)
+constexpr int kChunkCodes = 32;                // codes per chunk (bits words)
+constexpr int kMaxWeak = 1024;
+constexpr int kMaxGemvM = 16;
+
+struct Layer {
+  uint32_t magic;
+  int device;
+  int N, K, bits, group, G, k, k_ld;   // k_ld: row stride of w_weak (k rounded up to 8)
+  uint32_t* packed;     // N x (K*bits/32) words
+  __half* scales;       // N x G
+  __half* zeros;        // N x G
+  __half* w_weak;       // N x k_ld (zero padded)
+  int32_t* idx;         // k (device)
+  int32_t* blk_weak;    // K/128 + 1 offsets into idx: weak columns of packed block b are
+                        // idx[blk_weak[b] .. blk_weak[b+1])
+  int32_t* idx_host;    // k (host copy)
+  cudaStream_t stream;  // stream of owq_pack (used to order the release)
+  // tcgen05 GEMM tensor maps, encoded lazily on first use
+  bool maps_ready;
+  alignas(64) CUtensorMap map_packed;
+  alignas(64) CUtensorMap map_weak;
+};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device status word set by bounded waits (owq_device_status reads and clears it).
+int* device_status_ptr();
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_pack(const uint8_t* codes, const __half* zeros, const uint32_t* weak_mask,
+                        int N, int K, int bits, int group, uint32_t* packed, cudaStream_t s);
+cudaError_t launch_dequant(const Layer& L, __half* w_hat, uint8_t* codes, cudaStream_t s);
+
+struct GemvProblem {
+  const uint32_t* packed;
+  const __half* scales;
+  const __half* zeros;
+  const __half* w_weak;
+  const int32_t* idx;
+  const __half* x;
+  __half* y;
+  int N, K, G, k, k_ld;
+  int row_groups;     // ceil(N / rows_per_group)
+  int group_base;     // first global row-group index of this problem
+};
+cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cudaStream_t s);
+
+cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int T, int bits,
+                            int group, int k, uint8_t* codes, __half* scales, __half* zeros,
+                            int32_t* idx, __half* w_weak, cudaStream_t s);
+
+owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, cudaStream_t s);
+
+}  // namespace owq

@@ -1,0 +1,220 @@
+// OWQ quantiser on the GPU: Hessian diagonal, all-column RTN pre-quantisation, column
+// sensitivity, top-k weak-column selection, then min-max RTN of the dense columns.
+//
+// Pages: "OWQ: Outlier-Aware Weight Quantization for Efficient Fine-Tuning and Inference
+// of Large Language Models" (paperlayer.ai), "Weak-column selection" (paper p.4: the score
+// of a column combines its perturbation norm with its Hessian diagonal element; the top-k
+// columns stay in fp16 and are excluded from quantisation), "Error Analysis" / appendix
+// §1 Eq. (10) (second-order error dW H dW^T); min-max RTN is the simple quantiser named in
+// "OWQ -- paper by Lee et al. (2023) -- summary and ideas", Key points.
+//
+// Determinism: every fp64 sum runs over its index in ascending order with separate
+// multiply and add (no fused multiply-add), so the selection is a pure function of the
+// inputs.  Every float-to-integer decision uses IEEE fp32 division and round-half-to-even.
+#include "owq_internal.cuh"
+
+namespace owq {
+namespace {
+
+// min-max RTN parameters of one (row, group) from its range; returns s (fp16) and z.
+__device__ __forceinline__ void rtn_from_range(float mn, float mx, int qmax, __half* s_out,
+                                               float* s32_out, float* z32_out) {
+  if (mn == mx) { mn = -1.f; mx = 1.f; }
+  __half s = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)qmax));
+  if (__half2float(s) == 0.f) {            // range below fp16 resolution
+    mn = -1.f; mx = 1.f;
+    s = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), (float)qmax));
+  }
+  float s32 = __half2float(s);
+  float z = rintf(__fdiv_rn(-mn, s32));
+  z = fminf(fmaxf(z, 0.f), (float)qmax);
+  z = __fadd_rn(z, 0.f);                   // canonical +0
+  *s_out = s; *s32_out = s32; *z32_out = z;
+}
+
+__device__ __forceinline__ float rtn_code(float w, float s32, float z32, int qmax) {
+  float q = __fadd_rn(rintf(__fdiv_rn(w, s32)), z32);
+  return fminf(fmaxf(q, 0.f), (float)qmax);
+}
+
+// lambda_j = sum_t X[t, j]^2, t ascending.  One thread per column.
+__global__ void k_hessian_diag(const __half* __restrict__ X, int T, int K, double* __restrict__ lam) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= K) return;
+  double acc = 0.0;
+  const __half* p = X + j;
+  #pragma unroll 4
+  for (int t = 0; t < T; ++t) {
+    double v = (double)__half2float(p[(size_t)t * K]);
+    acc = __dadd_rn(acc, __dmul_rn(v, v));
+  }
+  lam[j] = acc;
+}
+
+// One warp per (row, group): range over the group's dense columns (weak ones read as 0,
+// which the range always contains), then s and z.
+__global__ void k_rtn_params(const __half* __restrict__ W, int N, int K, int group, int bits,
+                             const uint8_t* __restrict__ weak_mask,
+                             __half* __restrict__ scales, __half* __restrict__ zeros) {
+  const int G = K / group;
+  long long item = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (item >= (long long)N * G) return;
+  int lane = threadIdx.x & 31;
+  int i = (int)(item / G), g = (int)(item % G);
+  const __half* row = W + (size_t)i * K + (size_t)g * group;
+  float mn = 0.f, mx = 0.f;
+  for (int j = lane; j < group; j += 32) {
+    float v = __half2float(row[j]);
+    if (weak_mask && weak_mask[g * group + j]) v = 0.f;
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  #pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    __half s; float s32, z32;
+    rtn_from_range(mn, mx, (1 << bits) - 1, &s, &s32, &z32);
+    scales[item] = s;
+    zeros[item] = __float2half_rn(z32);
+  }
+}
+
+// colsum_j = sum_i (W[i,j] - W_hat0[i,j])^2, i ascending; W_hat0 = fp16_rn(s (q - z)) of the
+// all-column RTN (scales/zeros hold that quantisation here).  One thread per column.
+__global__ void k_colsum_dw2(const __half* __restrict__ W, int N, int K, int group, int bits,
+                             const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                             double* __restrict__ colsum) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= K) return;
+  const int G = K / group, g = j / group, qmax = (1 << bits) - 1;
+  double acc = 0.0;
+  #pragma unroll 4
+  for (int i = 0; i < N; ++i) {
+    float w = __half2float(W[(size_t)i * K + j]);
+    float s32 = __half2float(scales[(size_t)i * G + g]);
+    float z32 = __half2float(zeros[(size_t)i * G + g]);
+    float q = rtn_code(w, s32, z32, qmax);
+    float wh = __half2float(__float2half_rn(__fmul_rn(s32, __fsub_rn(q, z32))));
+    double d = __dsub_rn((double)w, (double)wh);
+    acc = __dadd_rn(acc, __dmul_rn(d, d));
+  }
+  colsum[j] = acc;
+}
+
+struct Cand { double v; int j; };
+
+__device__ __forceinline__ bool better(double av, int aj, double bv, int bj) {
+  return av > bv || (av == bv && aj < bj);
+}
+
+// sens_j = lambda_j * colsum_j; the k best (descending, ties to the lower index), written
+// ascending to idx; weak_mask[j] = 1 for those.  One block of 1024 threads.
+__global__ void __launch_bounds__(1024) k_topk(const double* __restrict__ lam, const double* __restrict__ colsum,
+                                               double* __restrict__ sens, int K, int k,
+                                               int32_t* __restrict__ idx, uint8_t* __restrict__ weak_mask) {
+  __shared__ double sv[32];
+  __shared__ int sj[32];
+  __shared__ int chosen[kMaxWeak];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  for (int j = tid; j < K; j += blockDim.x) {
+    sens[j] = __dmul_rn(lam[j], colsum[j]);
+    weak_mask[j] = 0;
+  }
+  __syncthreads();
+  for (int r = 0; r < k; ++r) {
+    double bv = -1.0; int bj = 0x7fffffff;
+    for (int j = tid; j < K; j += blockDim.x) {
+      double v = sens[j];
+      if (v >= 0.0 && better(v, j, bv, bj)) { bv = v; bj = j; }
+    }
+    #pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (better(ov, oj, bv, bj)) { bv = ov; bj = oj; }
+    }
+    if (lane == 0) { sv[wid] = bv; sj[wid] = bj; }
+    __syncthreads();
+    if (wid == 0) {
+      bv = lane < nw ? sv[lane] : -1.0;
+      bj = lane < nw ? sj[lane] : 0x7fffffff;
+      #pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+        if (better(ov, oj, bv, bj)) { bv = ov; bj = oj; }
+      }
+      if (lane == 0) {
+        if (bj >= K) bj = 0;           // unreachable for finite inputs (every sens >= 0)
+        chosen[r] = bj;
+        sens[bj] = -1.0;
+      }
+    }
+    __syncthreads();
+  }
+  // ascending order by rank
+  for (int t = tid; t < k; t += blockDim.x) {
+    int v = chosen[t], rank = 0;
+    for (int u = 0; u < k; ++u) rank += chosen[u] < v;
+    idx[rank] = v;
+    weak_mask[v] = 1;
+  }
+}
+
+__global__ void k_codes(const __half* __restrict__ W, int N, int K, int group, int bits,
+                        const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                        const uint8_t* __restrict__ weak_mask, uint8_t* __restrict__ codes) {
+  size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (size_t)N * K) return;
+  int i = (int)(e / K), j = (int)(e % K), G = K / group, g = j / group;
+  float s32 = __half2float(scales[(size_t)i * G + g]);
+  float z32 = __half2float(zeros[(size_t)i * G + g]);
+  float q = weak_mask[j] ? z32 : rtn_code(__half2float(W[e]), s32, z32, (1 << bits) - 1);
+  codes[e] = (uint8_t)q;
+}
+
+__global__ void k_gather_weak(const __half* __restrict__ W, int N, int K,
+                              const int32_t* __restrict__ idx, int k, __half* __restrict__ w_weak) {
+  size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (size_t)N * k) return;
+  int i = (int)(e / k), t = (int)(e % k);
+  w_weak[e] = W[(size_t)i * K + idx[t]];
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int T, int bits,
+                            int group, int k, uint8_t* codes, __half* scales, __half* zeros,
+                            int32_t* idx, __half* w_weak, cudaStream_t s) {
+  const size_t scratch = (size_t)K * (3 * sizeof(double)) + (size_t)K;
+  char* buf = nullptr;
+  cudaError_t e = cudaMallocAsync((void**)&buf, scratch, s);
+  if (e != cudaSuccess) return e;
+  double* lam = (double*)buf;
+  double* colsum = lam + K;
+  double* sens = colsum + K;
+  uint8_t* mask = (uint8_t*)(sens + K);
+  const int G = K / group;
+  const long long items = (long long)N * G;
+
+  k_hessian_diag<<<(K + 255) / 256, 256, 0, s>>>(X, T, K, lam);
+  // all-column RTN into the output scale/zero buffers (overwritten below)
+  k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, nullptr, scales, zeros);
+  k_colsum_dw2<<<(K + 127) / 128, 128, 0, s>>>(W, N, K, group, bits, scales, zeros, colsum);
+  k_topk<<<1, 1024, 0, s>>>(lam, colsum, sens, K, k, idx, mask);
+  k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, mask, scales, zeros);
+  const size_t NK = (size_t)N * K;
+  k_codes<<<(unsigned)((NK + 255) / 256), 256, 0, s>>>(W, N, K, group, bits, scales, zeros, mask, codes);
+  if (k > 0) {
+    const size_t Nk = (size_t)N * k;
+    k_gather_weak<<<(unsigned)((Nk + 255) / 256), 256, 0, s>>>(W, N, K, idx, k, w_weak);
+  }
+  e = cudaGetLastError();
+  cudaError_t e2 = cudaFreeAsync(buf, s);
+  return e != cudaSuccess ? e : e2;
+}
+
+}  // namespace owq
