@@ -1,0 +1,572 @@
+"""Benchmark of the OWQ mixed-precision weight-only matmul on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl owq|reference]
+                    [--workload opt-6.7b-decode|llama-7b-decode|opt-66b-decode] [--M m]
+
+Default workload (the decode configuration the metric is quoted on): OPT-6.7B-shaped decoder
+layer sets (q, k, v, out 4096x4096; fc1 16384x4096; fc2 4096x16384), 3-bit per-output-channel
+codes, k = K/128 fp16 weak columns, one token (M = 1).  A step is one token through a stack of
+32 such layer sets with distinct resident weights (2.5 GB, 20x the L2), i.e. 192 products;
+q/k/v share one launch (owq_gemv_multi).  Each step is a CUDA graph; the timed region replays
+exactly K of them between a barrier + synchronize on both sides.
+
+value = effective weight GB/s of the whole job (algorithmic bytes of all products / time),
+with inputs resident in HBM.  e2e = the same metric with each step's activations copied in
+from pinned host memory and its outputs read back inside the timed region.  With N > 1 every
+rank streams its own stack (independent replicas, weak scaling, no collective on the path);
+time is the max over ranks.  --impl reference times the CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import owq_synth  # noqa: E402
+
+METRIC = "decode GEMV µs/layer & effective weight GB/s (frac. of HBM peak); prefill TFLOP/s"
+UNIT = "GB/s"
+DEPTH = {"opt-6.7b-decode": 32, "llama-7b-decode": 32, "opt-66b-decode": 64}
+WID = {"opt-6.7b-decode": 1, "llama-7b-decode": 2, "opt-66b-decode": 3}
+# launches of one layer set: layers sharing an input (q/k/v, gate/up) are one multi launch
+GROUPS = {
+    "opt-6.7b-decode": [["q", "k", "v"], ["out"], ["fc1"], ["fc2"]],
+    "llama-7b-decode": [["q", "k", "v"], ["o"], ["gate", "up"], ["down"]],
+    "opt-66b-decode": [["q", "k", "v"], ["out"], ["fc1"], ["fc2"]],
+}
+
+
+# ---------------------------------------------------------------------------------- ranks
+def dist_setup():
+    """(rank, world, local_rank); initialises torch.distributed when WORLD_SIZE > 1."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------- helpers
+def layer_bytes(N, K, bits, group, k, M):
+    """Algorithmic bytes of one product: packed codes (weak slots included: the latency layout
+    stores them), fp16 scale+zero per (row, group), fp16 weak block, int32 indices, x, y."""
+    G = K // group
+    return N * K * bits // 8 + N * G * 4 + N * k * 2 + 4 * k + 2 * M * K + 2 * M * N
+
+
+def weight_bytes(N, K, bits, group, k):
+    G = K // group
+    return N * K * bits // 8 + N * G * 4 + N * k * 2 + 4 * k
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+            self.max_mhz = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        if self.nv is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._sample()
+        self._stop.set()
+        self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def ncu_traffic(kernel_tag: str):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or None when the
+    kernel's source changed after the capture (the summary stores the source digest)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.traffic.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                k, v = line.split("=", 1)
+                vals[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "weight_only_mixed_owq_b200", "csrc", vals.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if digest != vals.get("sha256_16"):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------------- owq arm
+def build_stack(owq, torch, spec, depth, M, dev):
+    """Quantise one layer set on the GPU and pack `depth` resident copies of it."""
+    sets, info = [], {}
+    inputs = {}
+    for li, L in enumerate(spec.layers):
+        short = L.name.split(".")[-1]
+        d = owq_synth.draw_layer(L, spec, M, owq_synth.seed_for(spec.wid, li))
+        W = torch.from_numpy(d["W"]).to(dev)
+        X = torch.from_numpy(d["X"]).to(dev)
+        q = owq.quantize(W, X, L.bits, L.group, L.k)
+        del W, X
+        inputs[short] = {"q": q, "x": torch.from_numpy(d["x"]).to(dev), "L": L}
+        info[short] = L
+    for c in range(depth):
+        layers = {}
+        for short, v in inputs.items():
+            q, L = v["q"], v["L"]
+            layers[short] = owq.OwqLayer(q["codes"], q["scales"], q["zeros"], q["idx"] if L.k else None,
+                                         q["w_weak"] if L.k else None, L.bits, L.group)
+        sets.append(layers)
+    for v in inputs.values():
+        del v["q"]
+    torch.cuda.synchronize()
+    return sets, inputs, info
+
+
+def run_owq(args, rank, world, local):
+    import torch
+
+    import weight_only_mixed_owq_b200 as owq
+    from cuda.bindings import runtime as rt
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = args.workload
+    spec = owq_synth.WORKLOADS[WID[wl]]
+    M = args.M
+    depth = args.depth or DEPTH[wl]
+    groups = GROUPS[wl]
+    sets, inputs, info = build_stack(owq, torch, spec, depth, M, dev)
+    ys = {s: torch.empty((M, info[s].N), dtype=torch.float16, device=dev) for s in info}
+
+    # per-launch algorithmic bytes
+    def launch_bytes(names):
+        return sum(layer_bytes(info[n].N, info[n].K, info[n].bits, info[n].group, info[n].k, M) for n in names)
+
+    step_bytes = depth * sum(launch_bytes(g) for g in groups)
+    step_wbytes = depth * sum(weight_bytes(info[n].N, info[n].K, info[n].bits, info[n].group, info[n].k)
+                              for g in groups for n in g)
+    launches_per_step = depth * len(groups)
+
+    def issue(c, stream_ptr, ev=None):
+        """Enqueue one layer set (copy c); optional external event pairs around each launch."""
+        for gi, g in enumerate(groups):
+            if ev is not None:
+                rt.cudaEventRecordWithFlags(ev[gi][0], stream_ptr, rt.cudaEventRecordExternal)
+            if len(g) == 1:
+                st = owq.owq_gemv(sets[c][g[0]].handle, inputs[g[0]]["x"], ys[g[0]], M, stream_ptr)
+            else:
+                st = owq.owq_gemv_multi([sets[c][n].handle for n in g], [inputs[n]["x"] for n in g],
+                                        [ys[n] for n in g], M, stream_ptr)
+            if st != 0:
+                raise RuntimeError(f"launch failed: {owq.owq_status_string(st)}")
+            if ev is not None:
+                rt.cudaEventRecordWithFlags(ev[gi][1], stream_ptr, rt.cudaEventRecordExternal)
+
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    # eager warm-up of every copy (loads modules, sets kernel attributes)
+    for c in range(depth):
+        issue(c, sp)
+    torch.cuda.synchronize()
+
+    # graphs: NG distinct step graphs, each with its own per-launch events
+    NG = 2
+    events = []
+    graphs = []
+    for gidx in range(NG):
+        ev = [[[rt.cudaEventCreate()[1], rt.cudaEventCreate()[1]] for _ in groups] for _ in range(depth)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            cs = torch.cuda.current_stream().cuda_stream
+            for c in range(depth):
+                issue(c, cs, ev[c])
+        graphs.append(g)
+        events.append(ev)
+
+    # e2e graph: pinned host activations in, outputs out, around the same step
+    host_x = {n: torch.empty_like(inputs[n]["x"], device="cpu").pin_memory() for n in inputs}
+    for n in inputs:
+        host_x[n].copy_(inputs[n]["x"].cpu())
+    host_y = {n: torch.empty_like(ys[n], device="cpu").pin_memory() for n in ys}
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=stream):
+        for n in inputs:
+            inputs[n]["x"].copy_(host_x[n], non_blocking=True)
+        cs = torch.cuda.current_stream().cuda_stream
+        for c in range(depth):
+            issue(c, cs)
+        for n in ys:
+            host_y[n].copy_(ys[n], non_blocking=True)
+    h2d = sum(v.numel() * v.element_size() for v in host_x.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_y.values())
+
+    for i in range(args.warmup):
+        graphs[i % NG].replay()
+    torch.cuda.synchronize()
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(args.steps):
+                graphs[i % NG].replay()
+            t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, world)
+
+    # per-launch durations of the dominant kernel (k_gemv) from the last replay of each graph
+    durs, dbytes = [], []
+    for gidx in range(min(NG, args.steps)):
+        for c in range(depth):
+            for gi, g in enumerate(groups):
+                err, t = rt.cudaEventElapsedTime(events[gidx][c][gi][0], events[gidx][c][gi][1])
+                if err == rt.cudaError_t.cudaSuccess:
+                    durs.append(t)
+                    dbytes.append(launch_bytes(g))
+    achieved = (sum(dbytes) / (sum(durs) * 1e-3) / 1e9) if durs else None
+    per_group = {}
+    for j, g in enumerate(groups):
+        sel = durs[j::len(groups)]
+        if sel:
+            us = 1e3 * sum(sel) / len(sel)
+            per_group["+".join(g)] = {"us": round(us, 3), "GBps": round(launch_bytes(g) / (us * 1e-6) / 1e9, 1)}
+
+    # e2e
+    for _ in range(max(1, args.warmup)):
+        g_e2e.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            g_e2e.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ems_max = max_over_ranks(e0.elapsed_time(e1), world)
+
+    total_bytes = sum_over_ranks(step_bytes * args.steps, world)
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+    e2e_value = total_bytes / (ems_max * 1e-3) / 1e9
+    peaks, peak_kind = measured_peaks()
+    per_layer_us = ms_max * 1e3 / args.steps / (depth * sum(len(g) for g in groups))
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{wl}: {depth} resident OPT/LLaMA-shaped decoder layer sets per token, M={M}",
+            "layers": {n: [info[n].N, info[n].K] for n in info},
+            "bits": spec.layers[0].bits, "group": "per-channel" if spec.layers[0].group == spec.layers[0].K else spec.layers[0].group,
+            "weak_cols": "K/128", "M": M, "products_per_step": depth * sum(len(g) for g in groups),
+            "launches_per_step": launches_per_step, "step_bytes": step_bytes, "step_weight_bytes": step_wbytes,
+            "l2": "inputs larger than L2 (distinct resident weights, no reuse within a step)",
+            "per_layer_us": round(per_layer_us, 3),
+            "weight_GBps": round(sum_over_ranks(step_wbytes * args.steps, world) / (ms_max * 1e-3) / 1e9, 2),
+            "parallelism": f"replicas x{world}",
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "k_gemv (decode GEMV)",
+            "achieved": round(achieved, 2) if achieved else None,
+            "peak": peaks["hbm_gbs"],
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
+            "frac_of_8TBps_spec": round(achieved / 8000.0, 4) if achieved else None,
+            "traffic": ncu_traffic("k_gemv_opt67b"),
+            "launches_sampled": len(durs),
+            "per_launch_group": per_group,
+        },
+        "clocks": clk.summary(),
+    }
+    for c in sets:
+        for L in c.values():
+            L.close()
+    return line
+
+
+def prefill_measure(args, dev):
+    """TFLOP/s of owq_gemm on the LLaMA-13B-shaped prefill layers (13824x5120, 5120x13824,
+    3-bit, g = 128, k = 40 / 108) for the token counts of that workload."""
+    import torch
+
+    import weight_only_mixed_owq_b200 as owq
+    spec = owq_synth.WORKLOADS[4]
+    out = {}
+    peaks, kind = measured_peaks()
+    layers = []
+    for li, L in enumerate(spec.layers):
+        d = owq_synth.draw_layer(L, spec, max(spec.Ms), owq_synth.seed_for(4, li))
+        W, X = torch.from_numpy(d["W"]).to(dev), torch.from_numpy(d["X"]).to(dev)
+        lay, _ = owq.quantize_pack(W, X, L.bits, L.group, L.k)
+        layers.append((L, lay, torch.from_numpy(d["x"]).to(dev)))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for M in spec.Ms:
+        tot_flop, tot_ms = 0.0, 0.0
+        for L, lay, x in layers:
+            xm = x[:M].contiguous()
+            y = torch.empty((M, L.N), dtype=torch.float16, device=dev)
+            for _ in range(3):
+                lay.gemm(xm, y)
+            times = []
+            for _ in range(10):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                lay.gemm(xm, y)
+                b.record()
+                torch.cuda.synchronize()
+                times.append(a.elapsed_time(b))
+            t = statistics.median(times)
+            tot_flop += 2.0 * M * L.N * L.K
+            tot_ms += t
+        tf = tot_flop / (tot_ms * 1e-3) / 1e12
+        out[str(M)] = {"tflops": round(tf, 2), "frac_burst": round(tf / peaks["bf16_tflops"], 4),
+                       "us_per_pair": round(tot_ms * 1e3, 2)}
+    for _, lay, _ in layers:
+        lay.close()
+    return {"layers": "13824x5120 + 5120x13824, 3-bit g128, k=40/108", "per_M": out,
+            "peak_tflops": peaks["bf16_tflops"], "peak_kind": kind,
+            "timing": "median of 10 single launches, L2 flushed between launches"}
+
+
+# ---------------------------------------------------------------------------------- oracle arm
+def oracle_sample(wl: str, rows: int):
+    """Quantise (oracle) one layer set and keep the first `rows` rows of each layer."""
+    import oracle
+    spec = owq_synth.WORKLOADS[WID[wl]]
+    out = []
+    for li, L in enumerate(spec.layers):
+        d = owq_synth.draw_layer(L, spec, 1, owq_synth.seed_for(spec.wid, li))
+        r = oracle.owq_quantize(d["W"], d["X"], L.bits, L.group, L.k)
+        n = min(rows, L.N)
+        packed = oracle.pack(r["codes"][:n], L.bits)
+        out.append({"L": L, "n": n, "packed": packed, "scales": r["scales"][:n], "zeros": r["zeros"][:n],
+                    "w_weak": r["w_weak"][:n], "idx": r["idx"], "x": d["x"]})
+    return out
+
+
+def oracle_step(sample) -> int:
+    """One pass of the oracle's product over the sample; returns its algorithmic bytes."""
+    import oracle
+    b = 0
+    for s in sample:
+        L = s["L"]
+        codes = oracle.unpack(s["packed"], L.K, L.bits)
+        W_hat = oracle.dequant(codes, s["scales"], s["zeros"])
+        oracle.matmul(W_hat, s["w_weak"], s["idx"], s["x"])
+        b += layer_bytes(s["n"], L.K, L.bits, L.group, L.k, 1)
+    return b
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl: str, budget_s: float = 12.0):
+    rows = 1024
+    sample = oracle_sample(wl, rows)
+    t0 = time.perf_counter()
+    b, n = 0, 0
+    while True:
+        b += oracle_step(sample)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(b / dt / 1e9, 4), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"first {rows} rows of each layer of one {wl} layer set, M=1, {n} passes, {dt:.1f} s "
+                      "(unpack, dequant, fp64 product)"}
+
+
+def run_reference(args):
+    """The oracle (numpy, fp64) on the host cores: each step one pass over a bounded sample."""
+    rows = 256
+    sample = oracle_sample(args.workload, rows)
+    for _ in range(args.warmup):
+        oracle_step(sample)
+    t0 = time.perf_counter()
+    b = 0
+    for _ in range(args.steps):
+        b += oracle_step(sample)
+    dt = time.perf_counter() - t0
+    v = b / dt / 1e9
+    sdesc = f"first {rows} rows of each layer of one {args.workload} layer set, M=1 (unpack, dequant, fp64 product)"
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload} (oracle sample)", "M": 1},
+        "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sdesc},
+        "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="owq", choices=["owq", "reference"])
+    ap.add_argument("--workload", default="opt-6.7b-decode", choices=sorted(DEPTH))
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--depth", type=int, default=0, help="resident layer sets per step (default: model depth)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    rank, world, local = dist_setup()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        teardown(world)
+        return 0
+
+    line = run_owq(args, rank, world, local)
+    if rank == 0 and world == 1:
+        import torch
+        if not args.no_prefill:
+            line["prefill"] = prefill_measure(args, torch.device("cuda", local))
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    teardown(world)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
