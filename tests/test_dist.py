@@ -1,0 +1,86 @@
+"""Host-side multi-rank logic of bench.py on CPU: world_size 2 over gloo.
+
+bench.py shards nothing (each rank streams its own layer stack); what needs checking is the
+rank plumbing: set-up from the torchrun environment, barriers, the max-over-ranks time and
+the sum-over-ranks work that make the whole-job number.
+"""
+import os
+import socket
+import subprocess
+import sys
+import textwrap
+
+import pytest
+
+from tests.conftest import ROOT
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+CHILD = textwrap.dedent(
+    """
+    import os, sys, json
+    sys.path.insert(0, {root!r})
+    import bench
+    rank, world, local = bench.dist_setup()
+    bench.barrier(world)
+    t = 10.0 + rank            # this rank's "elapsed ms"
+    work = 100.0 * (rank + 1)  # this rank's "bytes"
+    out = {{"rank": rank, "world": world, "max": bench.max_over_ranks(t, world),
+            "sum": bench.sum_over_ranks(work, world)}}
+    bench.barrier(world)
+    bench.teardown(world)
+    print(json.dumps(out))
+    """
+)
+
+
+def test_two_gloo_ranks_agree_on_max_time_and_total_work(tmp_path):
+    script = tmp_path / "child.py"
+    script.write_text(CHILD.format(root=ROOT))
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2",
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen([sys.executable, str(script)], env=env,
+                                      stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
+    outs = []
+    for p in procs:
+        o, e = p.communicate(timeout=180)
+        assert p.returncode == 0, e
+        outs.append(o.strip().splitlines()[-1])
+    import json
+    res = sorted((json.loads(o) for o in outs), key=lambda d: d["rank"])
+    for d in res:
+        assert d["world"] == 2
+        assert d["max"] == pytest.approx(11.0)
+        assert d["sum"] == pytest.approx(300.0)
+
+
+def test_single_rank_needs_no_process_group(monkeypatch):
+    import bench
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.dist_setup() == (0, 1, 0)
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.sum_over_ranks(2.0, 1) == 2.0
+
+
+def test_reference_arm_line_shape(monkeypatch):
+    """--impl reference prints one JSON line with the oracle's sample and no GPU use."""
+    import bench
+    monkeypatch.setattr(bench, "oracle_sample", lambda wl, rows: [])
+    monkeypatch.setattr(bench, "oracle_step", lambda s: 1000)
+    args = type("A", (), {"workload": "opt-6.7b-decode", "steps": 3, "warmup": 3})()
+    line = bench.run_reference(args)
+    assert line["impl"] == "reference"
+    assert line["unit"] == "GB/s" and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
