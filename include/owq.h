@@ -82,6 +82,28 @@ owq_status_t owq_quantize(const uint16_t* W, const uint16_t* X, int N, int K, in
                           int32_t* idx, uint16_t* w_weak, owq_stream_t stream);
 
 /*
+ * owq_quantize_noalloc -- owq_quantize without any device allocation.  (The paper has no
+ * counterpart: this is a deployment variant of the same computation.)
+ * For callers that cannot let a library allocate GPU memory -- serving processes that
+ * reserve nearly all device memory up front for their own pool (a library cudaMalloc would
+ * fail or fragment it) and processes that forbid allocation after start-up.  Same arguments,
+ * outputs and results (bit-identical) as owq_quantize, but its scratch lives in a static
+ * device array sized for K <= OWQ_NOALLOC_MAX_K columns (25 bytes per column, 1 MB), which
+ * every GPU that loads this library keeps until the process exits.  K above that limit
+ * returns OWQ_ERR_SHAPE and launches nothing.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it, so make that first call
+ * outside any stream capture.  All calls share the one array: calls that can overlap on the
+ * GPU (unordered streams) race on it and must be serialised by the caller.  No state carries
+ * over between calls (each kernel fully writes what it later reads).  Calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ */
+#define OWQ_NOALLOC_MAX_K 40960
+owq_status_t owq_quantize_noalloc(const uint16_t* W, const uint16_t* X, int N, int K, int T,
+                                  int bits, int group, int k,
+                                  uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                                  int32_t* idx, uint16_t* w_weak, owq_stream_t stream);
+
+/*
  * owq_pack -- build a layer handle in the packed, latency-favoured layout ("Storage
  * Methods", appendix §2: a full low-precision matrix, zero-filled at the weak columns,
  * plus a separate fp16 block of the weak columns).

@@ -10,7 +10,7 @@ import importlib
 _EXPORTS = (
     "LIB", "LIB_PATH", "OWQ_OK", "OwqError", "OwqLayer", "PROTOTYPES", "STATUS_NAMES",
     "owq_dequant", "owq_device_status", "owq_gemm", "owq_gemv", "owq_gemv_multi", "owq_layer_bytes",
-    "owq_layer_free", "owq_layer_info", "owq_pack", "owq_quantize",
+    "owq_layer_free", "owq_layer_info", "owq_pack", "owq_quantize", "owq_quantize_noalloc",
     "owq_status_string", "owq_version", "quantize", "quantize_pack",
 )
 

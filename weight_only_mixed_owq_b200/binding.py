@@ -23,6 +23,7 @@ STATUS_NAMES = {
 _P, _I, _SZ, _S = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t), ctypes.c_char_p
 PROTOTYPES = [
     ("owq_quantize", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    ("owq_quantize_noalloc", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     ("owq_pack", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     ("owq_gemv", _I, [_P, _P, _P, _I, _P]),
     ("owq_gemv_multi", _I, [ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _I, _P]),
@@ -89,6 +90,11 @@ def _check(st: int, where: str) -> None:
 def owq_quantize(W, X, N, K, T, bits, group, k, codes, scales, zeros, idx, w_weak, stream=None) -> int:
     return LIB.owq_quantize(_ptr(W), _ptr(X), N, K, T, bits, group, k, _ptr(codes), _ptr(scales),
                             _ptr(zeros), _ptr(idx), _ptr(w_weak), _stream(stream))
+
+
+def owq_quantize_noalloc(W, X, N, K, T, bits, group, k, codes, scales, zeros, idx, w_weak, stream=None) -> int:
+    return LIB.owq_quantize_noalloc(_ptr(W), _ptr(X), N, K, T, bits, group, k, _ptr(codes), _ptr(scales),
+                                    _ptr(zeros), _ptr(idx), _ptr(w_weak), _stream(stream))
 
 
 def owq_pack(codes, N, K, bits, group, scales, zeros, idx, k, w_weak, stream=None):

@@ -11,6 +11,8 @@
 // Determinism: every fp64 sum runs over its index in ascending order with separate
 // multiply and add (no fused multiply-add), so the selection is a pure function of the
 // inputs.  Every float-to-integer decision uses IEEE fp32 division and round-half-to-even.
+#include <mutex>
+
 #include "owq_internal.cuh"
 
 namespace owq {
@@ -218,3 +220,103 @@ cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int 
 }
 
 }  // namespace owq
+
+// ---------------------------------------------------------------------------------------
+// owq_quantize_noalloc: the same quantiser with its scratch in a fixed device array.
+//
+// Some callers cannot let a library allocate device memory: serving processes that reserve
+// (almost) all of the GPU's memory up front for their own pool, where a library-side
+// cudaMalloc fails or fragments that pool, and processes that forbid any allocation after
+// start-up.  This entry point therefore takes its scratch (lambda, column sums and scores in
+// fp64, plus a byte mask: 25 bytes per input column) from a file-scope device array of
+// OWQ_NOALLOC_MAX_K columns (1 MB), which every GPU that loads the library holds until the
+// process exits.  The array is shared by all calls: calls whose work overlaps on the GPU
+// (different streams, no ordering between them) race on it and must be serialised by the
+// caller.  Nothing in it has to start at zero: every kernel fully writes the part it reads
+// later (the mask is cleared by the selection kernel itself).
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char owq_noalloc_scratch[(size_t)OWQ_NOALLOC_MAX_K * (3 * sizeof(double) + 1)];
+
+namespace owq {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device (looked up once per device;
+// in host code the array's name is only a host-side stand-in, never a device address).
+cudaError_t noalloc_scratch(unsigned char** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, owq_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_quantize_static(const __half* W, const __half* X, int N, int K, int T, int bits,
+                                   int group, int k, uint8_t* codes, __half* scales, __half* zeros,
+                                   int32_t* idx, __half* w_weak, cudaStream_t s) {
+  unsigned char* buf = nullptr;
+  cudaError_t e = noalloc_scratch(&buf);
+  if (e != cudaSuccess) return e;
+  double* lam = reinterpret_cast<double*>(buf);
+  double* colsum = lam + K;
+  double* sens = colsum + K;
+  uint8_t* mask = reinterpret_cast<uint8_t*>(sens + K);
+  const int G = K / group;
+  const long long items = (long long)N * G;
+  k_hessian_diag<<<(K + 255) / 256, 256, 0, s>>>(X, T, K, lam);
+  k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, nullptr, scales, zeros);
+  k_colsum_dw2<<<(K + 127) / 128, 128, 0, s>>>(W, N, K, group, bits, scales, zeros, colsum);
+  k_topk<<<1, 1024, 0, s>>>(lam, colsum, sens, K, k, idx, mask);
+  k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, mask, scales, zeros);
+  const size_t NK = (size_t)N * K;
+  k_codes<<<(unsigned)((NK + 255) / 256), 256, 0, s>>>(W, N, K, group, bits, scales, zeros, mask, codes);
+  if (k > 0) {
+    const size_t Nk = (size_t)N * k;
+    k_gather_weak<<<(unsigned)((Nk + 255) / 256), 256, 0, s>>>(W, N, K, idx, k, w_weak);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace owq
+
+extern "C" owq_status_t owq_quantize_noalloc(const uint16_t* W, const uint16_t* X, int N, int K, int T,
+                                             int bits, int group, int k, uint8_t* codes, uint16_t* scales,
+                                             uint16_t* zeros, int32_t* idx, uint16_t* w_weak,
+                                             owq_stream_t stream) {
+  using namespace owq;
+  if (!W || !X || !codes || !scales || !zeros) return OWQ_ERR_NULL;
+  if (k > 0 && (!idx || !w_weak)) return OWQ_ERR_NULL;
+  if (bits != 3 && bits != 4) return OWQ_ERR_BITS;
+  if (N < 1 || N > (1 << 20) || K < kBlockCodes || K > 65536 || K % kBlockCodes) return OWQ_ERR_SHAPE;
+  if (group != K && group != 128) return OWQ_ERR_GROUP;
+  if (k < 0 || k > K || k > kMaxWeak) return OWQ_ERR_SHAPE;
+  if (T < 1 || T > (1 << 20)) return OWQ_ERR_SHAPE;
+  if (K > OWQ_NOALLOC_MAX_K) return OWQ_ERR_SHAPE;   // beyond the static scratch
+  if (!aligned16(W) || !aligned16(X) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros) ||
+      (k > 0 && (!aligned16(idx) || !aligned16(w_weak))))
+    return OWQ_ERR_ALIGN;
+  int dev = -1, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+    cudaGetLastError();
+    return OWQ_ERR_DEVICE;
+  }
+  cudaError_t e = launch_quantize_static(reinterpret_cast<const __half*>(W), reinterpret_cast<const __half*>(X),
+                                         N, K, T, bits, group, k, codes, reinterpret_cast<__half*>(scales),
+                                         reinterpret_cast<__half*>(zeros), idx, reinterpret_cast<__half*>(w_weak),
+                                         reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_CUDA; }
+  return OWQ_OK;
+}
