@@ -207,60 +207,65 @@ def owq_quantize(W: np.ndarray, X: np.ndarray, bits: int, group: int, k: int) ->
 # ----------------------------------------------------------------------------------------
 # Packed layout (latency-favoured, zero-filled; the format of this library)
 # ----------------------------------------------------------------------------------------
-# A row of K codes is cut into chunks of 32 consecutive codes; chunk c of row i is stored
-# as `bits` little-endian 32-bit words at word offset (i * K/32 + c) * bits.  Codes 2t and
-# 2t+1 of a chunk form pair t; the even code sits in the low 16 bits of a word and the odd
-# code in the high 16 bits, at the same offset.
-#   bits = 4: pair t is in word t // 4 at offset 4 * (t % 4) (and 16 + that).
-#   bits = 3: pair t < 15 is in word t // 5 at offset 3 * (t % 5) (and 16 + that);
-#             pair 15: bit e of code 30 is bit 15 of word e, bit e of code 31 is bit 31
+# A row of K codes is cut into blocks of 128 consecutive codes; block b of row i is
+# 4 * bits little-endian 32-bit words at word offset (i * K/128 + b) * 4 * bits.  Codes 2p and
+# 2p+1 of a block form pair p (p = 0..63).  The block is four chunks of `bits` words; chunk q
+# (words q*bits .. q*bits + bits - 1) holds the sixteen pairs p = 4j + q, j = 0..15.  Pair j
+# of a chunk sits at a slot (word w, bit offset o): the even code in bits o.., the odd code in
+# bits 16 + o.. of word w.
+#   bits = 4: w = 2 (j // 8) + (j % 2), o = 4 ((j % 8) // 2).
+#   bits = 3: slots of j = 0..15: (0,0) (1,0) (0,3) (1,3) (0,6) (1,6) (0,9) (1,9) (0,12) (1,12)
+#             (2,0) D (2,3) (2,12) (2,6) (2,9); slot D (j = 11) spreads its codes over the
+#             chunk: bit e of the even code is bit 15 of word e, bit e of the odd code is bit 31
 #             of word e (e = 0, 1, 2).
+SLOT3 = [(0, 0), (1, 0), (0, 3), (1, 3), (0, 6), (1, 6), (0, 9), (1, 9), (0, 12), (1, 12),
+         (2, 0), None, (2, 3), (2, 12), (2, 6), (2, 9)]
+SLOT4 = [(2 * (j // 8) + (j % 2), 4 * ((j % 8) // 2)) for j in range(16)]
+
+
 def pack(codes: np.ndarray, bits: int) -> np.ndarray:
     """Pack N x K codes into N x (K * bits / 32) uint32 words (format above)."""
     codes = np.asarray(codes, dtype=np.uint8)
     N, K = codes.shape
-    if K % 32:
-        raise ValueError("K must be a multiple of 32")
-    C = K // 32
-    c = codes.reshape(N, C, 32).astype(np.uint32)
-    words = np.zeros((N, C, bits), dtype=np.uint32)
-    if bits == 4:
-        for t in range(16):
-            j, off = t // 4, 4 * (t % 4)
-            words[:, :, j] |= (c[:, :, 2 * t] << off) | (c[:, :, 2 * t + 1] << (16 + off))
-    elif bits == 3:
-        for t in range(15):
-            j, off = t // 5, 3 * (t % 5)
-            words[:, :, j] |= (c[:, :, 2 * t] << off) | (c[:, :, 2 * t + 1] << (16 + off))
-        for e in range(3):
-            words[:, :, e] |= (((c[:, :, 30] >> e) & 1) << 15) | (((c[:, :, 31] >> e) & 1) << 31)
-    else:
+    if K % 128:
+        raise ValueError("K must be a multiple of 128")
+    if bits not in (3, 4):
         raise ValueError("bits must be 3 or 4")
-    return words.reshape(N, C * bits)
+    B = K // 128
+    c = codes.reshape(N, B, 64, 2).astype(np.uint32)          # [row, block, pair, even/odd]
+    words = np.zeros((N, B, 4, bits), dtype=np.uint32)        # [row, block, chunk, word]
+    slots = SLOT3 if bits == 3 else SLOT4
+    for q in range(4):
+        for j in range(16):
+            ev, od = c[:, :, 4 * j + q, 0], c[:, :, 4 * j + q, 1]
+            if slots[j] is None:
+                for e in range(3):
+                    words[:, :, q, e] |= (((ev >> e) & 1) << 15) | (((od >> e) & 1) << 31)
+            else:
+                w, o = slots[j]
+                words[:, :, q, w] |= (ev << o) | (od << (16 + o))
+    return words.reshape(N, B * 4 * bits)
 
 
 def unpack(words: np.ndarray, K: int, bits: int) -> np.ndarray:
     """Inverse of pack: N x (K * bits / 32) uint32 words -> N x K uint8 codes."""
     words = np.asarray(words, dtype=np.uint32)
     N = words.shape[0]
-    C = K // 32
-    w = words.reshape(N, C, bits)
-    c = np.zeros((N, C, 32), dtype=np.uint32)
-    if bits == 4:
-        for t in range(16):
-            j, off = t // 4, 4 * (t % 4)
-            c[:, :, 2 * t] = (w[:, :, j] >> off) & 0xF
-            c[:, :, 2 * t + 1] = (w[:, :, j] >> (16 + off)) & 0xF
-    elif bits == 3:
-        for t in range(15):
-            j, off = t // 5, 3 * (t % 5)
-            c[:, :, 2 * t] = (w[:, :, j] >> off) & 0x7
-            c[:, :, 2 * t + 1] = (w[:, :, j] >> (16 + off)) & 0x7
-        for e in range(3):
-            c[:, :, 30] |= ((w[:, :, e] >> 15) & 1) << e
-            c[:, :, 31] |= ((w[:, :, e] >> 31) & 1) << e
-    else:
-        raise ValueError("bits must be 3 or 4")
+    B = K // 128
+    w4 = words.reshape(N, B, 4, bits)
+    c = np.zeros((N, B, 64, 2), dtype=np.uint32)
+    mask = (1 << bits) - 1
+    slots = SLOT3 if bits == 3 else SLOT4
+    for q in range(4):
+        for j in range(16):
+            if slots[j] is None:
+                for e in range(3):
+                    c[:, :, 4 * j + q, 0] |= ((w4[:, :, q, e] >> 15) & 1) << e
+                    c[:, :, 4 * j + q, 1] |= ((w4[:, :, q, e] >> 31) & 1) << e
+            else:
+                w, o = slots[j]
+                c[:, :, 4 * j + q, 0] = (w4[:, :, q, w] >> o) & mask
+                c[:, :, 4 * j + q, 1] = (w4[:, :, q, w] >> (16 + o)) & mask
     return c.reshape(N, K).astype(np.uint8)
 
 

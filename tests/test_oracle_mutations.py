@@ -103,6 +103,28 @@ def test_mutant_swapped_pair_halves_is_caught(monkeypatch, golden_dir):
         pins.test_pack_hand_derived_words(golden_dir)
 
 
+def test_mutant_swapped_slots_is_caught(monkeypatch, golden_dir):
+    slots = list(oo.SLOT3)
+    slots[13], slots[15] = slots[15], slots[13]
+    monkeypatch.setattr(oo, "SLOT3", slots)
+    with pytest.raises(AssertionError):
+        pins.test_pack_hand_derived_words(golden_dir)
+
+
+def test_mutant_chunk_of_consecutive_pairs_is_caught(monkeypatch, golden_dir):
+    orig = oo.pack
+
+    def bad(codes, bits):
+        c = np.asarray(codes)
+        N, K = c.shape
+        # chunk q taking pairs 16q..16q+15 instead of 4j + q
+        perm = np.arange(K).reshape(K // 128, 16, 4, 2).transpose(0, 2, 1, 3).reshape(K)
+        return orig(c[:, perm], bits)
+    _patch(monkeypatch, "pack", bad)
+    with pytest.raises(AssertionError):
+        pins.test_pack_hand_derived_words(golden_dir)
+
+
 def test_mutant_latency_bits_without_zero_fill_is_caught(monkeypatch):
     orig = oo.bits_per_weight
 

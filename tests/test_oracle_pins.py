@@ -44,11 +44,12 @@ def test_rtn_hand_worked_rows(golden_dir):
 def test_pack_hand_derived_words(golden_dir):
     for bits, rule, words in _read_rows(os.path.join(golden_dir, "pack_words.txt")):
         bits = int(bits)
+        k = np.arange(128)
         mod = int(rule.split()[-1])
-        codes = (np.arange(32) % mod).astype(np.uint8)[None, :]
+        codes = ((k // 8 if "//" in rule else k) % mod).astype(np.uint8)[None, :]
         got = oracle.pack(codes, bits)[0]
         assert [f"{int(v):08x}" for v in got] == words.split()
-        assert oracle.unpack(got[None, :], 32, bits).tolist() == codes.tolist()
+        assert oracle.unpack(got[None, :], 128, bits).tolist() == codes.tolist()
 
 
 # ------------------------------------------------------------------ quantiser invariants
@@ -251,16 +252,25 @@ def test_pack_roundtrip_and_size(bits):
 
 @pytest.mark.parametrize("bits", [3, 4])
 def test_pack_single_code_moves_single_bits(bits):
-    """Each code occupies exactly `bits` bits and no two codes share a bit."""
-    seen = np.zeros(bits * 32, dtype=int)
-    for k in range(32):
-        codes = np.zeros((1, 32), np.uint8)
+    """Each code occupies exactly `bits` bits of its block and no two codes share a bit."""
+    seen = np.zeros(bits * 128, dtype=int)
+    for k in range(128):
+        codes = np.zeros((1, 128), np.uint8)
         codes[0, k] = (1 << bits) - 1
         w = oracle.pack(codes, bits)[0]
-        bitsset = [wi * 32 + b for wi in range(bits) for b in range(32) if (int(w[wi]) >> b) & 1]
+        bitsset = [wi * 32 + b for wi in range(4 * bits) for b in range(32) if (int(w[wi]) >> b) & 1]
         assert len(bitsset) == bits
         seen[bitsset] += 1
     assert np.all(seen == 1)
+
+
+def test_pack_blocks_are_independent():
+    """A code only moves bits of its own 128-code block (block b at words b * 4 * bits)."""
+    codes = np.zeros((1, 384), np.uint8)
+    codes[0, 200] = 5
+    w = oracle.pack(codes, 3)[0]
+    nz = np.nonzero(w)[0]
+    assert nz.min() >= 12 and nz.max() < 24
 
 
 # ------------------------------------------------------------------ storage accounting

@@ -151,7 +151,7 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   L->magic = kLayerMagic;
   cudaGetDevice(&L->device);
   L->N = N; L->K = K; L->bits = bits; L->group = group; L->G = K / group; L->k = k;
-  L->k_ld = std::max(8, (k + 7) & ~7);
+  L->k_ld = std::max(16, (k + 15) & ~15);   // 16-wide tensor-core k slices
   L->stream = s;
   L->maps_ready = false;
   const size_t packed_bytes = (size_t)N * K * bits / 8;

@@ -23,6 +23,7 @@
 // status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
 #include <cstring>
 
+#include "owq_format.cuh"
 #include "owq_internal.cuh"
 #include "owq_sm100.cuh"
 
@@ -76,36 +77,15 @@ __device__ __forceinline__ uint32_t h2_splat(float v) {
   return u | (u << 16);
 }
 
-// Dequantise one 32-code chunk into 16 fp16x2 values (k = 2t, 2t+1 in pair t).
-// A pair at bit offset o is lifted as (v & mask) | 0x6400 per half = 1024 + q 2^o, then
-// (1024 + q 2^o) * 2^-o - (1024 2^-o + z) = q - z exactly, then * s: fp16_rn(s (q - z)).
+// fp16_rn(s (q - z)) of pair j of a chunk (both halves).  The pair is lifted as
+// (bits | 0x6400) = 1024 + q 2^o per half, then (1024 + q 2^o) * 2^-o - (1024 2^-o + z) = q - z
+// exactly (one fma.rn.f16x2), then * s rounds once: bit-exact with the definition.
 template <int BITS>
-__device__ __forceinline__ void dequant_chunk(const uint32_t* w, uint32_t s2, const uint32_t* scl,
-                                              const uint32_t* nz, uint32_t* out) {
+__device__ __forceinline__ uint32_t dequant_pair(const uint32_t* w, int j, uint32_t s2, const uint32_t* scl,
+                                                 const uint32_t* nz) {
   constexpr uint32_t kMagic = 0x64006400u;
-  if constexpr (BITS == 3) {
-    #pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      const uint32_t v = w[j], u = v >> 9;
-      out[5 * j + 0] = h2_mul(h2_fma((v & 0x00070007u) | kMagic, scl[0], nz[0]), s2);
-      out[5 * j + 1] = h2_mul(h2_fma((v & 0x00380038u) | kMagic, scl[1], nz[1]), s2);
-      out[5 * j + 2] = h2_mul(h2_fma((v & 0x01C001C0u) | kMagic, scl[2], nz[2]), s2);
-      out[5 * j + 3] = h2_mul(h2_fma((u & 0x00070007u) | kMagic, scl[0], nz[0]), s2);
-      out[5 * j + 4] = h2_mul(h2_fma((u & 0x00380038u) | kMagic, scl[1], nz[1]), s2);
-    }
-    const uint32_t p15 = ((w[0] >> 15) & 0x00010001u) | ((w[1] >> 14) & 0x00020002u) |
-                         ((w[2] >> 13) & 0x00040004u);
-    out[15] = h2_mul(h2_fma(p15 | kMagic, scl[0], nz[0]), s2);
-  } else {
-    #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t v = w[j], u = v >> 8;
-      out[4 * j + 0] = h2_mul(h2_fma((v & 0x000F000Fu) | kMagic, scl[0], nz[0]), s2);
-      out[4 * j + 1] = h2_mul(h2_fma((v & 0x00F000F0u) | kMagic, scl[1], nz[1]), s2);
-      out[4 * j + 2] = h2_mul(h2_fma((u & 0x000F000Fu) | kMagic, scl[0], nz[0]), s2);
-      out[4 * j + 3] = h2_mul(h2_fma((u & 0x00F000F0u) | kMagic, scl[1], nz[1]), s2);
-    }
-  }
+  const int c = pair_class<BITS>(j);
+  return h2_mul(h2_fma(pair_bits<BITS>(w, j) | kMagic, scl[c], nz[c]), s2);
 }
 
 // byte offset of (row r, 16-byte chunk c) inside a 128-row, 128B-swizzled K-major slab
@@ -195,6 +175,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     }
   } else {
     // ---------------- dequantisation ----------------
+    // thread (r, h): row r of the tile, chunks 2h and 2h+1 of each 128-code block, i.e. the
+    // codes k = 8j + 4h .. 8j + 4h + 3 (j = 0..15): 8-byte halves of the 16-byte swizzle units
     const int td = threadIdx.x - 64;          // 0..255
     const int r = td & (kBM - 1), h = td >> 7;
     const int row = min(n0 + r, p.N - 1);
@@ -220,27 +202,29 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit);
       if (!ok) break;
       unsigned char* st = smem + s * L::kStage;
-      const uint32_t* pw = reinterpret_cast<const uint32_t*>(st + L::kX + L::kA + r * 16 * BITS) + h * 2 * BITS;
-      unsigned char* slab = st + L::kX + h * kBM * 128;
+      const uint32_t* pw = reinterpret_cast<const uint32_t*>(st + L::kX + L::kA + r * 16 * BITS);
+      uint32_t wa[BITS], wb[BITS];
       #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t w[BITS];
-        #pragma unroll
-        for (int j = 0; j < BITS; ++j) w[j] = pw[cc * BITS + j];
-        uint32_t o[16];
-        dequant_chunk<BITS>(w, s2, scl, nz, o);
-        #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(slab + sw128_off(r, cc * 4 + j)) =
-              make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      for (int j = 0; j < BITS; ++j) {
+        wa[j] = pw[(2 * h) * BITS + j];
+        wb[j] = pw[(2 * h + 1) * BITS + j];
       }
-      // weak columns of this 64-code slab: their fp16 values replace the zero-filled codes
+      unsigned char* abase = st + L::kX;
+      #pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t lo = dequant_pair<BITS>(wa, j, s2, scl, nz);   // k = 8j + 4h, +1
+        const uint32_t hi = dequant_pair<BITS>(wb, j, s2, scl, nz);   // k = 8j + 4h + 2, +3
+        unsigned char* slab = abase + (j >> 3) * kBM * 128;
+        *reinterpret_cast<uint2*>(slab + sw128_off(r, j & 7) + 8 * h) = make_uint2(lo, hi);
+      }
+      // weak columns of this block whose code falls in this thread's halves: their fp16
+      // values replace the zero-filled codes
       const int t0 = p.blk_weak[kb], t1 = p.blk_weak[kb + 1];
       for (int t = t0; t < t1; ++t) {
         const int col = p.idx[t] - kb * kStepCodes;
-        if ((col >> 6) != h) continue;
-        const int c = col & 63;
-        __half* dst = reinterpret_cast<__half*>(slab + sw128_off(r, c >> 3)) + (c & 7);
+        if (((col >> 2) & 1) != h) continue;
+        unsigned char* slab = abase + (col >> 6) * kBM * 128;
+        __half* dst = reinterpret_cast<__half*>(slab + sw128_off(r, (col >> 3) & 7)) + (col & 7);
         *dst = p.w_weak[(size_t)row * p.k_ld + t];
       }
       fence_proxy_async_smem();

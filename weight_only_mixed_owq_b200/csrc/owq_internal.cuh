@@ -20,7 +20,7 @@ constexpr int kMaxGemvM = 16;
 struct Layer {
   uint32_t magic;
   int device;
-  int N, K, bits, group, G, k, k_ld;   // k_ld: row stride of w_weak (k rounded up to 8)
+  int N, K, bits, group, G, k, k_ld;   // k_ld: row stride of w_weak (k rounded up to 16)
   uint32_t* packed;     // N x (K*bits/32) words
   __half* scales;       // N x G
   __half* zeros;        // N x G
@@ -56,7 +56,9 @@ struct GemvProblem {
   __half* y;
   int N, K, G, k, k_ld;
   int row_groups;     // ceil(N / rows_per_group)
-  int group_base;     // first global row-group index of this problem
+  int group_base;     // first global row-group index of this problem (register-pipelined kernel)
+  int cta_base;       // first CTA of this problem (bulk-copy kernel)
+  int ncta;           // CTAs serving this problem (bulk-copy kernel)
 };
 cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cudaStream_t s);
 
