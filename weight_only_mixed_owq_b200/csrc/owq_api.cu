@@ -154,7 +154,7 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   L->k_ld = std::max(16, (k + 15) & ~15);   // 16-wide tensor-core k slices
   L->stream = s;
   L->maps_ready = false;
-  const size_t packed_bytes = (size_t)N * K * bits / 8;
+  const size_t packed_bytes = (size_t)((N + 15) & ~15) * K * bits / 8;   // 16-row tiles
   const size_t sz_bytes = (size_t)N * L->G * sizeof(__half);
   const size_t weak_bytes = (size_t)N * L->k_ld * sizeof(__half);
   const int Kb = K / kBlockCodes;
@@ -183,6 +183,7 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
     blk[b] = t;
   }
 
+  if (e == cudaSuccess) e = cudaMemsetAsync(L->packed, 0, packed_bytes, s);   // padding rows of the last tile
   if (e == cudaSuccess) e = cudaMemcpyAsync(L->scales, scales, sz_bytes, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(L->zeros, zeros, sz_bytes, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(L->w_weak, 0, weak_bytes, s);

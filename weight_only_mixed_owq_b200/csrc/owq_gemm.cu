@@ -9,15 +9,16 @@
 //
 // One CTA computes a 128-weight-row x BN-token tile of y^T (MMA M = weight rows,
 // MMA N = tokens), looping over K in 128-code steps through an S-stage ring:
-//   warp 0      TMA producer: the packed 128 x (16*bits) byte tile (no swizzle) and two
-//               128B-swizzled BN x 64 fp16 activation boxes per step.
+//   warp 0      TMA producer: the packed 128 x (16*bits) byte tile (a 3-D box over the layer's
+//               16-row-tile storage, no swizzle) and two 128B-swizzled BN x 64 fp16
+//               activation boxes per step.
 //   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16,
 //               fp32 accumulator BN columns wide in tensor memory).
-//   warps 2-9   dequantisation: each thread owns one weight row and one 64-code half of a
-//               step, unpacks the codes in registers, forms fp16_rn(s (q - z)) with exact
-//               fp16x2 arithmetic, stores the 16-byte chunks into the K-major 128B-swizzled
-//               A tile, then overwrites the weak columns of that slab with their fp16
-//               values (no activation gather is needed).  The same warps run the epilogue
+//   warps 2-9   dequantisation: each thread owns one weight row and two chunks of each
+//               128-code step (codes 8j + 4h .. 8j + 4h + 3), unpacks them in registers, forms
+//               fp16_rn(s (q - z)) with exact fp16x2 arithmetic, stores 8-byte halves of the
+//               16-byte units of the K-major 128B-swizzled A tile, then overwrites its weak
+//               columns with their fp16 values (no activation gather is needed).  The same warps run the epilogue
 //               (tcgen05.ld of their TMEM lane quarter, fp16 rounding, coalesced stores).
 // Every mbarrier wait is bounded (clock64 limit): on expiry the thread records the device
 // status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
@@ -140,7 +141,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         if (!ok) break;
         unsigned char* st = smem + s * L::kStage;
         mbar_arrive_expect_tx(&full[s], kBytes);
-        tma_load_2d(st + L::kX + L::kA, &map_p, &full[s], kb * 16 * BITS, n0);
+        // packed: block kb of the 8 16-row tiles of this CTA (tile-major storage)
+        tma_load_3d(st + L::kX + L::kA, &map_p, &full[s], 0, kb, n0 / 16);
         tma_load_2d(st, &map_x, &full[s], kb * kStepCodes, m0);
         tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
       }
@@ -289,13 +291,24 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_packed_3d(CUtensorMap* m, const void* base, int K, int N, int bits) {
+  EncodeTiled enc = get_encoder();
+  if (!enc) return false;
+  const int Kb = K / kStepCodes;
+  const uint64_t tile_blk = 16ull * 16 * bits;          // bytes of one block of a 16-row tile
+  const cuuint64_t dims[3] = {tile_blk / 4, (cuuint64_t)Kb, (cuuint64_t)((N + 15) / 16)};
+  const cuuint64_t strides[2] = {tile_blk, tile_blk * Kb};
+  const cuuint32_t box[3] = {(cuuint32_t)(tile_blk / 4), 1, kBM / 16};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BITS, int BN, int S>
 owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
   if (!L.maps_ready) {
-    const uint64_t rb = (uint64_t)L.K * BITS / 8;
-    if (!encode_2d(&L.map_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.packed, rb, (uint64_t)L.N, rb,
-                   16 * BITS, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return OWQ_ERR_CUDA;
+    if (!encode_packed_3d(&L.map_packed, L.packed, L.K, L.N, BITS)) return OWQ_ERR_CUDA;
     L.maps_ready = true;
   }
   CUtensorMap mx;

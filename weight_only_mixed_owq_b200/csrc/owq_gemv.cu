@@ -8,9 +8,10 @@
 // Design (B200, HBM-bound):
 //  * Persistent CTAs, one per SM, 8 warps.  A CTA walks 16-row tiles of W; its warps split
 //    K into 8 contiguous ranges of 128-code blocks.  Each warp streams its (16 rows x up to
-//    kSub blocks) sub-tiles through a private S-stage shared-memory ring filled by
-//    cp.async.bulk (one copy per row, completion counted on the stage's mbarrier), so about
-//    150 KB per SM is in flight without costing registers.
+//    8 blocks) items through a private S-stage shared-memory ring: the layer stores every
+//    16-row tile block-major, so an item is one contiguous range and one cp.async.bulk,
+//    completion counted on the stage's mbarrier.  About 150 KB per SM is in flight without
+//    costing registers.
 //  * The contraction runs on the tensor cores (mma.sync m16n8k16, fp16 x fp16 -> fp32): with
 //    the packed layout of owq_format.cuh a lane's chunk of a block is exactly its A fragment,
 //    and one AND per code pair makes each A register (the codes as exact fp16 values
@@ -46,16 +47,14 @@ struct GemvArgs {
   int* status;   // device status word (bounded waits)
 };
 
-template <int BITS>
+template <int BITS, int S>
 struct Geo {
   static constexpr int kBlk = 16 * BITS;                       // bytes of one block of one row
-  static constexpr int kSub = BITS == 3 ? 8 : 4;               // blocks per ring stage
-  // padded row stride: the 32 lanes' fragment loads of one stage hit 32 distinct banks
-  static constexpr int kRowStride = BITS == 3 ? 400 : 320;
-  static constexpr int kStage = 16 * kRowStride;
-  static constexpr int kS = BITS == 3 ? 3 : 4;                 // stages per warp
-  static constexpr int kRing = kWarps * kS * kStage;
-  static constexpr int kBars = kWarps * kS * 8;
+  static constexpr int kTileBlk = 16 * kBlk;                   // one block of a 16-row tile (contiguous)
+  static constexpr int kSub = 8;                               // blocks per ring stage
+  static constexpr int kStage = kSub * kTileBlk;               // 6 KB (3-bit) / 8 KB (4-bit)
+  static constexpr int kRing = kWarps * S * kStage;
+  static constexpr int kBars = kWarps * S * 8;
 };
 
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
@@ -69,14 +68,12 @@ __device__ __forceinline__ uint4 ldg_u128(const void* p) {
   return r;
 }
 
-// D = A * B + C, m16n8k16, f16 inputs, f32 accumulators
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
-                                         const float (&c)[4]) {
+// D += A * B, m16n8k16, f16 inputs, f32 accumulators (in place)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-               "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
-               : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1),
-                 "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+               "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // sum_j q_j x_j from the class accumulators (exact power-of-two rescales)
@@ -86,111 +83,168 @@ __device__ __forceinline__ float combine(float a0, float a1, float a2) {
   else return 16777216.f * a0 + 1048576.f * a1;
 }
 
-template <int BITS, int NT>
+// P warps share a 16-row tile (each owns Kb / P consecutive blocks); the CTA's 8 warps work
+// on 8 / P row tiles at a time.
+template <int BITS, int NT, int S, int P, bool XSMEM>
 __global__ void __launch_bounds__(kWarps * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
-  using G_ = Geo<BITS>;
-  constexpr int S = G_::kS;
+  using G_ = Geo<BITS, S>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
   constexpr int MT = 8 * NT;                 // token capacity
+  constexpr int G8 = kWarps / P;             // row tiles per CTA round
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tig = lane & 3;
   const int M = args.M;
+  const int gw = warp / P, pw = warp % P;    // row tile of the round, part of K
 
   int pi = 0;
   #pragma unroll 1
   for (int q = 1; q < args.count; ++q)
     if ((int)blockIdx.x >= args.p[q].cta_base) pi = q;
-  const GemvProblem& P = args.p[pi];
-  const int K = P.K, Kb = K / kBlockCodes, Gn = P.G, k = P.k, N = P.N;
+  const GemvProblem& Pb = args.p[pi];
+  const int K = Pb.K, Kb = K / kBlockCodes, Gn = Pb.G, k = Pb.k, N = Pb.N;
   const bool per_group = Gn > 1;
-  const size_t row_bytes = (size_t)K * BITS / 8;
+  const int xstride = K / 2 + 4;             // words per token row of the staged activations
 
   unsigned char* ring = smem + warp * S * G_::kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_::kRing) + warp * S;
-  float* red = reinterpret_cast<float*>(smem + G_::kRing + G_::kBars);          // [2][warps][16][MT]
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + G_::kRing) + kWarps * S;
+  float* red = reinterpret_cast<float*>(smem + G_::kRing + G_::kBars + 16);     // [2][warps][16][MT]
   float* sx = red + 2 * kWarps * 16 * MT;                                        // [MT][Kb]
   __half* xw = reinterpret_cast<__half*>(sx + ((MT * Kb + 3) & ~3));           // [MT][k_ld]
+  uint32_t* xs = reinterpret_cast<uint32_t*>(xw + MT * Pb.k_ld);               // [M][xstride]
 
-  // this CTA's row tiles and this warp's block range
-  const int c = (int)blockIdx.x - P.cta_base;
+  // rounds of this CTA, this warp's block range
+  const int c = (int)blockIdx.x - Pb.cta_base;
   const int RT = (N + 15) / 16;
-  const int n_rt = c < RT ? (RT - c + P.ncta - 1) / P.ncta : 0;
-  const int b_lo = warp * Kb / kWarps, b_hi = (warp + 1) * Kb / kWarps;
+  const int units = (RT + G8 - 1) / G8;
+  const int n_rnd = c < units ? (units - c + Pb.ncta - 1) / Pb.ncta : 0;
+  const int b_lo = pw * Kb / P, b_hi = (pw + 1) * Kb / P;
   const int nb = b_hi - b_lo;
   const int n_sub = nb > 0 ? (nb + G_::kSub - 1) / G_::kSub : 1;   // an empty range still takes one empty item
-  const int T = n_rt * n_sub;
+  const int T = n_rnd * n_sub;
 
-  auto issue = [&](int it) {   // called by the whole warp
-    const int st = it % S, rt = c + (it / n_sub) * P.ncta, sub = it % n_sub;
+  // the layer stores each 16-row tile block-major (owq_pack.cu), so an item -- 16 rows x nbs
+  // consecutive blocks -- is one contiguous range: one bulk copy issued by lane 0
+  auto issue = [&](int it) {
+    const int st = it % S, rt = (c + (it / n_sub) * Pb.ncta) * G8 + gw, sub = it % n_sub;
     const int b0 = b_lo + sub * G_::kSub;
-    const int nbs = max(0, min(G_::kSub, b_hi - b0));
-    const int nrows = min(16, N - rt * 16);
-    const uint32_t bytes = (uint32_t)(nbs * G_::kBlk);
-    if (lane == 0) mbar_arrive_expect_tx(&bars[st], bytes * (uint32_t)nrows);
-    __syncwarp();
-    if (lane < nrows && bytes > 0) {
-      const unsigned char* src = reinterpret_cast<const unsigned char*>(P.packed) +
-                                 (size_t)(rt * 16 + lane) * row_bytes + (size_t)b0 * G_::kBlk;
-      bulk_load(ring + st * G_::kStage + lane * G_::kRowStride, src, bytes, &bars[st]);
+    const int nbs = rt < RT ? max(0, min(G_::kSub, b_hi - b0)) : 0;
+    const uint32_t bytes = (uint32_t)(nbs * G_::kTileBlk);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[st], bytes);
+      if (bytes > 0) {
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(Pb.packed) +
+                                   ((size_t)rt * Kb + b0) * G_::kTileBlk;
+        bulk_load(ring + st * G_::kStage, src, bytes, &bars[st]);
+      }
     }
   };
   if (lane == 0) {
     for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
+    if (warp == 0) mbar_init(xbar, 1);
     fence_mbar_init();
   }
-  __syncwarp();
+  __syncthreads();   // every barrier initialised before any thread waits on one
   int issued = 0;
   for (; issued < min(S, T); ++issued) issue(issued);
+  // the weights do not depend on the previous kernel in the stream: let the next one start
+  // and only now wait for the previous one before touching activations or outputs
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- CTA prologue: per-block activation sums (16 lanes per block) and the weak gather ----
-  const int pieces = MT * Kb * 16;
-  for (int p0 = 0; p0 < pieces; p0 += blockDim.x) {
-    const int p = p0 + threadIdx.x;
-    float v = 0.f;
-    const int m = p / (Kb * 16), rem = p % (Kb * 16);
-    if (p < pieces && m < M) {
-      const uint4 q = ldg_u128(P.x + (size_t)m * K + (size_t)rem * 8);
-      const uint32_t h[4] = {q.x, q.y, q.z, q.w};
-      #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
-        v += f.x;
-        v += f.y;
-      }
+  // ---- CTA prologue: activations into shared memory (one bulk copy per token row, padded
+  //      stride so the fragment reads of different tokens fall in different banks), then the
+  //      per-block activation sums and the weak-column gather from there ----
+  if constexpr (XSMEM) {
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(xbar, (uint32_t)(M * K * 2));
+      for (int m = 0; m < M; ++m) bulk_load(xs + m * xstride, Pb.x + (size_t)m * K, (uint32_t)(K * 2), xbar);
     }
-    #pragma unroll
-    for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (p < pieces && (p & 15) == 0) sx[p >> 4] = v;
+    const bool ok_x = mbar_wait(xbar, 0, args.status, kWaitLimit);
+    (void)ok_x;
   }
-  for (int e = threadIdx.x; e < MT * P.k_ld; e += blockDim.x) {
-    const int m = e / P.k_ld, t = e % P.k_ld;
-    xw[e] = (m < M && t < k) ? P.x[(size_t)m * K + P.idx[t]] : __float2half_rn(0.f);
+  {
+    const int pieces = M * Kb * 16;
+    for (int p0 = 0; p0 < pieces; p0 += blockDim.x) {
+      const int p = p0 + threadIdx.x;
+      float v = 0.f;
+      if (p < pieces) {
+        const int m = p / (Kb * 16), rem = p % (Kb * 16);
+        uint4 q;
+        if constexpr (XSMEM) q = *reinterpret_cast<const uint4*>(xs + m * xstride + rem * 4);
+        else q = ldg_u128(Pb.x + (size_t)m * K + (size_t)rem * 8);
+        const uint32_t h[4] = {q.x, q.y, q.z, q.w};
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
+          v += f.x;
+          v += f.y;
+        }
+      }
+      #pragma unroll
+      for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (p < pieces && (p & 15) == 0) sx[p >> 4] = v;
+    }
+  }
+  for (int e = threadIdx.x; e < MT * Pb.k_ld; e += blockDim.x) {
+    const int m = e / Pb.k_ld, t = e % Pb.k_ld;
+    __half v = __float2half_rn(0.f);
+    if (m < M && t < k) {
+      const int col = Pb.idx[t];
+      if constexpr (XSMEM) v = reinterpret_cast<const __half*>(xs + m * xstride)[col];
+      else v = Pb.x[(size_t)m * K + col];
+    }
+    xw[e] = v;
   }
   __syncthreads();
 
-  // activation sums over this warp's block range (per-channel fold), tokens 2tig, 2tig+1 (+8)
+  // activation sums over this warp's block range (per-channel fold), tokens 2tig, 2tig+1 (+8);
+  // tokens >= M only feed outputs that are never stored
   float sxw[NT][2];
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
     #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int tok = 8 * nt + 2 * tig + e;
+      const int tok = min(8 * nt + 2 * tig + e, M - 1);
       float v = 0.f;
       for (int b = b_lo; b < b_hi; ++b) v += sx[tok * Kb + b];
       sxw[nt][e] = v;
     }
 
-  const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+  // B fragment source rows (clamped: columns of tokens >= M are discarded)
+  int xtok[NT];
+  #pragma unroll
+  for (int nt = 0; nt < NT; ++nt) xtok[nt] = min(8 * nt + g, M - 1);
+
+  constexpr int kMaxWs = 8;   // weak k slices per warp kept in registers
   float D[NC][NT][4];
   float y[NT][4];
   int it = 0, fail_it = -1;
   bool ok = true;
   #pragma unroll 1
-  for (int rti = 0; rti < n_rt; ++rti) {
-    const int rt = c + rti * P.ncta;
+  for (int rnd = 0; rnd < n_rnd; ++rnd) {
+    const int rt = (c + rnd * Pb.ncta) * G8 + gw;
+    const bool live = rt < RT;
     const int row_a = min(rt * 16 + g, N - 1), row_b = min(rt * 16 + g + 8, N - 1);
+    // loads needed only at the end of the row tile: issue them now
+    float sa = 0.f, za = 0.f, sb = 0.f, zb = 0.f;
+    if (!per_group && live) {
+      sa = __half2float(Pb.scales[row_a]); za = __half2float(Pb.zeros[row_a]);
+      sb = __half2float(Pb.scales[row_b]); zb = __half2float(Pb.zeros[row_b]);
+    }
+    uint32_t wfr[kMaxWs][4];
+    #pragma unroll
+    for (int u = 0; u < kMaxWs; ++u) {
+      const int ws = pw + u * P;
+      if (live && ws * 16 < k) {
+        const __half* wr_a = Pb.w_weak + (size_t)row_a * Pb.k_ld + 16 * ws + 2 * tig;
+        const __half* wr_b = Pb.w_weak + (size_t)row_b * Pb.k_ld + 16 * ws + 2 * tig;
+        wfr[u][0] = ldg_u32(wr_a); wfr[u][1] = ldg_u32(wr_b);
+        wfr[u][2] = ldg_u32(wr_a + 8); wfr[u][3] = ldg_u32(wr_b + 8);
+      }
+    }
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
       #pragma unroll
@@ -208,16 +262,16 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         if (!ok) fail_it = it;
       }
       const int b0 = b_lo + sub * G_::kSub;
-      const int nbs = ok ? max(0, min(G_::kSub, b_hi - b0)) : 0;
-      const unsigned char* stage = ring + st * G_::kStage;
+      const int nbs = (ok && live) ? max(0, min(G_::kSub, b_hi - b0)) : 0;
+      const unsigned char* frag = ring + st * G_::kStage + g * G_::kBlk + tig * 4 * BITS;
       #pragma unroll 1
       for (int bb = 0; bb < nbs; ++bb) {
         const int b = b0 + bb;
-        // A fragments: chunk tig of rows g and g + 8
+        // A fragments: chunk tig of rows g and g + 8 (the 32 lanes hit 32 distinct banks)
         uint32_t wa[BITS], wb[BITS];
         {
-          const unsigned char* ra = stage + g * G_::kRowStride + bb * G_::kBlk + tig * 4 * BITS;
-          const unsigned char* rb = ra + 8 * G_::kRowStride;
+          const unsigned char* ra = frag + bb * G_::kTileBlk;
+          const unsigned char* rb = ra + 8 * G_::kBlk;
           if constexpr (BITS == 4) {
             const uint4 qa = *reinterpret_cast<const uint4*>(ra);
             const uint4 qb = *reinterpret_cast<const uint4*>(rb);
@@ -231,46 +285,49 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
             }
           }
         }
-        // B fragments: activation pairs p = 4j + tig of block b, token 8nt + g
+        // B fragments: activation pairs p = 4j + tig of block b for token xtok
         uint32_t xb[NT][16];
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const int tok = 8 * nt + g;
-          if (tok < M) {
-            const __half* xr = P.x + (size_t)tok * K + (size_t)b * kBlockCodes + 2 * tig;
+          if constexpr (XSMEM) {
+            const uint32_t* xr = xs + xtok[nt] * xstride + b * 64 + tig;
+            #pragma unroll
+            for (int j = 0; j < 16; ++j) xb[nt][j] = xr[4 * j];
+          } else {
+            const __half* xr = Pb.x + (size_t)xtok[nt] * K + (size_t)b * kBlockCodes + 2 * tig;
             #pragma unroll
             for (int j = 0; j < 16; ++j) xb[nt][j] = ldg_u32(xr + 8 * j);
-          } else {
-            #pragma unroll
-            for (int j = 0; j < 16; ++j) xb[nt][j] = 0u;
           }
+        }
+        if (per_group) {
+          #pragma unroll
+          for (int cl = 0; cl < NC; ++cl)
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              #pragma unroll
+              for (int i = 0; i < 4; ++i) D[cl][nt][i] = 0.f;
         }
         #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const int cl = pair_class<BITS>(2 * s);
-          // the first k slice of each offset class in a block restarts its accumulator
-          // when the layer has one scale per block (per-group)
-          const bool first = BITS == 3 ? (s < 3) : (s < 2);
           const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s), pair_bits<BITS>(wb, 2 * s),
                                  pair_bits<BITS>(wa, 2 * s + 1), pair_bits<BITS>(wb, 2 * s + 1)};
           #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (per_group && first) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1], zero4);
-            else mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1], D[cl][nt]);
-          }
+          for (int nt = 0; nt < NT; ++nt) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
         }
         if (per_group) {
-          const float sa = __half2float(P.scales[(size_t)row_a * Gn + b]);
-          const float za = __half2float(P.zeros[(size_t)row_a * Gn + b]);
-          const float sb = __half2float(P.scales[(size_t)row_b * Gn + b]);
-          const float zb = __half2float(P.zeros[(size_t)row_b * Gn + b]);
+          const float gsa = __half2float(Pb.scales[(size_t)row_a * Gn + b]);
+          const float gza = __half2float(Pb.zeros[(size_t)row_a * Gn + b]);
+          const float gsb = __half2float(Pb.scales[(size_t)row_b * Gn + b]);
+          const float gzb = __half2float(Pb.zeros[(size_t)row_b * Gn + b]);
           #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
             #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const float sxv = sx[(8 * nt + 2 * tig + (i & 1)) * Kb + b];
+              const int tok = min(8 * nt + 2 * tig + (i & 1), M - 1);
+              const float sxv = sx[tok * Kb + b];
               const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
-              const float sc = i < 2 ? sa : sb, z = i < 2 ? za : zb;
+              const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
               y[nt][i] = fmaf(sc, fmaf(-z, sxv, v), y[nt][i]);
             }
         }
@@ -285,8 +342,6 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
 
     // ---- this warp's part of the row tile is done: fold, weak columns, reduction ----
     if (!per_group) {
-      const float sa = __half2float(P.scales[row_a]), za = __half2float(P.zeros[row_a]);
-      const float sb = __half2float(P.scales[row_b]), zb = __half2float(P.zeros[row_b]);
       #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         #pragma unroll
@@ -296,37 +351,36 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           y[nt][i] = sc * fmaf(-z, sxw[nt][i & 1], v);
         }
     }
-    #pragma unroll 1
-    for (int ws = warp; ws * 16 < k; ws += kWarps) {
-      const __half* wr_a = P.w_weak + (size_t)row_a * P.k_ld + 16 * ws + 2 * tig;
-      const __half* wr_b = P.w_weak + (size_t)row_b * P.k_ld + 16 * ws + 2 * tig;
-      const uint32_t a[4] = {ldg_u32(wr_a), ldg_u32(wr_b), ldg_u32(wr_a + 8), ldg_u32(wr_b + 8)};
-      #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const __half* xr = xw + (8 * nt + g) * P.k_ld + 16 * ws + 2 * tig;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 8);
-        float dw[4];
-        mma16816(dw, a, b0, b1, zero4);
+    #pragma unroll
+    for (int u = 0; u < kMaxWs; ++u) {
+      const int ws = pw + u * P;
+      if (live && ws * 16 < k) {
         #pragma unroll
-        for (int i = 0; i < 4; ++i) y[nt][i] += dw[i];
+        for (int nt = 0; nt < NT; ++nt) {
+          const __half* xr = xw + (8 * nt + g) * Pb.k_ld + 16 * ws + 2 * tig;
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 8);
+          mma16816(y[nt], wfr[u], b0, b1);
+        }
       }
     }
-    float* rbuf = red + (size_t)(rti & 1) * kWarps * 16 * MT + (size_t)warp * 16 * MT;
+    float* rbuf = red + (size_t)(rnd & 1) * kWarps * 16 * MT + (size_t)warp * 16 * MT;
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
       #pragma unroll
       for (int i = 0; i < 4; ++i)
         rbuf[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
     __syncthreads();
-    if ((int)threadIdx.x < 16 * MT) {
-      const int r = threadIdx.x / MT, tok = threadIdx.x % MT;
-      const float* rs = red + (size_t)(rti & 1) * kWarps * 16 * MT + r * MT + tok;
+    // reduce: thread -> (row tile of the round, row, token), sum over the P warps of that tile
+    for (int e = threadIdx.x; e < G8 * 16 * MT; e += blockDim.x) {
+      const int tg = e / (16 * MT), r = (e / MT) % 16, tok = e % MT;
+      const int rtile = (c + rnd * Pb.ncta) * G8 + tg;
+      const float* rs = red + (size_t)(rnd & 1) * kWarps * 16 * MT + (size_t)(tg * P) * 16 * MT + r * MT + tok;
       float v = 0.f;
       #pragma unroll
-      for (int w = 0; w < kWarps; ++w) v += rs[w * 16 * MT];
-      const int row = rt * 16 + r;
-      if (ok && row < N && tok < M) P.y[(size_t)tok * N + row] = __float2half_rn(v);
+      for (int w = 0; w < P; ++w) v += rs[w * 16 * MT];
+      const int row = rtile * 16 + r;
+      if (ok && rtile < RT && row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(v);
     }
   }
   // after a timeout: never exit with bulk copies still writing into this CTA's memory
@@ -348,21 +402,46 @@ int sm_count() {
   return n;
 }
 
-template <int BITS, int NT>
-cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
-  using G_ = Geo<BITS>;
+template <int BITS, int NT, int S, int P, bool XSMEM>
+cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
+  auto kern = k_gemv_mma<BITS, NT, S, P, XSMEM>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int base = 0;
+  for (int q = 0; q < a.count; ++q) base += a.p[q].ncta;
+  // programmatic dependent launch: this kernel may start while the previous one in the stream
+  // drains; it waits (griddepcontrol.wait) before reading activations or writing outputs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(base);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int BITS, int NT, int P>
+cudaError_t launch_p(GemvArgs& a, cudaStream_t s) {
   constexpr int MT = 8 * NT;
+  constexpr int G8 = kWarps / P;
+  constexpr size_t kMaxSmem = 232448;
   const int C = sm_count();
   long long work[kMaxProblems], total = 0;
-  size_t extra = 0;
+  size_t extra = 0, xbytes = 0;
   for (int q = 0; q < a.count; ++q) {
-    GemvProblem& P = a.p[q];
-    const int Kb = P.K / kBlockCodes;
-    P.row_groups = (P.N + 15) / 16;
-    work[q] = (long long)P.row_groups * Kb;
+    GemvProblem& Pq = a.p[q];
+    const int Kb = Pq.K / kBlockCodes;
+    Pq.row_groups = ((Pq.N + 15) / 16 + G8 - 1) / G8;        // CTA rounds of work
+    work[q] = (long long)Pq.row_groups * Kb;
     total += work[q];
-    const size_t need = (size_t)((MT * Kb + 3) & ~3) * sizeof(float) + (size_t)MT * P.k_ld * sizeof(__half);
+    const size_t need = (size_t)((MT * Kb + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half);
     if (need > extra) extra = need;
+    const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
+    if (xb > xbytes) xbytes = xb;
   }
   // CTAs per problem in proportion to its work, at least one each, one resident wave in total
   int n[kMaxProblems], used = 0, big = 0;
@@ -388,14 +467,24 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
     a.p[q].ncta = n[q];
     base += n[q];
   }
-  const size_t smem = (size_t)G_::kRing + G_::kBars + (size_t)2 * kWarps * 16 * MT * sizeof(float) +
-                      ((extra + 15) & ~size_t(15));
-  if (smem > 232448) return cudaErrorInvalidValue;
-  auto kern = k_gemv_mma<BITS, NT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  kern<<<base, kWarps * 32, smem, s>>>(a);
-  return cudaGetLastError();
+  // shared memory: ring + barriers + reduction + sums/gather (+ staged activations)
+  auto smem_for = [&](int S, bool xs) {
+    const size_t ring = (size_t)kWarps * S * Geo<BITS, 1>::kStage;
+    return ring + (size_t)kWarps * S * 8 + 16 + (size_t)2 * kWarps * 16 * MT * sizeof(float) +
+           ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
+  };
+  if (smem_for(3, true) <= kMaxSmem) return launch_k<BITS, NT, 3, P, true>(a, smem_for(3, true), s);
+  if (smem_for(2, true) <= kMaxSmem) return launch_k<BITS, NT, 2, P, true>(a, smem_for(2, true), s);
+  if (smem_for(3, false) <= kMaxSmem) return launch_k<BITS, NT, 3, P, false>(a, smem_for(3, false), s);
+  return cudaErrorInvalidValue;
+}
+
+template <int BITS, int NT>
+cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
+  // short K: 4 warps per row tile (two row tiles per CTA round), else 8
+  int kb_max = 0;
+  for (int q = 0; q < a.count; ++q) kb_max = max(kb_max, a.p[q].K / kBlockCodes);
+  return kb_max < 64 ? launch_p<BITS, NT, 4>(a, s) : launch_p<BITS, NT, 8>(a, s);
 }
 
 template <int BITS>

@@ -5,6 +5,13 @@
 namespace owq {
 namespace {
 
+// Storage order of the blocks in a layer: rows are grouped in tiles of 16 (the last tile
+// padded with zero rows); a tile stores its blocks block-major, so block b of rows
+// 16t .. 16t+15 is one contiguous run of 16 blocks at block index (t * Kb + b) * 16 + row % 16.
+__host__ __device__ __forceinline__ size_t tiled_block(int row, int b, int Kb) {
+  return ((size_t)(row >> 4) * Kb + b) * 16 + (row & 15);
+}
+
 // One thread per 128-code block.  Codes of weak columns are replaced by the zero point of
 // their (row, group), so the packed dense matrix dequantises to exactly 0 there.
 template <int BITS>
@@ -40,7 +47,7 @@ __global__ void k_pack(const uint8_t* __restrict__ codes, const __half* __restri
   }
   uint32_t w[4 * BITS];
   encode_block<BITS>(c, w);
-  uint4* dst = reinterpret_cast<uint4*>(packed + item * 4 * BITS);
+  uint4* dst = reinterpret_cast<uint4*>(packed + tiled_block(i, b, Kb) * 4 * BITS);
   #pragma unroll
   for (int v = 0; v < BITS; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
 }
@@ -55,7 +62,7 @@ __global__ void k_dequant(const uint32_t* __restrict__ packed, const __half* __r
   if (item >= (size_t)N * Kb) return;
   const int i = (int)(item / Kb), b = (int)(item % Kb);
   uint32_t w[4 * BITS];
-  const uint4* src = reinterpret_cast<const uint4*>(packed + item * 4 * BITS);
+  const uint4* src = reinterpret_cast<const uint4*>(packed + tiled_block(i, b, Kb) * 4 * BITS);
   #pragma unroll
   for (int v = 0; v < BITS; ++v) {
     const uint4 a = src[v];
