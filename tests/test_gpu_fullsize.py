@@ -77,23 +77,34 @@ def test_fullsize_quantize_and_products(case):
     layer.close()
 
 
-def test_fullsize_qkv_multi_launch_matches_single():
-    """q, k, v of the OPT-6.7B set in one owq_gemv_multi launch (as bench.py runs them)."""
+def test_fullsize_qkv_multi_launch_matches_oracle():
+    """q, k, v of the OPT-6.7B set in one owq_gemv_multi launch (as bench.py runs them).
+
+    A multi launch may split K differently from three single launches (it has three times the
+    row tiles), so the two agree to fp32 rounding, not bit for bit; both must meet the
+    tolerance against the oracle."""
     import weight_only_mixed_owq_b200 as owq
     spec = owq_synth.WORKLOADS[1]
-    layers, xs, single = [], [], []
+    layers, xs, single, refs, xs_np = [], [], [], [], []
     for li in range(3):
         L = spec.layers[li]
         d = owq_synth.draw_layer(L, spec, 1, owq_synth.seed_for(1, li))
+        ref = oracle.owq_quantize(d["W"], d["X"], L.bits, L.group, L.k)
         lay, _ = owq.quantize_pack(torch.from_numpy(d["W"]).to(DEV), torch.from_numpy(d["X"]).to(DEV),
                                    L.bits, L.group, L.k)
         layers.append(lay)
         xs.append(torch.from_numpy(d["x"]).to(DEV))
+        xs_np.append(d["x"])
+        refs.append(ref)
         single.append(lay.gemv(xs[-1]))
     ys = [torch.empty_like(y) for y in single]
     assert owq.owq_gemv_multi([l.handle for l in layers], xs, ys, 1) == 0
     torch.cuda.synchronize()
-    for a, b in zip(ys, single):
-        assert torch.equal(a, b)
+    rows = _rows(4096, 99)
+    for a, b, ref, x in zip(ys, single, refs, xs_np):
+        assert float(torch.abs(a.float() - b.float()).max()) <= 1e-2
+        y64 = oracle.matmul_rows(ref["codes"], ref["scales"], ref["zeros"], ref["w_weak"], ref["idx"], x, rows)
+        check_output(a.cpu().numpy()[:, rows], y64, "qkv multi")
+        check_output(b.cpu().numpy()[:, rows], y64, "qkv single")
     for l in layers:
         l.close()

@@ -172,7 +172,8 @@ def test_gemv_multi_matches_single(owq):
     assert owq.owq_gemv_multi([L.handle for L in layers], xs, ys, 2) == 0
     torch.cuda.synchronize()
     for a, b in zip(ys, ys_single):
-        assert torch.equal(a, b)
+        # the multi launch may split K differently (fp32 sums in another order)
+        assert float(torch.abs(a.float() - b.float()).max()) <= 1e-2
     for L in layers:
         L.close()
 

@@ -37,7 +37,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kMaxProblems = 16;
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr long long kWaitLimit = 4000000000LL;   // ~2 s
 
 struct GemvArgs {
@@ -51,8 +51,8 @@ template <int BITS, int S>
 struct Geo {
   static constexpr int kBlk = 16 * BITS;                       // bytes of one block of one row
   static constexpr int kTileBlk = 16 * kBlk;                   // one block of a 16-row tile (contiguous)
-  static constexpr int kSub = 8;                               // blocks per ring stage
-  static constexpr int kStage = kSub * kTileBlk;               // 6 KB (3-bit) / 8 KB (4-bit)
+  static constexpr int kSub = 4;                               // blocks per ring stage
+  static constexpr int kStage = kSub * kTileBlk;               // 3 KB (3-bit) / 4 KB (4-bit)
   static constexpr int kRing = kWarps * S * kStage;
   static constexpr int kBars = kWarps * S * 8;
 };
@@ -83,15 +83,67 @@ __device__ __forceinline__ float combine(float a0, float a1, float a2) {
   else return 16777216.f * a0 + 1048576.f * a1;
 }
 
-// P warps share a 16-row tile (each owns Kb / P consecutive blocks); the CTA's 8 warps work
-// on 8 / P row tiles at a time.
+// Activations in fragment order: pair p = 4j + t of block b of token m is word
+// (m * xstride + b * 64 + t * 16 + 4 ((j / 4) ^ t) + j % 4) -- lane t's sixteen pairs of a block
+// are four 16-byte units, XOR-swizzled so that the four lanes t of a load hit four bank groups.
+__device__ __forceinline__ int xi_word(int b, int t, int v) { return b * 64 + t * 16 + 4 * (v ^ t); }
+
+// Per-block work of one warp: A fragments of rows g, g+8 from the staged tile, B fragments
+// from the staged activations, 8 k slices of m16n8k16 into the class accumulators.
+template <int BITS, int NT, bool XSMEM>
+__device__ __forceinline__ void block_mma(const unsigned char* frag, const uint32_t* xs, const __half* xg,
+                                          int xstride, int K, const int* xtok, int b, int tig,
+                                          float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+  constexpr int kBlk = 16 * BITS;
+  uint32_t wa[BITS], wb[BITS];
+  if constexpr (BITS == 4) {
+    const uint4 qa = *reinterpret_cast<const uint4*>(frag);
+    const uint4 qb = *reinterpret_cast<const uint4*>(frag + 8 * kBlk);
+    wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
+    wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
+  } else {
+    #pragma unroll
+    for (int j = 0; j < BITS; ++j) {
+      wa[j] = reinterpret_cast<const uint32_t*>(frag)[j];
+      wb[j] = reinterpret_cast<const uint32_t*>(frag + 8 * kBlk)[j];
+    }
+  }
+  uint32_t xb[NT][16];
+  #pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    if constexpr (XSMEM) {
+      const uint32_t* xr = xs + xtok[nt] * xstride;
+      #pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 q = *reinterpret_cast<const uint4*>(xr + xi_word(b, tig, v));
+        xb[nt][4 * v] = q.x; xb[nt][4 * v + 1] = q.y; xb[nt][4 * v + 2] = q.z; xb[nt][4 * v + 3] = q.w;
+      }
+    } else {
+      const __half* xr = xg + (size_t)xtok[nt] * K + (size_t)b * kBlockCodes + 2 * tig;
+      #pragma unroll
+      for (int j = 0; j < 16; ++j) xb[nt][j] = ldg_u32(xr + 8 * j);
+    }
+  }
+  #pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int cl = pair_class<BITS>(2 * s);
+    const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s), pair_bits<BITS>(wb, 2 * s),
+                           pair_bits<BITS>(wa, 2 * s + 1), pair_bits<BITS>(wb, 2 * s + 1)};
+    #pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
+  }
+}
+
+// P warps share a 16-row tile (each owns Kb / P consecutive blocks); the CTA's warps work on
+// kWarps / P row tiles at a time (a "round").
 template <int BITS, int NT, int S, int P, bool XSMEM>
 __global__ void __launch_bounds__(kWarps * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
   using G_ = Geo<BITS, S>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
   constexpr int MT = 8 * NT;                 // token capacity
-  constexpr int G8 = kWarps / P;             // row tiles per CTA round
+  constexpr int G8 = kWarps / P;             // row tiles per round
+  constexpr int UNR = NT == 1 ? 2 : 1;       // blocks per loop iteration (independent accumulators)
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tig = lane & 3;
@@ -103,17 +155,20 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   for (int q = 1; q < args.count; ++q)
     if ((int)blockIdx.x >= args.p[q].cta_base) pi = q;
   const GemvProblem& Pb = args.p[pi];
-  const int K = Pb.K, Kb = K / kBlockCodes, Gn = Pb.G, k = Pb.k, N = Pb.N;
+  const int K = Pb.K, Kb = K / kBlockCodes, Gn = Pb.G, k = Pb.k, N = Pb.N, k_ld = Pb.k_ld;
   const bool per_group = Gn > 1;
-  const int xstride = K / 2 + 4;             // words per token row of the staged activations
+  const int xstride = K / 2 + 4;             // words per staged token row
 
+  // shared memory carve-up (sizes computed identically on the host)
   unsigned char* ring = smem + warp * S * G_::kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_::kRing) + warp * S;
-  uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + G_::kRing) + kWarps * S;
-  float* red = reinterpret_cast<float*>(smem + G_::kRing + G_::kBars + 16);     // [2][warps][16][MT]
-  float* sx = red + 2 * kWarps * 16 * MT;                                        // [MT][Kb]
-  __half* xw = reinterpret_cast<__half*>(sx + ((MT * Kb + 3) & ~3));           // [MT][k_ld]
-  uint32_t* xs = reinterpret_cast<uint32_t*>(xw + MT * Pb.k_ld);               // [M][xstride]
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + G_::kRing) + kWarps * S;   // activations
+  uint64_t* wbar = xbar + 1;                                                      // [2] weak rows per round
+  float* red = reinterpret_cast<float*>(smem + G_::kRing + G_::kBars + 32);      // [2][warps][16][MT]
+  float* sx = red + 2 * kWarps * 16 * MT;                                         // [MT][Kb]
+  __half* xw = reinterpret_cast<__half*>(sx + ((MT * Kb + 3) & ~3));            // [MT][k_ld]
+  __half* wk = xw + MT * k_ld;                                                    // [2][G8*16][k_ld]
+  uint32_t* xs = reinterpret_cast<uint32_t*>(wk + 2 * G8 * 16 * k_ld);          // [M][xstride]
 
   // rounds of this CTA, this warp's block range
   const int c = (int)blockIdx.x - Pb.cta_base;
@@ -141,29 +196,39 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       }
     }
   };
+  // weak rows of the round's row tiles (consecutive rows of W_weak): one copy by thread 0
+  auto issue_weak = [&](int rnd) {
+    if (threadIdx.x != 0 || k == 0) return;
+    const int row0 = (c + rnd * Pb.ncta) * G8 * 16;
+    const int nrows = max(0, min(G8 * 16, N - row0));
+    const uint32_t bytes = (uint32_t)(nrows * k_ld * 2);
+    mbar_arrive_expect_tx(&wbar[rnd & 1], bytes);
+    if (bytes > 0) bulk_load(wk + (rnd & 1) * G8 * 16 * k_ld, Pb.w_weak + (size_t)row0 * k_ld, bytes, &wbar[rnd & 1]);
+  };
   if (lane == 0) {
     for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
-    if (warp == 0) mbar_init(xbar, 1);
+    if (warp == 0) { mbar_init(xbar, 1); mbar_init(&wbar[0], 1); mbar_init(&wbar[1], 1); }
     fence_mbar_init();
   }
   __syncthreads();   // every barrier initialised before any thread waits on one
   int issued = 0;
   for (; issued < min(S, T); ++issued) issue(issued);
+  if (n_rnd > 0) issue_weak(0);
+  if (n_rnd > 1) issue_weak(1);
   // the weights do not depend on the previous kernel in the stream: let the next one start
   // and only now wait for the previous one before touching activations or outputs
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- CTA prologue: activations into shared memory (one bulk copy per token row, padded
-  //      stride so the fragment reads of different tokens fall in different banks), then the
-  //      per-block activation sums and the weak-column gather from there ----
+  // ---- CTA prologue: activations into shared memory (one bulk copy per token row), the
+  //      per-block activation sums, the weak-column gather, then the activations are permuted
+  //      in place into fragment order ----
   if constexpr (XSMEM) {
     if (threadIdx.x == 0) {
       mbar_arrive_expect_tx(xbar, (uint32_t)(M * K * 2));
       for (int m = 0; m < M; ++m) bulk_load(xs + m * xstride, Pb.x + (size_t)m * K, (uint32_t)(K * 2), xbar);
     }
-    const bool ok_x = mbar_wait(xbar, 0, args.status, kWaitLimit);
-    (void)ok_x;
+    mbar_wait(xbar, 0, args.status, kWaitLimit);
   }
   {
     const int pieces = M * Kb * 16;
@@ -188,8 +253,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       if (p < pieces && (p & 15) == 0) sx[p >> 4] = v;
     }
   }
-  for (int e = threadIdx.x; e < MT * Pb.k_ld; e += blockDim.x) {
-    const int m = e / Pb.k_ld, t = e % Pb.k_ld;
+  for (int e = threadIdx.x; e < MT * k_ld; e += blockDim.x) {
+    const int m = e / k_ld, t = e % k_ld;
     __half v = __float2half_rn(0.f);
     if (m < M && t < k) {
       const int col = Pb.idx[t];
@@ -197,6 +262,24 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       else v = Pb.x[(size_t)m * K + col];
     }
     xw[e] = v;
+  }
+  if constexpr (XSMEM) {
+    __syncthreads();   // sums and gather read the natural order
+    for (int e = threadIdx.x; e < M * Kb; e += blockDim.x) {
+      uint32_t* blk = xs + (e / Kb) * xstride + (e % Kb) * 64;
+      uint32_t w[64];
+      #pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        const uint4 q = reinterpret_cast<const uint4*>(blk)[v];
+        w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
+      }
+      #pragma unroll
+      for (int t = 0; t < 4; ++t)
+        #pragma unroll
+        for (int v = 0; v < 4; ++v)   // pairs j = 4v .. 4v+3 of lane t: p = 4j + t
+          *reinterpret_cast<uint4*>(blk + t * 16 + 4 * (v ^ t)) =
+              make_uint4(w[4 * (4 * v) + t], w[4 * (4 * v + 1) + t], w[4 * (4 * v + 2) + t], w[4 * (4 * v + 3) + t]);
+    }
   }
   __syncthreads();
 
@@ -212,14 +295,10 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       for (int b = b_lo; b < b_hi; ++b) v += sx[tok * Kb + b];
       sxw[nt][e] = v;
     }
-
-  // B fragment source rows (clamped: columns of tokens >= M are discarded)
   int xtok[NT];
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt) xtok[nt] = min(8 * nt + g, M - 1);
 
-  constexpr int kMaxWs = 8;   // weak k slices per warp kept in registers
-  float D[NC][NT][4];
   float y[NT][4];
   int it = 0, fail_it = -1;
   bool ok = true;
@@ -228,31 +307,25 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     const int rt = (c + rnd * Pb.ncta) * G8 + gw;
     const bool live = rt < RT;
     const int row_a = min(rt * 16 + g, N - 1), row_b = min(rt * 16 + g + 8, N - 1);
-    // loads needed only at the end of the row tile: issue them now
-    float sa = 0.f, za = 0.f, sb = 0.f, zb = 0.f;
+    float sa = 0.f, za = 0.f, sb = 0.f, zb = 0.f;    // per-channel scale / zero, used at the end
     if (!per_group && live) {
       sa = __half2float(Pb.scales[row_a]); za = __half2float(Pb.zeros[row_a]);
       sb = __half2float(Pb.scales[row_b]); zb = __half2float(Pb.zeros[row_b]);
     }
-    uint32_t wfr[kMaxWs][4];
+    float D[UNR][NC][NT][4];
     #pragma unroll
-    for (int u = 0; u < kMaxWs; ++u) {
-      const int ws = pw + u * P;
-      if (live && ws * 16 < k) {
-        const __half* wr_a = Pb.w_weak + (size_t)row_a * Pb.k_ld + 16 * ws + 2 * tig;
-        const __half* wr_b = Pb.w_weak + (size_t)row_b * Pb.k_ld + 16 * ws + 2 * tig;
-        wfr[u][0] = ldg_u32(wr_a); wfr[u][1] = ldg_u32(wr_b);
-        wfr[u][2] = ldg_u32(wr_a + 8); wfr[u][3] = ldg_u32(wr_b + 8);
-      }
-    }
+    for (int u = 0; u < UNR; ++u)
+      #pragma unroll
+      for (int cl = 0; cl < NC; ++cl)
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) D[u][cl][nt][i] = 0.f;
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
       #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        y[nt][i] = 0.f;
-        #pragma unroll
-        for (int cl = 0; cl < NC; ++cl) D[cl][nt][i] = 0.f;
-      }
+      for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
+
     #pragma unroll 1
     for (int sub = 0; sub < n_sub; ++sub, ++it) {
       const int st = it % S;
@@ -265,71 +338,42 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       const int nbs = (ok && live) ? max(0, min(G_::kSub, b_hi - b0)) : 0;
       const unsigned char* frag = ring + st * G_::kStage + g * G_::kBlk + tig * 4 * BITS;
       #pragma unroll 1
-      for (int bb = 0; bb < nbs; ++bb) {
-        const int b = b0 + bb;
-        // A fragments: chunk tig of rows g and g + 8 (the 32 lanes hit 32 distinct banks)
-        uint32_t wa[BITS], wb[BITS];
-        {
-          const unsigned char* ra = frag + bb * G_::kTileBlk;
-          const unsigned char* rb = ra + 8 * G_::kBlk;
-          if constexpr (BITS == 4) {
-            const uint4 qa = *reinterpret_cast<const uint4*>(ra);
-            const uint4 qb = *reinterpret_cast<const uint4*>(rb);
-            wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
-            wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
-          } else {
-            #pragma unroll
-            for (int j = 0; j < BITS; ++j) {
-              wa[j] = reinterpret_cast<const uint32_t*>(ra)[j];
-              wb[j] = reinterpret_cast<const uint32_t*>(rb)[j];
-            }
-          }
-        }
-        // B fragments: activation pairs p = 4j + tig of block b for token xtok
-        uint32_t xb[NT][16];
-        #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if constexpr (XSMEM) {
-            const uint32_t* xr = xs + xtok[nt] * xstride + b * 64 + tig;
-            #pragma unroll
-            for (int j = 0; j < 16; ++j) xb[nt][j] = xr[4 * j];
-          } else {
-            const __half* xr = Pb.x + (size_t)xtok[nt] * K + (size_t)b * kBlockCodes + 2 * tig;
-            #pragma unroll
-            for (int j = 0; j < 16; ++j) xb[nt][j] = ldg_u32(xr + 8 * j);
-          }
-        }
+      for (int bb = 0; bb < nbs; bb += UNR) {
         if (per_group) {
           #pragma unroll
-          for (int cl = 0; cl < NC; ++cl)
+          for (int u = 0; u < UNR; ++u)
             #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int cl = 0; cl < NC; ++cl)
               #pragma unroll
-              for (int i = 0; i < 4; ++i) D[cl][nt][i] = 0.f;
+              for (int nt = 0; nt < NT; ++nt)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) D[u][cl][nt][i] = 0.f;
         }
-        #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int cl = pair_class<BITS>(2 * s);
-          const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s), pair_bits<BITS>(wb, 2 * s),
-                                 pair_bits<BITS>(wa, 2 * s + 1), pair_bits<BITS>(wb, 2 * s + 1)};
-          #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
+        block_mma<BITS, NT, XSMEM>(frag + bb * G_::kTileBlk, xs, Pb.x, xstride, K, xtok, b0 + bb, tig, D[0]);
+        if constexpr (UNR == 2) {
+          if (bb + 1 < nbs)
+            block_mma<BITS, NT, XSMEM>(frag + (bb + 1) * G_::kTileBlk, xs, Pb.x, xstride, K, xtok, b0 + bb + 1, tig, D[1]);
         }
         if (per_group) {
-          const float gsa = __half2float(Pb.scales[(size_t)row_a * Gn + b]);
-          const float gza = __half2float(Pb.zeros[(size_t)row_a * Gn + b]);
-          const float gsb = __half2float(Pb.scales[(size_t)row_b * Gn + b]);
-          const float gzb = __half2float(Pb.zeros[(size_t)row_b * Gn + b]);
           #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int tok = min(8 * nt + 2 * tig + (i & 1), M - 1);
-              const float sxv = sx[tok * Kb + b];
-              const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
-              const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
-              y[nt][i] = fmaf(sc, fmaf(-z, sxv, v), y[nt][i]);
+          for (int u = 0; u < UNR; ++u) {
+            const int b = b0 + bb + u;
+            if (u == 0 || bb + u < nbs) {
+              const float gsa = __half2float(Pb.scales[(size_t)row_a * Gn + b]);
+              const float gza = __half2float(Pb.zeros[(size_t)row_a * Gn + b]);
+              const float gsb = __half2float(Pb.scales[(size_t)row_b * Gn + b]);
+              const float gzb = __half2float(Pb.zeros[(size_t)row_b * Gn + b]);
+              #pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int tok = min(8 * nt + 2 * tig + (i & 1), M - 1);
+                  const float v = combine<BITS>(D[u][0][nt][i], D[u][1][nt][i], D[u][NC - 1][nt][i]);
+                  const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
+                  y[nt][i] = fmaf(sc, fmaf(-z, sx[tok * Kb + b], v), y[nt][i]);
+                }
             }
+          }
         }
       }
       __syncwarp();
@@ -346,21 +390,27 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       for (int nt = 0; nt < NT; ++nt)
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
+          float v = combine<BITS>(D[0][0][nt][i], D[0][1][nt][i], D[0][NC - 1][nt][i]);
+          if constexpr (UNR == 2) v += combine<BITS>(D[1][0][nt][i], D[1][1][nt][i], D[1][NC - 1][nt][i]);
           const float sc = i < 2 ? sa : sb, z = i < 2 ? za : zb;
           y[nt][i] = sc * fmaf(-z, sxw[nt][i & 1], v);
         }
     }
-    #pragma unroll
-    for (int u = 0; u < kMaxWs; ++u) {
-      const int ws = pw + u * P;
-      if (live && ws * 16 < k) {
-        #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const __half* xr = xw + (8 * nt + g) * Pb.k_ld + 16 * ws + 2 * tig;
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 8);
-          mma16816(y[nt], wfr[u], b0, b1);
+    if (k > 0) {
+      const bool ok_w = mbar_wait(&wbar[rnd & 1], (uint32_t)((rnd >> 1) & 1), args.status, kWaitLimit);
+      if (live && ok_w) {
+        const __half* wr = wk + (size_t)((rnd & 1) * G8 * 16 + gw * 16 + g) * k_ld + 2 * tig;
+        #pragma unroll 1
+        for (int ws = pw; ws * 16 < k; ws += P) {
+          const uint32_t a[4] = {*reinterpret_cast<const uint32_t*>(wr + 16 * ws),
+                                 *reinterpret_cast<const uint32_t*>(wr + 8 * k_ld + 16 * ws),
+                                 *reinterpret_cast<const uint32_t*>(wr + 16 * ws + 8),
+                                 *reinterpret_cast<const uint32_t*>(wr + 8 * k_ld + 16 * ws + 8)};
+          #pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const __half* xr = xw + (8 * nt + g) * k_ld + 16 * ws + 2 * tig;
+            mma16816(y[nt], a, *reinterpret_cast<const uint32_t*>(xr), *reinterpret_cast<const uint32_t*>(xr + 8));
+          }
         }
       }
     }
@@ -371,6 +421,11 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       for (int i = 0; i < 4; ++i)
         rbuf[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
     __syncthreads();
+    // the weak buffer of this round is free again: fetch the round after next into it
+    if (rnd + 2 < n_rnd) {
+      if (threadIdx.x == 0) fence_proxy_async_smem();
+      issue_weak(rnd + 2);
+    }
     // reduce: thread -> (row tile of the round, row, token), sum over the P warps of that tile
     for (int e = threadIdx.x; e < G8 * 16 * MT; e += blockDim.x) {
       const int tg = e / (16 * MT), r = (e / MT) % 16, tok = e % MT;
@@ -438,7 +493,8 @@ cudaError_t launch_p(GemvArgs& a, cudaStream_t s) {
     Pq.row_groups = ((Pq.N + 15) / 16 + G8 - 1) / G8;        // CTA rounds of work
     work[q] = (long long)Pq.row_groups * Kb;
     total += work[q];
-    const size_t need = (size_t)((MT * Kb + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half);
+    const size_t need = (size_t)((MT * Kb + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half) +
+                        (size_t)2 * G8 * 16 * Pq.k_ld * sizeof(__half);
     if (need > extra) extra = need;
     const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
     if (xb > xbytes) xbytes = xb;
@@ -467,24 +523,29 @@ cudaError_t launch_p(GemvArgs& a, cudaStream_t s) {
     a.p[q].ncta = n[q];
     base += n[q];
   }
-  // shared memory: ring + barriers + reduction + sums/gather (+ staged activations)
+  // shared memory: ring + barriers + reduction + sums / gather / weak rows (+ staged activations)
   auto smem_for = [&](int S, bool xs) {
     const size_t ring = (size_t)kWarps * S * Geo<BITS, 1>::kStage;
-    return ring + (size_t)kWarps * S * 8 + 16 + (size_t)2 * kWarps * 16 * MT * sizeof(float) +
+    return ring + (size_t)kWarps * S * 8 + 32 + (size_t)2 * kWarps * 16 * MT * sizeof(float) +
            ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
   };
   if (smem_for(3, true) <= kMaxSmem) return launch_k<BITS, NT, 3, P, true>(a, smem_for(3, true), s);
   if (smem_for(2, true) <= kMaxSmem) return launch_k<BITS, NT, 2, P, true>(a, smem_for(2, true), s);
   if (smem_for(3, false) <= kMaxSmem) return launch_k<BITS, NT, 3, P, false>(a, smem_for(3, false), s);
+  if (smem_for(2, false) <= kMaxSmem) return launch_k<BITS, NT, 2, P, false>(a, smem_for(2, false), s);
   return cudaErrorInvalidValue;
 }
 
 template <int BITS, int NT>
 cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
-  // short K: 4 warps per row tile (two row tiles per CTA round), else 8
-  int kb_max = 0;
-  for (int q = 0; q < a.count; ++q) kb_max = max(kb_max, a.p[q].K / kBlockCodes);
-  return kb_max < 64 ? launch_p<BITS, NT, 4>(a, s) : launch_p<BITS, NT, 8>(a, s);
+  // warps per 16-row tile: as few as possible (more K per warp) while the rounds still cover
+  // every SM once
+  int rt_total = 0;
+  for (int q = 0; q < a.count; ++q) rt_total += (a.p[q].N + 15) / 16;
+  const int C = sm_count();
+  if (rt_total >= 4 * C) return launch_p<BITS, NT, 4>(a, s);
+  if (rt_total >= 2 * C) return launch_p<BITS, NT, 8>(a, s);
+  return launch_p<BITS, NT, 16>(a, s);
 }
 
 template <int BITS>
