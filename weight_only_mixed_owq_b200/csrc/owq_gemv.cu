@@ -89,11 +89,11 @@ __device__ __forceinline__ float combine(float a0, float a1, float a2) {
 __device__ __forceinline__ int xi_word(int b, int t, int v) { return b * 64 + t * 16 + 4 * (v ^ t); }
 
 // Per-block work of one warp: A fragments of rows g, g+8 from the staged tile, B fragments
-// from the staged activations, 8 k slices of m16n8k16 into the class accumulators.
+// from the staged activations (xr: this lane's 64-byte unit row of block 0, xo: the four
+// swizzled unit offsets), 8 k slices of m16n8k16 into the class accumulators.
 template <int BITS, int NT, bool XSMEM>
-__device__ __forceinline__ void block_mma(const unsigned char* frag, const uint32_t* xs, const __half* xg,
-                                          int xstride, int K, const int* xtok, int b, int tig,
-                                          float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+__device__ __forceinline__ void block_mma(const unsigned char* frag, const uint32_t* const* xr, const int* xo,
+                                          const __half* const* xg, int b, float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
   constexpr int kBlk = 16 * BITS;
   uint32_t wa[BITS], wb[BITS];
   if constexpr (BITS == 4) {
@@ -112,16 +112,16 @@ __device__ __forceinline__ void block_mma(const unsigned char* frag, const uint3
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     if constexpr (XSMEM) {
-      const uint32_t* xr = xs + xtok[nt] * xstride;
+      const uint32_t* base = xr[nt] + b * 64;
       #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const uint4 q = *reinterpret_cast<const uint4*>(xr + xi_word(b, tig, v));
+        const uint4 q = *reinterpret_cast<const uint4*>(base + xo[v]);
         xb[nt][4 * v] = q.x; xb[nt][4 * v + 1] = q.y; xb[nt][4 * v + 2] = q.z; xb[nt][4 * v + 3] = q.w;
       }
     } else {
-      const __half* xr = xg + (size_t)xtok[nt] * K + (size_t)b * kBlockCodes + 2 * tig;
+      const __half* base = xg[nt] + (size_t)b * kBlockCodes;
       #pragma unroll
-      for (int j = 0; j < 16; ++j) xb[nt][j] = ldg_u32(xr + 8 * j);
+      for (int j = 0; j < 16; ++j) xb[nt][j] = ldg_u32(base + 8 * j);
     }
   }
   #pragma unroll
@@ -134,9 +134,19 @@ __device__ __forceinline__ void block_mma(const unsigned char* frag, const uint3
   }
 }
 
+template <int BITS, int NT>
+__device__ __forceinline__ void zero_acc(float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+  #pragma unroll
+  for (int cl = 0; cl < (BITS == 3 ? 3 : 2); ++cl)
+    #pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) D[cl][nt][i] = 0.f;
+}
+
 // P warps share a 16-row tile (each owns Kb / P consecutive blocks); the CTA's warps work on
 // kWarps / P row tiles at a time (a "round").
-template <int BITS, int NT, int S, int P, bool XSMEM>
+template <int BITS, int NT, int S, int P, bool XSMEM, bool PG>
 __global__ void __launch_bounds__(kWarps * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
   using G_ = Geo<BITS, S>;
@@ -156,7 +166,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     if ((int)blockIdx.x >= args.p[q].cta_base) pi = q;
   const GemvProblem& Pb = args.p[pi];
   const int K = Pb.K, Kb = K / kBlockCodes, Gn = Pb.G, k = Pb.k, N = Pb.N, k_ld = Pb.k_ld;
-  const bool per_group = Gn > 1;
+  constexpr bool per_group = PG;             // one scale / zero per 128-code block
   const int xstride = K / 2 + 4;             // words per staged token row
 
   // shared memory carve-up (sizes computed identically on the host)
@@ -295,9 +305,19 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       for (int b = b_lo; b < b_hi; ++b) v += sx[tok * Kb + b];
       sxw[nt][e] = v;
     }
-  int xtok[NT];
+  // per-lane operand pointers (tokens >= M are clamped: their columns are discarded)
+  const uint32_t* xr[NT];
+  const __half* xg[NT];
   #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) xtok[nt] = min(8 * nt + g, M - 1);
+  for (int nt = 0; nt < NT; ++nt) {
+    const int tok = min(8 * nt + g, M - 1);
+    xr[nt] = xs + tok * xstride + tig * 16;
+    xg[nt] = Pb.x + (size_t)tok * K + 2 * tig;
+  }
+  int xo[4];
+  #pragma unroll
+  for (int v = 0; v < 4; ++v) xo[v] = 4 * (v ^ tig);
+  const int frag_lane = g * G_::kBlk + tig * 4 * BITS;
 
   float y[NT][4];
   int it = 0, fail_it = -1;
@@ -314,17 +334,28 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     }
     float D[UNR][NC][NT][4];
     #pragma unroll
-    for (int u = 0; u < UNR; ++u)
-      #pragma unroll
-      for (int cl = 0; cl < NC; ++cl)
-        #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          #pragma unroll
-          for (int i = 0; i < 4; ++i) D[u][cl][nt][i] = 0.f;
+    for (int u = 0; u < UNR; ++u) zero_acc<BITS, NT>(D[u]);
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
       #pragma unroll
       for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
+
+    // per-group fold of one block's accumulators
+    auto fold = [&](float (&Du)[NC][NT][4], int b) {
+      const float gsa = __half2float(Pb.scales[(size_t)row_a * Gn + b]);
+      const float gza = __half2float(Pb.zeros[(size_t)row_a * Gn + b]);
+      const float gsb = __half2float(Pb.scales[(size_t)row_b * Gn + b]);
+      const float gzb = __half2float(Pb.zeros[(size_t)row_b * Gn + b]);
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = min(8 * nt + 2 * tig + (i & 1), M - 1);
+          const float v = combine<BITS>(Du[0][nt][i], Du[1][nt][i], Du[NC - 1][nt][i]);
+          const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
+          y[nt][i] = fmaf(sc, fmaf(-z, sx[tok * Kb + b], v), y[nt][i]);
+        }
+    };
 
     #pragma unroll 1
     for (int sub = 0; sub < n_sub; ++sub, ++it) {
@@ -336,44 +367,21 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       }
       const int b0 = b_lo + sub * G_::kSub;
       const int nbs = (ok && live) ? max(0, min(G_::kSub, b_hi - b0)) : 0;
-      const unsigned char* frag = ring + st * G_::kStage + g * G_::kBlk + tig * 4 * BITS;
-      #pragma unroll 1
-      for (int bb = 0; bb < nbs; bb += UNR) {
-        if (per_group) {
-          #pragma unroll
-          for (int u = 0; u < UNR; ++u)
-            #pragma unroll
-            for (int cl = 0; cl < NC; ++cl)
-              #pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                #pragma unroll
-                for (int i = 0; i < 4; ++i) D[u][cl][nt][i] = 0.f;
+      const unsigned char* frag = ring + st * G_::kStage + frag_lane;
+      if (nbs == G_::kSub) {
+        // full item: all kSub blocks unrolled, UNR independent accumulator sets
+        #pragma unroll
+        for (int bb = 0; bb < G_::kSub; ++bb) {
+          if (per_group) zero_acc<BITS, NT>(D[bb % UNR]);
+          block_mma<BITS, NT, XSMEM>(frag + bb * G_::kTileBlk, xr, xo, xg, b0 + bb, D[bb % UNR]);
+          if (per_group) fold(D[bb % UNR], b0 + bb);
         }
-        block_mma<BITS, NT, XSMEM>(frag + bb * G_::kTileBlk, xs, Pb.x, xstride, K, xtok, b0 + bb, tig, D[0]);
-        if constexpr (UNR == 2) {
-          if (bb + 1 < nbs)
-            block_mma<BITS, NT, XSMEM>(frag + (bb + 1) * G_::kTileBlk, xs, Pb.x, xstride, K, xtok, b0 + bb + 1, tig, D[1]);
-        }
-        if (per_group) {
-          #pragma unroll
-          for (int u = 0; u < UNR; ++u) {
-            const int b = b0 + bb + u;
-            if (u == 0 || bb + u < nbs) {
-              const float gsa = __half2float(Pb.scales[(size_t)row_a * Gn + b]);
-              const float gza = __half2float(Pb.zeros[(size_t)row_a * Gn + b]);
-              const float gsb = __half2float(Pb.scales[(size_t)row_b * Gn + b]);
-              const float gzb = __half2float(Pb.zeros[(size_t)row_b * Gn + b]);
-              #pragma unroll
-              for (int nt = 0; nt < NT; ++nt)
-                #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int tok = min(8 * nt + 2 * tig + (i & 1), M - 1);
-                  const float v = combine<BITS>(D[u][0][nt][i], D[u][1][nt][i], D[u][NC - 1][nt][i]);
-                  const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
-                  y[nt][i] = fmaf(sc, fmaf(-z, sx[tok * Kb + b], v), y[nt][i]);
-                }
-            }
-          }
+      } else {
+        #pragma unroll 1
+        for (int bb = 0; bb < nbs; ++bb) {
+          if (per_group) zero_acc<BITS, NT>(D[0]);
+          block_mma<BITS, NT, XSMEM>(frag + bb * G_::kTileBlk, xr, xo, xg, b0 + bb, D[0]);
+          if (per_group) fold(D[0], b0 + bb);
         }
       }
       __syncwarp();
@@ -459,7 +467,7 @@ int sm_count() {
 
 template <int BITS, int NT, int S, int P, bool XSMEM>
 cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
-  auto kern = k_gemv_mma<BITS, NT, S, P, XSMEM>;
+  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, S, P, XSMEM, true> : k_gemv_mma<BITS, NT, S, P, XSMEM, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int base = 0;
@@ -557,6 +565,15 @@ cudaError_t launch_bits(GemvArgs& a, cudaStream_t s) {
 
 cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cudaStream_t s) {
   if (count < 1 || count > kMaxProblems) return cudaErrorInvalidValue;
+  // one launch serves layers of one kind (per-channel or per-group scales)
+  for (int q = 1; q < count; ++q)
+    if ((probs[q].G > 1) != (probs[0].G > 1)) {
+      for (int j = 0; j < count; ++j) {
+        cudaError_t e = launch_gemv(probs + j, 1, bits, M, s);
+        if (e != cudaSuccess) return e;
+      }
+      return cudaSuccess;
+    }
   GemvArgs a{};
   for (int q = 0; q < count; ++q) a.p[q] = probs[q];
   a.count = count;
