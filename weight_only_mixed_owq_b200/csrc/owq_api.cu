@@ -67,6 +67,9 @@ void release(Layer* L) {
   cudaFree(L->w_weak);
   cudaFree(L->idx);
   cudaFree(L->blk_weak);
+  cudaFree(L->w_weak_t);
+  cudaFree(L->part);
+  cudaFree(L->cnt);
   delete[] L->idx_host;
   L->magic = 0;
   delete L;
@@ -170,6 +173,18 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   alloc((void**)&L->w_weak, weak_bytes);
   alloc((void**)&L->idx, sizeof(int32_t) * std::max(k, 1));
   alloc((void**)&L->blk_weak, sizeof(int32_t) * (Kb + 1));
+  const size_t RT = (size_t)(N + 15) / 16;
+  const size_t weak_t_bytes = RT * 16 * L->k_ld * sizeof(__half);
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, L->device) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  L->seg_cap = gemv_seg_cap(N, K, sms);
+  const size_t part_bytes = RT * L->seg_cap * 16 * 16 * sizeof(float);
+  alloc((void**)&L->w_weak_t, weak_t_bytes);
+  alloc((void**)&L->part, part_bytes);
+  alloc((void**)&L->cnt, RT * sizeof(int));
   uint32_t* mask_dev = nullptr;
   alloc((void**)&mask_dev, sizeof(uint32_t) * (K / 32));
   if (e != cudaSuccess) { cudaFree(mask_dev); release(L); return cuda_status(e); }
@@ -193,8 +208,10 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   if (e == cudaSuccess && k > 0) e = cudaMemcpyAsync(L->idx, idx, sizeof(int32_t) * k, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(L->blk_weak, blk.data(), sizeof(int32_t) * (Kb + 1), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(mask_dev, mask.data(), sizeof(uint32_t) * (K / 32), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(L->cnt, 0, RT * sizeof(int), s);
   if (e == cudaSuccess)
     e = launch_pack(codes, reinterpret_cast<const __half*>(zeros), mask_dev, N, K, bits, group, L->packed, s);
+  if (e == cudaSuccess) e = launch_weak_tiles(L->w_weak, N, L->k_ld, L->w_weak_t, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // host tables above must outlive the copies
   cudaFree(mask_dev);
   if (e != cudaSuccess) { release(L); return cuda_status(e); }
@@ -217,7 +234,8 @@ static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvP
   P->x = reinterpret_cast<const __half*>(x);
   P->y = reinterpret_cast<__half*>(y);
   P->N = L->N; P->K = L->K; P->G = L->G; P->k = L->k; P->k_ld = L->k_ld;
-  P->row_groups = 0; P->group_base = 0;
+  P->w_weak_t = L->w_weak_t; P->part = L->part; P->cnt = L->cnt; P->seg_cap = L->seg_cap;
+  P->row_groups = 0; P->cta_base = 0; P->ncta = 0; P->chunk = 0;
   return OWQ_OK;
 }
 
@@ -240,6 +258,8 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
   for (int q = 0; q < count; ++q) {
     Layer* L = lookup(layers[q]);
     if (!L) return OWQ_ERR_HANDLE;
+    for (int j = 0; j < q; ++j)   // each layer's split-tile workspace serves one product
+      if (layers[j] == layers[q]) return OWQ_ERR_HANDLE;
     if (q == 0) bits = L->bits;
     else if (L->bits != bits) return OWQ_ERR_BITS;
     owq_status_t st = make_problem(L, xs[q], ys[q], &P[q]);

@@ -6,27 +6,27 @@
 // dense matrix is zero-filled at the weak columns, so the dense and weak terms simply add.
 //
 // Design (B200, HBM-bound):
-//  * Persistent CTAs, one per SM, 8 warps.  A CTA walks 16-row tiles of W; its warps split
-//    K into 8 contiguous ranges of 128-code blocks.  Each warp streams its (16 rows x up to
-//    8 blocks) items through a private S-stage shared-memory ring: the layer stores every
-//    16-row tile block-major, so an item is one contiguous range and one cp.async.bulk,
-//    completion counted on the stage's mbarrier.  About 150 KB per SM is in flight without
-//    costing registers.
+//  * Work is the list of (16-row tile, 128-code block) units in row-tile order.  Every warp of
+//    a persistent grid (one CTA of 16 warps per SM) takes one equal contiguous chunk of it
+//    (stream-K), so no SM idles while another finishes and no warp waits for another: there
+//    is no barrier after the prologue.
+//  * A warp streams its chunk through a private S-stage shared-memory ring filled by
+//    cp.async.bulk: the layer stores each 16-row tile block-major, so an item (16 rows x up to
+//    4 blocks of one tile) is one contiguous copy; the weak block, stored tile-major too, is
+//    streamed the same way at the start of each tile.
 //  * The contraction runs on the tensor cores (mma.sync m16n8k16, fp16 x fp16 -> fp32): with
 //    the packed layout of owq_format.cuh a lane's chunk of a block is exactly its A fragment,
 //    and one AND per code pair makes each A register (the codes as exact fp16 values
-//    q * 2^(o - 24), o the bit offset; one accumulator per offset class).  Activations are
-//    the B fragment (up to 8 tokens per n8 tile, two tiles for M > 8).  This keeps the issued
-//    work below one instruction per code, which CUDA-core FMAs cannot reach.
+//    q * 2^(o - 24), o the bit offset; one accumulator per offset class).  Activations are the
+//    B fragment (up to 8 tokens per n8 tile, two tiles for M > 8), staged once per CTA in
+//    fragment order.  This keeps the issued work per code low enough for the HBM rate.
 //  * Scale and zero point: for a group with scale s and zero z,
 //        sum_j s (q_j - z) x_j = s * (sum_j q_j x_j - z * sum_j x_j);
-//    the per-block activation sums are computed once per CTA.  Per-channel layers fold once
-//    per row tile, per-group layers once per block.  (The exact fp16 rounding of each
-//    s (q - z) is not applied; the difference is far inside the output tolerance.)
-//  * Weak columns: the fp16 weak block is the A operand of extra k slices (exact fp16
-//    products) against the activations gathered once per CTA into shared memory.
-//  * The 8 warps' partial sums of a row tile are added in shared memory; one fp16 rounding
-//    per output.
+//    the activation sums come from per-block prefix sums computed once per CTA.  (The fp16
+//    rounding of each s (q - z) is not applied; the difference is far inside the tolerance.)
+//  * A row tile split between warps is finished by the last segment to
+//    arrive: it adds the other segments' partial sums, in segment order, from the layer's
+//    workspace (deterministic), and resets the tile's counter for the next call.
 #include "owq_format.cuh"
 #include "owq_internal.cuh"
 #include "owq_sm100.cuh"
@@ -37,8 +37,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kMaxProblems = 16;
-constexpr int kWarps = 16;
-constexpr long long kWaitLimit = 4000000000LL;   // ~2 s
+constexpr int kWarps = kGemvWarps;
+constexpr int kSub = 4;                          // blocks per ring item
+constexpr long long kWaitLimit = 4000000000LL;  // ~2 s
 
 struct GemvArgs {
   GemvProblem p[kMaxProblems];
@@ -47,14 +48,12 @@ struct GemvArgs {
   int* status;   // device status word (bounded waits)
 };
 
-template <int BITS, int S>
+template <int BITS>
 struct Geo {
   static constexpr int kBlk = 16 * BITS;                       // bytes of one block of one row
-  static constexpr int kTileBlk = 16 * kBlk;                   // one block of a 16-row tile (contiguous)
-  static constexpr int kSub = 4;                               // blocks per ring stage
+  static constexpr int kTileBlk = 16 * kBlk;                   // one block of a 16-row tile
   static constexpr int kStage = kSub * kTileBlk;               // 3 KB (3-bit) / 4 KB (4-bit)
-  static constexpr int kRing = kWarps * S * kStage;
-  static constexpr int kBars = kWarps * S * 8;
+  static constexpr int kWs = kStage / 512;                     // weak k slices per item
 };
 
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
@@ -83,39 +82,45 @@ __device__ __forceinline__ float combine(float a0, float a1, float a2) {
   else return 16777216.f * a0 + 1048576.f * a1;
 }
 
-// Activations in fragment order: pair p = 4j + t of block b of token m is word
-// (m * xstride + b * 64 + t * 16 + 4 ((j / 4) ^ t) + j % 4) -- lane t's sixteen pairs of a block
-// are four 16-byte units, XOR-swizzled so that the four lanes t of a load hit four bank groups.
-__device__ __forceinline__ int xi_word(int b, int t, int v) { return b * 64 + t * 16 + 4 * (v ^ t); }
+template <int BITS, int NT>
+__device__ __forceinline__ void zero_acc(float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+  #pragma unroll
+  for (int cl = 0; cl < (BITS == 3 ? 3 : 2); ++cl)
+    #pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) D[cl][nt][i] = 0.f;
+}
 
-// Per-block work of one warp: A fragments of rows g, g+8 from the staged tile, B fragments
-// from the staged activations (xr: this lane's 64-byte unit row of block 0, xo: the four
-// swizzled unit offsets), 8 k slices of m16n8k16 into the class accumulators.
+// One unit (one 128-code block of a 16-row tile) of one warp: A fragments of rows g, g+8
+// from the staged tile (fa: this lane's chunk), B fragments from the staged activations (xv:
+// this lane's four 16-byte fragment pieces of block 0, xoff: the block's word offset) or from
+// global memory (xg, block b), then 8 k slices of m16n8k16 into the offset-class accumulators.
 template <int BITS, int NT, bool XSMEM>
-__device__ __forceinline__ void block_mma(const unsigned char* frag, const uint32_t* const* xr, const int* xo,
-                                          const __half* const* xg, int b, float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+__device__ __forceinline__ void unit_mma(const unsigned char* fa, const uint32_t* const (&xv)[NT][4], int xoff,
+                                         const __half* const (&xg)[NT], int b,
+                                         float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
   constexpr int kBlk = 16 * BITS;
   uint32_t wa[BITS], wb[BITS];
   if constexpr (BITS == 4) {
-    const uint4 qa = *reinterpret_cast<const uint4*>(frag);
-    const uint4 qb = *reinterpret_cast<const uint4*>(frag + 8 * kBlk);
+    const uint4 qa = *reinterpret_cast<const uint4*>(fa);
+    const uint4 qb = *reinterpret_cast<const uint4*>(fa + 8 * kBlk);
     wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
     wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
   } else {
     #pragma unroll
     for (int j = 0; j < BITS; ++j) {
-      wa[j] = reinterpret_cast<const uint32_t*>(frag)[j];
-      wb[j] = reinterpret_cast<const uint32_t*>(frag + 8 * kBlk)[j];
+      wa[j] = reinterpret_cast<const uint32_t*>(fa)[j];
+      wb[j] = reinterpret_cast<const uint32_t*>(fa + 8 * kBlk)[j];
     }
   }
   uint32_t xb[NT][16];
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     if constexpr (XSMEM) {
-      const uint32_t* base = xr[nt] + b * 64;
       #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const uint4 q = *reinterpret_cast<const uint4*>(base + xo[v]);
+        const uint4 q = *reinterpret_cast<const uint4*>(xv[nt][v] + xoff);
         xb[nt][4 * v] = q.x; xb[nt][4 * v + 1] = q.y; xb[nt][4 * v + 2] = q.z; xb[nt][4 * v + 3] = q.w;
       }
     } else {
@@ -134,321 +139,360 @@ __device__ __forceinline__ void block_mma(const unsigned char* frag, const uint3
   }
 }
 
-template <int BITS, int NT>
-__device__ __forceinline__ void zero_acc(float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
-  #pragma unroll
-  for (int cl = 0; cl < (BITS == 3 ? 3 : 2); ++cl)
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      #pragma unroll
-      for (int i = 0; i < 4; ++i) D[cl][nt][i] = 0.f;
+// Arrival on a split row tile: one acquire-release atomic at GPU scope (the warp's partial
+// stores, ordered before it by the warp barrier, are released with it; the last arrival
+// acquires the other segments' partials with it).
+__device__ __forceinline__ int arrive_acq_rel(int* ctr) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
+  return old;
 }
 
-// P warps share a 16-row tile (each owns Kb / P consecutive blocks); the CTA's warps work on
-// kWarps / P row tiles at a time (a "round").
-template <int BITS, int NT, int S, int P, bool XSMEM, bool PG>
+// The sequence of ring items of one warp's chunk [lo, hi) of (tile, block) units: for every
+// tile segment that starts at block 0, first the weak k slices of the tile (kWs per item),
+// then its blocks (up to kSub per item, never crossing a tile).  Producer and consumer each
+// run their own copy, so they agree item by item.
+struct ItemGen {
+  int rt, b, rem, wpos, nsl, Kb, wsi;
+  __device__ void init(int rt0, int b0, int units, int Kb_, int nsl_, int wsi_) {
+    rt = rt0; b = b0; rem = units; Kb = Kb_; nsl = nsl_; wsi = wsi_;
+    wpos = (units > 0 && b0 == 0) ? 0 : nsl;
+  }
+  // kind 0: weak slices [first, first + cnt) of tile rt_; kind 1: blocks [first, first + cnt)
+  __device__ __forceinline__ bool next(int& kind, int& rt_, int& first, int& cnt) {
+    if (rem <= 0) return false;
+    rt_ = rt;
+    if (wpos < nsl) {
+      kind = 0; first = wpos; cnt = min(wsi, nsl - wpos); wpos += cnt;
+      return true;
+    }
+    kind = 1; first = b; cnt = min(kSub, min(Kb - b, rem));
+    b += cnt; rem -= cnt;
+    if (b == Kb) { b = 0; ++rt; wpos = 0; }
+    return true;
+  }
+  // after a block item: does it end a tile segment?
+  __device__ __forceinline__ bool segment_done() const { return rem <= 0 || b == 0; }
+};
+
+template <int BITS, int NT, int S, bool XSMEM, bool PG>
 __global__ void __launch_bounds__(kWarps * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
-  using G_ = Geo<BITS, S>;
+  using G_ = Geo<BITS>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
   constexpr int MT = 8 * NT;                 // token capacity
-  constexpr int G8 = kWarps / P;             // row tiles per round
-  constexpr int UNR = NT == 1 ? 2 : 1;       // blocks per loop iteration (independent accumulators)
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tig = lane & 3;
   const int M = args.M;
-  const int gw = warp / P, pw = warp % P;    // row tile of the round, part of K
 
   int pi = 0;
   #pragma unroll 1
   for (int q = 1; q < args.count; ++q)
     if ((int)blockIdx.x >= args.p[q].cta_base) pi = q;
   const GemvProblem& Pb = args.p[pi];
-  const int K = Pb.K, Kb = K / kBlockCodes, Gn = Pb.G, k = Pb.k, N = Pb.N, k_ld = Pb.k_ld;
-  constexpr bool per_group = PG;             // one scale / zero per 128-code block
+  const int K = Pb.K, Kb = K / kBlockCodes, k = Pb.k, N = Pb.N, k_ld = Pb.k_ld;
+  const int nsl = k > 0 ? k_ld / 16 : 0;     // weak k slices of a tile
   const int xstride = K / 2 + 4;             // words per staged token row
+  const int W = ((N + 15) / 16) * Kb;        // (tile, block) units
+  const int c = Pb.chunk;
 
   // shared memory carve-up (sizes computed identically on the host)
   unsigned char* ring = smem + warp * S * G_::kStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_::kRing) + warp * S;
-  uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + G_::kRing) + kWarps * S;   // activations
-  uint64_t* wbar = xbar + 1;                                                      // [2] weak rows per round
-  float* red = reinterpret_cast<float*>(smem + G_::kRing + G_::kBars + 32);      // [2][warps][16][MT]
-  float* sx = red + 2 * kWarps * 16 * MT;                                         // [MT][Kb]
-  __half* xw = reinterpret_cast<__half*>(sx + ((MT * Kb + 3) & ~3));            // [MT][k_ld]
-  __half* wk = xw + MT * k_ld;                                                    // [2][G8*16][k_ld]
-  uint32_t* xs = reinterpret_cast<uint32_t*>(wk + 2 * G8 * 16 * k_ld);          // [M][xstride]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * S * G_::kStage) + warp * S;
+  float* psx = reinterpret_cast<float*>(smem + kWarps * S * G_::kStage + kWarps * S * 8 + 16);   // [MT][Kb+1]
+  __half* xw = reinterpret_cast<__half*>(psx + ((MT * (Kb + 1) + 3) & ~3));                        // [MT][k_ld]
+  int32_t* sidx = reinterpret_cast<int32_t*>(xw + MT * k_ld);                                      // [k_ld]
+  uint32_t* xs = reinterpret_cast<uint32_t*>(sidx + k_ld);                                          // [M][xstride]
 
-  // rounds of this CTA, this warp's block range
-  const int c = (int)blockIdx.x - Pb.cta_base;
-  const int RT = (N + 15) / 16;
-  const int units = (RT + G8 - 1) / G8;
-  const int n_rnd = c < units ? (units - c + Pb.ncta - 1) / Pb.ncta : 0;
-  const int b_lo = pw * Kb / P, b_hi = (pw + 1) * Kb / P;
-  const int nb = b_hi - b_lo;
-  const int n_sub = nb > 0 ? (nb + G_::kSub - 1) / G_::kSub : 1;   // an empty range still takes one empty item
-  const int T = n_rnd * n_sub;
-
-  // the layer stores each 16-row tile block-major (owq_pack.cu), so an item -- 16 rows x nbs
-  // consecutive blocks -- is one contiguous range: one bulk copy issued by lane 0
-  auto issue = [&](int it) {
-    const int st = it % S, rt = (c + (it / n_sub) * Pb.ncta) * G8 + gw, sub = it % n_sub;
-    const int b0 = b_lo + sub * G_::kSub;
-    const int nbs = rt < RT ? max(0, min(G_::kSub, b_hi - b0)) : 0;
-    const uint32_t bytes = (uint32_t)(nbs * G_::kTileBlk);
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[st], bytes);
-      if (bytes > 0) {
-        const unsigned char* src = reinterpret_cast<const unsigned char*>(Pb.packed) +
-                                   ((size_t)rt * Kb + b0) * G_::kTileBlk;
-        bulk_load(ring + st * G_::kStage, src, bytes, &bars[st]);
-      }
+  // this warp's chunk of units
+  const int wi = ((int)blockIdx.x - Pb.cta_base) * kWarps + warp;
+  const int lo = min(wi * c, W), hi = min(lo + c, W);
+  const int rt0 = lo / Kb, b0 = lo - rt0 * Kb;
+  ItemGen prod, cons;
+  prod.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs);
+  cons.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs);
+  int issued = 0;
+  // lane 0 only: the next item of the chunk into stage st (false once the chunk is exhausted)
+  auto issue = [&](int st) -> bool {
+    int kind, rt, first, cnt;
+    if (!prod.next(kind, rt, first, cnt)) return false;
+    const unsigned char* src;
+    uint32_t bytes;
+    if (kind == 0) {
+      src = reinterpret_cast<const unsigned char*>(Pb.w_weak_t) + ((size_t)rt * nsl + first) * 512;
+      bytes = (uint32_t)(cnt * 512);
+    } else {
+      src = reinterpret_cast<const unsigned char*>(Pb.packed) + ((size_t)rt * Kb + first) * G_::kTileBlk;
+      bytes = (uint32_t)(cnt * G_::kTileBlk);
     }
+    mbar_arrive_expect_tx(&bars[st], bytes);
+    bulk_load(ring + st * G_::kStage, src, bytes, &bars[st]);
+    ++issued;
+    return true;
   };
-  // weak rows of the round's row tiles (consecutive rows of W_weak): one copy by thread 0
-  auto issue_weak = [&](int rnd) {
-    if (threadIdx.x != 0 || k == 0) return;
-    const int row0 = (c + rnd * Pb.ncta) * G8 * 16;
-    const int nrows = max(0, min(G8 * 16, N - row0));
-    const uint32_t bytes = (uint32_t)(nrows * k_ld * 2);
-    mbar_arrive_expect_tx(&wbar[rnd & 1], bytes);
-    if (bytes > 0) bulk_load(wk + (rnd & 1) * G8 * 16 * k_ld, Pb.w_weak + (size_t)row0 * k_ld, bytes, &wbar[rnd & 1]);
-  };
+
   if (lane == 0) {
     for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
-    if (warp == 0) { mbar_init(xbar, 1); mbar_init(&wbar[0], 1); mbar_init(&wbar[1], 1); }
     fence_mbar_init();
   }
-  __syncthreads();   // every barrier initialised before any thread waits on one
-  int issued = 0;
-  for (; issued < min(S, T); ++issued) issue(issued);
-  if (n_rnd > 0) issue_weak(0);
-  if (n_rnd > 1) issue_weak(1);
-  // the weights do not depend on the previous kernel in the stream: let the next one start
-  // and only now wait for the previous one before touching activations or outputs
+  // the weak-column indices are static: stage them before waiting for the previous kernel
+  for (int t = threadIdx.x; t < k; t += blockDim.x) sidx[t] = Pb.idx[t];
+  __syncthreads();   // barriers initialised and indices staged before any use
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // activations (and outputs) belong to the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- CTA prologue: activations into shared memory (one bulk copy per token row), the
-  //      per-block activation sums, the weak-column gather, then the activations are permuted
-  //      in place into fragment order ----
-  if constexpr (XSMEM) {
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(xbar, (uint32_t)(M * K * 2));
-      for (int m = 0; m < M; ++m) bulk_load(xs + m * xstride, Pb.x + (size_t)m * K, (uint32_t)(K * 2), xbar);
-    }
-    mbar_wait(xbar, 0, args.status, kWaitLimit);
-  }
+  // ---- CTA prologue.  The activation loads go out first, then each warp's first S ring items
+  //      (so the few activation bytes are not queued behind the weight stream).  The
+  //      activations go to shared memory already in fragment order (word 4j + t of a block, for
+  //      lane t, at t*16 + 4((j/4) ^ t) + j%4: 16-byte fragment loads spread over all banks),
+  //      with their per-block sums, prefix sums, and the weak-column activations ----
   {
-    const int pieces = M * Kb * 16;
-    for (int p0 = 0; p0 < pieces; p0 += blockDim.x) {
-      const int p = p0 + threadIdx.x;
-      float v = 0.f;
-      if (p < pieces) {
-        const int m = p / (Kb * 16), rem = p % (Kb * 16);
-        uint4 q;
-        if constexpr (XSMEM) q = *reinterpret_cast<const uint4*>(xs + m * xstride + rem * 4);
-        else q = ldg_u128(Pb.x + (size_t)m * K + (size_t)rem * 8);
-        const uint32_t h[4] = {q.x, q.y, q.z, q.w};
-        #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
-          v += f.x;
-          v += f.y;
+    const int pieces = K / 8;   // 16-byte pieces of one token row; 16 per block
+    const int total = M * pieces;
+    constexpr int kMaxIt = 4;   // pieces per thread kept in flight
+    #pragma unroll 1
+    for (int p0 = 0; p0 < total; p0 += kMaxIt * (int)blockDim.x) {
+      uint4 q[kMaxIt];
+      #pragma unroll
+      for (int it = 0; it < kMaxIt; ++it) {
+        const int p = p0 + it * blockDim.x + threadIdx.x;
+        if (p < total) q[it] = ldg_u128(Pb.x + (size_t)p * 8);
+      }
+      __half gx[2];
+      #pragma unroll
+      for (int it = 0; it < 2; ++it) {   // weak-column gather, in flight with the rows
+        const int e = (p0 / kMaxIt) * 2 + it * blockDim.x + threadIdx.x;
+        gx[it] = __float2half_rn(0.f);
+        if (e < MT * k_ld) {
+          const int m = e / k_ld, t = e - m * k_ld;
+          if (m < M && t < k) gx[it] = Pb.x[(size_t)m * K + sidx[t]];
         }
       }
+      if (p0 == 0 && lane == 0)
+        for (int st = 0; st < S; ++st)
+          if (!issue(st)) break;
       #pragma unroll
-      for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (p < pieces && (p & 15) == 0) sx[p >> 4] = v;
-    }
-  }
-  for (int e = threadIdx.x; e < MT * k_ld; e += blockDim.x) {
-    const int m = e / k_ld, t = e % k_ld;
-    __half v = __float2half_rn(0.f);
-    if (m < M && t < k) {
-      const int col = Pb.idx[t];
-      if constexpr (XSMEM) v = reinterpret_cast<const __half*>(xs + m * xstride)[col];
-      else v = Pb.x[(size_t)m * K + col];
-    }
-    xw[e] = v;
-  }
-  if constexpr (XSMEM) {
-    __syncthreads();   // sums and gather read the natural order
-    for (int e = threadIdx.x; e < M * Kb; e += blockDim.x) {
-      uint32_t* blk = xs + (e / Kb) * xstride + (e % Kb) * 64;
-      uint32_t w[64];
-      #pragma unroll
-      for (int v = 0; v < 16; ++v) {
-        const uint4 q = reinterpret_cast<const uint4*>(blk)[v];
-        w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
+      for (int it = 0; it < 2; ++it) {
+        const int e = (p0 / kMaxIt) * 2 + it * blockDim.x + threadIdx.x;
+        if (e < MT * k_ld) xw[e] = gx[it];
       }
       #pragma unroll
-      for (int t = 0; t < 4; ++t)
+      for (int it = 0; it < kMaxIt; ++it) {
+        const int p = p0 + it * blockDim.x + threadIdx.x;
+        float v = 0.f;
+        int m = 0, pp = 0;
+        if (p < total) {
+          m = p / pieces;
+          pp = p - m * pieces;
+          const uint32_t h[4] = {q[it].x, q[it].y, q[it].z, q[it].w};
+          #pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
+            v += f.x;
+            v += f.y;
+          }
+          if constexpr (XSMEM) {
+            uint32_t* blk = xs + m * xstride + (pp >> 4) * 64;
+            const int j = pp & 15;
+            #pragma unroll
+            for (int t = 0; t < 4; ++t) blk[t * 16 + 4 * ((j >> 2) ^ t) + (j & 3)] = h[t];
+          }
+        }
         #pragma unroll
-        for (int v = 0; v < 4; ++v)   // pairs j = 4v .. 4v+3 of lane t: p = 4j + t
-          *reinterpret_cast<uint4*>(blk + t * 16 + 4 * (v ^ t)) =
-              make_uint4(w[4 * (4 * v) + t], w[4 * (4 * v + 1) + t], w[4 * (4 * v + 2) + t], w[4 * (4 * v + 3) + t]);
+        for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (p < total && (pp & 15) == 0) psx[m * (Kb + 1) + (pp >> 4) + 1] = v;
+      }
+    }
+    // weak-column activations beyond what the loop above covered
+    #pragma unroll 1
+    for (int e = ((total + kMaxIt * (int)blockDim.x - 1) / (kMaxIt * (int)blockDim.x)) * 2 * blockDim.x + threadIdx.x;
+         e < MT * k_ld; e += blockDim.x) {
+      const int m = e / k_ld, t = e - m * k_ld;
+      xw[e] = (m < M && t < k) ? Pb.x[(size_t)m * K + sidx[t]] : __float2half_rn(0.f);
     }
   }
   __syncthreads();
-
-  // activation sums over this warp's block range (per-channel fold), tokens 2tig, 2tig+1 (+8);
-  // tokens >= M only feed outputs that are never stored
-  float sxw[NT][2];
-  #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  if (warp < MT) {   // prefix sums of the block sums, one warp per token (tokens >= M: zeros)
+    float* row = psx + warp * (Kb + 1);
+    const int per = (Kb + 31) / 32, b_lo = lane * per, b_hi = min(b_lo + per, Kb);
+    float run = 0.f;
+    for (int b = b_lo; b < b_hi; ++b) run += warp < M ? row[b + 1] : 0.f;
+    float incl = run;
     #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int tok = min(8 * nt + 2 * tig + e, M - 1);
-      float v = 0.f;
-      for (int b = b_lo; b < b_hi; ++b) v += sx[tok * Kb + b];
-      sxw[nt][e] = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const float t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
+    float acc = incl - run;
+    __syncwarp();
+    for (int b = b_lo; b < b_hi; ++b) {
+      acc += warp < M ? row[b + 1] : 0.f;
+      row[b + 1] = acc;
+    }
+    if (lane == 0) row[0] = 0.f;
+  }
+  __syncthreads();
+  if (lo >= hi) return;   // no work for this warp (no barrier follows)
+
   // per-lane operand pointers (tokens >= M are clamped: their columns are discarded)
-  const uint32_t* xr[NT];
+  const uint32_t* xv[NT][4];
   const __half* xg[NT];
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int tok = min(8 * nt + g, M - 1);
-    xr[nt] = xs + tok * xstride + tig * 16;
+    #pragma unroll
+    for (int v = 0; v < 4; ++v) xv[nt][v] = xs + tok * xstride + tig * 16 + 4 * (v ^ tig);
     xg[nt] = Pb.x + (size_t)tok * K + 2 * tig;
   }
-  int xo[4];
+  const unsigned char* fa0 = ring + g * G_::kBlk + tig * 4 * BITS;   // this lane's chunk in stage 0
+
+  float D[NC][NT][4], Dw[NT][4], y[NT][4];
+  zero_acc<BITS, NT>(D);
   #pragma unroll
-  for (int v = 0; v < 4; ++v) xo[v] = 4 * (v ^ tig);
-  const int frag_lane = g * G_::kBlk + tig * 4 * BITS;
-
-  float y[NT][4];
-  int it = 0, fail_it = -1;
+  for (int nt = 0; nt < NT; ++nt)
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) { Dw[nt][i] = 0.f; y[nt][i] = 0.f; }
+  int seg_b0 = b0;                 // first block of the current tile segment
+  int st = 0;                      // stage being consumed
+  uint32_t phase = 0;              // its barrier phase
+  int consumed = 0;
   bool ok = true;
+  int kind, rt, first, cnt;
   #pragma unroll 1
-  for (int rnd = 0; rnd < n_rnd; ++rnd) {
-    const int rt = (c + rnd * Pb.ncta) * G8 + gw;
-    const bool live = rt < RT;
-    const int row_a = min(rt * 16 + g, N - 1), row_b = min(rt * 16 + g + 8, N - 1);
-    float sa = 0.f, za = 0.f, sb = 0.f, zb = 0.f;    // per-channel scale / zero, used at the end
-    if (!per_group && live) {
-      sa = __half2float(Pb.scales[row_a]); za = __half2float(Pb.zeros[row_a]);
-      sb = __half2float(Pb.scales[row_b]); zb = __half2float(Pb.zeros[row_b]);
-    }
-    float D[UNR][NC][NT][4];
-    #pragma unroll
-    for (int u = 0; u < UNR; ++u) zero_acc<BITS, NT>(D[u]);
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      #pragma unroll
-      for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
-
-    // per-group fold of one block's accumulators
-    auto fold = [&](float (&Du)[NC][NT][4], int b) {
-      const float gsa = __half2float(Pb.scales[(size_t)row_a * Gn + b]);
-      const float gza = __half2float(Pb.zeros[(size_t)row_a * Gn + b]);
-      const float gsb = __half2float(Pb.scales[(size_t)row_b * Gn + b]);
-      const float gzb = __half2float(Pb.zeros[(size_t)row_b * Gn + b]);
-      #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+  while (cons.next(kind, rt, first, cnt)) {
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], phase, args.status, kWaitLimit));
+    const unsigned char* fa = fa0 + st * G_::kStage;
+    if (ok && kind == 0) {
+      // weak k slices: A = the fp16 weak rows (tile-major slice: [16 rows][16]), B = gathered x
+      #pragma unroll 1
+      for (int i = 0; i < cnt; ++i) {
+        const uint32_t* ws = reinterpret_cast<const uint32_t*>(ring + st * G_::kStage + i * 512);
+        const uint32_t a[4] = {ws[g * 8 + tig], ws[(g + 8) * 8 + tig], ws[g * 8 + 4 + tig], ws[(g + 8) * 8 + 4 + tig]};
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tok = min(8 * nt + 2 * tig + (i & 1), M - 1);
-          const float v = combine<BITS>(Du[0][nt][i], Du[1][nt][i], Du[NC - 1][nt][i]);
-          const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
-          y[nt][i] = fmaf(sc, fmaf(-z, sx[tok * Kb + b], v), y[nt][i]);
+        for (int nt = 0; nt < NT; ++nt) {
+          const __half* xr2 = xw + (8 * nt + g) * k_ld + 16 * (first + i) + 2 * tig;
+          mma16816(Dw[nt], a, *reinterpret_cast<const uint32_t*>(xr2), *reinterpret_cast<const uint32_t*>(xr2 + 8));
         }
-    };
-
-    #pragma unroll 1
-    for (int sub = 0; sub < n_sub; ++sub, ++it) {
-      const int st = it % S;
-      if (ok) {
-        const bool ok_lane = mbar_wait(&bars[st], (uint32_t)((it / S) & 1), args.status, kWaitLimit);
-        ok = __all_sync(0xffffffffu, ok_lane);
-        if (!ok) fail_it = it;
       }
-      const int b0 = b_lo + sub * G_::kSub;
-      const int nbs = (ok && live) ? max(0, min(G_::kSub, b_hi - b0)) : 0;
-      const unsigned char* frag = ring + st * G_::kStage + frag_lane;
-      if (nbs == G_::kSub) {
-        // full item: all kSub blocks unrolled, UNR independent accumulator sets
+    } else if (ok) {
+      auto fold_block = [&](int b) {   // per-group layers: one scale / zero per block
+        const int ra = min(rt * 16 + g, N - 1), rb = min(rt * 16 + g + 8, N - 1);
+        const float gsa = __half2float(Pb.scales[(size_t)ra * Kb + b]);
+        const float gza = __half2float(Pb.zeros[(size_t)ra * Kb + b]);
+        const float gsb = __half2float(Pb.scales[(size_t)rb * Kb + b]);
+        const float gzb = __half2float(Pb.zeros[(size_t)rb * Kb + b]);
         #pragma unroll
-        for (int bb = 0; bb < G_::kSub; ++bb) {
-          if (per_group) zero_acc<BITS, NT>(D[bb % UNR]);
-          block_mma<BITS, NT, XSMEM>(frag + bb * G_::kTileBlk, xr, xo, xg, b0 + bb, D[bb % UNR]);
-          if (per_group) fold(D[bb % UNR], b0 + bb);
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tok = 8 * nt + 2 * tig + (i & 1);
+            const float sxv = psx[tok * (Kb + 1) + b + 1] - psx[tok * (Kb + 1) + b];
+            const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
+            const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
+            y[nt][i] = fmaf(sc, fmaf(-z, sxv, v), y[nt][i]);
+          }
+        zero_acc<BITS, NT>(D);
+      };
+      const int xoff = first * 64;
+      if (cnt == kSub) {
+        #pragma unroll
+        for (int bb = 0; bb < kSub; ++bb) {
+          unit_mma<BITS, NT, XSMEM>(fa + bb * G_::kTileBlk, xv, xoff + bb * 64, xg, first + bb, D);
+          if constexpr (PG) fold_block(first + bb);
         }
       } else {
         #pragma unroll 1
-        for (int bb = 0; bb < nbs; ++bb) {
-          if (per_group) zero_acc<BITS, NT>(D[0]);
-          block_mma<BITS, NT, XSMEM>(frag + bb * G_::kTileBlk, xr, xo, xg, b0 + bb, D[0]);
-          if (per_group) fold(D[0], b0 + bb);
+        for (int bb = 0; bb < cnt; ++bb) {
+          unit_mma<BITS, NT, XSMEM>(fa + bb * G_::kTileBlk, xv, xoff + bb * 64, xg, first + bb, D);
+          if constexpr (PG) fold_block(first + bb);
         }
       }
-      __syncwarp();
-      if (ok && it + S < T) {
-        if (lane == 0) fence_proxy_async_smem();
-        issue(it + S);
-        ++issued;
-      }
     }
+    __syncwarp();
+    if (lane == 0 && ok) {   // refill the stage just consumed
+      fence_proxy_async_smem();
+      issue(st);
+    }
+    ++consumed;
+    if (++st == S) { st = 0; phase ^= 1u; }
 
-    // ---- this warp's part of the row tile is done: fold, weak columns, reduction ----
-    if (!per_group) {
+    // end of a tile segment: fold, then store (whole tile) or hand over (split tile)
+    if (kind == 1 && cons.segment_done()) {
+      const int seg_b1 = first + cnt;
+      const int ra = min(rt * 16 + g, N - 1), rb = min(rt * 16 + g + 8, N - 1);
+      if constexpr (!PG) {
+        const float sa = __half2float(Pb.scales[ra]), za = __half2float(Pb.zeros[ra]);
+        const float sb = __half2float(Pb.scales[rb]), zb = __half2float(Pb.zeros[rb]);
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tok = 8 * nt + 2 * tig + (i & 1);
+            const float sxv = psx[tok * (Kb + 1) + seg_b1] - psx[tok * (Kb + 1) + seg_b0];
+            const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
+            const float sc = i < 2 ? sa : sb, z = i < 2 ? za : zb;
+            y[nt][i] = sc * fmaf(-z, sxv, v);
+          }
+        zero_acc<BITS, NT>(D);
+      }
       #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float v = combine<BITS>(D[0][0][nt][i], D[0][1][nt][i], D[0][NC - 1][nt][i]);
-          if constexpr (UNR == 2) v += combine<BITS>(D[1][0][nt][i], D[1][1][nt][i], D[1][NC - 1][nt][i]);
-          const float sc = i < 2 ? sa : sb, z = i < 2 ? za : zb;
-          y[nt][i] = sc * fmaf(-z, sxw[nt][i & 1], v);
-        }
-    }
-    if (k > 0) {
-      const bool ok_w = mbar_wait(&wbar[rnd & 1], (uint32_t)((rnd >> 1) & 1), args.status, kWaitLimit);
-      if (live && ok_w) {
-        const __half* wr = wk + (size_t)((rnd & 1) * G8 * 16 + gw * 16 + g) * k_ld + 2 * tig;
-        #pragma unroll 1
-        for (int ws = pw; ws * 16 < k; ws += P) {
-          const uint32_t a[4] = {*reinterpret_cast<const uint32_t*>(wr + 16 * ws),
-                                 *reinterpret_cast<const uint32_t*>(wr + 8 * k_ld + 16 * ws),
-                                 *reinterpret_cast<const uint32_t*>(wr + 16 * ws + 8),
-                                 *reinterpret_cast<const uint32_t*>(wr + 8 * k_ld + 16 * ws + 8)};
+        for (int i = 0; i < 4; ++i) { y[nt][i] += Dw[nt][i]; Dw[nt][i] = 0.f; }
+
+      const int t0 = rt * Kb;
+      const int c_first = t0 / c, nseg = (t0 + Kb - 1) / c - c_first + 1;
+      bool write = ok;
+      if (nseg > 1) {
+        // split tile: publish this segment's partial; the last arrival finishes the tile
+        const int sid = (t0 + seg_b0) / c - c_first;
+        float* part = Pb.part + ((size_t)rt * Pb.seg_cap + sid) * 16 * 16;
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const __half* xr = xw + (8 * nt + g) * k_ld + 16 * ws + 2 * tig;
-            mma16816(y[nt], a, *reinterpret_cast<const uint32_t*>(xr), *reinterpret_cast<const uint32_t*>(xr + 8));
-          }
+          for (int i = 0; i < 4; ++i)
+            part[(g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = arrive_acq_rel(&Pb.cnt[rt]);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        const bool last = prev == nseg - 1;
+        if (last && lane == 0) Pb.cnt[rt] = 0;   // the tile's counter is ready for the next call
+        write = ok && last;
+        if (write) {
+          const float* pt = Pb.part + (size_t)rt * Pb.seg_cap * 16 * 16;
+          #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int off = (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1);
+              float v = 0.f;
+              for (int s2 = 0; s2 < nseg; ++s2) v += __ldcg(pt + s2 * 16 * 16 + off);
+              y[nt][i] = v;
+            }
         }
       }
-    }
-    float* rbuf = red + (size_t)(rnd & 1) * kWarps * 16 * MT + (size_t)warp * 16 * MT;
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      if (write) {
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
+            if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(y[nt][i]);
+          }
+      }
       #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        rbuf[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
-    __syncthreads();
-    // the weak buffer of this round is free again: fetch the round after next into it
-    if (rnd + 2 < n_rnd) {
-      if (threadIdx.x == 0) fence_proxy_async_smem();
-      issue_weak(rnd + 2);
-    }
-    // reduce: thread -> (row tile of the round, row, token), sum over the P warps of that tile
-    for (int e = threadIdx.x; e < G8 * 16 * MT; e += blockDim.x) {
-      const int tg = e / (16 * MT), r = (e / MT) % 16, tok = e % MT;
-      const int rtile = (c + rnd * Pb.ncta) * G8 + tg;
-      const float* rs = red + (size_t)(rnd & 1) * kWarps * 16 * MT + (size_t)(tg * P) * 16 * MT + r * MT + tok;
-      float v = 0.f;
-      #pragma unroll
-      for (int w = 0; w < P; ++w) v += rs[w * 16 * MT];
-      const int row = rtile * 16 + r;
-      if (ok && rtile < RT && row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(v);
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
+      seg_b0 = 0;
     }
   }
   // after a timeout: never exit with bulk copies still writing into this CTA's memory
-  if (fail_it >= 0 && lane == 0)
-    for (int j = fail_it; j < issued; ++j)
+  if (!ok && lane == 0)
+    for (int j = consumed; j < issued; ++j)
       mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1), args.status, kWaitLimit);
 }
 
@@ -465,9 +509,9 @@ int sm_count() {
   return n;
 }
 
-template <int BITS, int NT, int S, int P, bool XSMEM>
+template <int BITS, int NT, int S, bool XSMEM>
 cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
-  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, S, P, XSMEM, true> : k_gemv_mma<BITS, NT, S, P, XSMEM, false>;
+  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, S, XSMEM, true> : k_gemv_mma<BITS, NT, S, XSMEM, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int base = 0;
@@ -487,10 +531,9 @@ cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int BITS, int NT, int P>
-cudaError_t launch_p(GemvArgs& a, cudaStream_t s) {
+template <int BITS, int NT>
+cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
   constexpr int MT = 8 * NT;
-  constexpr int G8 = kWarps / P;
   constexpr size_t kMaxSmem = 232448;
   const int C = sm_count();
   long long work[kMaxProblems], total = 0;
@@ -498,19 +541,21 @@ cudaError_t launch_p(GemvArgs& a, cudaStream_t s) {
   for (int q = 0; q < a.count; ++q) {
     GemvProblem& Pq = a.p[q];
     const int Kb = Pq.K / kBlockCodes;
-    Pq.row_groups = ((Pq.N + 15) / 16 + G8 - 1) / G8;        // CTA rounds of work
+    Pq.row_groups = (Pq.N + 15) / 16;
     work[q] = (long long)Pq.row_groups * Kb;
     total += work[q];
-    const size_t need = (size_t)((MT * Kb + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half) +
-                        (size_t)2 * G8 * 16 * Pq.k_ld * sizeof(__half);
+    const size_t need = (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half) +
+                        (size_t)Pq.k_ld * sizeof(int32_t);
     if (need > extra) extra = need;
     const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
     if (xb > xbytes) xbytes = xb;
   }
-  // CTAs per problem in proportion to its work, at least one each, one resident wave in total
+  // CTAs per problem in proportion to its work (one resident wave in total), then an equal
+  // chunk of (tile, block) units per warp: at least kGemvMinChunk, and large enough that a
+  // row tile meets at most seg_cap warps (the size of the layer's partial-sum workspace)
   int n[kMaxProblems], used = 0, big = 0;
   for (int q = 0; q < a.count; ++q) {
-    n[q] = max(1, min(a.p[q].row_groups, (int)(work[q] * C / total)));
+    n[q] = max(1, (int)(work[q] * C / total));
     used += n[q];
     if (work[q] > work[big]) big = q;
   }
@@ -521,39 +566,30 @@ cudaError_t launch_p(GemvArgs& a, cudaStream_t s) {
     --n[q];
     --used;
   }
-  if (used < C) {
-    const int add = min(C - used, a.p[big].row_groups - n[big]);
-    if (add > 0) { n[big] += add; used += add; }
-  }
+  if (used < C) { n[big] += C - used; used = C; }
   int base = 0;
   for (int q = 0; q < a.count; ++q) {
-    a.p[q].cta_base = base;
-    a.p[q].ncta = n[q];
-    base += n[q];
+    GemvProblem& Pq = a.p[q];
+    const int Kb = Pq.K / kBlockCodes;
+    const long long warps = (long long)n[q] * kWarps;
+    int chunk = (int)((work[q] + warps - 1) / warps);
+    chunk = max(chunk, max(kGemvMinChunk, (Kb - 1) / (Pq.seg_cap - 1) + 1));
+    const int nchunks = (int)((work[q] + chunk - 1) / chunk);
+    Pq.chunk = chunk;
+    Pq.ncta = min(n[q], (nchunks + kWarps - 1) / kWarps);
+    Pq.cta_base = base;
+    base += Pq.ncta;
   }
-  // shared memory: ring + barriers + reduction + sums / gather / weak rows (+ staged activations)
   auto smem_for = [&](int S, bool xs) {
-    const size_t ring = (size_t)kWarps * S * Geo<BITS, 1>::kStage;
-    return ring + (size_t)kWarps * S * 8 + 32 + (size_t)2 * kWarps * 16 * MT * sizeof(float) +
+    return (size_t)kWarps * S * Geo<BITS>::kStage + (size_t)kWarps * S * 8 + 16 +
            ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
   };
-  if (smem_for(3, true) <= kMaxSmem) return launch_k<BITS, NT, 3, P, true>(a, smem_for(3, true), s);
-  if (smem_for(2, true) <= kMaxSmem) return launch_k<BITS, NT, 2, P, true>(a, smem_for(2, true), s);
-  if (smem_for(3, false) <= kMaxSmem) return launch_k<BITS, NT, 3, P, false>(a, smem_for(3, false), s);
-  if (smem_for(2, false) <= kMaxSmem) return launch_k<BITS, NT, 2, P, false>(a, smem_for(2, false), s);
+  if (smem_for(4, true) <= kMaxSmem) return launch_k<BITS, NT, 4, true>(a, smem_for(4, true), s);
+  if (smem_for(3, true) <= kMaxSmem) return launch_k<BITS, NT, 3, true>(a, smem_for(3, true), s);
+  if (smem_for(2, true) <= kMaxSmem) return launch_k<BITS, NT, 2, true>(a, smem_for(2, true), s);
+  if (smem_for(3, false) <= kMaxSmem) return launch_k<BITS, NT, 3, false>(a, smem_for(3, false), s);
+  if (smem_for(2, false) <= kMaxSmem) return launch_k<BITS, NT, 2, false>(a, smem_for(2, false), s);
   return cudaErrorInvalidValue;
-}
-
-template <int BITS, int NT>
-cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
-  // warps per 16-row tile: as few as possible (more K per warp) while the rounds still cover
-  // every SM once
-  int rt_total = 0;
-  for (int q = 0; q < a.count; ++q) rt_total += (a.p[q].N + 15) / 16;
-  const int C = sm_count();
-  if (rt_total >= 4 * C) return launch_p<BITS, NT, 4>(a, s);
-  if (rt_total >= 2 * C) return launch_p<BITS, NT, 8>(a, s);
-  return launch_p<BITS, NT, 16>(a, s);
 }
 
 template <int BITS>

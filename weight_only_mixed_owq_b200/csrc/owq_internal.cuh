@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <algorithm>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda.h>
@@ -29,6 +30,10 @@ struct Layer {
   int32_t* blk_weak;    // K/128 + 1 offsets into idx: weak columns of packed block b are
                         // idx[blk_weak[b] .. blk_weak[b+1])
   int32_t* idx_host;    // k (host copy)
+  __half* w_weak_t;     // the weak block tile-major: [N/16 tiles][k_ld/16 slices][16 rows][16]
+  float* part;          // decode workspace: partial sums [N/16 tiles][seg_cap][16 rows][16 tokens]
+  int* cnt;             // decode workspace: per-tile arrival counters (kept at 0 between calls)
+  int seg_cap;          // most warps that may share one row tile in the decode product
   cudaStream_t stream;  // stream of owq_pack (used to order the release)
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
@@ -45,6 +50,7 @@ int* device_status_ptr();
 cudaError_t launch_pack(const uint8_t* codes, const __half* zeros, const uint32_t* weak_mask,
                         int N, int K, int bits, int group, uint32_t* packed, cudaStream_t s);
 cudaError_t launch_dequant(const Layer& L, __half* w_hat, uint8_t* codes, cudaStream_t s);
+cudaError_t launch_weak_tiles(const __half* w_weak, int N, int k_ld, __half* w_weak_t, cudaStream_t s);
 
 struct GemvProblem {
   const uint32_t* packed;
@@ -55,11 +61,26 @@ struct GemvProblem {
   const __half* x;
   __half* y;
   int N, K, G, k, k_ld;
-  int row_groups;     // ceil(N / rows_per_group)
-  int group_base;     // first global row-group index of this problem (register-pipelined kernel)
-  int cta_base;       // first CTA of this problem (bulk-copy kernel)
-  int ncta;           // CTAs serving this problem (bulk-copy kernel)
+  const __half* w_weak_t;   // tile-major weak block
+  float* part;              // partial-sum workspace of split row tiles
+  int* cnt;                 // arrival counters of split row tiles
+  int seg_cap;              // partial-sum slots per row tile
+  int row_groups;     // 16-row tiles
+  int cta_base;       // first CTA of this problem
+  int ncta;           // CTAs serving this problem
+  int chunk;          // (row tile, block) units per warp
 };
+// Decode work split: each warp of the grid (kGemvWarps per SM) takes an equal contiguous chunk
+// of the (16-row tile, 128-code block) units, never fewer than kGemvMinChunk.  A row tile is
+// then shared by at most gemv_seg_cap warps, which sizes the layer's partial-sum workspace.
+constexpr int kGemvWarps = 16;
+constexpr int kGemvMinChunk = 8;
+inline int gemv_seg_cap(int N, int K, int sm_count) {
+  const long long units = (long long)((N + 15) / 16) * (K / kBlockCodes);
+  const long long warps = (long long)sm_count * kGemvWarps;
+  const int cmin = (int)std::max<long long>(kGemvMinChunk, (units + warps - 1) / warps);
+  return (K / kBlockCodes - 1) / cmin + 2;
+}
 cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cudaStream_t s);
 
 cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int T, int bits,

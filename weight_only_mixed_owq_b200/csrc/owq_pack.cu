@@ -101,7 +101,25 @@ __global__ void k_dequant(const uint32_t* __restrict__ packed, const __half* __r
   }
 }
 
+// Tile-major copy of the weak block for the decode kernel: element (row, t) of the row-major
+// [N][k_ld] block goes to [row / 16][t / 16][row % 16][t % 16] (rows past N are zero).
+__global__ void k_weak_tiles(const __half* __restrict__ w, int N, int k_ld, __half* __restrict__ wt) {
+  const size_t RT = (size_t)(N + 15) / 16;
+  size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= RT * 16 * k_ld) return;
+  const int col = (int)(e % 16), r = (int)((e / 16) % 16);
+  const size_t sl = (e / 256) % (size_t)(k_ld / 16), tile = e / ((size_t)256 * (k_ld / 16));
+  const size_t row = tile * 16 + r;
+  wt[e] = row < (size_t)N ? w[row * k_ld + sl * 16 + col] : __float2half_rn(0.f);
+}
+
 }  // namespace
+
+cudaError_t launch_weak_tiles(const __half* w_weak, int N, int k_ld, __half* w_weak_t, cudaStream_t s) {
+  const size_t n = (size_t)((N + 15) / 16) * 16 * k_ld;
+  k_weak_tiles<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w_weak, N, k_ld, w_weak_t);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const uint8_t* codes, const __half* zeros, const uint32_t* weak_mask,
                         int N, int K, int bits, int group, uint32_t* packed, cudaStream_t s) {
