@@ -215,11 +215,11 @@ def owq_quantize(W: np.ndarray, X: np.ndarray, bits: int, group: int, k: int) ->
 # bits 16 + o.. of word w.
 #   bits = 4: w = 2 (j // 8) + (j % 2), o = 4 ((j % 8) // 2).
 #   bits = 3: slots of j = 0..15: (0,0) (1,0) (0,3) (1,3) (0,6) (1,6) (0,9) (1,9) (0,12) (1,12)
-#             (2,0) D (2,3) (2,12) (2,6) (2,9); slot D (j = 11) spreads its codes over the
+#             (2,6) D (2,3) (2,12) (2,0) (2,9); slot D (j = 11) spreads its codes over the
 #             chunk: bit e of the even code is bit 15 of word e, bit e of the odd code is bit 31
 #             of word e (e = 0, 1, 2).
 SLOT3 = [(0, 0), (1, 0), (0, 3), (1, 3), (0, 6), (1, 6), (0, 9), (1, 9), (0, 12), (1, 12),
-         (2, 0), None, (2, 3), (2, 12), (2, 6), (2, 9)]
+         (2, 6), None, (2, 3), (2, 12), (2, 0), (2, 9)]
 SLOT4 = [(2 * (j // 8) + (j % 2), 4 * ((j % 8) // 2)) for j in range(16)]
 
 

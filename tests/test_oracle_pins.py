@@ -45,8 +45,11 @@ def test_pack_hand_derived_words(golden_dir):
     for bits, rule, words in _read_rows(os.path.join(golden_dir, "pack_words.txt")):
         bits = int(bits)
         k = np.arange(128)
-        mod = int(rule.split()[-1])
-        codes = ((k // 8 if "//" in rule else k) % mod).astype(np.uint8)[None, :]
+        if rule.startswith("pair"):   # pair p = (p mod 8, p // 8)
+            codes = np.where(k % 2 == 0, (k // 2) % 8, (k // 16) % 8).astype(np.uint8)[None, :]
+        else:
+            mod = int(rule.split()[-1])
+            codes = ((k // 8 if "//" in rule else k) % mod).astype(np.uint8)[None, :]
         got = oracle.pack(codes, bits)[0]
         assert [f"{int(v):08x}" for v in got] == words.split()
         assert oracle.unpack(got[None, :], 128, bits).tolist() == codes.tolist()

@@ -8,8 +8,8 @@
 // Pair j of a chunk sits at a slot (word, offset): even code at the offset, odd code 16 bits
 // higher in the same word.
 //   4-bit: word 2(j/8) + j%2, offset 4((j%8)/2).
-//   3-bit: (0,0) (1,0) (0,3) (1,3) (0,6) (1,6) (0,9) (1,9) (0,12) (1,12) (2,0) D (2,3) (2,12)
-//          (2,6) (2,9); slot D (j = 11): bit e of the even / odd code is bit 15 / 31 of word e.
+//   3-bit: (0,0) (1,0) (0,3) (1,3) (0,6) (1,6) (0,9) (1,9) (0,12) (1,12) (2,6) D (2,3) (2,12)
+//          (2,0) (2,9); slot D (j = 11): bit e of the even / odd code is bit 15 / 31 of word e.
 //
 // Why this layout.  The m16n8k16 tensor-core fragment gives lane (g, t) of a warp the k-pairs
 // t and t+4 of every 16-wide k slice, i.e. the block pairs p = 4j + t: one chunk per lane.
@@ -17,7 +17,10 @@
 // (after at most one shift), so one AND per pair lifts them into an fp16x2 register whose
 // halves equal code * 2^(o - 24) exactly (the code bits lie in the low 11 bits of each half,
 // where fp16 is linear in its bit pattern), and both registers of the slice share the scale
-// 2^(o - 24).  The prefill kernel reads the same pairs and forms fp16_rn(s (q - z)) from them.
+// 2^(o - 24).  With the 3-bit slots above, one right shift by 9 per word serves every pair
+// that is not at offset 0, 3 or 6 (offsets 9 and 12 become 0 and 3), and the spread pair D is
+// rebuilt at offset 6 from the same shifted words (bit 15 lands on bit 6).  The prefill kernel
+// reads the same pairs and forms fp16_rn(s (q - z)) from them.
 #pragma once
 #include <cstdint>
 
@@ -28,7 +31,7 @@ struct Slot { int word, off; };
 
 __host__ __device__ constexpr Slot slot3(int j) {
   constexpr int w[16] = {0, 1, 0, 1, 0, 1, 0, 1, 0, 1, 2, -1, 2, 2, 2, 2};
-  constexpr int o[16] = {0, 0, 3, 3, 6, 6, 9, 9, 12, 12, 0, -1, 3, 12, 6, 9};
+  constexpr int o[16] = {0, 0, 3, 3, 6, 6, 9, 9, 12, 12, 6, -1, 3, 12, 0, 9};
   return Slot{w[j], o[j]};
 }
 __host__ __device__ constexpr Slot slot4(int j) { return Slot{2 * (j / 8) + (j % 2), 4 * ((j % 8) / 2)}; }
@@ -79,12 +82,15 @@ __host__ __device__ __forceinline__ void decode_block(const uint32_t* w, uint32_
 }
 
 // ---- register extraction of pair j of a chunk (tensor-core and prefill kernels) ----
-// Returns the pair with both codes at bit offset pair_off<BITS>(j) of each 16-bit half and
-// every other bit clear.  All arguments are compile-time after unrolling.
+// Returns the pair with both codes at bit offset class_off(pair_class(j)) of each 16-bit half
+// and every other bit clear.  j is compile-time after unrolling.  The two pairs of one k slice
+// (j = 2s, 2s + 1) share a class.  k2 and k4 are 2 and 4: passed in at run time, they keep the
+// rebuild of pair D on the multiply-add pipe (as integer multiply-adds) instead of the integer
+// logic pipe that the other extractions load.
 template <int BITS>
 __host__ __device__ constexpr int pair_class(int j) {
   if (BITS == 3) {
-    constexpr int c[16] = {0, 0, 1, 1, 2, 2, 0, 0, 1, 1, 0, 0, 1, 1, 2, 2};
+    constexpr int c[16] = {0, 0, 1, 1, 2, 2, 0, 0, 1, 1, 2, 2, 1, 1, 0, 0};
     return c[j];
   } else {
     return (j / 2) % 2;   // offsets 0, 4, 0 (after >> 8), 4 (after >> 8)
@@ -94,9 +100,9 @@ template <int BITS>
 __host__ __device__ constexpr int class_off(int cls) { return BITS == 3 ? 3 * cls : 4 * cls; }
 
 template <int BITS>
-__device__ __forceinline__ uint32_t pair_bits(const uint32_t* w, int j) {
+__device__ __forceinline__ uint32_t pair_bits(const uint32_t* w, int j, uint32_t k2 = 2u, uint32_t k4 = 4u) {
   if constexpr (BITS == 3) {
-    constexpr uint32_t m0 = 0x00070007u, m1 = 0x00380038u, m2 = 0x01C001C0u;
+    constexpr uint32_t m0 = 0x00070007u, m1 = 0x00380038u, m2 = 0x01C001C0u, mD = 0x00400040u;
     switch (j) {
       case 0: return w[0] & m0;
       case 1: return w[1] & m0;
@@ -108,14 +114,16 @@ __device__ __forceinline__ uint32_t pair_bits(const uint32_t* w, int j) {
       case 7: return (w[1] >> 9) & m0;
       case 8: return (w[0] >> 9) & m1;
       case 9: return (w[1] >> 9) & m1;
-      case 10: return w[2] & m0;
-      case 11: return ((w[0] >> 15) & 0x00010001u) | ((w[1] >> 14) & 0x00020002u) | ((w[2] >> 13) & 0x00040004u);
+      case 10: return w[2] & m2;
+      case 11: return ((w[0] >> 9) & mD) + ((w[1] >> 9) & mD) * k2 + ((w[2] >> 9) & mD) * k4;
       case 12: return w[2] & m1;
       case 13: return (w[2] >> 9) & m1;
-      case 14: return w[2] & m2;
-      default: return (w[2] >> 3) & m2;
+      case 14: return w[2] & m0;
+      default: return (w[2] >> 9) & m0;
     }
   } else {
+    (void)k2;
+    (void)k4;
     const uint32_t v = w[2 * (j / 8) + (j % 2)];
     switch ((j % 8) / 2) {
       case 0: return v & 0x000F000Fu;

@@ -38,22 +38,26 @@ using namespace sm100;
 
 constexpr int kMaxProblems = 16;
 constexpr int kWarps = kGemvWarps;
-constexpr int kSub = 4;                          // blocks per ring item
+constexpr int kAhead = 2;                        // items in flight per warp (see GemvArgs::ahead)
 constexpr long long kWaitLimit = 4000000000LL;  // ~2 s
 
 struct GemvArgs {
   GemvProblem p[kMaxProblems];
   int count;
   int M;
+  int ahead;     // ring items a warp keeps in flight beyond the one it is reading (1 .. S)
+  uint32_t k2, k4;   // 2 and 4 (run-time values: see pair_bits)
   int* status;   // device status word (bounded waits)
 };
 
-template <int BITS>
+template <int BITS, int SUB>   // SUB: blocks per ring item
 struct Geo {
   static constexpr int kBlk = 16 * BITS;                       // bytes of one block of one row
   static constexpr int kTileBlk = 16 * kBlk;                   // one block of a 16-row tile
-  static constexpr int kStage = kSub * kTileBlk;               // 3 KB (3-bit) / 4 KB (4-bit)
-  static constexpr int kWs = kStage / 512;                     // weak k slices per item
+  static constexpr int kStageW = SUB * kTileBlk;               // weights of an item
+  static constexpr int kWs = kStageW / 512;                    // weak k slices per item
+  // a stage: the item's weights, then (per-group layers) its (scale, zero) pairs, 16 per block
+  static constexpr int stage_bytes(bool pg) { return kStageW + (pg ? SUB * 64 : 0); }
 };
 
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
@@ -93,25 +97,27 @@ __device__ __forceinline__ void zero_acc(float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
 }
 
 // One unit (one 128-code block of a 16-row tile) of one warp: A fragments of rows g, g+8
-// from the staged tile (fa: this lane's chunk), B fragments from the staged activations (xv:
-// this lane's four 16-byte fragment pieces of block 0, xoff: the block's word offset) or from
-// global memory (xg, block b), then 8 k slices of m16n8k16 into the offset-class accumulators.
+// from the staged tile (byte offset fa in shared memory: this lane's chunk), B fragments from
+// the staged activations (byte offsets xv: this lane's four 16-byte fragment pieces of block 0,
+// plus xoff for the block) or from global memory (xg, block b), then 8 k slices of m16n8k16
+// into the offset-class accumulators.  Shared memory is addressed as the kernel's shared array
+// plus 32-bit offsets, so each load is one shared load at register + immediate.
 template <int BITS, int NT, bool XSMEM>
-__device__ __forceinline__ void unit_mma(const unsigned char* fa, const uint32_t* const (&xv)[NT][4], int xoff,
-                                         const __half* const (&xg)[NT], int b,
+__device__ __forceinline__ void unit_mma(const unsigned char* sm, int fa, const int (&xv)[NT][4], int xoff,
+                                         const __half* const (&xg)[NT], int b, uint32_t k2, uint32_t k4,
                                          float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
   constexpr int kBlk = 16 * BITS;
   uint32_t wa[BITS], wb[BITS];
   if constexpr (BITS == 4) {
-    const uint4 qa = *reinterpret_cast<const uint4*>(fa);
-    const uint4 qb = *reinterpret_cast<const uint4*>(fa + 8 * kBlk);
+    const uint4 qa = *reinterpret_cast<const uint4*>(sm + fa);
+    const uint4 qb = *reinterpret_cast<const uint4*>(sm + fa + 8 * kBlk);
     wa[0] = qa.x; wa[1] = qa.y; wa[2] = qa.z; wa[3] = qa.w;
     wb[0] = qb.x; wb[1] = qb.y; wb[2] = qb.z; wb[3] = qb.w;
   } else {
     #pragma unroll
     for (int j = 0; j < BITS; ++j) {
-      wa[j] = reinterpret_cast<const uint32_t*>(fa)[j];
-      wb[j] = reinterpret_cast<const uint32_t*>(fa + 8 * kBlk)[j];
+      wa[j] = *reinterpret_cast<const uint32_t*>(sm + fa + 4 * j);
+      wb[j] = *reinterpret_cast<const uint32_t*>(sm + fa + 8 * kBlk + 4 * j);
     }
   }
   uint32_t xb[NT][16];
@@ -120,7 +126,7 @@ __device__ __forceinline__ void unit_mma(const unsigned char* fa, const uint32_t
     if constexpr (XSMEM) {
       #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const uint4 q = *reinterpret_cast<const uint4*>(xv[nt][v] + xoff);
+        const uint4 q = *reinterpret_cast<const uint4*>(sm + xv[nt][v] + xoff);
         xb[nt][4 * v] = q.x; xb[nt][4 * v + 1] = q.y; xb[nt][4 * v + 2] = q.z; xb[nt][4 * v + 3] = q.w;
       }
     } else {
@@ -132,8 +138,8 @@ __device__ __forceinline__ void unit_mma(const unsigned char* fa, const uint32_t
   #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int cl = pair_class<BITS>(2 * s);
-    const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s), pair_bits<BITS>(wb, 2 * s),
-                           pair_bits<BITS>(wa, 2 * s + 1), pair_bits<BITS>(wb, 2 * s + 1)};
+    const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s, k2, k4), pair_bits<BITS>(wb, 2 * s, k2, k4),
+                           pair_bits<BITS>(wa, 2 * s + 1, k2, k4), pair_bits<BITS>(wb, 2 * s + 1, k2, k4)};
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
   }
@@ -150,12 +156,12 @@ __device__ __forceinline__ int arrive_acq_rel(int* ctr) {
 
 // The sequence of ring items of one warp's chunk [lo, hi) of (tile, block) units: for every
 // tile segment that starts at block 0, first the weak k slices of the tile (kWs per item),
-// then its blocks (up to kSub per item, never crossing a tile).  Producer and consumer each
+// then its blocks (up to `sub` per item, never crossing a tile).  Producer and consumer each
 // run their own copy, so they agree item by item.
 struct ItemGen {
-  int rt, b, rem, wpos, nsl, Kb, wsi;
-  __device__ void init(int rt0, int b0, int units, int Kb_, int nsl_, int wsi_) {
-    rt = rt0; b = b0; rem = units; Kb = Kb_; nsl = nsl_; wsi = wsi_;
+  int rt, b, rem, wpos, nsl, Kb, wsi, sub;
+  __device__ void init(int rt0, int b0, int units, int Kb_, int nsl_, int wsi_, int sub_) {
+    rt = rt0; b = b0; rem = units; Kb = Kb_; nsl = nsl_; wsi = wsi_; sub = sub_;
     wpos = (units > 0 && b0 == 0) ? 0 : nsl;
   }
   // kind 0: weak slices [first, first + cnt) of tile rt_; kind 1: blocks [first, first + cnt)
@@ -166,7 +172,7 @@ struct ItemGen {
       kind = 0; first = wpos; cnt = min(wsi, nsl - wpos); wpos += cnt;
       return true;
     }
-    kind = 1; first = b; cnt = min(kSub, min(Kb - b, rem));
+    kind = 1; first = b; cnt = min(sub, min(Kb - b, rem));
     b += cnt; rem -= cnt;
     if (b == Kb) { b = 0; ++rt; wpos = 0; }
     return true;
@@ -175,12 +181,13 @@ struct ItemGen {
   __device__ __forceinline__ bool segment_done() const { return rem <= 0 || b == 0; }
 };
 
-template <int BITS, int NT, int S, bool XSMEM, bool PG>
+template <int BITS, int NT, int SUB, int S, bool XSMEM, bool PG>
 __global__ void __launch_bounds__(kWarps * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
-  using G_ = Geo<BITS>;
+  using G_ = Geo<BITS, SUB>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
   constexpr int MT = 8 * NT;                 // token capacity
+  constexpr int kStage = G_::stage_bytes(PG);
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tig = lane & 3;
@@ -196,27 +203,29 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   const int xstride = K / 2 + 4;             // words per staged token row
   const int W = ((N + 15) / 16) * Kb;        // (tile, block) units
   const int c = Pb.chunk;
+  const int ahead = min(args.ahead, S);
+  const uint32_t k2 = args.k2, k4 = args.k4;
 
   // shared memory carve-up (sizes computed identically on the host)
-  unsigned char* ring = smem + warp * S * G_::kStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * S * G_::kStage) + warp * S;
-  float* psx = reinterpret_cast<float*>(smem + kWarps * S * G_::kStage + kWarps * S * 8 + 16);   // [MT][Kb+1]
+  unsigned char* ring = smem + warp * S * kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * S * kStage) + warp * S;
+  float* psx = reinterpret_cast<float*>(smem + kWarps * S * kStage + kWarps * S * 8 + 16);   // [MT][Kb+1]
   __half* xw = reinterpret_cast<__half*>(psx + ((MT * (Kb + 1) + 3) & ~3));                        // [MT][k_ld]
-  int32_t* sidx = reinterpret_cast<int32_t*>(xw + MT * k_ld);                                      // [k_ld]
-  uint32_t* xs = reinterpret_cast<uint32_t*>(sidx + k_ld);                                          // [M][xstride]
+  uint32_t* xs = reinterpret_cast<uint32_t*>(xw + MT * k_ld);                                      // [M][xstride]
 
   // this warp's chunk of units
   const int wi = ((int)blockIdx.x - Pb.cta_base) * kWarps + warp;
   const int lo = min(wi * c, W), hi = min(lo + c, W);
   const int rt0 = lo / Kb, b0 = lo - rt0 * Kb;
   ItemGen prod, cons;
-  prod.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs);
-  cons.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs);
+  prod.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs, SUB);
+  cons.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs, SUB);
   int issued = 0;
-  // lane 0 only: the next item of the chunk into stage st (false once the chunk is exhausted)
-  auto issue = [&](int st) -> bool {
+  // lane 0 only: the next item of the chunk into the next stage (false once the chunk is exhausted)
+  auto issue = [&]() -> bool {
     int kind, rt, first, cnt;
     if (!prod.next(kind, rt, first, cnt)) return false;
+    const int st = issued % S;
     const unsigned char* src;
     uint32_t bytes;
     if (kind == 0) {
@@ -225,9 +234,17 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     } else {
       src = reinterpret_cast<const unsigned char*>(Pb.packed) + ((size_t)rt * Kb + first) * G_::kTileBlk;
       bytes = (uint32_t)(cnt * G_::kTileBlk);
+      if constexpr (PG) {
+        mbar_arrive_expect_tx(&bars[st], bytes + (uint32_t)(cnt * 64));
+        bulk_load(ring + st * kStage + G_::kStageW, Pb.sz_t + ((size_t)rt * Kb + first) * 16, (uint32_t)(cnt * 64),
+                  &bars[st]);
+        bulk_load(ring + st * kStage, src, bytes, &bars[st]);
+        ++issued;
+        return true;
+      }
     }
     mbar_arrive_expect_tx(&bars[st], bytes);
-    bulk_load(ring + st * G_::kStage, src, bytes, &bars[st]);
+    bulk_load(ring + st * kStage, src, bytes, &bars[st]);
     ++issued;
     return true;
   };
@@ -236,9 +253,15 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
   }
-  // the weak-column indices are static: stage them before waiting for the previous kernel
-  for (int t = threadIdx.x; t < k; t += blockDim.x) sidx[t] = Pb.idx[t];
-  __syncthreads();   // barriers initialised and indices staged before any use
+  // the weak-column indices are static: fetch this thread's before waiting for the previous
+  // kernel (gather elements e = threadIdx.x + it * blockDim.x, it < 2, of [MT][k_ld])
+  int gidx[2];
+  #pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int e = it * blockDim.x + threadIdx.x;
+    const int m = e / k_ld, t = e - m * k_ld;
+    gidx[it] = (e < MT * k_ld && m < M && t < k) ? Pb.idx[t] : -1;
+  }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // activations (and outputs) belong to the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -260,23 +283,22 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         const int p = p0 + it * blockDim.x + threadIdx.x;
         if (p < total) q[it] = ldg_u128(Pb.x + (size_t)p * 8);
       }
-      __half gx[2];
-      #pragma unroll
-      for (int it = 0; it < 2; ++it) {   // weak-column gather, in flight with the rows
-        const int e = (p0 / kMaxIt) * 2 + it * blockDim.x + threadIdx.x;
-        gx[it] = __float2half_rn(0.f);
-        if (e < MT * k_ld) {
-          const int m = e / k_ld, t = e - m * k_ld;
-          if (m < M && t < k) gx[it] = Pb.x[(size_t)m * K + sidx[t]];
+      if (p0 == 0) {
+        __half gx[2];
+        #pragma unroll
+        for (int it = 0; it < 2; ++it) {   // weak-column gather, in flight with the rows
+          const int e = it * blockDim.x + threadIdx.x;
+          gx[it] = __float2half_rn(0.f);
+          if (gidx[it] >= 0) gx[it] = Pb.x[(size_t)(e / k_ld) * K + gidx[it]];
         }
-      }
-      if (p0 == 0 && lane == 0)
-        for (int st = 0; st < S; ++st)
-          if (!issue(st)) break;
-      #pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int e = (p0 / kMaxIt) * 2 + it * blockDim.x + threadIdx.x;
-        if (e < MT * k_ld) xw[e] = gx[it];
+        if (lane == 0)
+          for (int j = 0; j < ahead; ++j)
+            if (!issue()) break;
+        #pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int e = it * blockDim.x + threadIdx.x;
+          if (e < MT * k_ld) xw[e] = gx[it];
+        }
       }
       #pragma unroll
       for (int it = 0; it < kMaxIt; ++it) {
@@ -307,10 +329,9 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     }
     // weak-column activations beyond what the loop above covered
     #pragma unroll 1
-    for (int e = ((total + kMaxIt * (int)blockDim.x - 1) / (kMaxIt * (int)blockDim.x)) * 2 * blockDim.x + threadIdx.x;
-         e < MT * k_ld; e += blockDim.x) {
+    for (int e = 2 * blockDim.x + threadIdx.x; e < MT * k_ld; e += blockDim.x) {
       const int m = e / k_ld, t = e - m * k_ld;
-      xw[e] = (m < M && t < k) ? Pb.x[(size_t)m * K + sidx[t]] : __float2half_rn(0.f);
+      xw[e] = (m < M && t < k) ? Pb.x[(size_t)m * K + Pb.idx[t]] : __float2half_rn(0.f);
     }
   }
   __syncthreads();
@@ -336,17 +357,19 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   __syncthreads();
   if (lo >= hi) return;   // no work for this warp (no barrier follows)
 
-  // per-lane operand pointers (tokens >= M are clamped: their columns are discarded)
-  const uint32_t* xv[NT][4];
+  // per-lane operand offsets in shared memory (tokens >= M are clamped: their columns are
+  // discarded)
+  const int xs_off = (int)(reinterpret_cast<const unsigned char*>(xs) - smem);
+  int xv[NT][4];
   const __half* xg[NT];
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int tok = min(8 * nt + g, M - 1);
     #pragma unroll
-    for (int v = 0; v < 4; ++v) xv[nt][v] = xs + tok * xstride + tig * 16 + 4 * (v ^ tig);
+    for (int v = 0; v < 4; ++v) xv[nt][v] = xs_off + 4 * (tok * xstride + tig * 16 + 4 * (v ^ tig));
     xg[nt] = Pb.x + (size_t)tok * K + 2 * tig;
   }
-  const unsigned char* fa0 = ring + g * G_::kBlk + tig * 4 * BITS;   // this lane's chunk in stage 0
+  const int fa0 = warp * S * kStage + g * G_::kBlk + tig * 4 * BITS;   // this lane's chunk in stage 0
 
   float D[NC][NT][4], Dw[NT][4], y[NT][4];
   zero_acc<BITS, NT>(D);
@@ -355,20 +378,33 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     #pragma unroll
     for (int i = 0; i < 4; ++i) { Dw[nt][i] = 0.f; y[nt][i] = 0.f; }
   int seg_b0 = b0;                 // first block of the current tile segment
+  int sz_rt = -1;                  // tile whose (scale, zero) pairs are in szA / szB
+  __half2 szA = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f)), szB = szA;
   int st = 0;                      // stage being consumed
   uint32_t phase = 0;              // its barrier phase
   int consumed = 0;
+  int failed_at = -1;              // item whose wait timed out
   bool ok = true;
   int kind, rt, first, cnt;
   #pragma unroll 1
   while (cons.next(kind, rt, first, cnt)) {
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], phase, args.status, kWaitLimit));
-    const unsigned char* fa = fa0 + st * G_::kStage;
+    if constexpr (!PG) {
+      if (rt != sz_rt) {   // per-channel pairs of a new tile: needed at its segment end
+        sz_rt = rt;
+        szA = Pb.sz_t[(size_t)rt * 16 + g];
+        szB = Pb.sz_t[(size_t)rt * 16 + g + 8];
+      }
+    }
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], phase, args.status, kWaitLimit));
+      if (!ok) failed_at = consumed;
+    }
+    const int fa = fa0 + st * kStage;
     if (ok && kind == 0) {
       // weak k slices: A = the fp16 weak rows (tile-major slice: [16 rows][16]), B = gathered x
       #pragma unroll 1
       for (int i = 0; i < cnt; ++i) {
-        const uint32_t* ws = reinterpret_cast<const uint32_t*>(ring + st * G_::kStage + i * 512);
+        const uint32_t* ws = reinterpret_cast<const uint32_t*>(ring + st * kStage + i * 512);
         const uint32_t a[4] = {ws[g * 8 + tig], ws[(g + 8) * 8 + tig], ws[g * 8 + 4 + tig], ws[(g + 8) * 8 + 4 + tig]};
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -377,12 +413,11 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         }
       }
     } else if (ok) {
-      auto fold_block = [&](int b) {   // per-group layers: one scale / zero per block
-        const int ra = min(rt * 16 + g, N - 1), rb = min(rt * 16 + g + 8, N - 1);
-        const float gsa = __half2float(Pb.scales[(size_t)ra * Kb + b]);
-        const float gza = __half2float(Pb.zeros[(size_t)ra * Kb + b]);
-        const float gsb = __half2float(Pb.scales[(size_t)rb * Kb + b]);
-        const float gzb = __half2float(Pb.zeros[(size_t)rb * Kb + b]);
+      const __half2* szs = reinterpret_cast<const __half2*>(ring + st * kStage + G_::kStageW);
+      auto fold_block = [&](int bb, int b) {   // per-group layers: one (scale, zero) pair per block
+        const float2 fa_ = __half22float2(szs[bb * 16 + g]);
+        const float2 fb_ = __half22float2(szs[bb * 16 + g + 8]);
+        const float gsa = fa_.x, gza = fa_.y, gsb = fb_.x, gzb = fb_.y;
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
@@ -395,36 +430,35 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           }
         zero_acc<BITS, NT>(D);
       };
-      const int xoff = first * 64;
-      if (cnt == kSub) {
-        #pragma unroll
-        for (int bb = 0; bb < kSub; ++bb) {
-          unit_mma<BITS, NT, XSMEM>(fa + bb * G_::kTileBlk, xv, xoff + bb * 64, xg, first + bb, D);
-          if constexpr (PG) fold_block(first + bb);
+      const int xoff = first * 256;
+      if (cnt == SUB) {
+        #pragma unroll 4
+        for (int bb = 0; bb < SUB; ++bb) {
+          unit_mma<BITS, NT, XSMEM>(smem, fa + bb * G_::kTileBlk, xv, xoff + bb * 256, xg, first + bb, k2, k4, D);
+          if constexpr (PG) fold_block(bb, first + bb);
         }
       } else {
         #pragma unroll 1
         for (int bb = 0; bb < cnt; ++bb) {
-          unit_mma<BITS, NT, XSMEM>(fa + bb * G_::kTileBlk, xv, xoff + bb * 64, xg, first + bb, D);
-          if constexpr (PG) fold_block(first + bb);
+          unit_mma<BITS, NT, XSMEM>(smem, fa + bb * G_::kTileBlk, xv, xoff + bb * 256, xg, first + bb, k2, k4, D);
+          if constexpr (PG) fold_block(bb, first + bb);
         }
       }
     }
     __syncwarp();
-    if (lane == 0 && ok) {   // refill the stage just consumed
-      fence_proxy_async_smem();
-      issue(st);
-    }
     ++consumed;
+    if (lane == 0 && ok && issued < consumed + ahead) {   // keep `ahead` items in flight
+      fence_proxy_async_smem();
+      issue();
+    }
     if (++st == S) { st = 0; phase ^= 1u; }
 
     // end of a tile segment: fold, then store (whole tile) or hand over (split tile)
     if (kind == 1 && cons.segment_done()) {
       const int seg_b1 = first + cnt;
-      const int ra = min(rt * 16 + g, N - 1), rb = min(rt * 16 + g + 8, N - 1);
       if constexpr (!PG) {
-        const float sa = __half2float(Pb.scales[ra]), za = __half2float(Pb.zeros[ra]);
-        const float sb = __half2float(Pb.scales[rb]), zb = __half2float(Pb.zeros[rb]);
+        const float2 fa_ = __half22float2(szA), fb_ = __half22float2(szB);
+        const float sa = fa_.x, za = fa_.y, sb = fb_.x, zb = fb_.y;
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
@@ -456,10 +490,10 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
             part[(g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
         __syncwarp();
         int prev = 0;
-        if (lane == 0) prev = arrive_acq_rel(&Pb.cnt[rt]);
+        if (lane == 0) prev = arrive_acq_rel(&Pb.cnt[(size_t)rt * kCntStride]);
         prev = __shfl_sync(0xffffffffu, prev, 0);
         const bool last = prev == nseg - 1;
-        if (last && lane == 0) Pb.cnt[rt] = 0;   // the tile's counter is ready for the next call
+        if (last && lane == 0) Pb.cnt[(size_t)rt * kCntStride] = 0;   // the tile's counter is ready for the next call
         write = ok && last;
         if (write) {
           const float* pt = Pb.part + (size_t)rt * Pb.seg_cap * 16 * 16;
@@ -491,8 +525,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     }
   }
   // after a timeout: never exit with bulk copies still writing into this CTA's memory
-  if (!ok && lane == 0)
-    for (int j = consumed; j < issued; ++j)
+  if (failed_at >= 0 && lane == 0)
+    for (int j = failed_at; j < issued; ++j)
       mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1), args.status, kWaitLimit);
 }
 
@@ -509,9 +543,9 @@ int sm_count() {
   return n;
 }
 
-template <int BITS, int NT, int S, bool XSMEM>
+template <int BITS, int NT, int SUB, int S, bool XSMEM>
 cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
-  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, S, XSMEM, true> : k_gemv_mma<BITS, NT, S, XSMEM, false>;
+  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, SUB, S, XSMEM, true> : k_gemv_mma<BITS, NT, SUB, S, XSMEM, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int base = 0;
@@ -544,8 +578,7 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
     Pq.row_groups = (Pq.N + 15) / 16;
     work[q] = (long long)Pq.row_groups * Kb;
     total += work[q];
-    const size_t need = (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half) +
-                        (size_t)Pq.k_ld * sizeof(int32_t);
+    const size_t need = (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half);
     if (need > extra) extra = need;
     const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
     if (xb > xbytes) xbytes = xb;
@@ -580,15 +613,19 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
     Pq.cta_base = base;
     base += Pq.ncta;
   }
-  auto smem_for = [&](int S, bool xs) {
-    return (size_t)kWarps * S * Geo<BITS>::kStage + (size_t)kWarps * S * 8 + 16 +
+  const bool pg = a.p[0].G > 1;
+  auto smem_for = [&](int sub, int S, bool xs) {
+    const size_t stage = sub == 8 ? Geo<BITS, 8>::stage_bytes(pg) : Geo<BITS, 4>::stage_bytes(pg);
+    return (size_t)kWarps * S * stage + (size_t)kWarps * S * 8 + 16 +
            ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
   };
-  if (smem_for(4, true) <= kMaxSmem) return launch_k<BITS, NT, 4, true>(a, smem_for(4, true), s);
-  if (smem_for(3, true) <= kMaxSmem) return launch_k<BITS, NT, 3, true>(a, smem_for(3, true), s);
-  if (smem_for(2, true) <= kMaxSmem) return launch_k<BITS, NT, 2, true>(a, smem_for(2, true), s);
-  if (smem_for(3, false) <= kMaxSmem) return launch_k<BITS, NT, 3, false>(a, smem_for(3, false), s);
-  if (smem_for(2, false) <= kMaxSmem) return launch_k<BITS, NT, 2, false>(a, smem_for(2, false), s);
+  // larger items first (fewer per-item steps per block), then deeper rings
+  if (smem_for(8, 2, true) <= kMaxSmem) return launch_k<BITS, NT, 8, 2, true>(a, smem_for(8, 2, true), s);
+  if (smem_for(4, 4, true) <= kMaxSmem) return launch_k<BITS, NT, 4, 4, true>(a, smem_for(4, 4, true), s);
+  if (smem_for(4, 3, true) <= kMaxSmem) return launch_k<BITS, NT, 4, 3, true>(a, smem_for(4, 3, true), s);
+  if (smem_for(4, 2, true) <= kMaxSmem) return launch_k<BITS, NT, 4, 2, true>(a, smem_for(4, 2, true), s);
+  if (smem_for(4, 3, false) <= kMaxSmem) return launch_k<BITS, NT, 4, 3, false>(a, smem_for(4, 3, false), s);
+  if (smem_for(4, 2, false) <= kMaxSmem) return launch_k<BITS, NT, 4, 2, false>(a, smem_for(4, 2, false), s);
   return cudaErrorInvalidValue;
 }
 
@@ -615,6 +652,9 @@ cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cu
   a.count = count;
   a.M = M;
   a.status = device_status_ptr();
+  a.ahead = kAhead;
+  a.k2 = 2u;
+  a.k4 = 4u;
   if (!a.status) return cudaErrorInvalidDevicePointer;
   return bits == 3 ? launch_bits<3>(a, s) : launch_bits<4>(a, s);
 }

@@ -31,8 +31,9 @@ struct Layer {
                         // idx[blk_weak[b] .. blk_weak[b+1])
   int32_t* idx_host;    // k (host copy)
   __half* w_weak_t;     // the weak block tile-major: [N/16 tiles][k_ld/16 slices][16 rows][16]
+  __half2* sz_t;        // (scale, zero) pairs tile-major: [N/16 tiles][G][16 rows] (rows >= N: (0, 0))
   float* part;          // decode workspace: partial sums [N/16 tiles][seg_cap][16 rows][16 tokens]
-  int* cnt;             // decode workspace: per-tile arrival counters (kept at 0 between calls)
+  int* cnt;             // decode workspace: per-tile arrival counters, kCntStride apart (0 between calls)
   int seg_cap;          // most warps that may share one row tile in the decode product
   cudaStream_t stream;  // stream of owq_pack (used to order the release)
   // tcgen05 GEMM tensor maps, encoded lazily on first use
@@ -51,6 +52,7 @@ cudaError_t launch_pack(const uint8_t* codes, const __half* zeros, const uint32_
                         int N, int K, int bits, int group, uint32_t* packed, cudaStream_t s);
 cudaError_t launch_dequant(const Layer& L, __half* w_hat, uint8_t* codes, cudaStream_t s);
 cudaError_t launch_weak_tiles(const __half* w_weak, int N, int k_ld, __half* w_weak_t, cudaStream_t s);
+cudaError_t launch_sz_tiles(const __half* scales, const __half* zeros, int N, int G, __half2* sz_t, cudaStream_t s);
 
 struct GemvProblem {
   const uint32_t* packed;
@@ -62,6 +64,7 @@ struct GemvProblem {
   __half* y;
   int N, K, G, k, k_ld;
   const __half* w_weak_t;   // tile-major weak block
+  const __half2* sz_t;      // tile-major (scale, zero) pairs
   float* part;              // partial-sum workspace of split row tiles
   int* cnt;                 // arrival counters of split row tiles
   int seg_cap;              // partial-sum slots per row tile
@@ -74,6 +77,7 @@ struct GemvProblem {
 // of the (16-row tile, 128-code block) units, never fewer than kGemvMinChunk.  A row tile is
 // then shared by at most gemv_seg_cap warps, which sizes the layer's partial-sum workspace.
 constexpr int kGemvWarps = 16;
+constexpr int kCntStride = 32;   // one split-tile counter per 128-byte line
 constexpr int kGemvMinChunk = 8;
 inline int gemv_seg_cap(int N, int K, int sm_count) {
   const long long units = (long long)((N + 15) / 16) * (K / kBlockCodes);

@@ -113,7 +113,27 @@ __global__ void k_weak_tiles(const __half* __restrict__ w, int N, int k_ld, __ha
   wt[e] = row < (size_t)N ? w[row * k_ld + sl * 16 + col] : __float2half_rn(0.f);
 }
 
+// Tile-major (scale, zero) pairs for the decode kernel: entry (row, grp) goes to
+// [row / 16][grp][row % 16] (rows past N are (0, 0)).
+__global__ void k_sz_tiles(const __half* __restrict__ scales, const __half* __restrict__ zeros, int N, int G,
+                           __half2* __restrict__ szt) {
+  const size_t RT = (size_t)(N + 15) / 16;
+  size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= RT * G * 16) return;
+  const int r = (int)(e % 16);
+  const size_t grp = (e / 16) % (size_t)G, tile = e / ((size_t)16 * G);
+  const size_t row = tile * 16 + r;
+  szt[e] = row < (size_t)N ? __halves2half2(scales[row * G + grp], zeros[row * G + grp])
+                           : __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f));
+}
+
 }  // namespace
+
+cudaError_t launch_sz_tiles(const __half* scales, const __half* zeros, int N, int G, __half2* sz_t, cudaStream_t s) {
+  const size_t n = (size_t)((N + 15) / 16) * G * 16;
+  k_sz_tiles<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(scales, zeros, N, G, sz_t);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_weak_tiles(const __half* w_weak, int N, int k_ld, __half* w_weak_t, cudaStream_t s) {
   const size_t n = (size_t)((N + 15) / 16) * 16 * k_ld;
