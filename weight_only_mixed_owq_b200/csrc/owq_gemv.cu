@@ -266,30 +266,30 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   // activations (and outputs) belong to the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- CTA prologue.  The activation loads go out first, then each warp's first S ring items
-  //      (so the few activation bytes are not queued behind the weight stream).  The
-  //      activations go to shared memory already in fragment order (word 4j + t of a block, for
-  //      lane t, at t*16 + 4((j/4) ^ t) + j%4: 16-byte fragment loads spread over all banks),
-  //      with their per-block sums, prefix sums, and the weak-column activations ----
-  {
+  // ---- CTA prologue ----
+  if constexpr (XSMEM) {
+    // The activations: every 16-byte piece of the rows is loaded at once (so the whole load is
+    // one round trip), the weight stream is issued behind these loads, then the pieces are
+    // stored in fragment order: word 4j + t of a block, for lane t, goes to t*16 + 4((j/4) ^ t)
+    // + j%4 (16-byte fragment loads spread over all banks).  The same pass forms the per-block
+    // activation sums; the weak-column activations are gathered alongside.
     const int pieces = K / 8;   // 16-byte pieces of one token row; 16 per block
     const int total = M * pieces;
-    constexpr int kMaxIt = 4;   // pieces per thread kept in flight
+    constexpr int kPer = 16;    // pieces per thread per pass
     #pragma unroll 1
-    for (int p0 = 0; p0 < total; p0 += kMaxIt * (int)blockDim.x) {
-      uint4 q[kMaxIt];
+    for (int p0 = 0; p0 < total; p0 += kPer * (int)blockDim.x) {
+      uint4 q[kPer];
       #pragma unroll
-      for (int it = 0; it < kMaxIt; ++it) {
+      for (int it = 0; it < kPer; ++it) {
         const int p = p0 + it * blockDim.x + threadIdx.x;
         if (p < total) q[it] = ldg_u128(Pb.x + (size_t)p * 8);
       }
+      __half gx[2];
       if (p0 == 0) {
-        __half gx[2];
         #pragma unroll
-        for (int it = 0; it < 2; ++it) {   // weak-column gather, in flight with the rows
+        for (int it = 0; it < 2; ++it) {
           const int e = it * blockDim.x + threadIdx.x;
-          gx[it] = __float2half_rn(0.f);
-          if (gidx[it] >= 0) gx[it] = Pb.x[(size_t)(e / k_ld) * K + gidx[it]];
+          gx[it] = gidx[it] >= 0 ? Pb.x[(size_t)(e / k_ld) * K + gidx[it]] : __float2half_rn(0.f);
         }
         if (lane == 0)
           for (int j = 0; j < ahead; ++j)
@@ -301,7 +301,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         }
       }
       #pragma unroll
-      for (int it = 0; it < kMaxIt; ++it) {
+      for (int it = 0; it < kPer; ++it) {
+        if (p0 + it * (int)blockDim.x >= total) break;   // uniform: whole passes of the CTA
         const int p = p0 + it * blockDim.x + threadIdx.x;
         float v = 0.f;
         int m = 0, pp = 0;
@@ -315,23 +316,54 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
             v += f.x;
             v += f.y;
           }
-          if constexpr (XSMEM) {
-            uint32_t* blk = xs + m * xstride + (pp >> 4) * 64;
-            const int j = pp & 15;
-            #pragma unroll
-            for (int t = 0; t < 4; ++t) blk[t * 16 + 4 * ((j >> 2) ^ t) + (j & 3)] = h[t];
-          }
+          uint32_t* blk = xs + m * xstride + (pp >> 4) * 64;
+          const int j = pp & 15;
+          #pragma unroll
+          for (int t = 0; t < 4; ++t) blk[t * 16 + 4 * ((j >> 2) ^ t) + (j & 3)] = h[t];
         }
         #pragma unroll
         for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (p < total && (pp & 15) == 0) psx[m * (Kb + 1) + (pp >> 4) + 1] = v;
       }
     }
-    // weak-column activations beyond what the loop above covered
     #pragma unroll 1
     for (int e = 2 * blockDim.x + threadIdx.x; e < MT * k_ld; e += blockDim.x) {
       const int m = e / k_ld, t = e - m * k_ld;
       xw[e] = (m < M && t < k) ? Pb.x[(size_t)m * K + Pb.idx[t]] : __float2half_rn(0.f);
+    }
+  } else {
+    // activations stay in global memory: per-block sums and the weak-column gather only
+    const int pieces = K / 8;
+    const int total = M * pieces;
+    #pragma unroll 4
+    for (int p0 = 0; p0 < total; p0 += blockDim.x) {
+      const int p = p0 + threadIdx.x;
+      float v = 0.f;
+      int m = 0, pp = 0;
+      if (p < total) {
+        m = p / pieces;
+        pp = p - m * pieces;
+        const uint4 q = ldg_u128(Pb.x + (size_t)p * 8);
+        const uint32_t h[4] = {q.x, q.y, q.z, q.w};
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
+          v += f.x;
+          v += f.y;
+        }
+      }
+      #pragma unroll
+      for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (p < total && (pp & 15) == 0) psx[m * (Kb + 1) + (pp >> 4) + 1] = v;
+      if (p0 == 0 && lane == 0)
+        for (int j = 0; j < ahead; ++j)
+          if (!issue()) break;
+    }
+    #pragma unroll 1
+    for (int e = threadIdx.x; e < MT * k_ld; e += blockDim.x) {
+      const int m = e / k_ld, t = e - m * k_ld;
+      const int col = e < (int)blockDim.x ? gidx[0] : e < 2 * (int)blockDim.x ? gidx[1] : ((m < M && t < k) ? Pb.idx[t] : -1);
+      xw[e] = col >= 0 ? Pb.x[(size_t)m * K + col] : __float2half_rn(0.f);
     }
   }
   __syncthreads();
