@@ -70,7 +70,6 @@ void release(Layer* L) {
   cudaFree(L->w_weak_t);
   cudaFree(L->sz_t);
   cudaFree(L->part);
-  cudaFree(L->cnt);
   delete[] L->idx_host;
   L->magic = 0;
   delete L;
@@ -182,11 +181,11 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
     sms = 148;
   }
   L->seg_cap = gemv_seg_cap(N, K, sms);
-  const size_t part_bytes = RT * L->seg_cap * 16 * 16 * sizeof(float);
+  const size_t part_bytes = RT * (L->seg_cap - 1) * 16 * 16 * sizeof(unsigned long long);
+  L->epoch = 0;
   alloc((void**)&L->w_weak_t, weak_t_bytes);
   alloc((void**)&L->sz_t, RT * L->G * 16 * sizeof(__half2));
   alloc((void**)&L->part, part_bytes);
-  alloc((void**)&L->cnt, RT * kCntStride * sizeof(int));
   uint32_t* mask_dev = nullptr;
   alloc((void**)&mask_dev, sizeof(uint32_t) * (K / 32));
   if (e != cudaSuccess) { cudaFree(mask_dev); release(L); return cuda_status(e); }
@@ -210,7 +209,7 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   if (e == cudaSuccess && k > 0) e = cudaMemcpyAsync(L->idx, idx, sizeof(int32_t) * k, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(L->blk_weak, blk.data(), sizeof(int32_t) * (Kb + 1), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(mask_dev, mask.data(), sizeof(uint32_t) * (K / 32), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(L->cnt, 0, RT * kCntStride * sizeof(int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(L->part, 0, part_bytes, s);   // epoch 0: never a live tag
   if (e == cudaSuccess)
     e = launch_pack(codes, reinterpret_cast<const __half*>(zeros), mask_dev, N, K, bits, group, L->packed, s);
   if (e == cudaSuccess) e = launch_weak_tiles(L->w_weak, N, L->k_ld, L->w_weak_t, s);
@@ -237,7 +236,9 @@ static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvP
   P->x = reinterpret_cast<const __half*>(x);
   P->y = reinterpret_cast<__half*>(y);
   P->N = L->N; P->K = L->K; P->G = L->G; P->k = L->k; P->k_ld = L->k_ld;
-  P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->part = L->part; P->cnt = L->cnt; P->seg_cap = L->seg_cap;
+  P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->part = L->part; P->seg_cap = L->seg_cap;
+  if (++L->epoch == 0) ++L->epoch;   // 0 marks the zeroed workspace
+  P->epoch = L->epoch;
   P->row_groups = 0; P->cta_base = 0; P->ncta = 0; P->chunk = 0;
   return OWQ_OK;
 }

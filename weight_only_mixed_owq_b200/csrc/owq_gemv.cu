@@ -24,9 +24,9 @@
 //        sum_j s (q_j - z) x_j = s * (sum_j q_j x_j - z * sum_j x_j);
 //    the activation sums come from per-block prefix sums computed once per CTA.  (The fp16
 //    rounding of each s (q - z) is not applied; the difference is far inside the tolerance.)
-//  * A row tile split between warps is finished by the last segment to
-//    arrive: it adds the other segments' partial sums, in segment order, from the layer's
-//    workspace (deterministic), and resets the tile's counter for the next call.
+//  * A row tile split between warps is finished by the warp holding its last unit, once that
+//    warp's own chunk is done: it adds the other segments' partial sums (tagged with the call's
+//    epoch, so they need no counter or fence) in segment order, then its own (deterministic).
 #include "owq_format.cuh"
 #include "owq_internal.cuh"
 #include "owq_sm100.cuh"
@@ -145,13 +145,17 @@ __device__ __forceinline__ void unit_mma(const unsigned char* sm, int fa, const 
   }
 }
 
-// Arrival on a split row tile: one acquire-release atomic at GPU scope (the warp's partial
-// stores, ordered before it by the warp barrier, are released with it; the last arrival
-// acquires the other segments' partials with it).
-__device__ __forceinline__ int arrive_acq_rel(int* ctr) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
-  return old;
+// Partial sums of split row tiles travel as 64-bit words (fp32 value in the low half, the
+// call's epoch in the high half): a 64-bit access is single-copy atomic, so a reader sees
+// either an older word or this call's complete value, and needs no fence or counter.
+__device__ __forceinline__ void st_tagged(unsigned long long* p, float v, uint32_t epoch) {
+  const unsigned long long w = (unsigned long long)__float_as_uint(v) | ((unsigned long long)epoch << 32);
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" :: "l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
 }
 
 // The sequence of ring items of one warp's chunk [lo, hi) of (tile, block) units: for every
@@ -410,6 +414,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     #pragma unroll
     for (int i = 0; i < 4; ++i) { Dw[nt][i] = 0.f; y[nt][i] = 0.f; }
   int seg_b0 = b0;                 // first block of the current tile segment
+  int fin_rt = -1, fin_nseg = 0;   // split tile whose last unit this warp holds (finished at the end)
+  float fin_y[NT][4];
   int sz_rt = -1;                  // tile whose (scale, zero) pairs are in szA / szB
   __half2 szA = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f)), szB = szA;
   int st = 0;                      // stage being consumed
@@ -510,50 +516,83 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
 
       const int t0 = rt * Kb;
       const int c_first = t0 / c, nseg = (t0 + Kb - 1) / c - c_first + 1;
-      bool write = ok;
-      if (nseg > 1) {
-        // split tile: publish this segment's partial; the last arrival finishes the tile
-        const int sid = (t0 + seg_b0) / c - c_first;
-        float* part = Pb.part + ((size_t)rt * Pb.seg_cap + sid) * 16 * 16;
-        #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            part[(g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
-        __syncwarp();
-        int prev = 0;
-        if (lane == 0) prev = arrive_acq_rel(&Pb.cnt[(size_t)rt * kCntStride]);
-        prev = __shfl_sync(0xffffffffu, prev, 0);
-        const bool last = prev == nseg - 1;
-        if (last && lane == 0) Pb.cnt[(size_t)rt * kCntStride] = 0;   // the tile's counter is ready for the next call
-        write = ok && last;
-        if (write) {
-          const float* pt = Pb.part + (size_t)rt * Pb.seg_cap * 16 * 16;
+      if (nseg == 1) {
+        if (ok) {
           #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
             #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int off = (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1);
-              float v = 0.f;
-              for (int s2 = 0; s2 < nseg; ++s2) v += __ldcg(pt + s2 * 16 * 16 + off);
-              y[nt][i] = v;
+              const int row = rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
+              if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(y[nt][i]);
             }
         }
-      }
-      if (write) {
+      } else if (seg_b1 == Kb) {
+        // this segment holds the tile's last unit: this warp finishes the tile once its own
+        // chunk is done, reading the other segments (lower chunks, earlier CTAs)
+        fin_rt = rt;
+        fin_nseg = nseg;
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int row = rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
-            if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(y[nt][i]);
-          }
+          for (int i = 0; i < 4; ++i) fin_y[nt][i] = y[nt][i];
+      } else {
+        // publish this segment's partial (segment sid < nseg - 1) and move on
+        const int sid = (t0 + seg_b0) / c - c_first;
+        unsigned long long* part = Pb.part + ((size_t)rt * (Pb.seg_cap - 1) + sid) * 256;
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st_tagged(part + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1), y[nt][i], Pb.epoch);
       }
       #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         #pragma unroll
         for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
       seg_b0 = 0;
+    }
+  }
+  // the split tile whose last unit this warp holds: add the other segments in segment order
+  // (bounded wait for each tagged word), then this warp's own part
+  if (fin_rt >= 0 && ok) {
+    const unsigned long long* pt = Pb.part + (size_t)fin_rt * (Pb.seg_cap - 1) * 256;
+    float acc[NT][4];
+    #pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+    bool good = true;
+    #pragma unroll 1
+    for (int s2 = 0; s2 < fin_nseg - 1 && good; ++s2) {
+      unsigned long long w[NT][4];
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) w[nt][i] = ld_tagged(pt + s2 * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1));
+      const long long t_start = clock64();
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          while ((uint32_t)(w[nt][i] >> 32) != Pb.epoch) {
+            if (clock64() - t_start > kWaitLimit) {
+              atomicExch(args.status, 1);
+              good = false;
+              break;
+            }
+            w[nt][i] = ld_tagged(pt + s2 * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1));
+          }
+          acc[nt][i] += __uint_as_float((uint32_t)w[nt][i]);
+        }
+    }
+    if (good) {
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = fin_rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
+          if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(acc[nt][i] + fin_y[nt][i]);
+        }
     }
   }
   // after a timeout: never exit with bulk copies still writing into this CTA's memory

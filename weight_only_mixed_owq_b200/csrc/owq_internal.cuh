@@ -32,9 +32,11 @@ struct Layer {
   int32_t* idx_host;    // k (host copy)
   __half* w_weak_t;     // the weak block tile-major: [N/16 tiles][k_ld/16 slices][16 rows][16]
   __half2* sz_t;        // (scale, zero) pairs tile-major: [N/16 tiles][G][16 rows] (rows >= N: (0, 0))
-  float* part;          // decode workspace: partial sums [N/16 tiles][seg_cap][16 rows][16 tokens]
-  int* cnt;             // decode workspace: per-tile arrival counters, kCntStride apart (0 between calls)
+  // decode workspace: partial sums of split row tiles, [N/16 tiles][seg_cap - 1][16 rows][16 tokens],
+  // each a 64-bit word (fp32 value | call epoch << 32); zero at pack time
+  unsigned long long* part;
   int seg_cap;          // most warps that may share one row tile in the decode product
+  uint32_t epoch;       // decode calls made on this handle (tags the partial sums of each call)
   cudaStream_t stream;  // stream of owq_pack (used to order the release)
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
@@ -65,9 +67,9 @@ struct GemvProblem {
   int N, K, G, k, k_ld;
   const __half* w_weak_t;   // tile-major weak block
   const __half2* sz_t;      // tile-major (scale, zero) pairs
-  float* part;              // partial-sum workspace of split row tiles
-  int* cnt;                 // arrival counters of split row tiles
-  int seg_cap;              // partial-sum slots per row tile
+  unsigned long long* part;  // tagged partial sums of split row tiles
+  int seg_cap;               // warps that may share a row tile (seg_cap - 1 slots per tile)
+  uint32_t epoch;            // tag of this call's partial sums (never 0)
   int row_groups;     // 16-row tiles
   int cta_base;       // first CTA of this problem
   int ncta;           // CTAs serving this problem
@@ -77,7 +79,6 @@ struct GemvProblem {
 // of the (16-row tile, 128-code block) units, never fewer than kGemvMinChunk.  A row tile is
 // then shared by at most gemv_seg_cap warps, which sizes the layer's partial-sum workspace.
 constexpr int kGemvWarps = 16;
-constexpr int kCntStride = 32;   // one split-tile counter per 128-byte line
 constexpr int kGemvMinChunk = 8;
 inline int gemv_seg_cap(int N, int K, int sm_count) {
   const long long units = (long long)((N + 15) / 16) * (K / kBlockCodes);
