@@ -335,8 +335,11 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
 
 template <int BITS>
 owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
+  // wider token tiles dequantise each weight tile once for more tokens (the dequantisation,
+  // not the MMA, bounds the narrower tiles); the widest one fits two stages
   if (M <= 64) return run<BITS, 64, 4>(L, x, y, M, s);
-  return run<BITS, 128, 3>(L, x, y, M, s);
+  if (M <= 256) return run<BITS, 128, 3>(L, x, y, M, s);
+  return run<BITS, 256, 2>(L, x, y, M, s);
 }
 
 }  // namespace
