@@ -23,6 +23,7 @@
 // Every mbarrier wait is bounded (clock64 limit): on expiry the thread records the device
 // status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
 #include <cstring>
+#include <type_traits>
 
 #include "owq_format.cuh"
 #include "owq_internal.cuh"
@@ -177,10 +178,11 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     }
   } else {
     // ---------------- dequantisation ----------------
-    // thread (r, h): row r of the tile, chunks 2h and 2h+1 of each 128-code block, i.e. the
-    // codes k = 8j + 4h .. 8j + 4h + 3 (j = 0..15): 8-byte halves of the 16-byte swizzle units
+    // thread (r, jh): row r of the tile and K-slab jh (codes 64 jh .. 64 jh + 63 of each
+    // 128-code block): for j = 8 jh .. 8 jh + 7, the four chunks' pair j are the 8 codes
+    // 8j .. 8j + 7, i.e. one whole 16-byte unit of the 128B-swizzled row (no bank conflicts)
     const int td = threadIdx.x - 64;          // 0..255
-    const int r = td & (kBM - 1), h = td >> 7;
+    const int r = td & (kBM - 1), jh = td >> 7;
     const int row = min(n0 + r, p.N - 1);
     const bool per_channel = p.G == 1;
     uint32_t s2 = 0, scl[3], nz[3];
@@ -188,50 +190,83 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     scl[0] = h2_splat(1.f);
     scl[1] = h2_splat(1.f / kOff[1]);
     scl[2] = h2_splat(1.f / kOff[2]);
-    auto load_sz = [&](int g) {
-      const __half sh = p.scales[(size_t)row * p.G + g];
-      const float z = __half2float(p.zeros[(size_t)row * p.G + g]);
-      const uint32_t su = __half_as_ushort(sh);
-      s2 = su | (su << 16);
-      #pragma unroll
-      for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
-    };
-    if (per_channel) load_sz(0);
+    // (scale, zero) of the next step, fetched one step ahead
+    __half sh_next = p.scales[(size_t)row * p.G];
+    __half z_next = p.zeros[(size_t)row * p.G];
+    // weak columns of the next step (up to 4 fetched one step ahead; more are read in place)
+    int wcol0, wcol1, wcol2, wcol3;
+    __half wval0, wval1, wval2, wval3;
+#define OWQ_FETCH_WEAK(KB)                                                                      \
+    {                                                                                           \
+      const int t0_ = p.blk_weak[KB], t1_ = p.blk_weak[(KB) + 1];                               \
+      const __half zero_ = __float2half_rn(0.f);                                                \
+      const __half* wr_ = p.w_weak + (size_t)row * p.k_ld;                                      \
+      wcol0 = t0_ < t1_ ? p.idx[t0_] - (KB) * kStepCodes : -1;                                  \
+      wcol1 = t0_ + 1 < t1_ ? p.idx[t0_ + 1] - (KB) * kStepCodes : -1;                          \
+      wcol2 = t0_ + 2 < t1_ ? p.idx[t0_ + 2] - (KB) * kStepCodes : -1;                          \
+      wcol3 = t0_ + 3 < t1_ ? p.idx[t0_ + 3] - (KB) * kStepCodes : -1;                          \
+      wval0 = t0_ < t1_ ? wr_[t0_] : zero_;                                                     \
+      wval1 = t0_ + 1 < t1_ ? wr_[t0_ + 1] : zero_;                                             \
+      wval2 = t0_ + 2 < t1_ ? wr_[t0_ + 2] : zero_;                                             \
+      wval3 = t0_ + 3 < t1_ ? wr_[t0_ + 3] : zero_;                                             \
+    }
+    OWQ_FETCH_WEAK(0)
     bool ok = true;
     for (int kb = 0; kb < nK && ok; ++kb) {
       const int s = kb % S, u = kb / S;
-      if (!per_channel) load_sz(kb);
+      if (kb == 0 || !per_channel) {
+        const uint32_t su = __half_as_ushort(sh_next);
+        const float z = __half2float(z_next);
+        s2 = su | (su << 16);
+        #pragma unroll
+        for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
+        if (!per_channel && kb + 1 < nK) {
+          sh_next = p.scales[(size_t)row * p.G + kb + 1];
+          z_next = p.zeros[(size_t)row * p.G + kb + 1];
+        }
+      }
+      const int wc[4] = {wcol0, wcol1, wcol2, wcol3};
+      const __half wv[4] = {wval0, wval1, wval2, wval3};
+      if (kb + 1 < nK) OWQ_FETCH_WEAK(kb + 1)
       ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit);
       if (!ok) break;
       unsigned char* st = smem + s * L::kStage;
-      const uint32_t* pw = reinterpret_cast<const uint32_t*>(st + L::kX + L::kA + r * 16 * BITS);
-      uint32_t wa[BITS], wb[BITS];
+      const uint4* pw = reinterpret_cast<const uint4*>(st + L::kX + L::kA + r * 16 * BITS);
+      uint32_t w[4 * BITS];
       #pragma unroll
-      for (int j = 0; j < BITS; ++j) {
-        wa[j] = pw[(2 * h) * BITS + j];
-        wb[j] = pw[(2 * h + 1) * BITS + j];
+      for (int v = 0; v < BITS; ++v) {
+        const uint4 q = pw[v];
+        w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
       }
-      unsigned char* abase = st + L::kX;
+      unsigned char* slab = st + L::kX + jh * kBM * 128;
+      // jh is uniform per warp: each branch sees compile-time pair indices
+      auto units = [&](auto jh_c) {
+        constexpr int JH = decltype(jh_c)::value;
+        #pragma unroll
+        for (int j8 = 0; j8 < 8; ++j8) {
+          uint32_t d[4];
+          #pragma unroll
+          for (int q = 0; q < 4; ++q) d[q] = dequant_pair<BITS>(w + q * BITS, 8 * JH + j8, s2, scl, nz);   // k = 8j + 2q, +1
+          *reinterpret_cast<uint4*>(slab + sw128_off(r, j8)) = make_uint4(d[0], d[1], d[2], d[3]);
+        }
+      };
+      if (jh == 0) units(std::integral_constant<int, 0>{});
+      else units(std::integral_constant<int, 1>{});
+      // weak columns of this block in this slab: their fp16 values replace the zero-filled codes
       #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const uint32_t lo = dequant_pair<BITS>(wa, j, s2, scl, nz);   // k = 8j + 4h, +1
-        const uint32_t hi = dequant_pair<BITS>(wb, j, s2, scl, nz);   // k = 8j + 4h + 2, +3
-        unsigned char* slab = abase + (j >> 3) * kBM * 128;
-        *reinterpret_cast<uint2*>(slab + sw128_off(r, j & 7) + 8 * h) = make_uint2(lo, hi);
-      }
-      // weak columns of this block whose code falls in this thread's halves: their fp16
-      // values replace the zero-filled codes
-      const int t0 = p.blk_weak[kb], t1 = p.blk_weak[kb + 1];
-      for (int t = t0; t < t1; ++t) {
+      for (int i = 0; i < 4; ++i)
+        if (wc[i] >= 0 && (wc[i] >> 6) == jh)
+          *(reinterpret_cast<__half*>(slab + sw128_off(r, (wc[i] >> 3) & 7)) + (wc[i] & 7)) = wv[i];
+      const int t1 = p.blk_weak[kb + 1];
+      for (int t = p.blk_weak[kb] + 4; t < t1; ++t) {   // blocks with more than four weak columns
         const int col = p.idx[t] - kb * kStepCodes;
-        if (((col >> 2) & 1) != h) continue;
-        unsigned char* slab = abase + (col >> 6) * kBM * 128;
-        __half* dst = reinterpret_cast<__half*>(slab + sw128_off(r, (col >> 3) & 7)) + (col & 7);
-        *dst = p.w_weak[(size_t)row * p.k_ld + t];
+        if ((col >> 6) != jh) continue;
+        *(reinterpret_cast<__half*>(slab + sw128_off(r, (col >> 3) & 7)) + (col & 7)) = p.w_weak[(size_t)row * p.k_ld + t];
       }
       fence_proxy_async_smem();
       mbar_arrive(&afull[s]);
     }
+#undef OWQ_FETCH_WEAK
 
     // ---------------- epilogue ----------------
     const int wd = warp - 2, q = warp & 3, chalf = wd >> 2;
