@@ -408,7 +408,7 @@ def run_owq(args, rank, world, local):
             "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
             "frac_of_8TBps_spec": round(achieved / 8000.0, 4) if achieved else None,
-            "traffic": ncu_traffic("k_gemv_opt67b"),
+            "traffic": ncu_traffic("k_gemv"),
             "launch_us": round(launch_us, 3),
             "basis": "algorithmic bytes of the timed launches / timed region (CUDA events); all launches are k_gemv",
             "per_launch_group_serialised": per_group,

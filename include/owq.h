@@ -113,10 +113,18 @@ owq_status_t owq_quantize_noalloc(const uint16_t* W, const uint16_t* X, int N, i
  *      idx and w_weak may be NULL when k == 0.
  * Out: *out = a new handle.  The handle owns copies of everything; the inputs may be
  *      freed once this call returns.
- * Packed format (per row, 32-code chunks of `bits` uint32 words, little-endian):
- *   pair t = codes (2t, 2t+1) of a chunk; even code in bits [o, o+bits) and odd code in
- *   bits [16+o, 16+o+bits) of the same word.  bits=4: word t/4, o = 4 (t%4).  bits=3:
- *   t < 15 -> word t/5, o = 3 (t%5); bit e of code 30 (31) is bit 15 (31) of word e.
+ * Packed format of one 128-code block of a row (4 * bits little-endian uint32 words):
+ *   codes 2p, 2p+1 form pair p (p = 0..63); the block is four chunks of `bits` words and
+ *   chunk q holds the pairs p = 4j + q (j = 0..15).  Pair j of a chunk sits at a slot
+ *   (word, offset): the even code at bit `offset`, the odd code at bit 16 + offset of
+ *   that word.  bits = 4: word 2(j/8) + j%2, offset 4((j%8)/2).  bits = 3: slots
+ *   (0,0) (1,0) (0,3) (1,3) (0,6) (1,6) (0,9) (1,9) (0,12) (1,12) (2,6) D (2,3) (2,12)
+ *   (2,0) (2,9) for j = 0..15, where D (j = 11) keeps bit e of its even / odd code in
+ *   bit 15 / 31 of word e.  (A tensor-core lane's operand fragment of a block is exactly
+ *   one chunk.)  The handle stores the blocks of each 16-row tile block-major (rows padded
+ *   to a multiple of 16 with zero words) and, for the decode kernel, tile-major copies of
+ *   the weak block and of the (scale, zero) pairs plus a split-tile workspace (about
+ *   8 * 256 bytes per 16-row tile per extra warp that may share it).
  * Synchronises `stream` once (idx is copied to the host and validated: OWQ_ERR_INDEX).
  */
 owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group,
@@ -127,11 +135,17 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group,
 /*
  * owq_gemv -- decode product for 1 <= M <= 16 tokens ("Real-device acceleration",
  * paper p.6: low-bit dense product plus fp16 weak columns on the activation channels
- * selected on the fly).  One kernel: 128-bit loads of the packed words, in-register
- * unpack, fp32 accumulation of exact fp16 products, the weak-column gather and product in
- * the same pass, warp-shuffle reduction, one fp16 rounding of each output.
+ * selected on the fly).  One kernel, one wave of one 16-warp CTA per SM: every warp
+ * streams an equal share of the layer's (16-row tile, 128-code block) units through its
+ * own shared-memory ring (bulk copies), lifts each code pair into an exact fp16x2 value with
+ * one AND, multiplies on the tensor cores (m16n8k16, fp32 accumulation), applies scale and
+ * zero point per row segment, and adds the weak columns (gathered activations x fp16 block)
+ * in the same pass; a row tile shared by several warps is summed by the warp holding its
+ * last unit.  One fp16 rounding of each output.
  * In:  x fp16 M x K row-major.   Out: y fp16 M x N row-major (fully overwritten).
- * Calls on the same handle may run concurrently (the handle is read-only here).
+ * Every call writes the handle's split-tile workspace and call counter: calls on one
+ * handle must be ordered (one stream, or events between streams); calls on different
+ * handles may overlap.  Bounded device waits: on a timeout (see owq_gemm) y is undefined.
  */
 owq_status_t owq_gemv(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
                       owq_stream_t stream);
@@ -140,8 +154,8 @@ owq_status_t owq_gemv(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
  * owq_gemv_multi -- `count` independent decode products in ONE launch (layers that
  * read their inputs before any of them writes, e.g. q/k/v of one attention block).
  * layers, xs, ys are HOST arrays of `count` entries; xs[i] is M x K_i and ys[i] is
- * M x N_i (device).  All layers must share bits; 1 <= count <= 16.  Output buffers must
- * not overlap inputs of another entry.
+ * M x N_i (device).  All layers must share bits; 1 <= count <= 16; a handle may appear
+ * only once (OWQ_ERR_HANDLE).  Output buffers must not overlap inputs of another entry.
  */
 owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs,
                             uint16_t* const* ys, int count, int M, owq_stream_t stream);
@@ -152,7 +166,8 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
  * to tcgen05 MMA with fp32 accumulators in tensor memory.  Same semantics and layouts as
  * owq_gemv; M <= 65536.  Bounded device waits: on a timeout the kernel abandons its tile,
  * sets the device status word and this call's later owq_device_status returns
- * OWQ_ERR_TIMEOUT (y is then undefined).
+ * OWQ_ERR_TIMEOUT (y is then undefined).  The first call on a handle builds its tensor
+ * map on the host: first calls from several host threads on one handle must be serialised.
  */
 owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
                       owq_stream_t stream);
@@ -167,8 +182,9 @@ owq_status_t owq_dequant(owq_layer_t layer, uint16_t* w_hat, uint8_t* codes,
 /* Shape of a layer (host outputs; any may be NULL). */
 owq_status_t owq_layer_info(owq_layer_t layer, int* N, int* K, int* bits, int* group, int* k);
 
-/* Bytes the layer stores, per part (host outputs; any may be NULL): packed codes
- * N*K*bits/8, scales+zeros 4*N*K/group, weak block 2*N*k, index list 4*k. */
+/* Bytes of the layer's data, per part (host outputs; any may be NULL): packed codes
+ * N*K*bits/8, scales+zeros 4*N*K/group, weak block 2*N*k, index list 4*k.  (The handle also
+ * keeps the working copies described at owq_pack.) */
 owq_status_t owq_layer_bytes(owq_layer_t layer, size_t* packed, size_t* scales_zeros,
                              size_t* weak, size_t* index);
 
