@@ -158,31 +158,40 @@ __device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long
   return w;
 }
 
-// The sequence of ring items of one warp's chunk [lo, hi) of (tile, block) units: for every
-// tile segment that starts at block 0, first the weak k slices of the tile (kWs per item),
-// then its blocks (up to `sub` per item, never crossing a tile).  Producer and consumer each
-// run their own copy, so they agree item by item.
+// The sequence of ring items of one warp's chunk [lo, hi) of (tile, block) units, walked from
+// the top down: for every tile segment that contains the tile's block 0, first the weak k
+// slices of the tile (kWs per item), then its blocks (up to `sub` per item, never crossing a
+// tile).  Walking down, the top segment of a chunk (the lower part of a tile the next warp
+// finishes) is published first and the bottom segment (the part that finishes a tile whose
+// lower part the previous warp published first) comes last.  Producer and consumer each run
+// their own copy, so they agree item by item.
 struct ItemGen {
-  int rt, b, rem, wpos, nsl, Kb, wsi, sub;
-  __device__ void init(int rt0, int b0, int units, int Kb_, int nsl_, int wsi_, int sub_) {
-    rt = rt0; b = b0; rem = units; Kb = Kb_; nsl = nsl_; wsi = wsi_; sub = sub_;
-    wpos = (units > 0 && b0 == 0) ? 0 : nsl;
+  int rt, bh, rem, wpos, nsl, Kb, wsi, sub;
+  bool seg_end;   // the last item returned closes its tile segment
+  __device__ void init(int hi, int units, int Kb_, int nsl_, int wsi_, int sub_) {
+    Kb = Kb_; nsl = nsl_; wsi = wsi_; sub = sub_; rem = units; seg_end = false;
+    rt = units > 0 ? (hi - 1) / Kb : 0;
+    bh = hi - rt * Kb;
+    wpos = (units > 0 && rem >= bh) ? 0 : nsl;   // the segment reaches block 0
   }
   // kind 0: weak slices [first, first + cnt) of tile rt_; kind 1: blocks [first, first + cnt)
   __device__ __forceinline__ bool next(int& kind, int& rt_, int& first, int& cnt) {
     if (rem <= 0) return false;
     rt_ = rt;
+    seg_end = false;
     if (wpos < nsl) {
       kind = 0; first = wpos; cnt = min(wsi, nsl - wpos); wpos += cnt;
       return true;
     }
-    kind = 1; first = b; cnt = min(sub, min(Kb - b, rem));
-    b += cnt; rem -= cnt;
-    if (b == Kb) { b = 0; ++rt; wpos = 0; }
+    kind = 1; cnt = min(sub, min(bh, rem)); first = bh - cnt;
+    bh -= cnt; rem -= cnt;
+    if (rem <= 0 || bh == 0) {
+      seg_end = true;
+      if (rem > 0) { --rt; bh = Kb; wpos = rem >= Kb ? 0 : nsl; }
+    }
     return true;
   }
-  // after a block item: does it end a tile segment?
-  __device__ __forceinline__ bool segment_done() const { return rem <= 0 || b == 0; }
+  __device__ __forceinline__ bool segment_done() const { return seg_end; }
 };
 
 template <int BITS, int NT, int SUB, int S, bool XSMEM, bool PG>
@@ -220,10 +229,10 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   // this warp's chunk of units
   const int wi = ((int)blockIdx.x - Pb.cta_base) * kWarps + warp;
   const int lo = min(wi * c, W), hi = min(lo + c, W);
-  const int rt0 = lo / Kb, b0 = lo - rt0 * Kb;
+  const int b_top = hi > lo ? hi - ((hi - 1) / Kb) * Kb : 0;   // block end of the top segment
   ItemGen prod, cons;
-  prod.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs, SUB);
-  cons.init(rt0, b0, hi - lo, Kb, nsl, G_::kWs, SUB);
+  prod.init(hi, hi - lo, Kb, nsl, G_::kWs, SUB);
+  cons.init(hi, hi - lo, Kb, nsl, G_::kWs, SUB);
   int issued = 0;
   // lane 0 only: the next item of the chunk into the next stage (false once the chunk is exhausted)
   auto issue = [&]() -> bool {
@@ -413,7 +422,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   for (int nt = 0; nt < NT; ++nt)
     #pragma unroll
     for (int i = 0; i < 4; ++i) { Dw[nt][i] = 0.f; y[nt][i] = 0.f; }
-  int seg_b0 = b0;                 // first block of the current tile segment
+  int seg_b1 = b_top;              // block end of the current tile segment (walking down)
   int fin_rt = -1, fin_nseg = 0;   // split tile whose last unit this warp holds (finished at the end)
   float fin_y[NT][4];
   int sz_rt = -1;                  // tile whose (scale, zero) pairs are in szA / szB
@@ -493,7 +502,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
 
     // end of a tile segment: fold, then store (whole tile) or hand over (split tile)
     if (kind == 1 && cons.segment_done()) {
-      const int seg_b1 = first + cnt;
+      const int seg_b0 = first;
       if constexpr (!PG) {
         const float2 fa_ = __half22float2(szA), fb_ = __half22float2(szB);
         const float sa = fa_.x, za = fa_.y, sb = fb_.x, zb = fb_.y;
@@ -549,7 +558,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       for (int nt = 0; nt < NT; ++nt)
         #pragma unroll
         for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
-      seg_b0 = 0;
+      seg_b1 = Kb;
     }
   }
   // the split tile whose last unit this warp holds: add the other segments in segment order
