@@ -69,6 +69,7 @@ void release(Layer* L) {
   cudaFree(L->blk_weak);
   cudaFree(L->w_weak_t);
   cudaFree(L->sz_t);
+  cudaFree(L->gemm_ws);
   cudaFree(L->part);
   delete[] L->idx_host;
   L->magic = 0;

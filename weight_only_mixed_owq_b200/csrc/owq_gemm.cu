@@ -22,6 +22,7 @@
 //               (tcgen05.ld of their TMEM lane quarter, fp16 rounding, coalesced stores).
 // Every mbarrier wait is bounded (clock64 limit): on expiry the thread records the device
 // status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
+#include <algorithm>
 #include <cstring>
 #include <type_traits>
 
@@ -58,8 +59,10 @@ struct GemmParams {
   const int32_t* idx;
   const int32_t* blk_weak;
   __half* y;
+  float* ws;        // split-K partial sums [split][M][N] (NULL: one split, fp16 y directly)
   int* status;
   int N, K, M, G, k_ld;
+  int ksteps;       // 128-code steps per split (blockIdx.z)
 };
 
 // fp16x2 helpers (exact integer arithmetic on small values)
@@ -112,7 +115,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kBM;      // first weight row
   const int m0 = blockIdx.y * BN;       // first token
-  const int nK = p.K / kStepCodes;
+  const int kb0 = blockIdx.z * p.ksteps;                       // first step of this split
+  const int nK = min(p.ksteps, p.K / kStepCodes - kb0);          // steps of this split
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -136,8 +140,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       // ---------------- TMA producer ----------------
       constexpr uint32_t kBytes = L::kX + L::kP;
       bool ok = true;
-      for (int kb = 0; kb < nK && ok; ++kb) {
-        const int s = kb % S, u = kb / S;
+      for (int i = 0; i < nK && ok; ++i) {
+        const int kb = kb0 + i, s = i % S, u = i / S;
         if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, p.status, kWaitLimit);
         if (!ok) break;
         unsigned char* st = smem + s * L::kStage;
@@ -148,16 +152,16 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
       }
       // never leave with copies in flight: wait for the last use of every stage
-      for (int kb = (nK > S ? nK - S : 0); kb < nK; ++kb)
-        mbar_wait(&full[kb % S], (kb / S) & 1, p.status, kWaitLimit);
+      for (int i = (nK > S ? nK - S : 0); i < nK; ++i)
+        mbar_wait(&full[i % S], (i / S) & 1, p.status, kWaitLimit);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc = idesc_f16_f32(kBM, BN);
       bool ok = true;
-      for (int kb = 0; kb < nK && ok; ++kb) {
-        const int s = kb % S, u = kb / S;
+      for (int i = 0; i < nK && ok; ++i) {
+        const int s = i % S, u = i / S;
         ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit) &&
              mbar_wait(&afull[s], u & 1, p.status, kWaitLimit);
         if (!ok) break;
@@ -170,7 +174,7 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = desc_sw128_kmajor(aa + a * kBM * 128 + kk * 32);
             const uint64_t bd = desc_sw128_kmajor(xa + a * BN * 128 + kk * 32);
-            mma_f16(tmem, ad, bd, idesc, (kb | a | kk) != 0);
+            mma_f16(tmem, ad, bd, idesc, (i | a | kk) != 0);
           }
         mma_commit(&empty[s]);
       }
@@ -191,8 +195,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     scl[1] = h2_splat(1.f / kOff[1]);
     scl[2] = h2_splat(1.f / kOff[2]);
     // (scale, zero) of the next step, fetched one step ahead
-    __half sh_next = p.scales[(size_t)row * p.G];
-    __half z_next = p.zeros[(size_t)row * p.G];
+    __half sh_next = p.scales[(size_t)row * p.G + (per_channel ? 0 : kb0)];
+    __half z_next = p.zeros[(size_t)row * p.G + (per_channel ? 0 : kb0)];
     // weak columns of the next step (up to 4 fetched one step ahead; more are read in place)
     int wcol0, wcol1, wcol2, wcol3;
     __half wval0, wval1, wval2, wval3;
@@ -210,24 +214,24 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       wval2 = t0_ + 2 < t1_ ? wr_[t0_ + 2] : zero_;                                             \
       wval3 = t0_ + 3 < t1_ ? wr_[t0_ + 3] : zero_;                                             \
     }
-    OWQ_FETCH_WEAK(0)
+    OWQ_FETCH_WEAK(kb0)
     bool ok = true;
-    for (int kb = 0; kb < nK && ok; ++kb) {
-      const int s = kb % S, u = kb / S;
-      if (kb == 0 || !per_channel) {
+    for (int i = 0; i < nK && ok; ++i) {
+      const int kb = kb0 + i, s = i % S, u = i / S;
+      if (i == 0 || !per_channel) {
         const uint32_t su = __half_as_ushort(sh_next);
         const float z = __half2float(z_next);
         s2 = su | (su << 16);
         #pragma unroll
         for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
-        if (!per_channel && kb + 1 < nK) {
+        if (!per_channel && i + 1 < nK) {
           sh_next = p.scales[(size_t)row * p.G + kb + 1];
           z_next = p.zeros[(size_t)row * p.G + kb + 1];
         }
       }
       const int wc[4] = {wcol0, wcol1, wcol2, wcol3};
       const __half wv[4] = {wval0, wval1, wval2, wval3};
-      if (kb + 1 < nK) OWQ_FETCH_WEAK(kb + 1)
+      if (i + 1 < nK) OWQ_FETCH_WEAK(kb + 1)
       ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit);
       if (!ok) break;
       unsigned char* st = smem + s * L::kStage;
@@ -279,10 +283,19 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
       tmem_ld_wait();
       if (acc_ok && orow < p.N) {
-        #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = m0 + c0 + j;
-          if (t < p.M) p.y[(size_t)t * p.N + orow] = __float2half_rn(__uint_as_float(v[j]));
+        if (p.ws) {   // split-K: fp32 partial of this split
+          float* w = p.ws + (size_t)blockIdx.z * p.M * p.N;
+          #pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = m0 + c0 + j;
+            if (t < p.M) w[(size_t)t * p.N + orow] = __uint_as_float(v[j]);
+          }
+        } else {
+          #pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = m0 + c0 + j;
+            if (t < p.M) p.y[(size_t)t * p.N + orow] = __float2half_rn(__uint_as_float(v[j]));
+          }
         }
       }
     }
@@ -294,6 +307,15 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     tc_fence_after();
     tmem_dealloc(tmem, BN);
     tmem_relinquish();
+  }
+}
+
+// Split-K: y = fp16_rn(sum of the splits' fp32 partials, in split order).
+__global__ void k_splitk_reduce(const float* __restrict__ ws, int splits, size_t MN, __half* __restrict__ y) {
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < MN; e += (size_t)gridDim.x * blockDim.x) {
+    float v = ws[e];
+    for (int z = 1; z < splits; ++z) v += ws[(size_t)z * MN + e];
+    y[e] = __float2half_rn(v);
   }
 }
 
@@ -355,6 +377,46 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
   prm.blk_weak = L.blk_weak; prm.y = y; prm.status = device_status_ptr();
   prm.N = L.N; prm.K = L.K; prm.M = M; prm.G = L.G; prm.k_ld = L.k_ld;
   if (!prm.status) return OWQ_ERR_CUDA;
+  // fewer tiles than SMs: split K over CTAs (at least 4 steps each), fp32 partials in the
+  // layer's workspace, then one reduction kernel; never grown during stream capture
+  const int nK = L.K / kStepCodes;
+  const long long tiles = (long long)((L.N + kBM - 1) / kBM) * ((M + BN - 1) / BN);
+  int splits = 1;
+  static int sms = 0;
+  if (!sms && (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, L.device) != cudaSuccess || sms <= 0)) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  if (tiles < sms) splits = (int)std::max<long long>(1, std::min<long long>(sms / tiles, nK / 4));
+  if (splits > 1) {
+    prm.ksteps = (nK + splits - 1) / splits;
+    splits = (nK + prm.ksteps - 1) / prm.ksteps;
+    const size_t need = (size_t)splits * M * L.N * sizeof(float);
+    if (need > L.gemm_ws_bytes) {
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+        cudaGetLastError();
+        splits = 1;
+      } else {
+        cudaFree(L.gemm_ws);
+        L.gemm_ws = nullptr;
+        L.gemm_ws_bytes = 0;
+        if (cudaMalloc(&L.gemm_ws, need) != cudaSuccess) {
+          cudaGetLastError();
+          L.gemm_ws = nullptr;
+          splits = 1;
+        } else {
+          L.gemm_ws_bytes = need;
+        }
+      }
+    }
+  }
+  if (splits == 1) {
+    prm.ksteps = nK;
+    prm.ws = nullptr;
+  } else {
+    prm.ws = L.gemm_ws;
+  }
   auto kern = k_gemm_sm100<BITS, BN, S>;
   constexpr int smem = smem_bytes<BITS, BN, S>();
   static_assert(smem <= 232448, "shared memory budget");
@@ -362,9 +424,14 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
     cudaGetLastError();
     return OWQ_ERR_CUDA;
   }
-  dim3 grid((L.N + kBM - 1) / kBM, (M + BN - 1) / BN);
+  dim3 grid((L.N + kBM - 1) / kBM, (M + BN - 1) / BN, splits);
   kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, prm);
   if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
+  if (splits > 1) {
+    const size_t MN = (size_t)M * L.N;
+    k_splitk_reduce<<<(unsigned)std::min<size_t>((MN + 255) / 256, 4096), 256, 0, s>>>(prm.ws, splits, MN, y);
+    if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
+  }
   return OWQ_OK;
 }
 

@@ -38,6 +38,8 @@ struct Layer {
   int seg_cap;          // most warps that may share one row tile in the decode product
   uint32_t epoch;       // decode calls made on this handle (tags the partial sums of each call)
   cudaStream_t stream;  // stream of owq_pack (used to order the release)
+  float* gemm_ws;       // prefill split-K partial sums (grown on first need, outside capture)
+  size_t gemm_ws_bytes;
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
   alignas(64) CUtensorMap map_packed;
