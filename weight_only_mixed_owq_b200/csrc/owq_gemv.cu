@@ -37,7 +37,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kMaxProblems = 16;
-constexpr int kWarps = kGemvWarps;
 constexpr int kAhead = 2;                        // items in flight per warp (see GemvArgs::ahead)
 constexpr long long kWaitLimit = 4000000000LL;  // ~2 s
 
@@ -194,9 +193,10 @@ struct ItemGen {
   __device__ __forceinline__ bool segment_done() const { return seg_end; }
 };
 
-template <int BITS, int NT, int SUB, int S, bool XSMEM, bool PG>
-__global__ void __launch_bounds__(kWarps * 32, 1)
+template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM, bool PG>
+__global__ void __launch_bounds__(WARPS * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
+  constexpr int kWarps = WARPS;
   using G_ = Geo<BITS, SUB>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
   constexpr int MT = 8 * NT;                 // token capacity
@@ -380,11 +380,12 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     }
   }
   __syncthreads();
-  if (warp < MT) {   // prefix sums of the block sums, one warp per token (tokens >= M: zeros)
-    float* row = psx + warp * (Kb + 1);
+  #pragma unroll 1
+  for (int tw = warp; tw < MT; tw += kWarps) {   // prefix sums of the block sums, a warp per token (tokens >= M: zeros)
+    float* row = psx + tw * (Kb + 1);
     const int per = (Kb + 31) / 32, b_lo = lane * per, b_hi = min(b_lo + per, Kb);
     float run = 0.f;
-    for (int b = b_lo; b < b_hi; ++b) run += warp < M ? row[b + 1] : 0.f;
+    for (int b = b_lo; b < b_hi; ++b) run += tw < M ? row[b + 1] : 0.f;
     float incl = run;
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -394,7 +395,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     float acc = incl - run;
     __syncwarp();
     for (int b = b_lo; b < b_hi; ++b) {
-      acc += warp < M ? row[b + 1] : 0.f;
+      acc += tw < M ? row[b + 1] : 0.f;
       row[b + 1] = acc;
     }
     if (lane == 0) row[0] = 0.f;
@@ -623,9 +624,10 @@ int sm_count() {
   return n;
 }
 
-template <int BITS, int NT, int SUB, int S, bool XSMEM>
+template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM>
 cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
-  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, SUB, S, XSMEM, true> : k_gemv_mma<BITS, NT, SUB, S, XSMEM, false>;
+  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, true>
+                           : k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int base = 0;
@@ -634,7 +636,7 @@ cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
   // drains; it waits (griddepcontrol.wait) before reading activations or writing outputs
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(base);
-  cfg.blockDim = dim3(kWarps * 32);
+  cfg.blockDim = dim3(WARPS * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -645,27 +647,18 @@ cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int BITS, int NT>
-cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
-  constexpr int MT = 8 * NT;
-  constexpr size_t kMaxSmem = 232448;
+// CTAs per problem in proportion to its work (one resident wave in total), then an equal
+// chunk of (tile, block) units per warp: at least kGemvMinChunk, and large enough that a row
+// tile meets at most seg_cap warps (the size of the layer's partial-sum workspace)
+void plan(GemvArgs& a, int warps_per_cta) {
   const int C = sm_count();
   long long work[kMaxProblems], total = 0;
-  size_t extra = 0, xbytes = 0;
   for (int q = 0; q < a.count; ++q) {
     GemvProblem& Pq = a.p[q];
-    const int Kb = Pq.K / kBlockCodes;
     Pq.row_groups = (Pq.N + 15) / 16;
-    work[q] = (long long)Pq.row_groups * Kb;
+    work[q] = (long long)Pq.row_groups * (Pq.K / kBlockCodes);
     total += work[q];
-    const size_t need = (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half);
-    if (need > extra) extra = need;
-    const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
-    if (xb > xbytes) xbytes = xb;
   }
-  // CTAs per problem in proportion to its work (one resident wave in total), then an equal
-  // chunk of (tile, block) units per warp: at least kGemvMinChunk, and large enough that a
-  // row tile meets at most seg_cap warps (the size of the layer's partial-sum workspace)
   int n[kMaxProblems], used = 0, big = 0;
   for (int q = 0; q < a.count; ++q) {
     n[q] = max(1, (int)(work[q] * C / total));
@@ -679,33 +672,59 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
     --n[q];
     --used;
   }
-  if (used < C) { n[big] += C - used; used = C; }
+  if (used < C) n[big] += C - used;
   int base = 0;
   for (int q = 0; q < a.count; ++q) {
     GemvProblem& Pq = a.p[q];
     const int Kb = Pq.K / kBlockCodes;
-    const long long warps = (long long)n[q] * kWarps;
+    const long long warps = (long long)n[q] * warps_per_cta;
     int chunk = (int)((work[q] + warps - 1) / warps);
     chunk = max(chunk, max(kGemvMinChunk, (Kb - 1) / (Pq.seg_cap - 1) + 1));
     const int nchunks = (int)((work[q] + chunk - 1) / chunk);
     Pq.chunk = chunk;
-    Pq.ncta = min(n[q], (nchunks + kWarps - 1) / kWarps);
+    Pq.ncta = min(n[q], (nchunks + warps_per_cta - 1) / warps_per_cta);
     Pq.cta_base = base;
     base += Pq.ncta;
   }
+}
+
+template <int BITS, int NT>
+cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
+  constexpr int MT = 8 * NT;
+  constexpr size_t kMaxSmem = 232448;
+  size_t extra = 0, xbytes = 0;
+  for (int q = 0; q < a.count; ++q) {
+    const GemvProblem& Pq = a.p[q];
+    const int Kb = Pq.K / kBlockCodes;
+    const size_t need = (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half);
+    if (need > extra) extra = need;
+    const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
+    if (xb > xbytes) xbytes = xb;
+  }
   const bool pg = a.p[0].G > 1;
-  auto smem_for = [&](int sub, int S, bool xs) {
+  auto smem_for = [&](int warps, int sub, int S, bool xs) {
     const size_t stage = sub == 8 ? Geo<BITS, 8>::stage_bytes(pg) : Geo<BITS, 4>::stage_bytes(pg);
-    return (size_t)kWarps * S * stage + (size_t)kWarps * S * 8 + 16 +
-           ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
+    return (size_t)warps * S * stage + (size_t)warps * S * 8 + 16 + ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
   };
-  // larger items first (fewer per-item steps per block), then deeper rings
-  if (smem_for(8, 2, true) <= kMaxSmem) return launch_k<BITS, NT, 8, 2, true>(a, smem_for(8, 2, true), s);
-  if (smem_for(4, 4, true) <= kMaxSmem) return launch_k<BITS, NT, 4, 4, true>(a, smem_for(4, 4, true), s);
-  if (smem_for(4, 3, true) <= kMaxSmem) return launch_k<BITS, NT, 4, 3, true>(a, smem_for(4, 3, true), s);
-  if (smem_for(4, 2, true) <= kMaxSmem) return launch_k<BITS, NT, 4, 2, true>(a, smem_for(4, 2, true), s);
-  if (smem_for(4, 3, false) <= kMaxSmem) return launch_k<BITS, NT, 4, 3, false>(a, smem_for(4, 3, false), s);
-  if (smem_for(4, 2, false) <= kMaxSmem) return launch_k<BITS, NT, 4, 2, false>(a, smem_for(4, 2, false), s);
+#define OWQ_TRY(W, SUB, S, XS)                                                           \
+  if (smem_for(W, SUB, S, XS) <= kMaxSmem) {                                             \
+    plan(a, W);                                                                          \
+    return launch_k<BITS, NT, W, SUB, S, XS>(a, smem_for(W, SUB, S, XS), s);            \
+  }
+  // 16 warps with the activations in shared memory: larger items first, then deeper rings
+  OWQ_TRY(16, 8, 2, true)
+  OWQ_TRY(16, 4, 4, true)
+  OWQ_TRY(16, 4, 3, true)
+  OWQ_TRY(16, 4, 2, true)
+  if constexpr (NT == 2) {
+    // more tokens than fit beside a 16-warp ring: 8 warps keep them in shared memory
+    OWQ_TRY(8, 4, 4, true)
+    OWQ_TRY(8, 4, 3, true)
+    OWQ_TRY(8, 4, 2, true)
+  }
+  OWQ_TRY(16, 4, 3, false)
+  OWQ_TRY(16, 4, 2, false)
+#undef OWQ_TRY
   return cudaErrorInvalidValue;
 }
 
