@@ -69,6 +69,7 @@ void release(Layer* L) {
   cudaFree(L->blk_weak);
   cudaFree(L->w_weak_t);
   cudaFree(L->sz_t);
+  cudaFree(L->xfrag);
   cudaFree(L->gemm_ws);
   cudaFree(L->part);
   delete[] L->idx_host;
@@ -186,6 +187,7 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   L->epoch = 0;
   alloc((void**)&L->w_weak_t, weak_t_bytes);
   alloc((void**)&L->sz_t, RT * L->G * 16 * sizeof(__half2));
+  alloc((void**)&L->xfrag, (size_t)16 * K * sizeof(__half));
   alloc((void**)&L->part, part_bytes);
   uint32_t* mask_dev = nullptr;
   alloc((void**)&mask_dev, sizeof(uint32_t) * (K / 32));
@@ -237,7 +239,7 @@ static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvP
   P->x = reinterpret_cast<const __half*>(x);
   P->y = reinterpret_cast<__half*>(y);
   P->N = L->N; P->K = L->K; P->G = L->G; P->k = L->k; P->k_ld = L->k_ld;
-  P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->part = L->part; P->seg_cap = L->seg_cap;
+  P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->xfrag = L->xfrag; P->part = L->part; P->seg_cap = L->seg_cap;
   if (++L->epoch == 0) ++L->epoch;   // 0 marks the zeroed workspace
   P->epoch = L->epoch;
   P->row_groups = 0; P->cta_base = 0; P->ncta = 0; P->chunk = 0;

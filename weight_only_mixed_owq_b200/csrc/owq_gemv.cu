@@ -103,7 +103,7 @@ __device__ __forceinline__ void zero_acc(float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
 // plus 32-bit offsets, so each load is one shared load at register + immediate.
 template <int BITS, int NT, bool XSMEM>
 __device__ __forceinline__ void unit_mma(const unsigned char* sm, int fa, const int (&xv)[NT][4], int xoff,
-                                         const __half* const (&xg)[NT], int b, uint32_t k2, uint32_t k4,
+                                         const uint4* const (&xg)[NT], int b, uint32_t k2, uint32_t k4,
                                          float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
   constexpr int kBlk = 16 * BITS;
   uint32_t wa[BITS], wb[BITS];
@@ -129,9 +129,13 @@ __device__ __forceinline__ void unit_mma(const unsigned char* sm, int fa, const 
         xb[nt][4 * v] = q.x; xb[nt][4 * v + 1] = q.y; xb[nt][4 * v + 2] = q.z; xb[nt][4 * v + 3] = q.w;
       }
     } else {
-      const __half* base = xg[nt] + (size_t)b * kBlockCodes;
+      // fragment-ordered activations in global memory: this lane's 16 words of block b
+      const uint4* base = xg[nt] + (size_t)b * 16;
       #pragma unroll
-      for (int j = 0; j < 16; ++j) xb[nt][j] = ldg_u32(base + 8 * j);
+      for (int v = 0; v < 4; ++v) {
+        const uint4 q = ldg_u128(base + v);
+        xb[nt][4 * v] = q.x; xb[nt][4 * v + 1] = q.y; xb[nt][4 * v + 2] = q.z; xb[nt][4 * v + 3] = q.w;
+      }
     }
   }
   #pragma unroll
@@ -192,6 +196,20 @@ struct ItemGen {
   }
   __device__ __forceinline__ bool segment_done() const { return seg_end; }
 };
+
+// Activations too large for shared memory are written once per call, before the product, in
+// fragment order: for token m, block b and lane t, the 16 words 4j + t (j = 0..15) of the
+// block, contiguous ([m][b][t][16 words]), so a lane fetches its B fragments of a block with
+// four 16-byte loads.
+__global__ void k_x_frag(const __half* __restrict__ x, int M, int K, uint32_t* __restrict__ xf) {
+  const int Kb = K / kBlockCodes;
+  const size_t n = (size_t)M * Kb * 64;   // words
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t mb = e / 64;             // (token, block)
+    const int w = (int)(e % 64), t = w / 16, j = w % 16;
+    xf[e] = reinterpret_cast<const uint32_t*>(x)[mb * 64 + 4 * j + t];
+  }
+}
 
 template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM, bool PG>
 __global__ void __launch_bounds__(WARPS * 32, 1)
@@ -407,13 +425,13 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   // discarded)
   const int xs_off = (int)(reinterpret_cast<const unsigned char*>(xs) - smem);
   int xv[NT][4];
-  const __half* xg[NT];
+  const uint4* xg[NT];
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int tok = min(8 * nt + g, M - 1);
     #pragma unroll
     for (int v = 0; v < 4; ++v) xv[nt][v] = xs_off + 4 * (tok * xstride + tig * 16 + 4 * (v ^ tig));
-    xg[nt] = Pb.x + (size_t)tok * K + 2 * tig;
+    xg[nt] = reinterpret_cast<const uint4*>(Pb.xfrag) + ((size_t)tok * Kb * 4 + tig) * 4;
   }
   const int fa0 = warp * S * kStage + g * G_::kBlk + tig * 4 * BITS;   // this lane's chunk in stage 0
 
@@ -626,6 +644,14 @@ int sm_count() {
 
 template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM>
 cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
+  if constexpr (!XSMEM) {
+    for (int q = 0; q < a.count; ++q) {
+      const size_t n = (size_t)a.M * a.p[q].K / 2;
+      k_x_frag<<<(unsigned)std::min<size_t>((n + 255) / 256, 2048), 256, 0, s>>>(a.p[q].x, a.M, a.p[q].K, a.p[q].xfrag);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, true>
                            : k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -717,10 +743,12 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
   OWQ_TRY(16, 4, 3, true)
   OWQ_TRY(16, 4, 2, true)
   if constexpr (NT == 2) {
-    // more tokens than fit beside a 16-warp ring: 8 warps keep them in shared memory
+    // more tokens than fit beside a 16-warp ring: 8 warps keep them in shared memory, or read
+    // them fragment-ordered from global memory with the register room of 8-warp CTAs
     OWQ_TRY(8, 4, 4, true)
     OWQ_TRY(8, 4, 3, true)
     OWQ_TRY(8, 4, 2, true)
+    OWQ_TRY(8, 4, 4, false)
   }
   OWQ_TRY(16, 4, 3, false)
   OWQ_TRY(16, 4, 2, false)

@@ -32,6 +32,7 @@ struct Layer {
   int32_t* idx_host;    // k (host copy)
   __half* w_weak_t;     // the weak block tile-major: [N/16 tiles][k_ld/16 slices][16 rows][16]
   __half2* sz_t;        // (scale, zero) pairs tile-major: [N/16 tiles][G][16 rows] (rows >= N: (0, 0))
+  uint32_t* xfrag;      // decode scratch: up to 16 activation rows in fragment order (see owq_gemv.cu)
   // decode workspace: partial sums of split row tiles, [N/16 tiles][seg_cap - 1][16 rows][16 tokens],
   // each a 64-bit word (fp32 value | call epoch << 32); zero at pack time
   unsigned long long* part;
@@ -69,6 +70,7 @@ struct GemvProblem {
   int N, K, G, k, k_ld;
   const __half* w_weak_t;   // tile-major weak block
   const __half2* sz_t;      // tile-major (scale, zero) pairs
+  uint32_t* xfrag;          // activations in fragment order (when they do not fit in shared memory)
   unsigned long long* part;  // tagged partial sums of split row tiles
   int seg_cap;               // warps that may share a row tile (seg_cap - 1 slots per tile)
   uint32_t epoch;            // tag of this call's partial sums (never 0)
