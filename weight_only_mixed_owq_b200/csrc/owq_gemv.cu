@@ -294,6 +294,9 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     gidx[it] = (e < MT * k_ld && m < M && t < k) ? Pb.idx[t] : -1;
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the weights do not depend on the previous kernel: each warp's first item streams while this
+  // CTA waits for it (the rest follow the activation loads)
+  if (lane == 0) issue();
   // activations (and outputs) belong to the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
@@ -323,7 +326,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           gx[it] = gidx[it] >= 0 ? Pb.x[(size_t)(e / k_ld) * K + gidx[it]] : __float2half_rn(0.f);
         }
         if (lane == 0)
-          for (int j = 0; j < ahead; ++j)
+          for (int j = 1; j < ahead; ++j)
             if (!issue()) break;
         #pragma unroll
         for (int it = 0; it < 2; ++it) {
@@ -387,7 +390,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (p < total && (pp & 15) == 0) psx[m * (Kb + 1) + (pp >> 4) + 1] = v;
       if (p0 == 0 && lane == 0)
-        for (int j = 0; j < ahead; ++j)
+        for (int j = 1; j < ahead; ++j)
           if (!issue()) break;
     }
     #pragma unroll 1
