@@ -242,7 +242,7 @@ static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvP
   P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->xfrag = L->xfrag; P->part = L->part; P->seg_cap = L->seg_cap;
   if (++L->epoch == 0) ++L->epoch;   // 0 marks the zeroed workspace
   P->epoch = L->epoch;
-  P->row_groups = 0; P->cta_base = 0; P->ncta = 0; P->chunk = 0;
+  P->row_groups = 0; P->cta_base = 0; P->ncta = 0; P->chunk = 0; P->lt_cap = 0;
   return OWQ_OK;
 }
 

@@ -155,6 +155,14 @@ __device__ __forceinline__ void st_tagged(unsigned long long* p, float v, uint32
   const unsigned long long w = (unsigned long long)__float_as_uint(v) | ((unsigned long long)epoch << 32);
   asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" :: "l"(p), "l"(w) : "memory");
 }
+// Segments still expected by a row tile whose segments are all in this CTA: count down one,
+// acquire-release at CTA scope (the segment's accumulator adds are released with it; the
+// segment that reaches 0 acquires all of them).
+__device__ __forceinline__ int count_down_cta(int* c) {
+  int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], -1;" : "=r"(old) : "r"(smem_u32(c)) : "memory");
+  return old;
+}
 __device__ __forceinline__ unsigned long long ld_tagged(const unsigned long long* p) {
   unsigned long long w;
   asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
@@ -232,7 +240,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   const int K = Pb.K, Kb = K / kBlockCodes, k = Pb.k, N = Pb.N, k_ld = Pb.k_ld;
   const int nsl = k > 0 ? k_ld / 16 : 0;     // weak k slices of a tile
   const int xstride = K / 2 + 4;             // words per staged token row
-  const int W = ((N + 15) / 16) * Kb;        // (tile, block) units
+  const int RT = (N + 15) / 16;              // row tiles
+  const int W = RT * Kb;                     // (tile, block) units
   const int c = Pb.chunk;
   const int ahead = min(args.ahead, S);
   const uint32_t k2 = args.k2, k4 = args.k4;
@@ -243,6 +252,12 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   float* psx = reinterpret_cast<float*>(smem + kWarps * S * kStage + kWarps * S * 8 + 16);   // [MT][Kb+1]
   __half* xw = reinterpret_cast<__half*>(psx + ((MT * (Kb + 1) + 3) & ~3));                        // [MT][k_ld]
   uint32_t* xs = reinterpret_cast<uint32_t*>(xw + MT * k_ld);                                      // [M][xstride]
+  // row tiles whose segments are all in this CTA: accumulators [lt][16][MT] and segment counts
+  const int lcap = Pb.lt_cap;
+  float* lacc = reinterpret_cast<float*>(xs + (XSMEM ? M * xstride : 0));
+  int* lcnt = reinterpret_cast<int*>(lacc + lcap * 16 * MT);
+  const int cta_c0 = ((int)blockIdx.x - Pb.cta_base) * kWarps;   // first chunk of this CTA
+  const int t_lo = min(cta_c0 * c, W) / Kb;                        // first tile it touches
 
   // this warp's chunk of units
   const int wi = ((int)blockIdx.x - Pb.cta_base) * kWarps + warp;
@@ -283,6 +298,11 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   if (lane == 0) {
     for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
+  }
+  for (int e = threadIdx.x; e < lcap * 16 * MT; e += blockDim.x) lacc[e] = 0.f;
+  for (int lt = threadIdx.x; lt < lcap; lt += blockDim.x) {
+    const int t = t_lo + lt, cf = (t * Kb) / c, cl = ((t + 1) * Kb - 1) / c;
+    lcnt[lt] = (t < RT && cl > cf && cf >= cta_c0 && cl < cta_c0 + kWarps) ? cl - cf + 1 : 0;
   }
   // the weak-column indices are static: fetch this thread's before waiting for the previous
   // kernel (gather elements e = threadIdx.x + it * blockDim.x, it < 2, of [MT][k_ld])
@@ -557,6 +577,30 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
               if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(y[nt][i]);
             }
         }
+      } else if (rt - t_lo < lcap && c_first >= cta_c0 && c_first + nseg <= cta_c0 + kWarps) {
+        // every segment of this tile is in this CTA: add into its shared accumulator; the last
+        // segment to arrive stores the tile
+        float* acc = lacc + (rt - t_lo) * 16 * MT;
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i)
+            atomicAdd(acc + (g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1), y[nt][i]);
+        __syncwarp();   // the warp's adds precede lane 0's release
+        int old = 0;
+        if (lane == 0) old = count_down_cta(&lcnt[rt - t_lo]);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == 1 && ok) {
+          __syncwarp();
+          #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
+              const float v = acc[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)];
+              if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(v);
+            }
+        }
       } else if (seg_b1 == Kb) {
         // this segment holds the tile's last unit: this warp finishes the tile once its own
         // chunk is done, reading the other segments (lower chunks, earlier CTAs)
@@ -711,6 +755,7 @@ void plan(GemvArgs& a, int warps_per_cta) {
     chunk = max(chunk, max(kGemvMinChunk, (Kb - 1) / (Pq.seg_cap - 1) + 1));
     const int nchunks = (int)((work[q] + chunk - 1) / chunk);
     Pq.chunk = chunk;
+    Pq.lt_cap = (warps_per_cta * chunk - 1) / Kb + 2;
     Pq.ncta = min(n[q], (nchunks + warps_per_cta - 1) / warps_per_cta);
     Pq.cta_base = base;
     base += Pq.ncta;
@@ -735,10 +780,23 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
     const size_t stage = sub == 8 ? Geo<BITS, 8>::stage_bytes(pg) : Geo<BITS, 4>::stage_bytes(pg);
     return (size_t)warps * S * stage + (size_t)warps * S * 8 + 16 + ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
   };
+  // the in-CTA hand-off area (accumulators and counts of the tiles one CTA touches), used when
+  // it fits beside the ring
+  auto local_bytes = [&]() {
+    size_t b = 0;
+    for (int q = 0; q < a.count; ++q)
+      b = std::max(b, (size_t)a.p[q].lt_cap * 16 * MT * sizeof(float) + (size_t)((a.p[q].lt_cap + 3) & ~3) * sizeof(int));
+    return b;
+  };
 #define OWQ_TRY(W, SUB, S, XS)                                                           \
   if (smem_for(W, SUB, S, XS) <= kMaxSmem) {                                             \
     plan(a, W);                                                                          \
-    return launch_k<BITS, NT, W, SUB, S, XS>(a, smem_for(W, SUB, S, XS), s);            \
+    size_t sm = smem_for(W, SUB, S, XS) + local_bytes();                                 \
+    if (sm > kMaxSmem) {                                                                 \
+      for (int q = 0; q < a.count; ++q) a.p[q].lt_cap = 0;                               \
+      sm = smem_for(W, SUB, S, XS);                                                      \
+    }                                                                                    \
+    return launch_k<BITS, NT, W, SUB, S, XS>(a, sm, s);                                 \
   }
   // 16 warps with the activations in shared memory: larger items first, then deeper rings
   OWQ_TRY(16, 8, 2, true)

@@ -78,6 +78,7 @@ struct GemvProblem {
   int cta_base;       // first CTA of this problem
   int ncta;           // CTAs serving this problem
   int chunk;          // (row tile, block) units per warp
+  int lt_cap;         // row tiles one CTA's chunks touch, if their in-CTA hand-off fits in shared memory (else 0)
 };
 // Decode work split: each warp of the grid (kGemvWarps per SM) takes an equal contiguous chunk
 // of the (16-row tile, 128-code block) units, never fewer than kGemvMinChunk.  A row tile is
