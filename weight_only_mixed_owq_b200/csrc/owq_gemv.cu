@@ -59,11 +59,6 @@ struct Geo {
   static constexpr int stage_bytes(bool pg) { return kStageW + (pg ? SUB * 64 : 0); }
 };
 
-__device__ __forceinline__ uint32_t ldg_u32(const void* p) {
-  uint32_t r;
-  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
-}
 __device__ __forceinline__ uint4 ldg_u128(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
@@ -300,9 +295,9 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     fence_mbar_init();
   }
   for (int e = threadIdx.x; e < lcap * 16 * MT; e += blockDim.x) lacc[e] = 0.f;
-  for (int lt = threadIdx.x; lt < lcap; lt += blockDim.x) {
+  for (int lt = threadIdx.x; lt < lcap; lt += blockDim.x) {   // segments of each split tile in this CTA
     const int t = t_lo + lt, cf = (t * Kb) / c, cl = ((t + 1) * Kb - 1) / c;
-    lcnt[lt] = (t < RT && cl > cf && cf >= cta_c0 && cl < cta_c0 + kWarps) ? cl - cf + 1 : 0;
+    lcnt[lt] = (t < RT && cl > cf) ? max(0, min(cl, cta_c0 + kWarps - 1) - max(cf, cta_c0) + 1) : 0;
   }
   // the weak-column indices are static: fetch this thread's before waiting for the previous
   // kernel (gather elements e = threadIdx.x + it * blockDim.x, it < 2, of [MT][k_ld])
@@ -577,9 +572,11 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
               if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(y[nt][i]);
             }
         }
-      } else if (rt - t_lo < lcap && c_first >= cta_c0 && c_first + nseg <= cta_c0 + kWarps) {
-        // every segment of this tile is in this CTA: add into its shared accumulator; the last
-        // segment to arrive stores the tile
+      } else if (lcap > 0) {
+        // split tile, two-level hand-off: the segments in this CTA add into a shared
+        // accumulator; the last of them stores the tile (all segments here), publishes this
+        // CTA's partial (a higher CTA holds the tile's last units), or adds the lower CTAs'
+        // partials (bounded wait on the epoch tag, CTA order) and stores the tile
         float* acc = lacc + (rt - t_lo) * 16 * MT;
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -590,16 +587,62 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         int old = 0;
         if (lane == 0) old = count_down_cta(&lcnt[rt - t_lo]);
         old = __shfl_sync(0xffffffffu, old, 0);
-        if (old == 1 && ok) {
+        if (old == 1) {
           __syncwarp();
+          float v[NT][4];
           #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
             #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int row = rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
-              const float v = acc[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)];
-              if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(v);
+            for (int i = 0; i < 4; ++i) v[nt][i] = acc[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)];
+          const int jf = c_first / kWarps, jl = (c_first + nseg - 1) / kWarps, j = cta_c0 / kWarps;
+          const unsigned long long* pt = Pb.part + (size_t)rt * (Pb.seg_cap - 1) * 256;
+          if (j < jl) {
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              #pragma unroll
+              for (int i = 0; i < 4; ++i)
+                st_tagged(const_cast<unsigned long long*>(pt) + (j - jf) * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1),
+                          v[nt][i], Pb.epoch);
+          } else {
+            float tot[NT][4];
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              #pragma unroll
+              for (int i = 0; i < 4; ++i) tot[nt][i] = 0.f;
+            bool good = ok;
+            #pragma unroll 1
+            for (int s2 = 0; s2 < j - jf && good; ++s2) {
+              unsigned long long w[NT][4];
+              #pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) w[nt][i] = ld_tagged(pt + s2 * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1));
+              const long long t_start = clock64();
+              #pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  while ((uint32_t)(w[nt][i] >> 32) != Pb.epoch) {
+                    if (clock64() - t_start > kWaitLimit) {
+                      atomicExch(args.status, 1);
+                      good = false;
+                      break;
+                    }
+                    w[nt][i] = ld_tagged(pt + s2 * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1));
+                  }
+                  tot[nt][i] += __uint_as_float((uint32_t)w[nt][i]);
+                }
             }
+            if (good) {
+              #pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int row = rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
+                  if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(tot[nt][i] + v[nt][i]);
+                }
+            }
+          }
         }
       } else if (seg_b1 == Kb) {
         // this segment holds the tile's last unit: this warp finishes the tile once its own
