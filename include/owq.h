@@ -51,6 +51,12 @@ typedef int owq_status_t;
 #define OWQ_ERR_NOMEM     9   /* a device or host allocation failed                           */
 #define OWQ_ERR_HANDLE    10  /* the layer handle is NULL or not one this library made         */
 #define OWQ_ERR_DEVICE    11  /* no CUDA device, or the device is not sm_100                   */
+#define OWQ_ERR_ARG       12  /* an argument outside its documented set (owq_debug_inject)      */
+
+/* Failures owq_debug_inject can arm. */
+#define OWQ_INJECT_NONE         0
+#define OWQ_INJECT_GEMV_TAG     1
+#define OWQ_INJECT_GEMM_ARRIVE  2
 
 /* Opaque handle of one packed layer; owns the device buffers owq_pack allocated. */
 typedef struct owq_layer_s* owq_layer_t;
@@ -194,6 +200,25 @@ owq_status_t owq_layer_free(owq_layer_t layer);
 /* Synchronises the device, then returns and clears the device status word that bounded
  * waits set (OWQ_OK, or OWQ_ERR_TIMEOUT). */
 owq_status_t owq_device_status(void);
+
+/*
+ * owq_debug_inject -- test hook for the bounded-wait error path (host only, process-wide,
+ * not thread-safe).  Arms one injected failure, consumed by the next call of its kind:
+ *   OWQ_INJECT_GEMV_TAG     next owq_gemv / owq_gemv_multi: the partial sums of row tiles that
+ *                           are split across CTAs are published under a tag no reader accepts,
+ *                           so each cross-CTA wait runs out and its tile is not written (a
+ *                           layer whose tiles all stay inside one CTA has no such wait);
+ *   OWQ_INJECT_GEMM_ARRIVE  next owq_gemm: one dequantisation thread of every CTA skips its
+ *                           arrival for its first K step, so the MMA issuer's wait runs out,
+ *                           then the producer's and the dequantisation threads' waits.
+ * wait_cycles (>= 1) bounds every device wait of that call, in SM clock cycles (otherwise the
+ * bound is 4e9 cycles, about 2 s).  The kernel records the timeout in the device status
+ * word, leaves y undefined, lets its own bulk copies land, frees its tensor memory and
+ * returns: the next owq_device_status returns OWQ_ERR_TIMEOUT and the context stays usable.
+ * OWQ_INJECT_NONE disarms (wait_cycles ignored).  Errors: OWQ_ERR_ARG for an unknown `what`
+ * or wait_cycles < 1.
+ */
+owq_status_t owq_debug_inject(int what, long long wait_cycles);
 
 /* Static, human-readable name of a status code. */
 const char* owq_status_string(owq_status_t status);

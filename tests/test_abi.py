@@ -74,6 +74,11 @@ def test_host_validation_rejects_bad_arguments(owq):
     assert owq.owq_layer_free(None) == 0
     assert owq.owq_layer_info(A)[0] == 10
     assert owq.owq_layer_bytes(A)[0] == 10
+    # fault-injection hook: unknown kinds and empty wait bounds are refused
+    assert owq.owq_debug_inject(3, 1000) == 12
+    assert owq.owq_debug_inject(-1, 1000) == 12
+    assert owq.owq_debug_inject(owq.OWQ_INJECT_GEMV_TAG, 0) == 12
+    assert owq.owq_debug_inject(owq.OWQ_INJECT_NONE, 0) == 0
 
 
 @pytest.mark.skipif(_gpu_present(), reason="checks the no-device path; needs a machine without a GPU")

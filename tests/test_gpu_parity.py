@@ -196,3 +196,26 @@ def test_gpu_error_paths(owq):
     assert owq.owq_gemv(layer.handle, x[:, 1:], y, 1) == 6
     layer.close()
     assert owq.owq_gemv(layer.handle or 0, x, y, 1) == 10
+
+
+# Shapes whose row tiles are split inside CTAs and across CTAs in the decode launch (N x K,
+# bits, group, k): every partial sum is added in a fixed order, so repeated calls agree bit
+# for bit.
+DETERMINISM_SHAPES = [(4096, 11008, 4, 128, 86), (16384, 4096, 3, 4096, 32), (4096, 4096, 3, 4096, 32)]
+
+
+@pytest.mark.parametrize("shape", DETERMINISM_SHAPES, ids=[f"{s[0]}x{s[1]}" for s in DETERMINISM_SHAPES])
+def test_repeated_calls_are_bit_identical(owq, shape):
+    N, K, bits, group, k = shape
+    d = owq_synth.draw_small(N, K, 64, 64, seed=300 + bits)
+    layer, _ = owq.quantize_pack(_gpu(d["W"]), _gpu(d["X"]), bits, group, k)
+    x = _gpu(d["x"])
+    for M in (1, 5, 9, 16):
+        xm = x[:M].contiguous()
+        y0 = layer.gemv(xm)
+        for _ in range(3):
+            assert torch.equal(layer.gemv(xm).view(torch.int16), y0.view(torch.int16)), M
+    y0 = layer.gemm(x)
+    assert torch.equal(layer.gemm(x).view(torch.int16), y0.view(torch.int16))
+    assert owq.owq_device_status() == 0
+    layer.close()

@@ -16,8 +16,9 @@ OWQ_OK = 0
 STATUS_NAMES = {
     0: "OWQ_OK", 1: "OWQ_ERR_NULL", 2: "OWQ_ERR_SHAPE", 3: "OWQ_ERR_BITS", 4: "OWQ_ERR_GROUP",
     5: "OWQ_ERR_INDEX", 6: "OWQ_ERR_ALIGN", 7: "OWQ_ERR_CUDA", 8: "OWQ_ERR_TIMEOUT",
-    9: "OWQ_ERR_NOMEM", 10: "OWQ_ERR_HANDLE", 11: "OWQ_ERR_DEVICE",
+    9: "OWQ_ERR_NOMEM", 10: "OWQ_ERR_HANDLE", 11: "OWQ_ERR_DEVICE", 12: "OWQ_ERR_ARG",
 }
+OWQ_INJECT_NONE, OWQ_INJECT_GEMV_TAG, OWQ_INJECT_GEMM_ARRIVE = 0, 1, 2
 
 # (name, restype, argtypes) of every exported symbol of include/owq.h
 _P, _I, _SZ, _S = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t), ctypes.c_char_p
@@ -33,6 +34,7 @@ PROTOTYPES = [
     ("owq_layer_bytes", _I, [_P, _SZ, _SZ, _SZ, _SZ]),
     ("owq_layer_free", _I, [_P]),
     ("owq_device_status", _I, []),
+    ("owq_debug_inject", _I, [_I, ctypes.c_longlong]),
     ("owq_status_string", _S, [_I]),
     ("owq_version", _S, []),
 ]
@@ -143,6 +145,10 @@ def owq_layer_free(layer) -> int:
 
 def owq_device_status() -> int:
     return LIB.owq_device_status()
+
+
+def owq_debug_inject(what: int, wait_cycles: int) -> int:
+    return LIB.owq_debug_inject(what, wait_cycles)
 
 
 def owq_status_string(st: int) -> str:

@@ -98,6 +98,7 @@ const char* owq_status_string(owq_status_t s) {
     case OWQ_ERR_NOMEM: return "OWQ_ERR_NOMEM: allocation failed";
     case OWQ_ERR_HANDLE: return "OWQ_ERR_HANDLE: not a live layer handle";
     case OWQ_ERR_DEVICE: return "OWQ_ERR_DEVICE: no sm_100 CUDA device";
+    case OWQ_ERR_ARG: return "OWQ_ERR_ARG: argument outside its documented set";
     default: return "OWQ: unknown status";
   }
 }
@@ -228,6 +229,27 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   return OWQ_OK;
 }
 
+// one armed test failure (owq_debug_inject), taken by the next call of its kind
+static int g_inject = OWQ_INJECT_NONE;
+static long long g_inject_wait = kDefaultWaitLimit;
+
+// wait bound of this call; true if the armed failure is of kind `what` (then disarmed)
+static bool take_inject(int what, long long* wait_limit) {
+  *wait_limit = kDefaultWaitLimit;
+  if (g_inject != what) return false;
+  *wait_limit = g_inject_wait;
+  g_inject = OWQ_INJECT_NONE;
+  return true;
+}
+
+owq_status_t owq_debug_inject(int what, long long wait_cycles) {
+  if (what == OWQ_INJECT_NONE) { g_inject = what; return OWQ_OK; }
+  if ((what != OWQ_INJECT_GEMV_TAG && what != OWQ_INJECT_GEMM_ARRIVE) || wait_cycles < 1) return OWQ_ERR_ARG;
+  g_inject = what;
+  g_inject_wait = wait_cycles;
+  return OWQ_OK;
+}
+
 static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvProblem* P) {
   if (!x || !y) return OWQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(y)) return OWQ_ERR_ALIGN;
@@ -242,6 +264,7 @@ static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvP
   P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->xfrag = L->xfrag; P->part = L->part; P->seg_cap = L->seg_cap;
   if (++L->epoch == 0) ++L->epoch;   // 0 marks the zeroed workspace
   P->epoch = L->epoch;
+  P->wtag = L->epoch;
   P->row_groups = 0; P->cta_base = 0; P->ncta = 0; P->chunk = 0; P->lt_cap = 0;
   return OWQ_OK;
 }
@@ -253,7 +276,9 @@ owq_status_t owq_gemv(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, 
   GemvProblem P;
   owq_status_t st = make_problem(L, x, y, &P);
   if (st) return st;
-  return cuda_status(launch_gemv(&P, 1, L->bits, M, reinterpret_cast<cudaStream_t>(stream)));
+  long long wl;
+  if (take_inject(OWQ_INJECT_GEMV_TAG, &wl)) P.wtag = 0;
+  return cuda_status(launch_gemv(&P, 1, L->bits, M, wl, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs, uint16_t* const* ys,
@@ -272,7 +297,10 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
     owq_status_t st = make_problem(L, xs[q], ys[q], &P[q]);
     if (st) return st;
   }
-  return cuda_status(launch_gemv(P, count, bits, M, reinterpret_cast<cudaStream_t>(stream)));
+  long long wl;
+  if (take_inject(OWQ_INJECT_GEMV_TAG, &wl))
+    for (int q = 0; q < count; ++q) P[q].wtag = 0;
+  return cuda_status(launch_gemv(P, count, bits, M, wl, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, owq_stream_t stream) {
@@ -281,7 +309,9 @@ owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, 
   if (M < 1 || M > 65536) return OWQ_ERR_SHAPE;
   if (!x || !y) return OWQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(y)) return OWQ_ERR_ALIGN;
-  return gemm_sm100(*L, reinterpret_cast<const __half*>(x), reinterpret_cast<__half*>(y), M,
+  long long wl;
+  const bool skip = take_inject(OWQ_INJECT_GEMM_ARRIVE, &wl);
+  return gemm_sm100(*L, reinterpret_cast<const __half*>(x), reinterpret_cast<__half*>(y), M, wl, skip,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -39,7 +39,6 @@ constexpr int kBM = 128;               // weight rows per tile (MMA M)
 constexpr int kStepCodes = 128;        // K per pipeline step
 constexpr int kDequantWarps = 8;
 constexpr int kThreads = 32 * (2 + kDequantWarps);
-constexpr long long kWaitLimit = 4000000000LL;  // ~2 s at 2 GHz
 
 template <int BITS, int BN>
 struct Smem {
@@ -63,6 +62,8 @@ struct GemmParams {
   int* status;
   int N, K, M, G, k_ld;
   int ksteps;       // 128-code steps per split (blockIdx.z)
+  long long wait_limit;   // bound of every mbarrier wait, in SM clock cycles
+  int skip_arrive;  // test-injected lost arrival: dequantisation thread 0 skips its first one
 };
 
 // fp16x2 helpers (exact integer arithmetic on small values)
@@ -140,9 +141,10 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       // ---------------- TMA producer ----------------
       constexpr uint32_t kBytes = L::kX + L::kP;
       bool ok = true;
+      int issued = 0;
       for (int i = 0; i < nK && ok; ++i) {
         const int kb = kb0 + i, s = i % S, u = i / S;
-        if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, p.status, kWaitLimit);
+        if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, p.status, p.wait_limit);
         if (!ok) break;
         unsigned char* st = smem + s * L::kStage;
         mbar_arrive_expect_tx(&full[s], kBytes);
@@ -150,10 +152,11 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         tma_load_3d(st + L::kX + L::kA, &map_p, &full[s], 0, kb, n0 / 16);
         tma_load_2d(st, &map_x, &full[s], kb * kStepCodes, m0);
         tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
+        issued = i + 1;
       }
-      // never leave with copies in flight: wait for the last use of every stage
-      for (int i = (nK > S ? nK - S : 0); i < nK; ++i)
-        mbar_wait(&full[i % S], (i / S) & 1, p.status, kWaitLimit);
+      // never leave with copies in flight: wait for the last issued use of every stage
+      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait(&full[i % S], (i / S) & 1, p.status, p.wait_limit);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -162,8 +165,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       bool ok = true;
       for (int i = 0; i < nK && ok; ++i) {
         const int s = i % S, u = i / S;
-        ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit) &&
-             mbar_wait(&afull[s], u & 1, p.status, kWaitLimit);
+        ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit) &&
+             mbar_wait(&afull[s], u & 1, p.status, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
         unsigned char* st = smem + s * L::kStage;
@@ -232,7 +235,7 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       const int wc[4] = {wcol0, wcol1, wcol2, wcol3};
       const __half wv[4] = {wval0, wval1, wval2, wval3};
       if (i + 1 < nK) OWQ_FETCH_WEAK(kb + 1)
-      ok = mbar_wait(&full[s], u & 1, p.status, kWaitLimit);
+      ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);
       if (!ok) break;
       unsigned char* st = smem + s * L::kStage;
       const uint4* pw = reinterpret_cast<const uint4*>(st + L::kX + L::kA + r * 16 * BITS);
@@ -268,13 +271,13 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         *(reinterpret_cast<__half*>(slab + sw128_off(r, (col >> 3) & 7)) + (col & 7)) = p.w_weak[(size_t)row * p.k_ld + t];
       }
       fence_proxy_async_smem();
-      mbar_arrive(&afull[s]);
+      if (!(p.skip_arrive && i == 0 && td == 0)) mbar_arrive(&afull[s]);
     }
 #undef OWQ_FETCH_WEAK
 
     // ---------------- epilogue ----------------
     const int wd = warp - 2, q = warp & 3, chalf = wd >> 2;
-    const bool acc_ok = mbar_wait(accf, 0, p.status, kWaitLimit);
+    const bool acc_ok = mbar_wait(accf, 0, p.status, p.wait_limit);
     tc_fence_after();
     const int orow = n0 + 32 * q + lane;
     #pragma unroll 1
@@ -363,7 +366,8 @@ bool encode_packed_3d(CUtensorMap* m, const void* base, int K, int N, int bits) 
 }
 
 template <int BITS, int BN, int S>
-owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
+owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_limit, bool skip_arrive,
+                 cudaStream_t s) {
   if (!L.maps_ready) {
     if (!encode_packed_3d(&L.map_packed, L.packed, L.K, L.N, BITS)) return OWQ_ERR_CUDA;
     L.maps_ready = true;
@@ -376,6 +380,7 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
   prm.scales = L.scales; prm.zeros = L.zeros; prm.w_weak = L.w_weak; prm.idx = L.idx;
   prm.blk_weak = L.blk_weak; prm.y = y; prm.status = device_status_ptr();
   prm.N = L.N; prm.K = L.K; prm.M = M; prm.G = L.G; prm.k_ld = L.k_ld;
+  prm.wait_limit = wait_limit; prm.skip_arrive = skip_arrive ? 1 : 0;
   if (!prm.status) return OWQ_ERR_CUDA;
   // fewer tiles than SMs: split K over CTAs (at least 4 steps each), fp32 partials in the
   // layer's workspace, then one reduction kernel; never grown during stream capture
@@ -436,18 +441,20 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
 }
 
 template <int BITS>
-owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
+owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, long long wl, bool skip, cudaStream_t s) {
   // wider token tiles dequantise each weight tile once for more tokens (the dequantisation,
   // not the MMA, bounds the narrower tiles); the widest one fits two stages
-  if (M <= 64) return run<BITS, 64, 4>(L, x, y, M, s);
-  if (M <= 256) return run<BITS, 128, 3>(L, x, y, M, s);
-  return run<BITS, 256, 2>(L, x, y, M, s);
+  if (M <= 64) return run<BITS, 64, 4>(L, x, y, M, wl, skip, s);
+  if (M <= 256) return run<BITS, 128, 3>(L, x, y, M, wl, skip, s);
+  return run<BITS, 256, 2>(L, x, y, M, wl, skip, s);
 }
 
 }  // namespace
 
-owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, cudaStream_t s) {
-  return L.bits == 3 ? dispatch<3>(L, x, y, M, s) : dispatch<4>(L, x, y, M, s);
+owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, long long wait_limit,
+                        bool skip_arrive, cudaStream_t s) {
+  return L.bits == 3 ? dispatch<3>(L, x, y, M, wait_limit, skip_arrive, s)
+                     : dispatch<4>(L, x, y, M, wait_limit, skip_arrive, s);
 }
 
 }  // namespace owq

@@ -24,9 +24,13 @@
 //        sum_j s (q_j - z) x_j = s * (sum_j q_j x_j - z * sum_j x_j);
 //    the activation sums come from per-block prefix sums computed once per CTA.  (The fp16
 //    rounding of each s (q - z) is not applied; the difference is far inside the tolerance.)
-//  * A row tile split between warps is finished by the warp holding its last unit, once that
-//    warp's own chunk is done: it adds the other segments' partial sums (tagged with the call's
-//    epoch, so they need no counter or fence) in segment order, then its own (deterministic).
+//  * A row tile split between warps: the segments inside one CTA leave their partial sums in
+//    shared memory and the last to arrive (a CTA-scope counter) adds them in unit order; across
+//    CTAs, each CTA's sum is published as 64-bit words tagged with the call's epoch (no counter
+//    or fence) and the CTA holding the tile's last units adds them in CTA order.  Without room
+//    for the in-CTA area, each segment is published the same way and the warp holding the last
+//    unit adds them in segment order.  Every sum runs in a fixed order: the output is the same
+//    bit for bit on every call.
 #include "owq_format.cuh"
 #include "owq_internal.cuh"
 #include "owq_sm100.cuh"
@@ -38,7 +42,6 @@ using namespace sm100;
 
 constexpr int kMaxProblems = 16;
 constexpr int kAhead = 2;                        // items in flight per warp (see GemvArgs::ahead)
-constexpr long long kWaitLimit = 4000000000LL;  // ~2 s
 
 struct GemvArgs {
   GemvProblem p[kMaxProblems];
@@ -47,6 +50,7 @@ struct GemvArgs {
   int ahead;     // ring items a warp keeps in flight beyond the one it is reading (1 .. S)
   uint32_t k2, k4;   // 2 and 4 (run-time values: see pair_bits)
   int* status;   // device status word (bounded waits)
+  long long wait_limit;   // bound of every device wait, in SM clock cycles
 };
 
 template <int BITS, int SUB>   // SUB: blocks per ring item
@@ -294,7 +298,6 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
     fence_mbar_init();
   }
-  for (int e = threadIdx.x; e < lcap * 16 * MT; e += blockDim.x) lacc[e] = 0.f;
   for (int lt = threadIdx.x; lt < lcap; lt += blockDim.x) {   // segments of each split tile in this CTA
     const int t = t_lo + lt, cf = (t * Kb) / c, cl = ((t + 1) * Kb - 1) / c;
     lcnt[lt] = (t < RT && cl > cf) ? max(0, min(cl, cta_c0 + kWarps - 1) - max(cf, cta_c0) + 1) : 0;
@@ -480,7 +483,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       }
     }
     if (ok) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], phase, args.status, kWaitLimit));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], phase, args.status, args.wait_limit));
       if (!ok) failed_at = consumed;
     }
     const int fa = fa0 + st * kStage;
@@ -573,17 +576,20 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
             }
         }
       } else if (lcap > 0) {
-        // split tile, two-level hand-off: the segments in this CTA add into a shared
-        // accumulator; the last of them stores the tile (all segments here), publishes this
-        // CTA's partial (a higher CTA holds the tile's last units), or adds the lower CTAs'
-        // partials (bounded wait on the epoch tag, CTA order) and stores the tile
-        float* acc = lacc + (rt - t_lo) * 16 * MT;
+        // split tile, two-level hand-off.  Each segment in this CTA leaves its partial in shared
+        // memory: the tile's lowest segment, when its warp walks it first (the warp's chunk
+        // reaches below the tile), in the tile's slot; every other segment is the last one its
+        // warp walks, so in that warp's ring, idle from then on.  The last segment to arrive
+        // adds them in unit order (the same order every call), then stores the tile (all its
+        // segments are here), publishes this CTA's partial (a higher CTA holds the tile's last
+        // units), or adds the lower CTAs' partials (bounded wait on the tag, CTA order)
+        float* slot = lacc + (rt - t_lo) * 16 * MT;
+        float* mine = lo < t0 ? slot : reinterpret_cast<float*>(ring);
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            atomicAdd(acc + (g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1), y[nt][i]);
-        __syncwarp();   // the warp's adds precede lane 0's release
+          for (int i = 0; i < 4; ++i) mine[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
+        __syncwarp();   // the warp's stores precede lane 0's release
         int old = 0;
         if (lane == 0) old = count_down_cta(&lcnt[rt - t_lo]);
         old = __shfl_sync(0xffffffffu, old, 0);
@@ -593,7 +599,17 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
             #pragma unroll
-            for (int i = 0; i < 4; ++i) v[nt][i] = acc[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)];
+            for (int i = 0; i < 4; ++i) v[nt][i] = 0.f;
+          const int cw0 = max(c_first, cta_c0), cw1 = min(c_first + nseg - 1, cta_c0 + kWarps - 1);
+          #pragma unroll 1
+          for (int cw = cw0; cw <= cw1; ++cw) {
+            const float* src = (cw == c_first && c_first * c < t0)
+                                   ? slot : reinterpret_cast<const float*>(smem + (cw - cta_c0) * S * kStage);
+            #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              #pragma unroll
+              for (int i = 0; i < 4; ++i) v[nt][i] += src[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)];
+          }
           const int jf = c_first / kWarps, jl = (c_first + nseg - 1) / kWarps, j = cta_c0 / kWarps;
           const unsigned long long* pt = Pb.part + (size_t)rt * (Pb.seg_cap - 1) * 256;
           if (j < jl) {
@@ -602,7 +618,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
               #pragma unroll
               for (int i = 0; i < 4; ++i)
                 st_tagged(const_cast<unsigned long long*>(pt) + (j - jf) * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1),
-                          v[nt][i], Pb.epoch);
+                          v[nt][i], Pb.wtag);
           } else {
             float tot[NT][4];
             #pragma unroll
@@ -623,7 +639,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
                 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   while ((uint32_t)(w[nt][i] >> 32) != Pb.epoch) {
-                    if (clock64() - t_start > kWaitLimit) {
+                    if (clock64() - t_start > args.wait_limit) {
                       atomicExch(args.status, 1);
                       good = false;
                       break;
@@ -661,7 +677,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
           for (int i = 0; i < 4; ++i)
-            st_tagged(part + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1), y[nt][i], Pb.epoch);
+            st_tagged(part + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1), y[nt][i], Pb.wtag);
       }
       #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -693,7 +709,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
           while ((uint32_t)(w[nt][i] >> 32) != Pb.epoch) {
-            if (clock64() - t_start > kWaitLimit) {
+            if (clock64() - t_start > args.wait_limit) {
               atomicExch(args.status, 1);
               good = false;
               break;
@@ -716,7 +732,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   // after a timeout: never exit with bulk copies still writing into this CTA's memory
   if (failed_at >= 0 && lane == 0)
     for (int j = failed_at; j < issued; ++j)
-      mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1), args.status, kWaitLimit);
+      mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1), args.status, args.wait_limit);
 }
 
 int sm_count() {
@@ -867,13 +883,14 @@ cudaError_t launch_bits(GemvArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cudaStream_t s) {
+cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, long long wait_limit,
+                        cudaStream_t s) {
   if (count < 1 || count > kMaxProblems) return cudaErrorInvalidValue;
   // one launch serves layers of one kind (per-channel or per-group scales)
   for (int q = 1; q < count; ++q)
     if ((probs[q].G > 1) != (probs[0].G > 1)) {
       for (int j = 0; j < count; ++j) {
-        cudaError_t e = launch_gemv(probs + j, 1, bits, M, s);
+        cudaError_t e = launch_gemv(probs + j, 1, bits, M, wait_limit, s);
         if (e != cudaSuccess) return e;
       }
       return cudaSuccess;
@@ -883,6 +900,7 @@ cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cu
   a.count = count;
   a.M = M;
   a.status = device_status_ptr();
+  a.wait_limit = wait_limit;
   a.ahead = kAhead;
   a.k2 = 2u;
   a.k4 = 4u;

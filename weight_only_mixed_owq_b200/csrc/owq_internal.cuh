@@ -51,6 +51,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Device status word set by bounded waits (owq_device_status reads and clears it).
 int* device_status_ptr();
+// Bound of a device wait when no test shortens it: about 2 s at the B200's clock.
+constexpr long long kDefaultWaitLimit = 4000000000LL;
 
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_pack(const uint8_t* codes, const __half* zeros, const uint32_t* weak_mask,
@@ -74,6 +76,8 @@ struct GemvProblem {
   unsigned long long* part;  // tagged partial sums of split row tiles
   int seg_cap;               // warps that may share a row tile (seg_cap - 1 slots per tile)
   uint32_t epoch;            // tag of this call's partial sums (never 0)
+  uint32_t wtag;             // tag the partial sums are published under: epoch (0 only when a
+                             // test injects a lost hand-off)
   int row_groups;     // 16-row tiles
   int cta_base;       // first CTA of this problem
   int ncta;           // CTAs serving this problem
@@ -91,12 +95,16 @@ inline int gemv_seg_cap(int N, int K, int sm_count) {
   const int cmin = (int)std::max<long long>(kGemvMinChunk, (units + warps - 1) / warps);
   return (K / kBlockCodes - 1) / cmin + 2;
 }
-cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, cudaStream_t s);
+cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, long long wait_limit,
+                        cudaStream_t s);
 
 cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int T, int bits,
                             int group, int k, uint8_t* codes, __half* scales, __half* zeros,
                             int32_t* idx, __half* w_weak, cudaStream_t s);
 
-owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, cudaStream_t s);
+// skip_arrive: a test-injected lost arrival (one dequantisation thread per CTA skips its first
+// arrival), so that the bounded waits run out
+owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, long long wait_limit,
+                        bool skip_arrive, cudaStream_t s);
 
 }  // namespace owq
