@@ -61,7 +61,10 @@ def dist_setup():
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        # a short timeout: a rank that dies or never joins ends the others' next collective
+        # with an error instead of a wait
+        secs = float(os.environ.get("OWQ_PG_TIMEOUT_S", "120"))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=secs))
     return rank, world, local
 
 

@@ -84,3 +84,52 @@ def test_reference_arm_line_shape(monkeypatch):
     assert line["unit"] == "GB/s" and line["higher_is_better"] is True
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+FAILING_CHILD = textwrap.dedent(
+    """
+    import os, sys, time
+    sys.path.insert(0, {root!r})
+    import bench
+    rank, world, local = bench.dist_setup()
+    if rank == 1:
+        raise RuntimeError("rank 1 fails between steps")
+    t0 = time.time()
+    try:
+        bench.barrier(world)
+    except Exception as e:
+        print("collective-error after %.1f s: %s" % (time.time() - t0, type(e).__name__))
+        sys.exit(3)
+    print("no error")
+    """
+)
+
+
+def _launch(script, ranks, world, port, timeout_s):
+    procs = {}
+    for r in ranks:
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(world),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="",
+                   OWQ_PG_TIMEOUT_S=str(timeout_s))
+        procs[r] = subprocess.Popen([sys.executable, str(script)], env=env,
+                                    stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+    return procs
+
+
+def test_a_rank_that_raises_ends_the_others_collective_with_an_error(tmp_path):
+    script = tmp_path / "failing.py"
+    script.write_text(FAILING_CHILD.format(root=ROOT))
+    procs = _launch(script, (0, 1), 2, _free_port(), 10)
+    out = {r: p.communicate(timeout=120) for r, p in procs.items()}
+    assert procs[1].returncode != 0 and "rank 1 fails" in out[1][1]
+    assert procs[0].returncode == 3, out[0]
+    assert "collective-error" in out[0][0]
+
+
+def test_a_rank_that_never_joins_ends_set_up_with_an_error(tmp_path):
+    script = tmp_path / "failing.py"
+    script.write_text(FAILING_CHILD.format(root=ROOT))
+    procs = _launch(script, (0,), 2, _free_port(), 5)   # rank 1 is never started
+    o, e = procs[0].communicate(timeout=120)
+    assert procs[0].returncode != 0
+    assert "no error" not in o
