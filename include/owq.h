@@ -129,8 +129,8 @@ owq_status_t owq_quantize_noalloc(const uint16_t* W, const uint16_t* X, int N, i
  *   bit 15 / 31 of word e.  (A tensor-core lane's operand fragment of a block is exactly
  *   one chunk.)  The handle stores the blocks of each 16-row tile block-major (rows padded
  *   to a multiple of 16 with zero words) and, for the decode kernel, tile-major copies of
- *   the weak block and of the (scale, zero) pairs plus a split-tile workspace (about
- *   8 * 256 bytes per 16-row tile per extra warp that may share it).
+ *   the weak block and of the (scale, zero) pairs plus a split-tile workspace (2 KB per
+ *   16-row tile and per extra CTA that may share it: one for most layers, N/16 * 2 KB).
  * Synchronises `stream` once (idx is copied to the host and validated: OWQ_ERR_INDEX).
  */
 owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group,

@@ -183,8 +183,8 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
     cudaGetLastError();
     sms = 148;
   }
-  L->seg_cap = gemv_seg_cap(N, K, sms);
-  const size_t part_bytes = RT * (L->seg_cap - 1) * 16 * 16 * sizeof(unsigned long long);
+  L->cta_slots = gemv_cta_slots(N, K, sms);
+  const size_t part_bytes = RT * L->cta_slots * 16 * 16 * sizeof(unsigned long long);
   L->epoch = 0;
   alloc((void**)&L->w_weak_t, weak_t_bytes);
   alloc((void**)&L->sz_t, RT * L->G * 16 * sizeof(__half2));
@@ -261,7 +261,7 @@ static owq_status_t make_problem(Layer* L, const uint16_t* x, uint16_t* y, GemvP
   P->x = reinterpret_cast<const __half*>(x);
   P->y = reinterpret_cast<__half*>(y);
   P->N = L->N; P->K = L->K; P->G = L->G; P->k = L->k; P->k_ld = L->k_ld;
-  P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->xfrag = L->xfrag; P->part = L->part; P->seg_cap = L->seg_cap;
+  P->w_weak_t = L->w_weak_t; P->sz_t = L->sz_t; P->xfrag = L->xfrag; P->part = L->part; P->cta_slots = L->cta_slots;
   if (++L->epoch == 0) ++L->epoch;   // 0 marks the zeroed workspace
   P->epoch = L->epoch;
   P->wtag = L->epoch;

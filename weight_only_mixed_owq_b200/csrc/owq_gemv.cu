@@ -252,9 +252,13 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   __half* xw = reinterpret_cast<__half*>(psx + ((MT * (Kb + 1) + 3) & ~3));                        // [MT][k_ld]
   uint32_t* xs = reinterpret_cast<uint32_t*>(xw + MT * k_ld);                                      // [M][xstride]
   // row tiles whose segments are all in this CTA: accumulators [lt][16][MT] and segment counts
+  // split row tiles: early slots [min(lt_cap, warps)][16][MT] (indexed by tile, or by warp when
+  // the CTA touches more tiles than it has warps: a warp walks at most one early segment) and
+  // the segment counts of the tiles the CTA touches
   const int lcap = Pb.lt_cap;
+  const bool by_tile = lcap <= kWarps;
   float* lacc = reinterpret_cast<float*>(xs + (XSMEM ? M * xstride : 0));
-  int* lcnt = reinterpret_cast<int*>(lacc + lcap * 16 * MT);
+  int* lcnt = reinterpret_cast<int*>(lacc + (by_tile ? lcap : kWarps) * 16 * MT);
   const int cta_c0 = ((int)blockIdx.x - Pb.cta_base) * kWarps;   // first chunk of this CTA
   const int t_lo = min(cta_c0 * c, W) / Kb;                        // first tile it touches
 
@@ -463,8 +467,6 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     #pragma unroll
     for (int i = 0; i < 4; ++i) { Dw[nt][i] = 0.f; y[nt][i] = 0.f; }
   int seg_b1 = b_top;              // block end of the current tile segment (walking down)
-  int fin_rt = -1, fin_nseg = 0;   // split tile whose last unit this warp holds (finished at the end)
-  float fin_y[NT][4];
   int sz_rt = -1;                  // tile whose (scale, zero) pairs are in szA / szB
   __half2 szA = __halves2half2(__float2half_rn(0.f), __float2half_rn(0.f)), szB = szA;
   int st = 0;                      // stage being consumed
@@ -564,8 +566,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         for (int i = 0; i < 4; ++i) { y[nt][i] += Dw[nt][i]; Dw[nt][i] = 0.f; }
 
       const int t0 = rt * Kb;
-      const int c_first = t0 / c, nseg = (t0 + Kb - 1) / c - c_first + 1;
-      if (nseg == 1) {
+      if ((t0 + Kb - 1) / c == t0 / c) {   // the whole tile is in this chunk
         if (ok) {
           #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
@@ -575,20 +576,34 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
               if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(y[nt][i]);
             }
         }
-      } else if (lcap > 0) {
-        // split tile, two-level hand-off.  Each segment in this CTA leaves its partial in shared
-        // memory: the tile's lowest segment, when its warp walks it first (the warp's chunk
-        // reaches below the tile), in the tile's slot; every other segment is the last one its
-        // warp walks, so in that warp's ring, idle from then on.  The last segment to arrive
-        // adds them in unit order (the same order every call), then stores the tile (all its
-        // segments are here), publishes this CTA's partial (a higher CTA holds the tile's last
-        // units), or adds the lower CTAs' partials (bounded wait on the tag, CTA order)
-        float* slot = lacc + (rt - t_lo) * 16 * MT;
-        float* mine = lo < t0 ? slot : reinterpret_cast<float*>(ring);
+      } else if (lo < t0 && wi == cta_c0 + kWarps - 1) {
+        // the top segment of the CTA's top warp (walked first): all this CTA holds of a tile
+        // that a higher CTA finishes, so it is published at once, long before that CTA reaches
+        // the tile's lowest units (it walks down too)
+        unsigned long long* pt = Pb.part + ((size_t)rt * Pb.cta_slots + cta_c0 / kWarps - (t0 / c) / kWarps) * 256;
         #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
           #pragma unroll
-          for (int i = 0; i < 4; ++i) mine[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
+          for (int i = 0; i < 4; ++i)
+            st_tagged(pt + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1), y[nt][i], Pb.wtag);
+      } else {
+        // split tile, two-level hand-off.  Each segment in this CTA leaves its partial in shared
+        // memory: the tile's lowest segment, when its warp walks it first (the warp's chunk
+        // reaches below the tile), in an early slot; every other segment is the last one its
+        // warp walks, so in that warp's ring, idle from then on.  The last segment to arrive
+        // adds them in unit order (the same order every call), then stores the tile (all its
+        // segments are here), publishes this CTA's sum (a higher CTA holds the tile's last
+        // units), or adds the lower CTAs' sums (bounded wait on the tag, CTA order).
+        const int c_first = t0 / c, c_last = (t0 + Kb - 1) / c;
+        const bool early = c_first * c < t0;   // the tile's lowest segment is walked first
+        float* eslot = lacc + (by_tile ? rt - t_lo : c_first - cta_c0) * 16 * MT;
+        if (lo < t0 || failed_at < 0) {       // (after a timeout, copies may still reach the ring)
+          float* mine = lo < t0 ? eslot : reinterpret_cast<float*>(ring);
+          #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) mine[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)] = y[nt][i];
+        }
         __syncwarp();   // the warp's stores precede lane 0's release
         int old = 0;
         if (lane == 0) old = count_down_cta(&lcnt[rt - t_lo]);
@@ -600,18 +615,18 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           for (int nt = 0; nt < NT; ++nt)
             #pragma unroll
             for (int i = 0; i < 4; ++i) v[nt][i] = 0.f;
-          const int cw0 = max(c_first, cta_c0), cw1 = min(c_first + nseg - 1, cta_c0 + kWarps - 1);
+          const int cw0 = max(c_first, cta_c0), cw1 = min(c_last, cta_c0 + kWarps - 1);
           #pragma unroll 1
           for (int cw = cw0; cw <= cw1; ++cw) {
-            const float* src = (cw == c_first && c_first * c < t0)
-                                   ? slot : reinterpret_cast<const float*>(smem + (cw - cta_c0) * S * kStage);
+            const float* src = (cw == c_first && early)
+                                   ? eslot : reinterpret_cast<const float*>(smem + (cw - cta_c0) * S * kStage);
             #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
               #pragma unroll
               for (int i = 0; i < 4; ++i) v[nt][i] += src[(g + 8 * (i >> 1)) * MT + 8 * nt + 2 * tig + (i & 1)];
           }
-          const int jf = c_first / kWarps, jl = (c_first + nseg - 1) / kWarps, j = cta_c0 / kWarps;
-          const unsigned long long* pt = Pb.part + (size_t)rt * (Pb.seg_cap - 1) * 256;
+          const int jf = c_first / kWarps, jl = c_last / kWarps, j = cta_c0 / kWarps;
+          const unsigned long long* pt = Pb.part + (size_t)rt * Pb.cta_slots * 256;
           if (j < jl) {
             #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -660,73 +675,12 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
             }
           }
         }
-      } else if (seg_b1 == Kb) {
-        // this segment holds the tile's last unit: this warp finishes the tile once its own
-        // chunk is done, reading the other segments (lower chunks, earlier CTAs)
-        fin_rt = rt;
-        fin_nseg = nseg;
-        #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          #pragma unroll
-          for (int i = 0; i < 4; ++i) fin_y[nt][i] = y[nt][i];
-      } else {
-        // publish this segment's partial (segment sid < nseg - 1) and move on
-        const int sid = (t0 + seg_b0) / c - c_first;
-        unsigned long long* part = Pb.part + ((size_t)rt * (Pb.seg_cap - 1) + sid) * 256;
-        #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            st_tagged(part + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1), y[nt][i], Pb.wtag);
       }
       #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         #pragma unroll
         for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
       seg_b1 = Kb;
-    }
-  }
-  // the split tile whose last unit this warp holds: add the other segments in segment order
-  // (bounded wait for each tagged word), then this warp's own part
-  if (fin_rt >= 0 && ok) {
-    const unsigned long long* pt = Pb.part + (size_t)fin_rt * (Pb.seg_cap - 1) * 256;
-    float acc[NT][4];
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    bool good = true;
-    #pragma unroll 1
-    for (int s2 = 0; s2 < fin_nseg - 1 && good; ++s2) {
-      unsigned long long w[NT][4];
-      #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        #pragma unroll
-        for (int i = 0; i < 4; ++i) w[nt][i] = ld_tagged(pt + s2 * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1));
-      const long long t_start = clock64();
-      #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          while ((uint32_t)(w[nt][i] >> 32) != Pb.epoch) {
-            if (clock64() - t_start > args.wait_limit) {
-              atomicExch(args.status, 1);
-              good = false;
-              break;
-            }
-            w[nt][i] = ld_tagged(pt + s2 * 256 + (g + 8 * (i >> 1)) * 16 + 8 * nt + 2 * tig + (i & 1));
-          }
-          acc[nt][i] += __uint_as_float((uint32_t)w[nt][i]);
-        }
-    }
-    if (good) {
-      #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = fin_rt * 16 + g + 8 * (i >> 1), tok = 8 * nt + 2 * tig + (i & 1);
-          if (row < N && tok < M) Pb.y[(size_t)tok * N + row] = __float2half_rn(acc[nt][i] + fin_y[nt][i]);
-        }
     }
   }
   // after a timeout: never exit with bulk copies still writing into this CTA's memory
@@ -781,7 +735,7 @@ cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
 
 // CTAs per problem in proportion to its work (one resident wave in total), then an equal
 // chunk of (tile, block) units per warp: at least kGemvMinChunk, and large enough that a row
-// tile meets at most seg_cap warps (the size of the layer's partial-sum workspace)
+// tile meets at most cta_slots + 1 CTAs (the size of the layer's partial-sum workspace)
 void plan(GemvArgs& a, int warps_per_cta) {
   const int C = sm_count();
   long long work[kMaxProblems], total = 0;
@@ -811,7 +765,10 @@ void plan(GemvArgs& a, int warps_per_cta) {
     const int Kb = Pq.K / kBlockCodes;
     const long long warps = (long long)n[q] * warps_per_cta;
     int chunk = (int)((work[q] + warps - 1) / warps);
-    chunk = max(chunk, max(kGemvMinChunk, (Kb - 1) / (Pq.seg_cap - 1) + 1));
+    // at least kGemvMinChunk units, and a CTA span large enough that a tile meets at most
+    // cta_slots + 1 CTAs (the layer's workspace; the minimum already guarantees it)
+    const int span = (Kb - 1 + Pq.cta_slots - 1) / Pq.cta_slots;
+    chunk = max(chunk, max(kGemvMinChunk, (span + warps_per_cta - 1) / warps_per_cta));
     const int nchunks = (int)((work[q] + chunk - 1) / chunk);
     Pq.chunk = chunk;
     Pq.lt_cap = (warps_per_cta * chunk - 1) / Kb + 2;
@@ -839,23 +796,20 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
     const size_t stage = sub == 8 ? Geo<BITS, 8>::stage_bytes(pg) : Geo<BITS, 4>::stage_bytes(pg);
     return (size_t)warps * S * stage + (size_t)warps * S * 8 + 16 + ((extra + 15) & ~size_t(15)) + (xs ? xbytes : 0);
   };
-  // the in-CTA hand-off area (accumulators and counts of the tiles one CTA touches), used when
-  // it fits beside the ring
-  auto local_bytes = [&]() {
+  // the split-tile hand-off area: early slots and segment counters (see the kernel)
+  auto local_bytes = [&](int warps) {
     size_t b = 0;
-    for (int q = 0; q < a.count; ++q)
-      b = std::max(b, (size_t)a.p[q].lt_cap * 16 * MT * sizeof(float) + (size_t)((a.p[q].lt_cap + 3) & ~3) * sizeof(int));
+    for (int q = 0; q < a.count; ++q) {
+      const int lt = a.p[q].lt_cap;
+      b = std::max(b, (size_t)std::min(lt, warps) * 16 * MT * sizeof(float) + (size_t)((lt + 3) & ~3) * sizeof(int));
+    }
     return b;
   };
 #define OWQ_TRY(W, SUB, S, XS)                                                           \
   if (smem_for(W, SUB, S, XS) <= kMaxSmem) {                                             \
     plan(a, W);                                                                          \
-    size_t sm = smem_for(W, SUB, S, XS) + local_bytes();                                 \
-    if (sm > kMaxSmem) {                                                                 \
-      for (int q = 0; q < a.count; ++q) a.p[q].lt_cap = 0;                               \
-      sm = smem_for(W, SUB, S, XS);                                                      \
-    }                                                                                    \
-    return launch_k<BITS, NT, W, SUB, S, XS>(a, sm, s);                                 \
+    const size_t sm = smem_for(W, SUB, S, XS) + local_bytes(W);                          \
+    if (sm <= kMaxSmem) return launch_k<BITS, NT, W, SUB, S, XS>(a, sm, s);              \
   }
   // 16 warps with the activations in shared memory: larger items first, then deeper rings
   OWQ_TRY(16, 8, 2, true)

@@ -33,10 +33,11 @@ struct Layer {
   __half* w_weak_t;     // the weak block tile-major: [N/16 tiles][k_ld/16 slices][16 rows][16]
   __half2* sz_t;        // (scale, zero) pairs tile-major: [N/16 tiles][G][16 rows] (rows >= N: (0, 0))
   uint32_t* xfrag;      // decode scratch: up to 16 activation rows in fragment order (see owq_gemv.cu)
-  // decode workspace: partial sums of split row tiles, [N/16 tiles][seg_cap - 1][16 rows][16 tokens],
-  // each a 64-bit word (fp32 value | call epoch << 32); zero at pack time
+  // decode workspace: the partial sums a CTA publishes for a row tile shared with higher CTAs,
+  // [N/16 tiles][cta_slots][16 rows][16 tokens], each a 64-bit word (fp32 value | call epoch
+  // << 32); zero at pack time
   unsigned long long* part;
-  int seg_cap;          // most warps that may share one row tile in the decode product
+  int cta_slots;        // most CTAs below the one finishing a row tile in the decode product
   uint32_t epoch;       // decode calls made on this handle (tags the partial sums of each call)
   cudaStream_t stream;  // stream of owq_pack (used to order the release)
   float* gemm_ws;       // prefill split-K partial sums (grown on first need, outside capture)
@@ -74,7 +75,7 @@ struct GemvProblem {
   const __half2* sz_t;      // tile-major (scale, zero) pairs
   uint32_t* xfrag;          // activations in fragment order (when they do not fit in shared memory)
   unsigned long long* part;  // tagged partial sums of split row tiles
-  int seg_cap;               // warps that may share a row tile (seg_cap - 1 slots per tile)
+  int cta_slots;             // partial-sum slots per row tile (CTAs that may share a tile, minus 1)
   uint32_t epoch;            // tag of this call's partial sums (never 0)
   uint32_t wtag;             // tag the partial sums are published under: epoch (0 only when a
                              // test injects a lost hand-off)
@@ -82,18 +83,23 @@ struct GemvProblem {
   int cta_base;       // first CTA of this problem
   int ncta;           // CTAs serving this problem
   int chunk;          // (row tile, block) units per warp
-  int lt_cap;         // row tiles one CTA's chunks touch, if their in-CTA hand-off fits in shared memory (else 0)
+  int lt_cap;         // row tiles one CTA's chunks touch (segment counters in shared memory)
 };
 // Decode work split: each warp of the grid (kGemvWarps per SM) takes an equal contiguous chunk
-// of the (16-row tile, 128-code block) units, never fewer than kGemvMinChunk.  A row tile is
-// then shared by at most gemv_seg_cap warps, which sizes the layer's partial-sum workspace.
+// of the (16-row tile, 128-code block) units, never fewer than kGemvMinChunk.  A CTA (at least
+// kGemvMinWarps warps) then spans at least kGemvMinWarps * cmin units, so a row tile of K/128
+// units meets at most gemv_cta_slots + 1 CTAs; the slots size the layer's partial-sum workspace.
 constexpr int kGemvWarps = 16;
-constexpr int kGemvMinChunk = 8;
-inline int gemv_seg_cap(int N, int K, int sm_count) {
+constexpr int kGemvMinWarps = 8;
+constexpr int kGemvMinChunk = 4;
+inline int gemv_min_chunk(int N, int K, int sm_count) {
   const long long units = (long long)((N + 15) / 16) * (K / kBlockCodes);
   const long long warps = (long long)sm_count * kGemvWarps;
-  const int cmin = (int)std::max<long long>(kGemvMinChunk, (units + warps - 1) / warps);
-  return (K / kBlockCodes - 1) / cmin + 2;
+  return (int)std::max<long long>(kGemvMinChunk, (units + warps - 1) / warps);
+}
+inline int gemv_cta_slots(int N, int K, int sm_count) {
+  const int span = kGemvMinWarps * gemv_min_chunk(N, K, sm_count);
+  return std::max(1, (K / kBlockCodes - 1 + span - 1) / span);
 }
 cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, long long wait_limit,
                         cudaStream_t s);
