@@ -168,12 +168,17 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
 
 /*
  * owq_gemm -- prefill product for any M >= 1 (tuned for M >= 64): TMA-staged packed tiles,
- * dequantised into shared memory (weak columns patched in as their fp16 values) and fed
- * to tcgen05 MMA with fp32 accumulators in tensor memory.  Same semantics and layouts as
- * owq_gemv; M <= 65536.  Bounded device waits: on a timeout the kernel abandons its tile,
- * sets the device status word and this call's later owq_device_status returns
+ * dequantised into shared memory and fed to tcgen05 MMA with fp32 accumulators in tensor
+ * memory; the weak block and the weak activations (gathered by a small kernel into the
+ * handle's scratch) run as extra K-steps into the same accumulator.  Same semantics and
+ * layouts as owq_gemv; M <= 65536.  Bounded device waits: on a timeout the kernel abandons
+ * its tile, sets the device status word and this call's later owq_device_status returns
  * OWQ_ERR_TIMEOUT (y is then undefined).  The first call on a handle builds its tensor
- * map on the host: first calls from several host threads on one handle must be serialised.
+ * maps on the host: first calls from several host threads on one handle must be
+ * serialised.  The handle's scratch (M * k_ld * 2 bytes of weak activations; for few row
+ * tiles also a split-K workspace) grows on the first call that needs more, which must not
+ * be inside a stream capture: there a too-small weak-activation scratch gives OWQ_ERR_NOMEM
+ * (the split-K workspace falls back to one split).
  */
 owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
                       owq_stream_t stream);

@@ -71,6 +71,7 @@ void release(Layer* L) {
   cudaFree(L->sz_t);
   cudaFree(L->xfrag);
   cudaFree(L->gemm_ws);
+  cudaFree(L->gemm_xw);
   cudaFree(L->part);
   delete[] L->idx_host;
   L->magic = 0;

@@ -9,17 +9,20 @@
 //
 // One CTA computes a 128-weight-row x BN-token tile of y^T (MMA M = weight rows,
 // MMA N = tokens), looping over K in 128-code steps through an S-stage ring:
-//   warp 0      TMA producer: the packed 128 x (16*bits) byte tile (a 3-D box over the layer's
-//               16-row-tile storage, no swizzle) and two 128B-swizzled BN x 64 fp16
-//               activation boxes per step.
+//   warp 0      TMA producer.  Dense step: the packed 128 x (16*bits) byte tile (a 3-D box over
+//               the layer's 16-row-tile storage), for per-group layers the step's (scale, zero)
+//               pairs of the 8 tiles, and two 128B-swizzled BN x 64 fp16 activation boxes.
+//               Weak step (after the dense ones): two 128 x 64 boxes of the fp16 weak block
+//               straight into the A slabs and two boxes of the gathered weak activations.
 //   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16,
 //               fp32 accumulator BN columns wide in tensor memory).
-//   warps 2-9   dequantisation: each thread owns one weight row and two chunks of each
-//               128-code step (codes 8j + 4h .. 8j + 4h + 3), unpacks them in registers, forms
-//               fp16_rn(s (q - z)) with exact fp16x2 arithmetic, stores 8-byte halves of the
-//               16-byte units of the K-major 128B-swizzled A tile, then overwrites its weak
-//               columns with their fp16 values (no activation gather is needed).  The same warps run the epilogue
-//               (tcgen05.ld of their TMEM lane quarter, fp16 rounding, coalesced stores).
+//   warps 2-9   dequantisation of the dense steps: each thread owns one weight row and one
+//               64-code slab of each step, unpacks in registers, forms fp16_rn(s (q - z)) with
+//               exact fp16x2 arithmetic and stores whole 16-byte units of the K-major
+//               128B-swizzled A tile.  The weak columns hold q = z, so their dequantised value
+//               is exactly 0 and the weak steps add W_weak x[idx] into the same accumulator.
+//               The same warps run the epilogue (tcgen05.ld of their TMEM lane quarter, fp16
+//               rounding, coalesced stores).
 // Every mbarrier wait is bounded (clock64 limit): on expiry the thread records the device
 // status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
 #include <algorithm>
@@ -45,23 +48,22 @@ struct Smem {
   static constexpr int kX = 2 * BN * 128;           // two 64-column swizzled boxes
   static constexpr int kA = 2 * kBM * 128;          // two 64-column swizzled slabs
   static constexpr int kP = kBM * 16 * BITS;        // packed tile
-  static constexpr int kStage = ((kX + kA + kP) + 1023) & ~1023;
+  static constexpr int kSZ = kBM * 4;               // (scale, zero) pairs of the step (per-group layers)
+  static constexpr int kStage = ((kX + kA + kP + kSZ) + 1023) & ~1023;
 };
 
 template <int BITS, int BN, int S>
 constexpr int smem_bytes() { return S * Smem<BITS, BN>::kStage + 1024 /*barriers*/ + 1024 /*align slack*/; }
 
 struct GemmParams {
-  const __half* scales;
+  const __half* scales;   // per-channel layers: read once per row (per-group: staged by TMA)
   const __half* zeros;
-  const __half* w_weak;
-  const int32_t* idx;
-  const int32_t* blk_weak;
   __half* y;
   float* ws;        // split-K partial sums [split][M][N] (NULL: one split, fp16 y directly)
   int* status;
-  int N, K, M, G, k_ld;
-  int ksteps;       // 128-code steps per split (blockIdx.z)
+  int N, K, M, G;
+  int ksteps;       // dense 128-code steps per split (blockIdx.z)
+  int nw;           // weak steps: 128 columns of the weak block each (run by the last split)
   long long wait_limit;   // bound of every mbarrier wait, in SM clock cycles
   int skip_arrive;  // test-injected lost arrival: dequantisation thread 0 skips its first one
 };
@@ -102,7 +104,8 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 template <int BITS, int BN, int S>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_p,
-             const __grid_constant__ GemmParams p) {
+             const __grid_constant__ CUtensorMap map_ww, const __grid_constant__ CUtensorMap map_xw,
+             const __grid_constant__ CUtensorMap map_sz, const __grid_constant__ GemmParams p) {
   using L = Smem<BITS, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,8 +119,10 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kBM;      // first weight row
   const int m0 = blockIdx.y * BN;       // first token
-  const int kb0 = blockIdx.z * p.ksteps;                       // first step of this split
-  const int nK = min(p.ksteps, p.K / kStepCodes - kb0);          // steps of this split
+  const int kb0 = blockIdx.z * p.ksteps;                          // first dense step of this split
+  const int nD = max(0, min(p.ksteps, p.K / kStepCodes - kb0));   // dense steps of this split
+  const int nK = nD + (blockIdx.z == gridDim.z - 1 ? p.nw : 0);   // + the weak steps (last split)
+  const bool per_group = p.G > 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -139,19 +144,34 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      constexpr uint32_t kBytes = L::kX + L::kP;
+      // dense step: the packed block of the 8 16-row tiles of this CTA (tile-major storage),
+      // their (scale, zero) pairs (per-group layers) and two activation boxes; weak step: the
+      // fp16 weak block (two 64-column boxes straight into the A slabs) and the gathered weak
+      // activations
+      const uint32_t kDense = L::kX + L::kP + (per_group ? L::kSZ : 0);
+      constexpr uint32_t kWeak = L::kX + L::kA;
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < nK && ok; ++i) {
-        const int kb = kb0 + i, s = i % S, u = i / S;
+        const int s = i % S, u = i / S;
         if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, p.status, p.wait_limit);
         if (!ok) break;
         unsigned char* st = smem + s * L::kStage;
-        mbar_arrive_expect_tx(&full[s], kBytes);
-        // packed: block kb of the 8 16-row tiles of this CTA (tile-major storage)
-        tma_load_3d(st + L::kX + L::kA, &map_p, &full[s], 0, kb, n0 / 16);
-        tma_load_2d(st, &map_x, &full[s], kb * kStepCodes, m0);
-        tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
+        if (i < nD) {
+          const int kb = kb0 + i;
+          mbar_arrive_expect_tx(&full[s], kDense);
+          tma_load_3d(st + L::kX + L::kA, &map_p, &full[s], 0, kb, n0 / 16);
+          if (per_group) tma_load_3d(st + L::kX + L::kA + L::kP, &map_sz, &full[s], 0, kb, n0 / 16);
+          tma_load_2d(st, &map_x, &full[s], kb * kStepCodes, m0);
+          tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
+        } else {
+          const int c0 = (i - nD) * kStepCodes;
+          mbar_arrive_expect_tx(&full[s], kWeak);
+          tma_load_2d(st + L::kX, &map_ww, &full[s], c0, n0);
+          tma_load_2d(st + L::kX + kBM * 128, &map_ww, &full[s], c0 + 64, n0);
+          tma_load_2d(st, &map_xw, &full[s], c0, m0);
+          tma_load_2d(st + BN * 128, &map_xw, &full[s], c0 + 64, m0);
+        }
         issued = i + 1;
       }
       // never leave with copies in flight: wait for the last issued use of every stage
@@ -190,54 +210,32 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     // 8j .. 8j + 7, i.e. one whole 16-byte unit of the 128B-swizzled row (no bank conflicts)
     const int td = threadIdx.x - 64;          // 0..255
     const int r = td & (kBM - 1), jh = td >> 7;
-    const int row = min(n0 + r, p.N - 1);
-    const bool per_channel = p.G == 1;
     uint32_t s2 = 0, scl[3], nz[3];
     constexpr float kOff[3] = {1.f, BITS == 3 ? 8.f : 16.f, 64.f};
     scl[0] = h2_splat(1.f);
     scl[1] = h2_splat(1.f / kOff[1]);
     scl[2] = h2_splat(1.f / kOff[2]);
-    // (scale, zero) of the next step, fetched one step ahead
-    __half sh_next = p.scales[(size_t)row * p.G + (per_channel ? 0 : kb0)];
-    __half z_next = p.zeros[(size_t)row * p.G + (per_channel ? 0 : kb0)];
-    // weak columns of the next step (up to 4 fetched one step ahead; more are read in place)
-    int wcol0, wcol1, wcol2, wcol3;
-    __half wval0, wval1, wval2, wval3;
-#define OWQ_FETCH_WEAK(KB)                                                                      \
-    {                                                                                           \
-      const int t0_ = p.blk_weak[KB], t1_ = p.blk_weak[(KB) + 1];                               \
-      const __half zero_ = __float2half_rn(0.f);                                                \
-      const __half* wr_ = p.w_weak + (size_t)row * p.k_ld;                                      \
-      wcol0 = t0_ < t1_ ? p.idx[t0_] - (KB) * kStepCodes : -1;                                  \
-      wcol1 = t0_ + 1 < t1_ ? p.idx[t0_ + 1] - (KB) * kStepCodes : -1;                          \
-      wcol2 = t0_ + 2 < t1_ ? p.idx[t0_ + 2] - (KB) * kStepCodes : -1;                          \
-      wcol3 = t0_ + 3 < t1_ ? p.idx[t0_ + 3] - (KB) * kStepCodes : -1;                          \
-      wval0 = t0_ < t1_ ? wr_[t0_] : zero_;                                                     \
-      wval1 = t0_ + 1 < t1_ ? wr_[t0_ + 1] : zero_;                                             \
-      wval2 = t0_ + 2 < t1_ ? wr_[t0_ + 2] : zero_;                                             \
-      wval3 = t0_ + 3 < t1_ ? wr_[t0_ + 3] : zero_;                                             \
+    auto set_sz = [&](__half sh, __half zh) {
+      const uint32_t su = __half_as_ushort(sh);
+      const float z = __half2float(zh);
+      s2 = su | (su << 16);
+      #pragma unroll
+      for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
+    };
+    if (!per_group) {   // per-channel: one (scale, zero) pair for the whole row
+      const int row = min(n0 + r, p.N - 1);
+      set_sz(p.scales[row], p.zeros[row]);
     }
-    OWQ_FETCH_WEAK(kb0)
     bool ok = true;
-    for (int i = 0; i < nK && ok; ++i) {
-      const int kb = kb0 + i, s = i % S, u = i / S;
-      if (i == 0 || !per_channel) {
-        const uint32_t su = __half_as_ushort(sh_next);
-        const float z = __half2float(z_next);
-        s2 = su | (su << 16);
-        #pragma unroll
-        for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
-        if (!per_channel && i + 1 < nK) {
-          sh_next = p.scales[(size_t)row * p.G + kb + 1];
-          z_next = p.zeros[(size_t)row * p.G + kb + 1];
-        }
-      }
-      const int wc[4] = {wcol0, wcol1, wcol2, wcol3};
-      const __half wv[4] = {wval0, wval1, wval2, wval3};
-      if (i + 1 < nK) OWQ_FETCH_WEAK(kb + 1)
+    for (int i = 0; i < nD && ok; ++i) {
+      const int s = i % S, u = i / S;
       ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);
       if (!ok) break;
       unsigned char* st = smem + s * L::kStage;
+      if (per_group) {   // this step's pair, staged with the packed tile ([8 tiles][16 rows])
+        const __half2 sz = *reinterpret_cast<const __half2*>(st + L::kX + L::kA + L::kP + r * 4);
+        set_sz(__low2half(sz), __high2half(sz));
+      }
       const uint4* pw = reinterpret_cast<const uint4*>(st + L::kX + L::kA + r * 16 * BITS);
       uint32_t w[4 * BITS];
       #pragma unroll
@@ -259,21 +257,15 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       };
       if (jh == 0) units(std::integral_constant<int, 0>{});
       else units(std::integral_constant<int, 1>{});
-      // weak columns of this block in this slab: their fp16 values replace the zero-filled codes
-      #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (wc[i] >= 0 && (wc[i] >> 6) == jh)
-          *(reinterpret_cast<__half*>(slab + sw128_off(r, (wc[i] >> 3) & 7)) + (wc[i] & 7)) = wv[i];
-      const int t1 = p.blk_weak[kb + 1];
-      for (int t = p.blk_weak[kb] + 4; t < t1; ++t) {   // blocks with more than four weak columns
-        const int col = p.idx[t] - kb * kStepCodes;
-        if ((col >> 6) != jh) continue;
-        *(reinterpret_cast<__half*>(slab + sw128_off(r, (col >> 3) & 7)) + (col & 7)) = p.w_weak[(size_t)row * p.k_ld + t];
-      }
+      // the weak columns hold q = z: their dequantised value is exactly 0 (the weak steps add them)
       fence_proxy_async_smem();
       if (!(p.skip_arrive && i == 0 && td == 0)) mbar_arrive(&afull[s]);
     }
-#undef OWQ_FETCH_WEAK
+    // weak steps: the A tile arrives by TMA; keep pace with the ring, then release the MMA
+    for (int i = nD; i < nK && ok; ++i) {
+      ok = mbar_wait(&full[i % S], (i / S) & 1, p.status, p.wait_limit);
+      if (ok) mbar_arrive(&afull[i % S]);
+    }
 
     // ---------------- epilogue ----------------
     const int wd = warp - 2, q = warp & 3, chalf = wd >> 2;
@@ -310,6 +302,17 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     tc_fence_after();
     tmem_dealloc(tmem, BN);
     tmem_relinquish();
+  }
+}
+
+// Weak activations of every token, in the weak block's column order: xw[m][t] = x[m][idx[t]]
+// (t < k), 0 for t in [k, k_ld).
+__global__ void k_gather_weak_x(const __half* __restrict__ x, int M, int K, const int32_t* __restrict__ idx,
+                                int k, int k_ld, __half* __restrict__ xw) {
+  const size_t n = (size_t)M * k_ld;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(e / k_ld), t = (int)(e % k_ld);
+    xw[e] = t < k ? x[(size_t)m * K + idx[t]] : __float2half_rn(0.f);
   }
 }
 
@@ -365,11 +368,49 @@ bool encode_packed_3d(CUtensorMap* m, const void* base, int K, int N, int bits) 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// (scale, zero) pairs of the 16-row tiles, tile-major [RT][G][16] 32-bit words: one box is
+// the pairs of one group for the 8 tiles of a CTA
+bool encode_sz_3d(CUtensorMap* m, const void* base, int G, int N) {
+  EncodeTiled enc = get_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {16, (cuuint64_t)G, (cuuint64_t)((N + 15) / 16)};
+  const cuuint64_t strides[2] = {64, 64ull * G};
+  const cuuint32_t box[3] = {16, 1, kBM / 16};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// grow a per-layer device scratch outside stream capture (false: too small and not growable)
+bool ensure_scratch(void** buf, size_t* have, size_t need, cudaStream_t s) {
+  if (need <= *have) return true;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaFree(*buf);
+  *buf = nullptr;
+  *have = 0;
+  if (cudaMalloc(buf, need) != cudaSuccess) {
+    cudaGetLastError();
+    *buf = nullptr;
+    return false;
+  }
+  *have = need;
+  return true;
+}
+
 template <int BITS, int BN, int S>
 owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_limit, bool skip_arrive,
                  cudaStream_t s) {
   if (!L.maps_ready) {
     if (!encode_packed_3d(&L.map_packed, L.packed, L.K, L.N, BITS)) return OWQ_ERR_CUDA;
+    if (L.G > 1 && !encode_sz_3d(&L.map_sz, L.sz_t, L.G, L.N)) return OWQ_ERR_CUDA;
+    if (L.k > 0 && !encode_2d(&L.map_weak, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, L.w_weak, (uint64_t)L.k_ld, (uint64_t)L.N,
+                              (uint64_t)L.k_ld * 2, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+      return OWQ_ERR_CUDA;
     L.maps_ready = true;
   }
   CUtensorMap mx;
@@ -377,9 +418,9 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return OWQ_ERR_CUDA;
   GemmParams prm;
-  prm.scales = L.scales; prm.zeros = L.zeros; prm.w_weak = L.w_weak; prm.idx = L.idx;
-  prm.blk_weak = L.blk_weak; prm.y = y; prm.status = device_status_ptr();
-  prm.N = L.N; prm.K = L.K; prm.M = M; prm.G = L.G; prm.k_ld = L.k_ld;
+  prm.scales = L.scales; prm.zeros = L.zeros; prm.y = y; prm.status = device_status_ptr();
+  prm.N = L.N; prm.K = L.K; prm.M = M; prm.G = L.G;
+  prm.nw = L.k > 0 ? (L.k_ld + kStepCodes - 1) / kStepCodes : 0;
   prm.wait_limit = wait_limit; prm.skip_arrive = skip_arrive ? 1 : 0;
   if (!prm.status) return OWQ_ERR_CUDA;
   // fewer tiles than SMs: split K over CTAs (at least 4 steps each), fp32 partials in the
@@ -430,7 +471,19 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
     return OWQ_ERR_CUDA;
   }
   dim3 grid((L.N + kBM - 1) / kBM, (M + BN - 1) / BN, splits);
-  kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, prm);
+  // the weak activations, gathered once per call into the layer's scratch (grown outside capture)
+  CUtensorMap mxw = mx;
+  if (L.k > 0) {
+    if (!ensure_scratch(reinterpret_cast<void**>(&L.gemm_xw), &L.gemm_xw_bytes, (size_t)M * L.k_ld * sizeof(__half), s))
+      return OWQ_ERR_NOMEM;
+    const size_t n = (size_t)M * L.k_ld;
+    k_gather_weak_x<<<(unsigned)std::min<size_t>((n + 255) / 256, 2048), 256, 0, s>>>(x, M, L.K, L.idx, L.k, L.k_ld, L.gemm_xw);
+    if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
+    if (!encode_2d(&mxw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, L.gemm_xw, (uint64_t)L.k_ld, (uint64_t)M, (uint64_t)L.k_ld * 2,
+                   64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      return OWQ_ERR_CUDA;
+  }
+  kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, L.k > 0 ? L.map_weak : mx, mxw, L.G > 1 ? L.map_sz : mx, prm);
   if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
   if (splits > 1) {
     const size_t MN = (size_t)M * L.N;
@@ -444,7 +497,7 @@ template <int BITS>
 owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, long long wl, bool skip, cudaStream_t s) {
   // wider token tiles dequantise each weight tile once for more tokens (the dequantisation,
   // not the MMA, bounds the narrower tiles); the widest one fits two stages
-  if (M <= 64) return run<BITS, 64, 4>(L, x, y, M, wl, skip, s);
+  if (M <= 64) return run<BITS, 64, BITS == 3 ? 4 : 3>(L, x, y, M, wl, skip, s);
   if (M <= 256) return run<BITS, 128, 3>(L, x, y, M, wl, skip, s);
   return run<BITS, 256, 2>(L, x, y, M, wl, skip, s);
 }

@@ -42,10 +42,13 @@ struct Layer {
   cudaStream_t stream;  // stream of owq_pack (used to order the release)
   float* gemm_ws;       // prefill split-K partial sums (grown on first need, outside capture)
   size_t gemm_ws_bytes;
+  __half* gemm_xw;      // prefill weak activations [M][k_ld] (grown on first need, outside capture)
+  size_t gemm_xw_bytes;
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
   alignas(64) CUtensorMap map_packed;
-  alignas(64) CUtensorMap map_weak;
+  alignas(64) CUtensorMap map_weak;    // the weak block [N][k_ld], 128 x 64 boxes, 128B swizzle
+  alignas(64) CUtensorMap map_sz;      // (scale, zero) pairs of per-group layers
 };
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
