@@ -12,16 +12,17 @@
 //   warp 0      TMA producer.  Dense step: the packed 128 x (16*bits) byte tile (a 3-D box over
 //               the layer's 16-row-tile storage), for per-group layers the step's (scale, zero)
 //               pairs of the 8 tiles, and two 128B-swizzled BN x 64 fp16 activation boxes.
-//               Weak step (after the dense ones): two 128 x 64 boxes of the fp16 weak block
-//               straight into the A slabs and two boxes of the gathered weak activations.
-//   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16,
-//               fp32 accumulator BN columns wide in tensor memory).
-//   warps 2-9   dequantisation of the dense steps: each thread owns one weight row and one
-//               64-code slab of each step, unpacks in registers, forms fp16_rn(s (q - z)) with
-//               exact fp16x2 arithmetic and stores whole 16-byte units of the K-major
-//               128B-swizzled A tile.  The weak columns hold q = z, so their dequantised value
-//               is exactly 0 and the weak steps add W_weak x[idx] into the same accumulator.
-//               The same warps run the epilogue (tcgen05.ld of their TMEM lane quarter, fp16
+//               Weak step (after the dense ones): two boxes of the gathered weak activations.
+//   warp 1      TMEM allocation and the single MMA-issuing thread (tcgen05.mma kind::f16 with
+//               the A operand in tensor memory, B from shared memory, fp32 accumulator BN
+//               columns wide in tensor memory).
+//   warps 2-9   the A operand: each thread owns one weight row (its warp's TMEM lane quarter)
+//               and one 64-code slab of each step.  Dense step: unpack in registers, form
+//               fp16_rn(s (q - z)) with exact fp16x2 arithmetic, tcgen05.st into the step's A
+//               stage in tensor memory (no shared-memory A tile, so the ring holds more
+//               stages).  The weak columns hold q = z, so their dequantised value is exactly 0;
+//               the weak steps load the fp16 weak block rows instead, adding W_weak x[idx] into
+//               the same accumulator.  The same warps run the epilogue (tcgen05.ld, fp16
 //               rounding, coalesced stores).
 // Every mbarrier wait is bounded (clock64 limit): on expiry the thread records the device
 // status word and leaves its loop, so a broken pipeline ends the kernel instead of hanging.
@@ -41,15 +42,15 @@ using namespace sm100;
 constexpr int kBM = 128;               // weight rows per tile (MMA M)
 constexpr int kStepCodes = 128;        // K per pipeline step
 constexpr int kDequantWarps = 8;
+constexpr uint32_t kTmemCols = 512;    // accumulator (BN <= 256 columns) + S <= 4 A stages of 64
 constexpr int kThreads = 32 * (2 + kDequantWarps);
 
 template <int BITS, int BN>
 struct Smem {
-  static constexpr int kX = 2 * BN * 128;           // two 64-column swizzled boxes
-  static constexpr int kA = 2 * kBM * 128;          // two 64-column swizzled slabs
+  static constexpr int kX = 2 * BN * 128;           // two 64-column swizzled activation boxes
   static constexpr int kP = kBM * 16 * BITS;        // packed tile
   static constexpr int kSZ = kBM * 4;               // (scale, zero) pairs of the step (per-group layers)
-  static constexpr int kStage = ((kX + kA + kP + kSZ) + 1023) & ~1023;
+  static constexpr int kStage = ((kX + kP + kSZ) + 1023) & ~1023;
 };
 
 template <int BITS, int BN, int S>
@@ -58,6 +59,8 @@ constexpr int smem_bytes() { return S * Smem<BITS, BN>::kStage + 1024 /*barriers
 struct GemmParams {
   const __half* scales;   // per-channel layers: read once per row (per-group: staged by TMA)
   const __half* zeros;
+  const __half* w_weak;   // the weak block [N][k_ld] (read by the A-operand warps in weak steps)
+  int k_ld;
   __half* y;
   float* ws;        // split-K partial sums [split][M][N] (NULL: one split, fp16 y directly)
   int* status;
@@ -104,15 +107,15 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 template <int BITS, int BN, int S>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_p,
-             const __grid_constant__ CUtensorMap map_ww, const __grid_constant__ CUtensorMap map_xw,
-             const __grid_constant__ CUtensorMap map_sz, const __grid_constant__ GemmParams p) {
+             const __grid_constant__ CUtensorMap map_xw, const __grid_constant__ CUtensorMap map_sz,
+             const __grid_constant__ GemmParams p) {
   using L = Smem<BITS, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage);
   uint64_t* full = bars;            // [S] TMA landed
   uint64_t* empty = bars + S;       // [S] MMAs of the stage done
-  uint64_t* afull = bars + 2 * S;   // [S] A tile written
+  uint64_t* afull = bars + 2 * S;   // [S] A tile written to tensor memory
   uint64_t* accf = bars + 3 * S;    // accumulator complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
 
@@ -135,7 +138,9 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     prefetch_tmap(&map_x);
     prefetch_tmap(&map_p);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, BN);
+  // tensor memory: the accumulator (BN columns) then S A stages of 64 columns (128 rows x 128
+  // fp16 codes, two per 32-bit column)
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -145,11 +150,9 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       // dense step: the packed block of the 8 16-row tiles of this CTA (tile-major storage),
-      // their (scale, zero) pairs (per-group layers) and two activation boxes; weak step: the
-      // fp16 weak block (two 64-column boxes straight into the A slabs) and the gathered weak
-      // activations
+      // their (scale, zero) pairs (per-group layers) and two activation boxes; weak step: two
+      // boxes of the gathered weak activations
       const uint32_t kDense = L::kX + L::kP + (per_group ? L::kSZ : 0);
-      constexpr uint32_t kWeak = L::kX + L::kA;
       bool ok = true;
       int issued = 0;
       for (int i = 0; i < nK && ok; ++i) {
@@ -160,15 +163,13 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
         if (i < nD) {
           const int kb = kb0 + i;
           mbar_arrive_expect_tx(&full[s], kDense);
-          tma_load_3d(st + L::kX + L::kA, &map_p, &full[s], 0, kb, n0 / 16);
-          if (per_group) tma_load_3d(st + L::kX + L::kA + L::kP, &map_sz, &full[s], 0, kb, n0 / 16);
+          tma_load_3d(st + L::kX, &map_p, &full[s], 0, kb, n0 / 16);
+          if (per_group) tma_load_3d(st + L::kX + L::kP, &map_sz, &full[s], 0, kb, n0 / 16);
           tma_load_2d(st, &map_x, &full[s], kb * kStepCodes, m0);
           tma_load_2d(st + BN * 128, &map_x, &full[s], kb * kStepCodes + 64, m0);
         } else {
           const int c0 = (i - nD) * kStepCodes;
-          mbar_arrive_expect_tx(&full[s], kWeak);
-          tma_load_2d(st + L::kX, &map_ww, &full[s], c0, n0);
-          tma_load_2d(st + L::kX + kBM * 128, &map_ww, &full[s], c0 + 64, n0);
+          mbar_arrive_expect_tx(&full[s], L::kX);
           tma_load_2d(st, &map_xw, &full[s], c0, m0);
           tma_load_2d(st + BN * 128, &map_xw, &full[s], c0 + 64, m0);
         }
@@ -189,27 +190,27 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
              mbar_wait(&afull[s], u & 1, p.status, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
-        unsigned char* st = smem + s * L::kStage;
-        const uint32_t xa = smem_u32(st), aa = smem_u32(st + L::kX);
+        const uint32_t xa = smem_u32(smem + s * L::kStage);
+        const uint32_t at = tmem + BN + 64 * s;
         #pragma unroll
-        for (int a = 0; a < 2; ++a)
-          #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = desc_sw128_kmajor(aa + a * kBM * 128 + kk * 32);
-            const uint64_t bd = desc_sw128_kmajor(xa + a * BN * 128 + kk * 32);
-            mma_f16(tmem, ad, bd, idesc, (i | a | kk) != 0);
-          }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = desc_sw128_kmajor(xa + (kk >> 2) * BN * 128 + (kk & 3) * 32);
+          mma_f16_ts(tmem, at + 8 * kk, bd, idesc, (i | kk) != 0);
+        }
         mma_commit(&empty[s]);
       }
       mma_commit(accf);
     }
   } else {
-    // ---------------- dequantisation ----------------
-    // thread (r, jh): row r of the tile and K-slab jh (codes 64 jh .. 64 jh + 63 of each
-    // 128-code block): for j = 8 jh .. 8 jh + 7, the four chunks' pair j are the 8 codes
-    // 8j .. 8j + 7, i.e. one whole 16-byte unit of the 128B-swizzled row (no bank conflicts)
-    const int td = threadIdx.x - 64;          // 0..255
-    const int r = td & (kBM - 1), jh = td >> 7;
+    // ---------------- A operand ----------------
+    // warp w owns the lane quarter w % 4 of tensor memory: thread (row r = 32 (w % 4) + lane,
+    // slab jh = (w - 2) / 4) writes codes 64 jh .. 64 jh + 63 of its row, columns
+    // 32 jh .. 32 jh + 31 of the step's A stage.  For j = 8 jh .. 8 jh + 7 the four chunks'
+    // pair j are the codes 8j .. 8j + 7.
+    const int quarter = warp & 3, jh = (warp - 2) >> 2;
+    const int r = 32 * quarter + lane;
+    const int row = min(n0 + r, p.N - 1);
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
     uint32_t s2 = 0, scl[3], nz[3];
     constexpr float kOff[3] = {1.f, BITS == 3 ? 8.f : 16.f, 64.f};
     scl[0] = h2_splat(1.f);
@@ -222,60 +223,67 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       #pragma unroll
       for (int c = 0; c < 3; ++c) nz[c] = h2_splat(-(1024.f / kOff[c] + z));
     };
-    if (!per_group) {   // per-channel: one (scale, zero) pair for the whole row
-      const int row = min(n0 + r, p.N - 1);
-      set_sz(p.scales[row], p.zeros[row]);
-    }
+    if (!per_group) set_sz(p.scales[row], p.zeros[row]);   // per-channel: one pair per row
     bool ok = true;
-    for (int i = 0; i < nD && ok; ++i) {
+    for (int i = 0; i < nK && ok; ++i) {
       const int s = i % S, u = i / S;
-      ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);
+      ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);   // (also: the stage's previous MMAs are done)
       if (!ok) break;
-      unsigned char* st = smem + s * L::kStage;
-      if (per_group) {   // this step's pair, staged with the packed tile ([8 tiles][16 rows])
-        const __half2 sz = *reinterpret_cast<const __half2*>(st + L::kX + L::kA + L::kP + r * 4);
-        set_sz(__low2half(sz), __high2half(sz));
-      }
-      const uint4* pw = reinterpret_cast<const uint4*>(st + L::kX + L::kA + r * 16 * BITS);
-      uint32_t w[4 * BITS];
-      #pragma unroll
-      for (int v = 0; v < BITS; ++v) {
-        const uint4 q = pw[v];
-        w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
-      }
-      unsigned char* slab = st + L::kX + jh * kBM * 128;
-      // jh is uniform per warp: each branch sees compile-time pair indices
-      auto units = [&](auto jh_c) {
-        constexpr int JH = decltype(jh_c)::value;
-        #pragma unroll
-        for (int j8 = 0; j8 < 8; ++j8) {
-          uint32_t d[4];
-          #pragma unroll
-          for (int q = 0; q < 4; ++q) d[q] = dequant_pair<BITS>(w + q * BITS, 8 * JH + j8, s2, scl, nz);   // k = 8j + 2q, +1
-          *reinterpret_cast<uint4*>(slab + sw128_off(r, j8)) = make_uint4(d[0], d[1], d[2], d[3]);
+      tc_fence_after();
+      const unsigned char* st = smem + s * L::kStage;
+      const uint32_t at = tmem + lane_base + BN + 64 * s + 32 * jh;
+      uint32_t d[2][16];
+      if (i < nD) {
+        if (per_group) {   // this step's pair, staged with the packed tile ([8 tiles][16 rows])
+          const __half2 sz = *reinterpret_cast<const __half2*>(st + L::kX + L::kP + r * 4);
+          set_sz(__low2half(sz), __high2half(sz));
         }
-      };
-      if (jh == 0) units(std::integral_constant<int, 0>{});
-      else units(std::integral_constant<int, 1>{});
-      // the weak columns hold q = z: their dequantised value is exactly 0 (the weak steps add them)
-      fence_proxy_async_smem();
-      if (!(p.skip_arrive && i == 0 && td == 0)) mbar_arrive(&afull[s]);
-    }
-    // weak steps: the A tile arrives by TMA; keep pace with the ring, then release the MMA
-    for (int i = nD; i < nK && ok; ++i) {
-      ok = mbar_wait(&full[i % S], (i / S) & 1, p.status, p.wait_limit);
-      if (ok) mbar_arrive(&afull[i % S]);
+        const uint4* pw = reinterpret_cast<const uint4*>(st + L::kX + r * 16 * BITS);
+        uint32_t w[4 * BITS];
+        #pragma unroll
+        for (int v = 0; v < BITS; ++v) {
+          const uint4 q = pw[v];
+          w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
+        }
+        // jh is uniform per warp: each branch sees compile-time pair indices.  The weak columns
+        // hold q = z: their value is exactly 0 (the weak steps add them).
+        auto units = [&](auto jh_c) {
+          constexpr int JH = decltype(jh_c)::value;
+          #pragma unroll
+          for (int j8 = 0; j8 < 8; ++j8)
+            #pragma unroll
+            for (int q = 0; q < 4; ++q)   // codes 8j + 2q, 8j + 2q + 1 -> column 4 j8 + q
+              d[j8 >> 2][4 * (j8 & 3) + q] = dequant_pair<BITS>(w + q * BITS, 8 * JH + j8, s2, scl, nz);
+        };
+        if (jh == 0) units(std::integral_constant<int, 0>{});
+        else units(std::integral_constant<int, 1>{});
+      } else {
+        // weak step: the fp16 weak block, columns c0 + 64 jh .. + 63 of this row (0 past k_ld)
+        const int c0 = (i - nD) * kStepCodes + 64 * jh;
+        const uint4* src = reinterpret_cast<const uint4*>(p.w_weak + (size_t)row * p.k_ld + c0);
+        #pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint4 q = (n0 + r < p.N && c0 + 8 * v < p.k_ld) ? src[v] : make_uint4(0, 0, 0, 0);
+          d[v >> 2][4 * (v & 3)] = q.x; d[v >> 2][4 * (v & 3) + 1] = q.y;
+          d[v >> 2][4 * (v & 3) + 2] = q.z; d[v >> 2][4 * (v & 3) + 3] = q.w;
+        }
+      }
+      tmem_st16(at, d[0]);
+      tmem_st16(at + 16, d[1]);
+      tmem_st_wait();
+      tc_fence_before();
+      if (!(p.skip_arrive && i == 0 && threadIdx.x == 64)) mbar_arrive(&afull[s]);
     }
 
     // ---------------- epilogue ----------------
-    const int wd = warp - 2, q = warp & 3, chalf = wd >> 2;
+    const int chalf = jh;
     const bool acc_ok = mbar_wait(accf, 0, p.status, p.wait_limit);
     tc_fence_after();
-    const int orow = n0 + 32 * q + lane;
+    const int orow = n0 + r;
     #pragma unroll 1
     for (int c0 = chalf * (BN / 2); c0 < (chalf + 1) * (BN / 2); c0 += 16) {
       uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+      tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
       tmem_ld_wait();
       if (acc_ok && orow < p.N) {
         if (p.ws) {   // split-K: fp32 partial of this split
@@ -300,7 +308,7 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, kTmemCols);
     tmem_relinquish();
   }
 }
@@ -408,9 +416,6 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   if (!L.maps_ready) {
     if (!encode_packed_3d(&L.map_packed, L.packed, L.K, L.N, BITS)) return OWQ_ERR_CUDA;
     if (L.G > 1 && !encode_sz_3d(&L.map_sz, L.sz_t, L.G, L.N)) return OWQ_ERR_CUDA;
-    if (L.k > 0 && !encode_2d(&L.map_weak, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, L.w_weak, (uint64_t)L.k_ld, (uint64_t)L.N,
-                              (uint64_t)L.k_ld * 2, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
-      return OWQ_ERR_CUDA;
     L.maps_ready = true;
   }
   CUtensorMap mx;
@@ -418,7 +423,8 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return OWQ_ERR_CUDA;
   GemmParams prm;
-  prm.scales = L.scales; prm.zeros = L.zeros; prm.y = y; prm.status = device_status_ptr();
+  prm.scales = L.scales; prm.zeros = L.zeros; prm.w_weak = L.w_weak; prm.k_ld = L.k_ld;
+  prm.y = y; prm.status = device_status_ptr();
   prm.N = L.N; prm.K = L.K; prm.M = M; prm.G = L.G;
   prm.nw = L.k > 0 ? (L.k_ld + kStepCodes - 1) / kStepCodes : 0;
   prm.wait_limit = wait_limit; prm.skip_arrive = skip_arrive ? 1 : 0;
@@ -466,6 +472,9 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   auto kern = k_gemm_sm100<BITS, BN, S>;
   constexpr int smem = smem_bytes<BITS, BN, S>();
   static_assert(smem <= 232448, "shared memory budget");
+  // one CTA per SM (more than half the shared memory), so its 512 tensor-memory columns are free
+  static_assert(smem > 232448 / 2, "one CTA per SM");
+  static_assert(BN + 64 * S <= (int)kTmemCols, "tensor memory: accumulator + A stages");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return OWQ_ERR_CUDA;
@@ -483,7 +492,7 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
                    64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
       return OWQ_ERR_CUDA;
   }
-  kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, L.k > 0 ? L.map_weak : mx, mxw, L.G > 1 ? L.map_sz : mx, prm);
+  kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, mxw, L.G > 1 ? L.map_sz : mx, prm);
   if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
   if (splits > 1) {
     const size_t MN = (size_t)M * L.N;
@@ -497,9 +506,9 @@ template <int BITS>
 owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, long long wl, bool skip, cudaStream_t s) {
   // wider token tiles dequantise each weight tile once for more tokens (the dequantisation,
   // not the MMA, bounds the narrower tiles); the widest one fits two stages
-  if (M <= 64) return run<BITS, 64, BITS == 3 ? 4 : 3>(L, x, y, M, wl, skip, s);
-  if (M <= 256) return run<BITS, 128, 3>(L, x, y, M, wl, skip, s);
-  return run<BITS, 256, 2>(L, x, y, M, wl, skip, s);
+  if (M <= 64) return run<BITS, 64, 6>(L, x, y, M, wl, skip, s);
+  if (M <= 256) return run<BITS, 128, 4>(L, x, y, M, wl, skip, s);
+  return run<BITS, 256, 3>(L, x, y, M, wl, skip, s);
 }
 
 }  // namespace
