@@ -41,9 +41,7 @@ using namespace sm100;
 
 constexpr int kBM = 128;               // weight rows per tile (MMA M)
 constexpr int kStepCodes = 128;        // K per pipeline step
-constexpr int kDequantWarps = 8;
 constexpr uint32_t kTmemCols = 512;    // accumulator (BN <= 256 columns) + S <= 4 A stages of 64
-constexpr int kThreads = 32 * (2 + kDequantWarps);
 
 template <int BITS, int BN>
 struct Smem {
@@ -104,8 +102,8 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int BITS, int BN, int S>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BITS, int BN, int S, int DW>
+__global__ void __launch_bounds__(32 * (2 + DW), 1)
 k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_p,
              const __grid_constant__ CUtensorMap map_xw, const __grid_constant__ CUtensorMap map_sz,
              const __grid_constant__ GemmParams p) {
@@ -131,7 +129,7 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], 32 * kDequantWarps);
+      mbar_init(&afull[s], 32 * DW);
     }
     mbar_init(accf, 1);
     fence_mbar_init();
@@ -203,10 +201,12 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
     }
   } else {
     // ---------------- A operand ----------------
-    // warp w owns the lane quarter w % 4 of tensor memory: thread (row r = 32 (w % 4) + lane,
-    // slab jh = (w - 2) / 4) writes codes 64 jh .. 64 jh + 63 of its row, columns
-    // 32 jh .. 32 jh + 31 of the step's A stage.  For j = 8 jh .. 8 jh + 7 the four chunks'
-    // pair j are the codes 8j .. 8j + 7.
+    // DW warps, NSL = DW / 4 per lane quarter: warp w owns the lane quarter w % 4 of tensor
+    // memory and slab sl = (w - 2) / 4 of each step.  Thread (row r = 32 (w % 4) + lane, sl)
+    // writes codes 8U sl .. 8U sl + 8U - 1 of its row (U = 16 / NSL units of 8 codes), columns
+    // 4U sl .. 4U sl + 4U - 1 of the step's A stage.  For unit j the four chunks' pair j are
+    // the codes 8j .. 8j + 7.
+    constexpr int NSL = DW / 4, U = 16 / NSL;
     const int quarter = warp & 3, jh = (warp - 2) >> 2;
     const int r = 32 * quarter + lane;
     const int row = min(n0 + r, p.N - 1);
@@ -231,8 +231,8 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       if (!ok) break;
       tc_fence_after();
       const unsigned char* st = smem + s * L::kStage;
-      const uint32_t at = tmem + lane_base + BN + 64 * s + 32 * jh;
-      uint32_t d[2][16];
+      const uint32_t at = tmem + lane_base + BN + 64 * s + 4 * U * jh;
+      uint32_t d[U / 4][16];
       if (i < nD) {
         if (per_group) {   // this step's pair, staged with the packed tile ([8 tiles][16 rows])
           const __half2 sz = *reinterpret_cast<const __half2*>(st + L::kX + L::kP + r * 4);
@@ -245,43 +245,51 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
           const uint4 q = pw[v];
           w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
         }
-        // jh is uniform per warp: each branch sees compile-time pair indices.  The weak columns
-        // hold q = z: their value is exactly 0 (the weak steps add them).
-        auto units = [&](auto jh_c) {
-          constexpr int JH = decltype(jh_c)::value;
+        // the slab is uniform per warp: each branch sees compile-time pair indices.  The weak
+        // columns hold q = z: their value is exactly 0 (the weak steps add them).
+        auto units = [&](auto sl_c) {
+          constexpr int SL = decltype(sl_c)::value;
           #pragma unroll
-          for (int j8 = 0; j8 < 8; ++j8)
+          for (int ju = 0; ju < U; ++ju)
             #pragma unroll
-            for (int q = 0; q < 4; ++q)   // codes 8j + 2q, 8j + 2q + 1 -> column 4 j8 + q
-              d[j8 >> 2][4 * (j8 & 3) + q] = dequant_pair<BITS>(w + q * BITS, 8 * JH + j8, s2, scl, nz);
+            for (int q = 0; q < 4; ++q)   // codes 8j + 2q, 8j + 2q + 1 -> column 4 ju + q of the slab
+              d[ju >> 2][4 * (ju & 3) + q] = dequant_pair<BITS>(w + q * BITS, U * SL + ju, s2, scl, nz);
         };
-        if (jh == 0) units(std::integral_constant<int, 0>{});
-        else units(std::integral_constant<int, 1>{});
+        if constexpr (NSL == 2) {
+          if (jh == 0) units(std::integral_constant<int, 0>{});
+          else units(std::integral_constant<int, 1>{});
+        } else {
+          switch (jh) {
+            case 0: units(std::integral_constant<int, 0>{}); break;
+            case 1: units(std::integral_constant<int, 1>{}); break;
+            case 2: units(std::integral_constant<int, 2>{}); break;
+            default: units(std::integral_constant<int, 3>{}); break;
+          }
+        }
       } else {
-        // weak step: the fp16 weak block, columns c0 + 64 jh .. + 63 of this row (0 past k_ld)
-        const int c0 = (i - nD) * kStepCodes + 64 * jh;
+        // weak step: the fp16 weak block, columns c0 .. c0 + 8U - 1 of this row (0 past k_ld)
+        const int c0 = (i - nD) * kStepCodes + 8 * U * jh;
         const uint4* src = reinterpret_cast<const uint4*>(p.w_weak + (size_t)row * p.k_ld + c0);
         #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < U; ++v) {
           const uint4 q = (n0 + r < p.N && c0 + 8 * v < p.k_ld) ? src[v] : make_uint4(0, 0, 0, 0);
           d[v >> 2][4 * (v & 3)] = q.x; d[v >> 2][4 * (v & 3) + 1] = q.y;
           d[v >> 2][4 * (v & 3) + 2] = q.z; d[v >> 2][4 * (v & 3) + 3] = q.w;
         }
       }
-      tmem_st16(at, d[0]);
-      tmem_st16(at + 16, d[1]);
+      #pragma unroll
+      for (int h = 0; h < U / 4; ++h) tmem_st16(at + 16 * h, d[h]);
       tmem_st_wait();
       tc_fence_before();
       if (!(p.skip_arrive && i == 0 && threadIdx.x == 64)) mbar_arrive(&afull[s]);
     }
 
     // ---------------- epilogue ----------------
-    const int chalf = jh;
     const bool acc_ok = mbar_wait(accf, 0, p.status, p.wait_limit);
     tc_fence_after();
     const int orow = n0 + r;
     #pragma unroll 1
-    for (int c0 = chalf * (BN / 2); c0 < (chalf + 1) * (BN / 2); c0 += 16) {
+    for (int c0 = jh * (BN / NSL); c0 < (jh + 1) * (BN / NSL); c0 += 16) {
       uint32_t v[16];
       tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
       tmem_ld_wait();
@@ -410,7 +418,7 @@ bool ensure_scratch(void** buf, size_t* have, size_t need, cudaStream_t s) {
   return true;
 }
 
-template <int BITS, int BN, int S>
+template <int BITS, int BN, int S, int DW>
 owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_limit, bool skip_arrive,
                  cudaStream_t s) {
   if (!L.maps_ready) {
@@ -469,7 +477,7 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   } else {
     prm.ws = L.gemm_ws;
   }
-  auto kern = k_gemm_sm100<BITS, BN, S>;
+  auto kern = k_gemm_sm100<BITS, BN, S, DW>;
   constexpr int smem = smem_bytes<BITS, BN, S>();
   static_assert(smem <= 232448, "shared memory budget");
   // one CTA per SM (more than half the shared memory), so its 512 tensor-memory columns are free
@@ -492,7 +500,7 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
                    64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
       return OWQ_ERR_CUDA;
   }
-  kern<<<grid, kThreads, smem, s>>>(mx, L.map_packed, mxw, L.G > 1 ? L.map_sz : mx, prm);
+  kern<<<grid, 32 * (2 + DW), smem, s>>>(mx, L.map_packed, mxw, L.G > 1 ? L.map_sz : mx, prm);
   if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
   if (splits > 1) {
     const size_t MN = (size_t)M * L.N;
@@ -506,9 +514,9 @@ template <int BITS>
 owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, long long wl, bool skip, cudaStream_t s) {
   // wider token tiles dequantise each weight tile once for more tokens (the dequantisation,
   // not the MMA, bounds the narrower tiles); the widest one fits two stages
-  if (M <= 64) return run<BITS, 64, 6>(L, x, y, M, wl, skip, s);
-  if (M <= 256) return run<BITS, 128, 4>(L, x, y, M, wl, skip, s);
-  return run<BITS, 256, 3>(L, x, y, M, wl, skip, s);
+  if (M <= 64) return run<BITS, 64, 6, 8>(L, x, y, M, wl, skip, s);
+  if (M <= 256) return run<BITS, 128, 4, 8>(L, x, y, M, wl, skip, s);
+  return run<BITS, 256, 3, 16>(L, x, y, M, wl, skip, s);
 }
 
 }  // namespace
