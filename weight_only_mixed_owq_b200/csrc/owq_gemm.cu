@@ -97,11 +97,6 @@ __device__ __forceinline__ uint32_t dequant_pair(const uint32_t* w, int j, uint3
   return h2_mul(h2_fma(pair_bits<BITS>(w, j) | kMagic, scl[c], nz[c]), s2);
 }
 
-// byte offset of (row r, 16-byte chunk c) inside a 128-row, 128B-swizzled K-major slab
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
-
 template <int BITS, int BN, int S, int DW>
 __global__ void __launch_bounds__(32 * (2 + DW), 1)
 k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_p,

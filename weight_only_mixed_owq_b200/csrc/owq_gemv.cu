@@ -84,26 +84,64 @@ __device__ __forceinline__ float combine(float a0, float a1, float a2) {
   else return 16777216.f * a0 + 1048576.f * a1;
 }
 
-template <int BITS, int NT>
-__device__ __forceinline__ void zero_acc(float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+template <int NCA, int NT>
+__device__ __forceinline__ void zero_acc(float (&D)[NCA][NT][4]) {
   #pragma unroll
-  for (int cl = 0; cl < (BITS == 3 ? 3 : 2); ++cl)
+  for (int cl = 0; cl < NCA; ++cl)
     #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
       #pragma unroll
       for (int i = 0; i < 4; ++i) D[cl][nt][i] = 0.f;
 }
 
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_splat(__half h) {
+  const uint32_t u = __half_as_ushort(h);
+  return u | (u << 16);
+}
+
+// Dequantisation constants of the two rows (g, g + 8) a lane holds: the scale splat s and,
+// per offset class c, -(1024 / 2^o_c + z) splat.  A code pair at offset o lifted as
+// (bits | 0x6400) = 1024 + q 2^o per half gives (1024 + q 2^o) 2^-o - (1024 2^-o + z) = q - z
+// exactly (one fma.rn.f16x2), then * s rounds once: W_hat = fp16_rn(s (q - z)) bit for bit.
+template <int BITS>
+struct RowDq {
+  static constexpr int NC = BITS == 3 ? 3 : 2;
+  uint32_t s2[2], nz[2][NC];
+  __device__ __forceinline__ void set(int h, __half2 sz) {   // h: 0 = row g, 1 = row g + 8
+    s2[h] = h2_splat(__low2half(sz));
+    const float z = __half2float(__high2half(sz));
+    #pragma unroll
+    for (int c = 0; c < NC; ++c)
+      nz[h][c] = h2_splat(__float2half_rn(-(1024.f / (float)(1 << class_off<BITS>(c)) + z)));
+  }
+};
+template <int BITS>
+__device__ __forceinline__ uint32_t class_scale(int c) {   // 2^-o_c splat (exact)
+  return h2_splat(__float2half_rn(1.f / (float)(1 << class_off<BITS>(c))));
+}
+
+
 // One unit (one 128-code block of a 16-row tile) of one warp: A fragments of rows g, g+8
 // from the staged tile (byte offset fa in shared memory: this lane's chunk), B fragments from
 // the staged activations (byte offsets xv: this lane's four 16-byte fragment pieces of block 0,
 // plus xoff for the block) or from global memory (xg, block b), then 8 k slices of m16n8k16
-// into the offset-class accumulators.  Shared memory is addressed as the kernel's shared array
-// plus 32-bit offsets, so each load is one shared load at register + immediate.
-template <int BITS, int NT, bool XSMEM>
+// into the offset-class accumulators (EXACT: each code pair first dequantised to
+// fp16_rn(s (q - z)), one accumulator).  Shared memory is addressed as the kernel's shared
+// array plus 32-bit offsets, so each load is one shared load at register + immediate.
+template <int BITS, int NT, bool XSMEM, bool EXACT>
 __device__ __forceinline__ void unit_mma(const unsigned char* sm, int fa, const int (&xv)[NT][4], int xoff,
                                          const uint4* const (&xg)[NT], int b, uint32_t k2, uint32_t k4,
-                                         float (&D)[BITS == 3 ? 3 : 2][NT][4]) {
+                                         const RowDq<BITS>& dq, float (&D)[EXACT ? 1 : (BITS == 3 ? 3 : 2)][NT][4]) {
   constexpr int kBlk = 16 * BITS;
   uint32_t wa[BITS], wb[BITS];
   if constexpr (BITS == 4) {
@@ -137,13 +175,25 @@ __device__ __forceinline__ void unit_mma(const unsigned char* sm, int fa, const 
       }
     }
   }
+  constexpr uint32_t kMagic = 0x64006400u;
   #pragma unroll
   for (int s = 0; s < 8; ++s) {
-    const int cl = pair_class<BITS>(2 * s);
-    const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s, k2, k4), pair_bits<BITS>(wb, 2 * s, k2, k4),
-                           pair_bits<BITS>(wa, 2 * s + 1, k2, k4), pair_bits<BITS>(wb, 2 * s + 1, k2, k4)};
-    #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
+    const int cl = pair_class<BITS>(2 * s);   // (pairs 2s and 2s + 1 share the class)
+    if constexpr (EXACT) {
+      const uint32_t sc = class_scale<BITS>(cl);
+      const uint32_t a[4] = {h2_mul(h2_fma(pair_bits<BITS>(wa, 2 * s, k2, k4) | kMagic, sc, dq.nz[0][cl]), dq.s2[0]),
+                             h2_mul(h2_fma(pair_bits<BITS>(wb, 2 * s, k2, k4) | kMagic, sc, dq.nz[1][cl]), dq.s2[1]),
+                             h2_mul(h2_fma(pair_bits<BITS>(wa, 2 * s + 1, k2, k4) | kMagic, sc, dq.nz[0][cl]), dq.s2[0]),
+                             h2_mul(h2_fma(pair_bits<BITS>(wb, 2 * s + 1, k2, k4) | kMagic, sc, dq.nz[1][cl]), dq.s2[1])};
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma16816(D[0][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
+    } else {
+      (void)kMagic;
+      const uint32_t a[4] = {pair_bits<BITS>(wa, 2 * s, k2, k4), pair_bits<BITS>(wb, 2 * s, k2, k4),
+                             pair_bits<BITS>(wa, 2 * s + 1, k2, k4), pair_bits<BITS>(wb, 2 * s + 1, k2, k4)};
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma16816(D[cl][nt], a, xb[nt][2 * s], xb[nt][2 * s + 1]);
+    }
   }
 }
 
@@ -224,6 +274,12 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   constexpr int kWarps = WARPS;
   using G_ = Geo<BITS, SUB>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
+  // 9-16 tokens: each code pair is dequantised to fp16_rn(s (q - z)) in registers (one
+  // accumulator; its cost is shared by two token tiles).  1-8 tokens: the codes are multiplied
+  // as exact q 2^(o - 24) values into offset-class accumulators and the scale and zero point are
+  // applied to each segment's sums (fewer instructions per code).
+  constexpr bool EXACT = NT == 2;
+  constexpr int NCA = EXACT ? 1 : NC;
   constexpr int MT = 8 * NT;                 // token capacity
   constexpr int kStage = G_::stage_bytes(PG);
   extern __shared__ __align__(128) unsigned char smem[];
@@ -248,8 +304,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   // shared memory carve-up (sizes computed identically on the host)
   unsigned char* ring = smem + warp * S * kStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * S * kStage) + warp * S;
-  float* psx = reinterpret_cast<float*>(smem + kWarps * S * kStage + kWarps * S * 8 + 16);   // [MT][Kb+1]
-  __half* xw = reinterpret_cast<__half*>(psx + ((MT * (Kb + 1) + 3) & ~3));                        // [MT][k_ld]
+  float* psx = reinterpret_cast<float*>(smem + kWarps * S * kStage + kWarps * S * 8 + 16);   // [MT][Kb+1] (!EXACT)
+  __half* xw = reinterpret_cast<__half*>(psx + (EXACT ? 0 : ((MT * (Kb + 1) + 3) & ~3)));        // [MT][k_ld]
   uint32_t* xs = reinterpret_cast<uint32_t*>(xw + MT * k_ld);                                      // [M][xstride]
   // row tiles whose segments are all in this CTA: accumulators [lt][16][MT] and segment counts
   // split row tiles: early slots [min(lt_cap, warps)][16][MT] (indexed by tile, or by warp when
@@ -366,20 +422,24 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           m = p / pieces;
           pp = p - m * pieces;
           const uint32_t h[4] = {q[it].x, q[it].y, q[it].z, q[it].w};
-          #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
-            v += f.x;
-            v += f.y;
+          if constexpr (!EXACT) {
+            #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[u]));
+              v += f.x;
+              v += f.y;
+            }
           }
           uint32_t* blk = xs + m * xstride + (pp >> 4) * 64;
           const int j = pp & 15;
           #pragma unroll
           for (int t = 0; t < 4; ++t) blk[t * 16 + 4 * ((j >> 2) ^ t) + (j & 3)] = h[t];
         }
-        #pragma unroll
-        for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (p < total && (pp & 15) == 0) psx[m * (Kb + 1) + (pp >> 4) + 1] = v;
+        if constexpr (!EXACT) {
+          #pragma unroll
+          for (int o = 8; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (p < total && (pp & 15) == 0) psx[m * (Kb + 1) + (pp >> 4) + 1] = v;
+        }
       }
     }
     #pragma unroll 1
@@ -388,9 +448,13 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       xw[e] = (m < M && t < k) ? Pb.x[(size_t)m * K + Pb.idx[t]] : __float2half_rn(0.f);
     }
   } else {
-    // activations stay in global memory: per-block sums and the weak-column gather only
+    // activations stay in global memory (fragment-ordered by k_x_frag): per-block sums (for
+    // the offset-class products) and the weak-column gather only
     const int pieces = K / 8;
-    const int total = M * pieces;
+    const int total = EXACT ? 0 : M * pieces;
+    if (EXACT && lane == 0)
+      for (int j = 1; j < ahead; ++j)
+        if (!issue()) break;
     #pragma unroll 4
     for (int p0 = 0; p0 < total; p0 += blockDim.x) {
       const int p = p0 + threadIdx.x;
@@ -424,7 +488,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   }
   __syncthreads();
   #pragma unroll 1
-  for (int tw = warp; tw < MT; tw += kWarps) {   // prefix sums of the block sums, a warp per token (tokens >= M: zeros)
+  for (int tw = warp; tw < (EXACT ? 0 : MT); tw += kWarps) {   // prefix sums of the block sums, a warp per token (tokens >= M: zeros)
     float* row = psx + tw * (Kb + 1);
     const int per = (Kb + 31) / 32, b_lo = lane * per, b_hi = min(b_lo + per, Kb);
     float run = 0.f;
@@ -443,7 +507,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     }
     if (lane == 0) row[0] = 0.f;
   }
-  __syncthreads();
+  if constexpr (!EXACT) __syncthreads();
   if (lo >= hi) return;   // no work for this warp (no barrier follows)
 
   // per-lane operand offsets in shared memory (tokens >= M are clamped: their columns are
@@ -460,8 +524,9 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   }
   const int fa0 = warp * S * kStage + g * G_::kBlk + tig * 4 * BITS;   // this lane's chunk in stage 0
 
-  float D[NC][NT][4], Dw[NT][4], y[NT][4];
-  zero_acc<BITS, NT>(D);
+  float D[NCA][NT][4], Dw[NT][4], y[NT][4];
+  zero_acc<NCA, NT>(D);
+  RowDq<BITS> dq;
   #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
     #pragma unroll
@@ -478,10 +543,11 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   #pragma unroll 1
   while (cons.next(kind, rt, first, cnt)) {
     if constexpr (!PG) {
-      if (rt != sz_rt) {   // per-channel pairs of a new tile: needed at its segment end
+      if (rt != sz_rt) {   // per-channel pairs of a new tile (EXACT: before its units; else at its segment end)
         sz_rt = rt;
         szA = Pb.sz_t[(size_t)rt * 16 + g];
         szB = Pb.sz_t[(size_t)rt * 16 + g + 8];
+        if constexpr (EXACT) { dq.set(0, szA); dq.set(1, szB); }
       }
     }
     if (ok) {
@@ -513,24 +579,26 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           for (int i = 0; i < 4; ++i) {
             const int tok = 8 * nt + 2 * tig + (i & 1);
             const float sxv = psx[tok * (Kb + 1) + b + 1] - psx[tok * (Kb + 1) + b];
-            const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
+            const float v = combine<BITS>(D[0][nt][i], D[NCA > 1 ? 1 : 0][nt][i], D[NCA - 1][nt][i]);
             const float sc = i < 2 ? gsa : gsb, z = i < 2 ? gza : gzb;
             y[nt][i] = fmaf(sc, fmaf(-z, sxv, v), y[nt][i]);
           }
-        zero_acc<BITS, NT>(D);
+        zero_acc<NCA, NT>(D);
       };
       const int xoff = first * 256;
       if (cnt == SUB) {
         #pragma unroll 4
         for (int bb = 0; bb < SUB; ++bb) {
-          unit_mma<BITS, NT, XSMEM>(smem, fa + bb * G_::kTileBlk, xv, xoff + bb * 256, xg, first + bb, k2, k4, D);
-          if constexpr (PG) fold_block(bb, first + bb);
+          if constexpr (PG && EXACT) { dq.set(0, szs[bb * 16 + g]); dq.set(1, szs[bb * 16 + g + 8]); }
+          unit_mma<BITS, NT, XSMEM, EXACT>(smem, fa + bb * G_::kTileBlk, xv, xoff + bb * 256, xg, first + bb, k2, k4, dq, D);
+          if constexpr (PG && !EXACT) fold_block(bb, first + bb);
         }
       } else {
         #pragma unroll 1
         for (int bb = 0; bb < cnt; ++bb) {
-          unit_mma<BITS, NT, XSMEM>(smem, fa + bb * G_::kTileBlk, xv, xoff + bb * 256, xg, first + bb, k2, k4, D);
-          if constexpr (PG) fold_block(bb, first + bb);
+          if constexpr (PG && EXACT) { dq.set(0, szs[bb * 16 + g]); dq.set(1, szs[bb * 16 + g + 8]); }
+          unit_mma<BITS, NT, XSMEM, EXACT>(smem, fa + bb * G_::kTileBlk, xv, xoff + bb * 256, xg, first + bb, k2, k4, dq, D);
+          if constexpr (PG && !EXACT) fold_block(bb, first + bb);
         }
       }
     }
@@ -545,7 +613,12 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     // end of a tile segment: fold, then store (whole tile) or hand over (split tile)
     if (kind == 1 && cons.segment_done()) {
       const int seg_b0 = first;
-      if constexpr (!PG) {
+      if constexpr (EXACT) {   // the sums are already scaled
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) { y[nt][i] = D[0][nt][i]; D[0][nt][i] = 0.f; }
+      } else if constexpr (!PG) {
         const float2 fa_ = __half22float2(szA), fb_ = __half22float2(szB);
         const float sa = fa_.x, za = fa_.y, sb = fb_.x, zb = fb_.y;
         #pragma unroll
@@ -554,11 +627,11 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
           for (int i = 0; i < 4; ++i) {
             const int tok = 8 * nt + 2 * tig + (i & 1);
             const float sxv = psx[tok * (Kb + 1) + seg_b1] - psx[tok * (Kb + 1) + seg_b0];
-            const float v = combine<BITS>(D[0][nt][i], D[1][nt][i], D[NC - 1][nt][i]);
+            const float v = combine<BITS>(D[0][nt][i], D[NCA > 1 ? 1 : 0][nt][i], D[NCA - 1][nt][i]);
             const float sc = i < 2 ? sa : sb, z = i < 2 ? za : zb;
             y[nt][i] = sc * fmaf(-z, sxv, v);
           }
-        zero_acc<BITS, NT>(D);
+        zero_acc<NCA, NT>(D);
       }
       #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
@@ -786,7 +859,7 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
   for (int q = 0; q < a.count; ++q) {
     const GemvProblem& Pq = a.p[q];
     const int Kb = Pq.K / kBlockCodes;
-    const size_t need = (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float) + (size_t)MT * Pq.k_ld * sizeof(__half);
+    const size_t need = (NT == 2 ? 0 : (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float)) + (size_t)MT * Pq.k_ld * sizeof(__half);
     if (need > extra) extra = need;
     const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
     if (xb > xbytes) xbytes = xb;
