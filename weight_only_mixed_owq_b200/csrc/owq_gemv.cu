@@ -268,17 +268,17 @@ __global__ void k_x_frag(const __half* __restrict__ x, int M, int K, uint32_t* _
   }
 }
 
-template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM, bool PG>
+template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM, bool PG, bool EXACT>
 __global__ void __launch_bounds__(WARPS * 32, 1)
 k_gemv_mma(const __grid_constant__ GemvArgs args) {
   constexpr int kWarps = WARPS;
   using G_ = Geo<BITS, SUB>;
   constexpr int NC = BITS == 3 ? 3 : 2;      // offset classes
-  // 9-16 tokens: each code pair is dequantised to fp16_rn(s (q - z)) in registers (one
-  // accumulator; its cost is shared by two token tiles).  1-8 tokens: the codes are multiplied
-  // as exact q 2^(o - 24) values into offset-class accumulators and the scale and zero point are
-  // applied to each segment's sums (fewer instructions per code).
-  constexpr bool EXACT = NT == 2;
+  // EXACT (9-16 tokens; per-group layers from 4 tokens): each code pair is dequantised to
+  // fp16_rn(s (q - z)) in registers, one accumulator, the cost shared by the tokens.
+  // Otherwise the codes are multiplied as exact q 2^(o - 24) values into offset-class
+  // accumulators and the scale and zero point are applied to the sums (fewer instructions
+  // per code at 1 token).
   constexpr int NCA = EXACT ? 1 : NC;
   constexpr int MT = 8 * NT;                 // token capacity
   constexpr int kStage = G_::stage_bytes(PG);
@@ -775,6 +775,10 @@ int sm_count() {
   return n;
 }
 
+// Exact per-pair dequantisation (see the kernel) for two token tiles, and for per-group layers
+// from 4 tokens (their per-block scale fold costs more than the exact form there)
+inline bool gemv_exact(int NT, bool pg, int M) { return NT == 2 || (pg && M >= 4); }
+
 template <int BITS, int NT, int WARPS, int SUB, int S, bool XSMEM>
 cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
   if constexpr (!XSMEM) {
@@ -785,8 +789,16 @@ cudaError_t launch_k(GemvArgs& a, size_t smem, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  auto kern = a.p[0].G > 1 ? k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, true>
-                           : k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, false>;
+  void (*kern)(GemvArgs);
+  const bool pg = a.p[0].G > 1;
+  if constexpr (NT == 2) {
+    kern = pg ? k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, true, true>
+              : k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, false, true>;
+  } else {
+    kern = pg ? (gemv_exact(NT, true, a.M) ? k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, true, true>
+                                           : k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, true, false>)
+              : k_gemv_mma<BITS, NT, WARPS, SUB, S, XSMEM, false, false>;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int base = 0;
@@ -859,7 +871,8 @@ cudaError_t launch_t(GemvArgs& a, cudaStream_t s) {
   for (int q = 0; q < a.count; ++q) {
     const GemvProblem& Pq = a.p[q];
     const int Kb = Pq.K / kBlockCodes;
-    const size_t need = (NT == 2 ? 0 : (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float)) + (size_t)MT * Pq.k_ld * sizeof(__half);
+    const size_t need = (gemv_exact(NT, Pq.G > 1, a.M) ? 0 : (size_t)((MT * (Kb + 1) + 3) & ~3) * sizeof(float)) +
+                        (size_t)MT * Pq.k_ld * sizeof(__half);
     if (need > extra) extra = need;
     const size_t xb = (size_t)a.M * (Pq.K / 2 + 4) * sizeof(uint32_t);
     if (xb > xbytes) xbytes = xb;
