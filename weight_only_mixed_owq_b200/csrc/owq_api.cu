@@ -66,14 +66,12 @@ void release(Layer* L) {
   cudaFree(L->zeros);
   cudaFree(L->w_weak);
   cudaFree(L->idx);
-  cudaFree(L->blk_weak);
   cudaFree(L->w_weak_t);
   cudaFree(L->sz_t);
   cudaFree(L->xfrag);
   cudaFree(L->gemm_ws);
   cudaFree(L->gemm_xw);
   cudaFree(L->part);
-  delete[] L->idx_host;
   L->magic = 0;
   delete L;
 }
@@ -164,10 +162,6 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   const size_t packed_bytes = (size_t)((N + 15) & ~15) * K * bits / 8;   // 16-row tiles
   const size_t sz_bytes = (size_t)N * L->G * sizeof(__half);
   const size_t weak_bytes = (size_t)N * L->k_ld * sizeof(__half);
-  const int Kb = K / kBlockCodes;
-  L->idx_host = new (std::nothrow) int32_t[std::max(k, 1)];
-  if (!L->idx_host) { release(L); return OWQ_ERR_NOMEM; }
-  std::copy(hidx.begin(), hidx.end(), L->idx_host);
 
   cudaError_t e = cudaSuccess;
   auto alloc = [&](void** p, size_t n) { if (e == cudaSuccess) e = cudaMalloc(p, std::max<size_t>(n, 16)); };
@@ -176,7 +170,6 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   alloc((void**)&L->zeros, sz_bytes);
   alloc((void**)&L->w_weak, weak_bytes);
   alloc((void**)&L->idx, sizeof(int32_t) * std::max(k, 1));
-  alloc((void**)&L->blk_weak, sizeof(int32_t) * (Kb + 1));
   const size_t RT = (size_t)(N + 15) / 16;
   const size_t weak_t_bytes = RT * 16 * L->k_ld * sizeof(__half);
   int sms = 0;
@@ -195,14 +188,9 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   alloc((void**)&mask_dev, sizeof(uint32_t) * (K / 32));
   if (e != cudaSuccess) { cudaFree(mask_dev); release(L); return cuda_status(e); }
 
-  // host-side tables: weak bitmask per 32-code chunk, weak range per 128-code block
+  // host-side table: weak bitmask per 32-code chunk
   std::vector<uint32_t> mask(K / 32, 0u);
-  std::vector<int32_t> blk(Kb + 1, 0);
   for (int t = 0; t < k; ++t) mask[hidx[t] / 32] |= 1u << (hidx[t] % 32);
-  for (int b = 0, t = 0; b <= Kb; ++b) {
-    while (t < k && hidx[t] < b * kBlockCodes) ++t;
-    blk[b] = t;
-  }
 
   if (e == cudaSuccess) e = cudaMemsetAsync(L->packed, 0, packed_bytes, s);   // padding rows of the last tile
   if (e == cudaSuccess) e = cudaMemcpyAsync(L->scales, scales, sz_bytes, cudaMemcpyDeviceToDevice, s);
@@ -212,7 +200,6 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
     e = cudaMemcpy2DAsync(L->w_weak, (size_t)L->k_ld * sizeof(__half), w_weak, (size_t)k * sizeof(__half),
                           (size_t)k * sizeof(__half), N, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess && k > 0) e = cudaMemcpyAsync(L->idx, idx, sizeof(int32_t) * k, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(L->blk_weak, blk.data(), sizeof(int32_t) * (Kb + 1), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(mask_dev, mask.data(), sizeof(uint32_t) * (K / 32), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(L->part, 0, part_bytes, s);   // epoch 0: never a live tag
   if (e == cudaSuccess)

@@ -27,9 +27,6 @@ struct Layer {
   __half* zeros;        // N x G
   __half* w_weak;       // N x k_ld (zero padded)
   int32_t* idx;         // k (device)
-  int32_t* blk_weak;    // K/128 + 1 offsets into idx: weak columns of packed block b are
-                        // idx[blk_weak[b] .. blk_weak[b+1])
-  int32_t* idx_host;    // k (host copy)
   __half* w_weak_t;     // the weak block tile-major: [N/16 tiles][k_ld/16 slices][16 rows][16]
   __half2* sz_t;        // (scale, zero) pairs tile-major: [N/16 tiles][G][16 rows] (rows >= N: (0, 0))
   uint32_t* xfrag;      // decode scratch: up to 16 activation rows in fragment order (see owq_gemv.cu)
@@ -47,7 +44,6 @@ struct Layer {
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
   alignas(64) CUtensorMap map_packed;
-  alignas(64) CUtensorMap map_weak;    // the weak block [N][k_ld], 128 x 64 boxes, 128B swizzle
   alignas(64) CUtensorMap map_sz;      // (scale, zero) pairs of per-group layers
 };
 
