@@ -293,3 +293,30 @@ def test_bits_per_weight_reproduces_page_numbers():
     b = oracle.layer_bytes(4096, 4096, 3, 4096, 32)
     tot = 8.0 * sum(b.values()) / (4096 * 4096)
     assert tot == pytest.approx(oracle.bits_per_weight(4096, 3, 32, "latency", group=4096, N=4096))
+
+
+def test_single_output_bound_accepts_unrounded_weights_and_rejects_mistakes():
+    """The analytic check used for one-element decode outputs (tests/owq_checks.py) holds for the
+    product of the unrounded dequantised weights s (q - z) and fails for a dropped weak term, a
+    zero point off by one or a 10% scale error."""
+    from tests.owq_checks import check_output_short
+    N, K, bits, group, k = 1, 128, 3, 128, 1
+    d = owq_synth.draw_small(N, K, 8, 16, seed=4129, n_outliers=1)
+    ref = oracle.owq_quantize(d["W"], d["X"], bits, group, k)
+    W_hat = oracle.dequant(ref["codes"], ref["scales"], ref["zeros"])
+    x = d["x"][:1]
+    y64 = oracle.matmul(W_hat, ref["w_weak"], ref["idx"], x)
+    s = ref["scales"].astype(np.float64)[:, :1]
+    z = ref["zeros"].astype(np.float64)[:, :1]
+    xw = x[:, ref["idx"]].astype(np.float64) @ ref["w_weak"].astype(np.float64).T
+
+    def product(scale, zero, weak):
+        w = scale * (ref["codes"].astype(np.float64) - zero)
+        w[:, ref["idx"]] = 0.0
+        return (x.astype(np.float64) @ w.T + weak).astype(np.float16)
+
+    check_output_short(product(s, z, xw), W_hat, ref["w_weak"], ref["idx"], x, y64, "unrounded")
+    # (at this near-cancelled output the bound is ~5% of |y|: a 10% scale error must fail)
+    for bad in (product(s, z, 0.0 * xw), product(s, z + 1, xw), product(s * 1.1, z, xw)):
+        with pytest.raises(AssertionError):
+            check_output_short(bad, W_hat, ref["w_weak"], ref["idx"], x, y64, "planted")
