@@ -178,7 +178,8 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
  * serialised.  The handle's scratch (M * k_ld * 2 bytes of weak activations; for few row
  * tiles also a split-K workspace) grows on the first call that needs more, which must not
  * be inside a stream capture: there a too-small weak-activation scratch gives OWQ_ERR_NOMEM
- * (the split-K workspace falls back to one split).
+ * (the split-K workspace falls back to one split).  Calls on one handle must be ordered
+ * (same stream, or synchronised): they share that scratch.
  */
 owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
                       owq_stream_t stream);
