@@ -12,25 +12,25 @@
 //    is no barrier after the prologue.
 //  * A warp streams its chunk through a private S-stage shared-memory ring filled by
 //    cp.async.bulk: the layer stores each 16-row tile block-major, so an item (16 rows x up to
-//    4 blocks of one tile) is one contiguous copy; the weak block, stored tile-major too, is
-//    streamed the same way at the start of each tile.
+//    4 or 8 blocks of one tile) is one contiguous copy; the weak block, stored tile-major too,
+//    is streamed the same way at the start of each tile.
 //  * The contraction runs on the tensor cores (mma.sync m16n8k16, fp16 x fp16 -> fp32): with
 //    the packed layout of owq_format.cuh a lane's chunk of a block is exactly its A fragment,
 //    and one AND per code pair makes each A register (the codes as exact fp16 values
 //    q * 2^(o - 24), o the bit offset; one accumulator per offset class).  Activations are the
 //    B fragment (up to 8 tokens per n8 tile, two tiles for M > 8), staged once per CTA in
 //    fragment order.  This keeps the issued work per code low enough for the HBM rate.
-//  * Scale and zero point: for a group with scale s and zero z,
+//  * Scale and zero point, 1-8 tokens: for a group with scale s and zero z,
 //        sum_j s (q_j - z) x_j = s * (sum_j q_j x_j - z * sum_j x_j);
-//    the activation sums come from per-block prefix sums computed once per CTA.  (The fp16
-//    rounding of each s (q - z) is not applied; the difference is far inside the tolerance.)
+//    the activation sums come from per-block prefix sums computed once per CTA (the product
+//    of the unrounded dequantised weights).  9-16 tokens, and per-group layers from 4 tokens:
+//    each code pair is dequantised in registers to fp16_rn(s (q - z)), the oracle's W_hat bit
+//    for bit (two fp16x2 operations per pair, shared by the tokens), into one accumulator.
 //  * A row tile split between warps: the segments inside one CTA leave their partial sums in
 //    shared memory and the last to arrive (a CTA-scope counter) adds them in unit order; across
 //    CTAs, each CTA's sum is published as 64-bit words tagged with the call's epoch (no counter
-//    or fence) and the CTA holding the tile's last units adds them in CTA order.  Without room
-//    for the in-CTA area, each segment is published the same way and the warp holding the last
-//    unit adds them in segment order.  Every sum runs in a fixed order: the output is the same
-//    bit for bit on every call.
+//    or fence) and the CTA holding the tile's last units adds them in CTA order.  Every sum
+//    runs in a fixed order: the output is the same bit for bit on every call.
 #include "owq_format.cuh"
 #include "owq_internal.cuh"
 #include "owq_sm100.cuh"
