@@ -41,7 +41,10 @@ using namespace sm100;
 
 constexpr int kBM = 128;               // weight rows per tile (MMA M)
 constexpr int kStepCodes = 128;        // K per pipeline step
-constexpr uint32_t kTmemCols = 512;    // accumulator (BN <= 256 columns) + S <= 4 A stages of 64
+// tensor-memory columns of a CTA: the accumulator (BN) + S A stages of 64, as a power of two;
+// 256 lets two CTAs share an SM
+template <int BN, int S>
+constexpr uint32_t tmem_cols() { return BN + 64 * S <= 256 ? 256u : 512u; }
 
 template <int BITS, int BN>
 struct Smem {
@@ -133,7 +136,7 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   }
   // tensor memory: the accumulator (BN columns) then S A stages of 64 columns (128 rows x 128
   // fp16 codes, two per 32-bit column)
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 1) tmem_alloc(tmem_slot, tmem_cols<BN, S>());
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -311,7 +314,7 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, tmem_cols<BN, S>());
     tmem_relinquish();
   }
 }
@@ -475,9 +478,10 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   auto kern = k_gemm_sm100<BITS, BN, S, DW>;
   constexpr int smem = smem_bytes<BITS, BN, S>();
   static_assert(smem <= 232448, "shared memory budget");
-  // one CTA per SM (more than half the shared memory), so its 512 tensor-memory columns are free
-  static_assert(smem > 232448 / 2, "one CTA per SM");
-  static_assert(BN + 64 * S <= (int)kTmemCols, "tensor memory: accumulator + A stages");
+  // the CTAs an SM can hold (by shared memory) never need more than its 512 tensor-memory
+  // columns, so an allocation never waits
+  static_assert(BN + 64 * S <= (int)tmem_cols<BN, S>(), "tensor memory: accumulator + A stages");
+  static_assert((232448 / smem) * tmem_cols<BN, S>() <= 512, "tensor memory per SM");
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return OWQ_ERR_CUDA;
