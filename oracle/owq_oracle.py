@@ -37,6 +37,9 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
   matmul                      pinned: k = K reproduces W x exactly; k = 0 is the plain quantised
                               product; the RTN error bound; brute force on tiny shapes.
   bits_per_weight             pinned: the pages' 3.01 -> 3.012 and 0.21% figures.
+  weak_grad                   pinned: directional derivative of the pinned forward product
+                              (the loss is linear in the weak block).
+  input_grad                  pinned: adjoint identity against the pinned forward product.
 """
 from __future__ import annotations
 
@@ -53,6 +56,8 @@ __all__ = [
     "unpack",
     "matmul",
     "matmul_rows",
+    "weak_grad",
+    "input_grad",
     "bits_per_weight",
     "layer_bytes",
 ]
@@ -297,6 +302,41 @@ def matmul_rows(codes, scales, zeros, w_weak, idx, x, rows) -> np.ndarray:
     rows = np.asarray(rows, dtype=np.int64)
     W_hat = dequant(np.asarray(codes)[rows], np.asarray(scales)[rows], np.asarray(zeros)[rows])
     return matmul(W_hat, np.asarray(w_weak)[rows], idx, x)
+
+
+# ----------------------------------------------------------------------------------------
+# Weak column tuning: the two gradients a frozen OWQ layer passes back
+# ----------------------------------------------------------------------------------------
+def weak_grad(x: np.ndarray, dy: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """dW_weak[i, t] = sum_m dy[m, i] x[m, idx[t]]   (fp64, N x k).
+
+    [PL] "Weak Column Tuning" (paper "PEFT with Weak Column Tuning", p.5) and "WCT-based
+    fine-tuning" (p.7): only the fp16 weak columns are trained, the packed low-bit matrix stays
+    frozen.  The forward term that holds them is sum_t W_weak[i, t] x[m, idx[t]], so the
+    gradient of a loss with output gradient dy is the product of dy^T and the gathered
+    activation columns.
+    """
+    dy64 = np.asarray(dy, dtype=F16).astype(F64)
+    x64 = np.asarray(x, dtype=F16).astype(F64)
+    idx = np.asarray(idx, dtype=np.int64)
+    return dy64.T @ x64[:, idx]
+
+
+def input_grad(W_hat: np.ndarray, w_weak: np.ndarray, idx: np.ndarray, dy: np.ndarray) -> np.ndarray:
+    """dX[m, j] = sum_i dy[m, i] W_hat[i, j] + sum_{t: idx[t] = j} sum_i dy[m, i] W_weak[i, t]
+    (fp64, M x K).
+
+    The gradient a frozen OWQ layer passes to the layer below during weak column tuning
+    ([PL] "Weak Column Tuning", p.5: the dense matrix stays frozen, earlier layers' weak
+    columns still need it): the transpose of the forward product of [PL] "Real-device
+    acceleration", with the weak columns' fp16 values in place of the zero-filled codes.
+    """
+    dy64 = np.asarray(dy, dtype=F16).astype(F64)
+    dx = dy64 @ np.asarray(W_hat, dtype=F16).astype(F64)
+    idx = np.asarray(idx, dtype=np.int64)
+    if idx.size:
+        dx[:, idx] += dy64 @ np.asarray(w_weak, dtype=F16).astype(F64)
+    return dx
 
 
 # ----------------------------------------------------------------------------------------

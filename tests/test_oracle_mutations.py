@@ -133,3 +133,30 @@ def test_mutant_latency_bits_without_zero_fill_is_caught(monkeypatch):
     _patch(monkeypatch, "bits_per_weight", bad)
     with pytest.raises(AssertionError):
         pins.test_bits_per_weight_reproduces_page_numbers()
+
+
+def test_mutant_input_grad_without_weak_term_is_caught(monkeypatch):
+    def bad(W_hat, w_weak, idx, dy):
+        return np.asarray(dy, dtype=F16).astype(F64) @ np.asarray(W_hat, dtype=F16).astype(F64)
+    _patch(monkeypatch, "input_grad", bad)
+    with pytest.raises(AssertionError):
+        pins.test_input_grad_is_adjoint_of_forward_product(3, 256, 5, 3)
+
+
+def test_mutant_input_grad_weak_term_at_wrong_columns_is_caught(monkeypatch):
+    orig = oo.input_grad
+
+    def bad(W_hat, w_weak, idx, dy):
+        return orig(W_hat, w_weak, np.minimum(np.asarray(idx) + 1, np.asarray(W_hat).shape[1] - 1), dy)
+    _patch(monkeypatch, "input_grad", bad)
+    with pytest.raises(AssertionError):
+        pins.test_input_grad_is_adjoint_of_forward_product(4, 128, 9, 1)
+
+
+def test_mutant_weak_grad_wrong_gather_is_caught(monkeypatch):
+    def bad(x, dy, idx):
+        k = len(idx)
+        return np.asarray(dy, dtype=F16).astype(F64).T @ np.asarray(x, dtype=F16).astype(F64)[:, :k]
+    _patch(monkeypatch, "weak_grad", bad)
+    with pytest.raises(AssertionError):
+        pins.test_weak_grad_is_directional_derivative_of_forward_product(5, 3)

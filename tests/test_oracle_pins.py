@@ -320,3 +320,57 @@ def test_single_output_bound_accepts_unrounded_weights_and_rejects_mistakes():
     for bad in (product(s, z, 0.0 * xw), product(s, z + 1, xw), product(s * 1.1, z, xw)):
         with pytest.raises(AssertionError):
             check_output_short(bad, W_hat, ref["w_weak"], ref["idx"], x, y64, "planted")
+
+
+# ------------------------------------------------------------------ weak column tuning gradients
+def _wct_case(bits, group, k, M, seed):
+    d = owq_synth.draw_small(12, 256, M, 32, seed=seed)
+    r = oracle.owq_quantize(d["W"], d["X"], bits, group, k)
+    W_hat = oracle.dequant(r["codes"], r["scales"], r["zeros"])
+    rng = np.random.default_rng(seed + 1)
+    dy = rng.standard_normal((M, 12)).astype(F16)
+    return d, r, W_hat, dy
+
+
+@pytest.mark.parametrize("bits,group,k,M", [(3, 256, 5, 3), (4, 128, 9, 1), (3, 128, 0, 2)])
+def test_input_grad_is_adjoint_of_forward_product(bits, group, k, M):
+    """<dy, y(x)> = <dX(dy), x> for every x: the forward product (pinned above) is linear in
+    x, so its adjoint is fixed by it; checked on several random x."""
+    d, r, W_hat, dy = _wct_case(bits, group, k, M, seed=70 + k)
+    dx = oracle.input_grad(W_hat, r["w_weak"], r["idx"], dy)
+    rng = np.random.default_rng(5)
+    for _ in range(3):
+        x = rng.standard_normal((M, 256)).astype(F16)
+        y = oracle.matmul(W_hat, r["w_weak"], r["idx"], x)
+        lhs = float((dy.astype(F64) * y).sum())
+        rhs = float((dx * x.astype(F64)).sum())
+        assert rhs == pytest.approx(lhs, rel=1e-12, abs=1e-12)
+    # one-hot x reads single entries: dX[m, j] = <dy[m], y(e_j)[m]>
+    for j in [0, 17, 255] + [int(v) for v in r["idx"][:2]]:
+        x = np.zeros((M, 256), dtype=F16)
+        x[:, j] = 1
+        y = oracle.matmul(W_hat, r["w_weak"], r["idx"], x)
+        for m in range(M):
+            assert dx[m, j] == pytest.approx(float((dy[m].astype(F64) * y[m]).sum()), rel=1e-12, abs=1e-14)
+
+
+@pytest.mark.parametrize("k,M", [(5, 3), (1, 7)])
+def test_weak_grad_is_directional_derivative_of_forward_product(k, M):
+    """The loss <dy, y> is linear in the weak block, so for any direction V the derivative
+    <dW_weak, V> equals <dy, y(W_hat = 0, W_weak = V)> exactly (the forward product pinned
+    above, with the dense part switched off)."""
+    d, r, W_hat, dy = _wct_case(3, 256, k, M, seed=90 + k)
+    g = oracle.weak_grad(d["x"], dy, r["idx"])
+    assert g.shape == (12, k)
+    rng = np.random.default_rng(9)
+    zero = np.zeros_like(W_hat)
+    for _ in range(3):
+        V = rng.standard_normal((12, k)).astype(F16)
+        y = oracle.matmul(zero, V, r["idx"], d["x"])
+        assert float((g * V.astype(F64)).sum()) == pytest.approx(float((dy.astype(F64) * y).sum()), rel=1e-12)
+    # a unit direction isolates one entry
+    for i, t in [(0, 0), (11, k - 1), (5, k // 2)]:
+        V = np.zeros((12, k), dtype=F16)
+        V[i, t] = 1
+        y = oracle.matmul(zero, V, r["idx"], d["x"])
+        assert g[i, t] == pytest.approx(float((dy.astype(F64) * y).sum()), rel=1e-12, abs=1e-14)
