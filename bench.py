@@ -469,6 +469,62 @@ def prefill_measure(args, dev):
             "timing": "median of 10 single launches, L2 flushed between launches"}
 
 
+def wct_measure(args, dev):
+    """Weak column tuning kernels on the OPT-6.7B-shaped layers (3-bit per channel, k = K/128):
+    owq_input_grad (dX = dY W_eff from the packed layout; HBM-bound, GB/s of its algorithmic
+    bytes: packed + scales/zeros + weak block + idx + dY + dX) and owq_weak_grad
+    (dW_weak = dY^T x[:, idx]; bytes dY + the gathered x columns + fp32 dW_weak)."""
+    import torch
+
+    import weight_only_mixed_owq_b200 as owq
+    spec = owq_synth.WORKLOADS[1]
+    peaks, kind = measured_peaks()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        times = []
+        for _ in range(10):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        return statistics.median(times) * 1e-3
+
+    out = {}
+    for li in (0, 4, 5):   # q (4096 x 4096), fc1 (16384 x 4096), fc2 (4096 x 16384)
+        L = spec.layers[li]
+        d = owq_synth.draw_layer(L, spec, 16, owq_synth.seed_for(1, li))
+        W, X = torch.from_numpy(d["W"]).to(dev), torch.from_numpy(d["X"]).to(dev)
+        lay, _ = owq.quantize_pack(W, X, L.bits, L.group, L.k)
+        del W, X
+        wbytes = L.N * L.K * L.bits // 8 + L.N * (L.K // L.group) * 4 + L.N * L.k * 2 + 4 * L.k
+        row = {}
+        for M in (1, 16):
+            dy = torch.randn((M, L.N), device=dev).half()
+            dx = torch.empty((M, L.K), dtype=torch.float16, device=dev)
+            t = timed(lambda: lay.input_grad(dy, dx))
+            B = wbytes + 2 * M * L.N + 2 * M * L.K
+            row[f"input_grad_M{M}"] = {"us": round(t * 1e6, 2), "GBps": round(B / t / 1e9, 1),
+                                       "frac_hbm": round(B / t / 1e9 / peaks["hbm_gbs"], 4)}
+        for M in (16, 2048):
+            x = torch.randn((M, L.K), device=dev).half()
+            dy = torch.randn((M, L.N), device=dev).half()
+            dw = torch.empty((L.N, L.k), dtype=torch.float32, device=dev)
+            t = timed(lambda: lay.weak_grad(x, dy, dw))
+            B = 2 * M * L.N + 2 * M * L.k + 4 * L.N * L.k
+            row[f"weak_grad_M{M}"] = {"us": round(t * 1e6, 2), "GBps": round(B / t / 1e9, 1),
+                                      "TFLOPs": round(2.0 * M * L.N * L.k / t / 1e12, 2)}
+        out[f"{L.name} {L.N}x{L.K} k={L.k}"] = row
+        lay.close()
+    return {"layers": out, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_kind": kind,
+            "timing": "median of 10 single launches, L2 flushed between launches"}
+
+
 # ---------------------------------------------------------------------------------- oracle arm
 def oracle_sample(wl: str, rows: int):
     """Quantise (oracle) one layer set and keep the first `rows` rows of each layer."""
@@ -559,6 +615,7 @@ def main(argv=None):
     ap.add_argument("--depth", type=int, default=0, help="resident layer sets per step (default: model depth)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-wct", action="store_true", help="skip the weak column tuning kernels")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
@@ -574,6 +631,8 @@ def main(argv=None):
         import torch
         if not args.no_prefill:
             line["prefill"] = prefill_measure(args, torch.device("cuda", local))
+        if not args.no_wct:
+            line["wct"] = wct_measure(args, torch.device("cuda", local))
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload)
     if rank == 0:

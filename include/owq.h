@@ -185,6 +185,40 @@ owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
                       owq_stream_t stream);
 
 /*
+ * owq_weak_grad -- weak column tuning: gradient of a loss with respect to the layer's fp16
+ * weak block ("PEFT with Weak Column Tuning", paper p.5, and "WCT-based fine-tuning",
+ * p.7: only the weak columns are trained, the packed low-bit matrix stays frozen).
+ *   dw_weak[i][t] = sum_m dy[m][i] * x[m][idx[t]]
+ * In:  x fp16 M x K row-major (the layer's forward input), dy fp16 M x N row-major (the
+ *      gradient of its output); 1 <= M <= 65536.
+ * Out: dw_weak fp32 N x k row-major (fully overwritten; may be NULL when k == 0, and then
+ *      nothing is launched).  fp32 accumulation in token order.  No scratch, no waits.
+ * Device pointers, 16-byte aligned (OWQ_ERR_ALIGN); asynchronous on `stream`.
+ */
+owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t* dy,
+                           float* dw_weak, int M, owq_stream_t stream);
+
+/*
+ * owq_input_grad -- weak column tuning: the gradient the frozen layer passes to its input
+ * (same pages; earlier layers' weak columns need it), the transposed product
+ *   dx[m][j] = sum_i dy[m][i] * W_eff[i][j],
+ * W_eff = W_hat = fp16_rn(s * (q - z)) except at the weak columns, which take their fp16
+ * values from the weak block.  Read straight from the packed layout (no W_hat in memory),
+ * fp32 accumulation, one fp16 rounding of each output.
+ * In:  dy fp16 M x N row-major; 1 <= M <= 65536 (one pass over the packed weights per 16
+ *      tokens).  Out: dx fp16 M x K row-major (fully overwritten).
+ * The rows are split over CTAs; their fp32 partial sums go to a workspace the handle owns
+ * (slices x 16 tokens x K x 4 bytes, with about 2 x SMs / (K / 128) slices: 2.6 MB at
+ * K = 4096 on 148 SMs), allocated on the first call that needs it; that first call must not be inside a stream capture (inside one, a
+ * handle without the workspace runs one slice per column block: slower, same result).
+ * The last CTA of each column block adds the slices in a fixed order: repeated calls give
+ * identical bits.  Calls on one handle must be ordered (one stream, or events between
+ * streams): they share that workspace.  Device pointers, 16-byte aligned; asynchronous.
+ */
+owq_status_t owq_input_grad(owq_layer_t layer, const uint16_t* dy, uint16_t* dx, int M,
+                            owq_stream_t stream);
+
+/*
  * owq_dequant -- test hook: write W_hat = fp16_rn(s * (q - z)) (N x K fp16, 0 at the weak
  * columns) and, if codes is not NULL, the unpacked codes (N x K uint8).
  */

@@ -1,0 +1,130 @@
+"""Parity of the weak column tuning kernels with the CPU oracle, through the C ABI.
+
+owq_input_grad (fp16 dX = dY W_eff, read from the packed layout) is held to the output
+tolerance of tests/owq_checks.py against the oracle's fp64 input_grad.  owq_weak_grad (fp32
+dW_weak = dY^T x[:, idx]) is held to the fp32 accumulation bound: the fp16 x fp16 products
+are exact in fp32, so each of the M additions adds at most 2^-24 of the running sum.
+Layers are quantised by the oracle and packed by owq_pack; no expected value comes from the
+GPU.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import owq_synth
+from tests.owq_checks import check_output
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+F64 = np.float64
+
+# (name, N, K, bits, group, k, token counts, channels forced weak)
+CASES = [
+    ("one-slice", 48, 256, 3, 256, 3, (1, 2), None),
+    ("ragged-n200", 200, 640, 3, 640, 7, (1, 5, 16), None),
+    ("g128-b4-two-passes", 200, 640, 4, 128, 7, (3, 37), None),
+    ("k0", 96, 384, 3, 128, 0, (4,), None),
+    ("many-slices", 1000, 1280, 3, 128, 13, (16,), None),
+    ("edges-pair-weak", 130, 1024, 4, 1024, 6, (8,), (0, 1023, 2, 3, 511, 512)),
+]
+
+
+def _gpu(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def _layer(owq, ref, bits, group):
+    k = len(ref["idx"])
+    return owq.OwqLayer(_gpu(ref["codes"]), _gpu(ref["scales"]), _gpu(ref["zeros"]),
+                        _gpu(ref["idx"]) if k else None, _gpu(ref["w_weak"]) if k else None, bits, group)
+
+
+def _dy(M, N, seed):
+    return owq_synth.rng(seed).standard_normal((M, N), dtype=np.float32).astype(np.float16)
+
+
+def _check_weak_grad(got, x, dy, idx, where):
+    want = oracle.weak_grad(x, dy, idx)
+    got = np.asarray(got, dtype=F64)
+    assert got.shape == want.shape
+    terms = np.abs(dy.astype(F64)).T @ np.abs(x.astype(F64)[:, idx])
+    bound = dy.shape[0] * 2.0 ** -24 * terms + 1e-30
+    err = np.abs(got - want)
+    assert np.all(err <= bound), f"{where}: weak grad error {float(err.max()):.3g}"
+
+
+def _case(case):
+    name, N, K, bits, group, k, Ms, forced = case
+    d = owq_synth.draw_small(N, K, max(Ms), 48, seed=2000 + N + K + k, n_outliers=0 if forced else min(3, k))
+    if forced:
+        ch = np.array(forced)
+        d["X"][:, ch] = (d["X"][:, ch].astype(np.float32) * 50).astype(np.float16)
+    ref = oracle.owq_quantize(d["W"], d["X"], bits, group, k)
+    if forced:
+        assert set(forced) <= set(ref["idx"].tolist())
+    return d, ref
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_wct_gradients_match_oracle(case):
+    import weight_only_mixed_owq_b200 as owq
+    name, N, K, bits, group, k, Ms, forced = case
+    d, ref = _case(case)
+    W_hat = oracle.dequant(ref["codes"], ref["scales"], ref["zeros"])
+    layer = _layer(owq, ref, bits, group)
+    for M in Ms:
+        dy = _dy(M, N, 31 + M)
+        x = d["x"][:M]
+        dy_g, x_g = _gpu(dy), _gpu(x)
+        dx = layer.input_grad(dy_g)
+        dx2 = layer.input_grad(dy_g)
+        dw = layer.weak_grad(x_g, dy_g)
+        torch.cuda.synchronize()
+        check_output(dx.cpu().numpy(), oracle.input_grad(W_hat, ref["w_weak"], ref["idx"], dy),
+                     f"{name} input_grad M={M}")
+        assert torch.equal(dx.view(torch.int16), dx2.view(torch.int16)), "repeat differs"
+        if k:
+            _check_weak_grad(dw.cpu().numpy(), x, dy, ref["idx"], f"{name} M={M}")
+    layer.close()
+
+
+def test_wct_gradients_fullsize_opt67b_attention_layer():
+    """4096 x 4096, 3-bit per channel, k = 32 (the OPT-6.7B q/k/v/out shape), in the launch
+    configuration bench.py times; every output compared."""
+    import weight_only_mixed_owq_b200 as owq
+    spec = owq_synth.WORKLOADS[1]
+    L = spec.layers[0]
+    d = owq_synth.draw_layer(L, spec, 16, owq_synth.seed_for(1, 0))
+    ref = oracle.owq_quantize(d["W"], d["X"], L.bits, L.group, L.k)
+    W_hat = oracle.dequant(ref["codes"], ref["scales"], ref["zeros"])
+    layer = _layer(owq, ref, L.bits, L.group)
+    for M in (1, 16):
+        dy = _dy(M, L.N, 77 + M)
+        x = d["x"][:M]
+        dx = layer.input_grad(_gpu(dy))
+        dw = layer.weak_grad(_gpu(x), _gpu(dy))
+        torch.cuda.synchronize()
+        check_output(dx.cpu().numpy(), oracle.input_grad(W_hat, ref["w_weak"], ref["idx"], dy),
+                     f"{L.name} input_grad M={M}")
+        _check_weak_grad(dw.cpu().numpy(), x, dy, ref["idx"], f"{L.name} M={M}")
+    layer.close()
+
+
+def test_wct_error_paths():
+    import weight_only_mixed_owq_b200 as owq
+    d, ref = _case(CASES[0])
+    layer = _layer(owq, ref, 3, 256)
+    buf = torch.zeros(4096, dtype=torch.float16, device=DEV)
+    f32 = torch.zeros(4096, dtype=torch.float32, device=DEV)
+    h = layer.handle
+    assert owq.owq_input_grad(h, buf, buf, 0) == 2            # OWQ_ERR_SHAPE
+    assert owq.owq_input_grad(h, buf, buf, 65537) == 2
+    assert owq.owq_input_grad(h, None, buf, 1) == 1           # OWQ_ERR_NULL
+    assert owq.owq_input_grad(h, buf.data_ptr() + 2, buf, 1) == 6   # OWQ_ERR_ALIGN
+    assert owq.owq_weak_grad(h, buf, buf, None, 1) == 1       # k > 0 needs an output
+    assert owq.owq_weak_grad(h, buf, buf, f32.data_ptr() + 4, 1) == 6
+    assert owq.owq_weak_grad(h, buf, buf, f32, 0) == 2
+    assert owq.owq_weak_grad(None, buf, buf, f32, 1) == owq.owq_input_grad(None, buf, buf, 1)
+    layer.close()

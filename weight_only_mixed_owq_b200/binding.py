@@ -29,6 +29,8 @@ PROTOTYPES = [
     ("owq_gemv", _I, [_P, _P, _P, _I, _P]),
     ("owq_gemv_multi", _I, [ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _I, _P]),
     ("owq_gemm", _I, [_P, _P, _P, _I, _P]),
+    ("owq_weak_grad", _I, [_P, _P, _P, _P, _I, _P]),
+    ("owq_input_grad", _I, [_P, _P, _P, _I, _P]),
     ("owq_dequant", _I, [_P, _P, _P, _P]),
     ("owq_layer_info", _I, [_P] + [ctypes.POINTER(_I)] * 5),
     ("owq_layer_bytes", _I, [_P, _SZ, _SZ, _SZ, _SZ]),
@@ -123,6 +125,14 @@ def owq_gemm(layer, x, y, M, stream=None) -> int:
     return LIB.owq_gemm(layer, _ptr(x), _ptr(y), M, _stream(stream))
 
 
+def owq_weak_grad(layer, x, dy, dw_weak, M, stream=None) -> int:
+    return LIB.owq_weak_grad(layer, _ptr(x), _ptr(dy), _ptr(dw_weak), M, _stream(stream))
+
+
+def owq_input_grad(layer, dy, dx, M, stream=None) -> int:
+    return LIB.owq_input_grad(layer, _ptr(dy), _ptr(dx), M, _stream(stream))
+
+
 def owq_dequant(layer, w_hat, codes=None, stream=None) -> int:
     return LIB.owq_dequant(layer, _ptr(w_hat), _ptr(codes), _stream(stream))
 
@@ -205,6 +215,24 @@ class OwqLayer:
             y = torch.empty((M, self.N), dtype=torch.float16, device=x.device)
         _check(owq_gemm(self.handle, x, y, M, stream), "owq_gemm")
         return y
+
+    def weak_grad(self, x, dy, dw=None, stream=None):
+        """dW_weak = dy^T x[:, idx] (fp32 N x k)."""
+        import torch
+        M = x.shape[0]
+        if dw is None:
+            dw = torch.empty((self.N, self.k), dtype=torch.float32, device=x.device)
+        _check(owq_weak_grad(self.handle, x, dy, dw if self.k else None, M, stream), "owq_weak_grad")
+        return dw
+
+    def input_grad(self, dy, dx=None, stream=None):
+        """dX = dy W_eff (fp16 M x K)."""
+        import torch
+        M = dy.shape[0]
+        if dx is None:
+            dx = torch.empty((M, self.K), dtype=torch.float16, device=dy.device)
+        _check(owq_input_grad(self.handle, dy, dx, M, stream), "owq_input_grad")
+        return dx
 
     def dequant(self, with_codes: bool = False, stream=None):
         import torch

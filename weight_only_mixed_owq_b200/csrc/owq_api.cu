@@ -71,6 +71,7 @@ void release(Layer* L) {
   cudaFree(L->xfrag);
   cudaFree(L->gemm_ws);
   cudaFree(L->gemm_xw);
+  cudaFree(L->ig_ws);
   cudaFree(L->part);
   L->magic = 0;
   delete L;
@@ -301,6 +302,30 @@ owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, 
   const bool skip = take_inject(OWQ_INJECT_GEMM_ARRIVE, &wl);
   return gemm_sm100(*L, reinterpret_cast<const __half*>(x), reinterpret_cast<__half*>(y), M, wl, skip,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t* dy, float* dw_weak,
+                           int M, owq_stream_t stream) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (M < 1 || M > 65536) return OWQ_ERR_SHAPE;
+  if (!x || !dy || (L->k > 0 && !dw_weak)) return OWQ_ERR_NULL;
+  if (!aligned16(x) || !aligned16(dy) || (dw_weak && !aligned16(dw_weak))) return OWQ_ERR_ALIGN;
+  return cuda_status(launch_weak_grad(*L, reinterpret_cast<const __half*>(x),
+                                      reinterpret_cast<const __half*>(dy), dw_weak, M,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+owq_status_t owq_input_grad(owq_layer_t layer, const uint16_t* dy, uint16_t* dx, int M,
+                            owq_stream_t stream) {
+  Layer* L = lookup(layer);
+  if (!L) return OWQ_ERR_HANDLE;
+  if (M < 1 || M > 65536) return OWQ_ERR_SHAPE;
+  if (!dy || !dx) return OWQ_ERR_NULL;
+  if (!aligned16(dy) || !aligned16(dx)) return OWQ_ERR_ALIGN;
+  return cuda_status(launch_input_grad(*L, reinterpret_cast<const __half*>(dy),
+                                       reinterpret_cast<__half*>(dx), M,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 owq_status_t owq_dequant(owq_layer_t layer, uint16_t* w_hat, uint8_t* codes, owq_stream_t stream) {

@@ -41,6 +41,8 @@ struct Layer {
   size_t gemm_ws_bytes;
   __half* gemm_xw;      // prefill weak activations [M][k_ld] (grown on first need, outside capture)
   size_t gemm_xw_bytes;
+  void* ig_ws;          // input-gradient workspace: arrival counters per column block (zero
+  size_t ig_ws_bytes;   // between calls), then per-slice partial sums (grown on first need)
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
   alignas(64) CUtensorMap map_packed;
@@ -106,6 +108,11 @@ cudaError_t launch_gemv(const GemvProblem* probs, int count, int bits, int M, lo
 cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int T, int bits,
                             int group, int k, uint8_t* codes, __half* scales, __half* zeros,
                             int32_t* idx, __half* w_weak, cudaStream_t s);
+
+// weak column tuning: dW_weak = dY^T x[:, idx] (fp32 N x k) and dX = dY W_eff (fp16 M x K)
+cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, float* dw, int M,
+                             cudaStream_t s);
+cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s);
 
 // skip_arrive: a test-injected lost arrival (one dequantisation thread per CTA skips its first
 // arrival), so that the bounded waits run out
