@@ -104,6 +104,7 @@ k_input_grad(const IgArgs a) {
   __shared__ __align__(16) float s_dy[2][kIgStageRows][TOK];
   __shared__ float2 s_red[3][TOK][64];
   __shared__ int s_last;
+  __shared__ int s_slot[kBlockCodes];
 
   const int tid = threadIdx.x, p = tid & 63, h = tid >> 6;
   const int b = blockIdx.x, slice = blockIdx.y, S = gridDim.y;
@@ -118,17 +119,16 @@ k_input_grad(const IgArgs a) {
   const int word = chunk * BITS + (spread ? 0 : sl.word);
   const int shift = spread ? 0 : sl.off;
 
-  // weak slots of the two columns (idx is strictly ascending)
-  int tw[2] = {-1, -1};
-  #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    int lo = 0, hi = a.k;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (a.idx[mid] < col + e) lo = mid + 1; else hi = mid;
-    }
-    if (lo < a.k && a.idx[lo] == col + e) tw[e] = lo;
+  // weak slots of the block's columns: one parallel pass over idx into a shared table
+  if (tid < kBlockCodes) s_slot[tid] = -1;
+  __syncthreads();
+  for (int t = tid; t < a.k; t += kIgThreads) {
+    const int c = a.idx[t] - b * kBlockCodes;
+    if (c >= 0 && c < kBlockCodes) s_slot[c] = t;
   }
+  __syncthreads();
+  const int tw0 = s_slot[2 * p], tw1 = s_slot[2 * p + 1];
+  const bool weak = tw0 >= 0 || tw1 >= 0;
 
   const int nstages = (tiles + 3) / 4;
   const int st0 = slice * a.stages_per_slice;
@@ -138,7 +138,18 @@ k_input_grad(const IgArgs a) {
   uint4 r_words = make_uint4(0, 0, 0, 0);
   __half r_s = __float2half(0.f), r_z = __float2half(0.f);
   __half r_dy[(TOK * kIgStageRows + kIgThreads - 1) / kIgThreads];
+  // weak values of this thread's rows, one stage ahead (threads with a weak column only)
+  __half2 wk_next[16], wk_cur[16];
   auto load = [&](int st) {
+    if (weak) {
+      #pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        const int row = st * kIgStageRows + h * 16 + rr;
+        const __half* wr = a.w_weak + (size_t)row * a.k_ld;
+        wk_next[rr] = __halves2half2(tw0 >= 0 && row < a.N ? wr[tw0] : __float2half(0.f),
+                                     tw1 >= 0 && row < a.N ? wr[tw1] : __float2half(0.f));
+      }
+    }
     if (tid < kStageWords4) {
       const int tile = st * 4 + tid / (16 * BITS);
       r_words = make_uint4(0, 0, 0, 0);
@@ -158,6 +169,10 @@ k_input_grad(const IgArgs a) {
     }
   };
   auto store = [&](int buf) {
+    if (weak) {
+      #pragma unroll
+      for (int rr = 0; rr < 16; ++rr) wk_cur[rr] = wk_next[rr];
+    }
     if (tid < kStageWords4) s_words[buf][tid] = r_words;
     if (tid < kIgStageRows) {
       s_scale[buf][tid] = __halves2half2(r_s, r_s);
@@ -184,16 +199,18 @@ k_input_grad(const IgArgs a) {
     const int buf = (st - st0) & 1;
     if (st + 1 < st1) load(st + 1);
     const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_words[buf]);
-    #pragma unroll 4
+    #pragma unroll
     for (int rr = 0; rr < 16; ++rr) {
       const int r = h * 16 + rr;               // row within the stage
-      const int row = st * kIgStageRows + r;
       // row r of the stage is row r % 16 of tile r / 16: block (r / 16) * 16 + r % 16 = r
       const uint32_t v = pair_codes<BITS>(sw + r * 4 * BITS, word, shift, spread) | 0x64006400u;
       const __half2 qz = __hsub2(*reinterpret_cast<const __half2*>(&v), s_zb[buf][r]);
       float2 wv = __half22float2(__hmul2(s_scale[buf][r], qz));
-      if (tw[0] >= 0) wv.x = row < a.N ? __half2float(a.w_weak[(size_t)row * a.k_ld + tw[0]]) : 0.f;
-      if (tw[1] >= 0) wv.y = row < a.N ? __half2float(a.w_weak[(size_t)row * a.k_ld + tw[1]]) : 0.f;
+      if (weak) {
+        const float2 wk = __half22float2(wk_cur[rr]);
+        if (tw0 >= 0) wv.x = wk.x;
+        if (tw1 >= 0) wv.y = wk.y;
+      }
       const float* d = s_dy[buf][r];
       #pragma unroll
       for (int m = 0; m < TOK; ++m) {
@@ -240,8 +257,19 @@ k_input_grad(const IgArgs a) {
   __threadfence();
   for (int e = tid; e < TOK * kBlockCodes; e += kIgThreads) {
     const int m = e / kBlockCodes, c = b * kBlockCodes + e % kBlockCodes;
+    const float* src = a.part + (size_t)m * a.K + c;
+    const size_t step = (size_t)kIgMaxTok * a.K;
     float sum = 0.f;
-    for (int s = 0; s < S; ++s) sum += __ldcg(a.part + ((size_t)s * kIgMaxTok + m) * a.K + c);
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {   // four loads in flight, added in slice order
+      const float v0 = __ldcg(src + s * step), v1 = __ldcg(src + (s + 1) * step);
+      const float v2 = __ldcg(src + (s + 2) * step), v3 = __ldcg(src + (s + 3) * step);
+      sum += v0;
+      sum += v1;
+      sum += v2;
+      sum += v3;
+    }
+    for (; s < S; ++s) sum += __ldcg(src + s * step);
     if (m < a.M) a.dx[(size_t)m * a.K + c] = __float2half_rn(sum);
   }
   if (tid == 0) a.count[b] = 0u;   // ready for the next call on this stream
@@ -284,7 +312,7 @@ cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, 
 cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s) {
   const int Kb = L.K / kBlockCodes;
   const int nstages = ((L.N + 15) / 16 + 3) / 4;
-  // about two CTAs per SM over the column blocks and row slices
+  // about two CTAs per SM (what the registers allow) over the column blocks and row slices
   int slices = std::max(1, std::min(nstages, (2 * wct_sm_count(L.device) + Kb - 1) / Kb));
   int per = (nstages + slices - 1) / slices;
   slices = (nstages + per - 1) / per;
