@@ -312,8 +312,9 @@ cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, 
 cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s) {
   const int Kb = L.K / kBlockCodes;
   const int nstages = ((L.N + 15) / 16 + 3) / 4;
-  // about two CTAs per SM (what the registers allow) over the column blocks and row slices
-  int slices = std::max(1, std::min(nstages, (2 * wct_sm_count(L.device) + Kb - 1) / Kb));
+  // two CTAs per SM (what the registers allow) over the column blocks and row slices, rounded
+  // down so that the grid is one wave
+  int slices = std::max(1, std::min(nstages, (2 * wct_sm_count(L.device)) / Kb));
   int per = (nstages + slices - 1) / slices;
   slices = (nstages + per - 1) / per;
   // workspace: one arrival counter per column block (zero between calls), then the partial sums
