@@ -70,6 +70,10 @@ def test_host_validation_rejects_bad_arguments(owq):
     assert owq.owq_gemv(A, A, A, 1) == 10
     assert owq.owq_gemm(A, A, A, 64) == 10
     assert owq.owq_dequant(A, A) == 10
+    assert owq.owq_weak_grad(A, A, A, A, 1) == 10
+    assert owq.owq_weak_grad(None, A, A, A, 16) == 10
+    assert owq.owq_input_grad(A, A, A, 1) == 10
+    assert owq.owq_input_grad(None, A, A, 16) == 10
     assert owq.owq_layer_free(A) == 10
     assert owq.owq_layer_free(None) == 0
     assert owq.owq_layer_info(A)[0] == 10
