@@ -208,8 +208,8 @@ owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t*
  * In:  dy fp16 M x N row-major; 1 <= M <= 65536 (one pass over the packed weights per 16
  *      tokens).  Out: dx fp16 M x K row-major (fully overwritten).
  * The rows are split over CTAs; their fp32 partial sums go to a workspace the handle owns
- * (slices x 16 tokens x K x 4 bytes, with about 2 x SMs / (K / 128) slices: 2.6 MB at
- * K = 4096 on 148 SMs), allocated on the first call that needs it; that first call must not be inside a stream capture (inside one, a
+ * (slices x 16 tokens x K x 4 bytes, with at most 2 x SMs / (K / 128) slices so that the
+ * grid is one wave: 2.1 MB at K = 4096 on 148 SMs), allocated on the first call that needs it; that first call must not be inside a stream capture (inside one, a
  * handle without the workspace runs one slice per column block: slower, same result).
  * The last CTA of each column block adds the slices in a fixed order: repeated calls give
  * identical bits.  Calls on one handle must be ordered (one stream, or events between
