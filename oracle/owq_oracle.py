@@ -40,6 +40,12 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
   weak_grad                   pinned: directional derivative of the pinned forward product
                               (the loss is linear in the weak block).
   input_grad                  pinned: adjoint identity against the pinned forward product.
+  search_params               pinned: never worse than min-max RTN (whose parameters are a
+                              grid point); exact rows reproduced with zero error; a planted
+                              outlier is truncated.  The grid itself is a reading.
+  optq_quantize               pinned: a diagonal Hessian reduces it to RTN; the compensated
+                              weak columns equal the least-squares optimum given the
+                              quantised dense columns (a different route: lstsq on X).
 """
 from __future__ import annotations
 
@@ -58,6 +64,8 @@ __all__ = [
     "matmul_rows",
     "weak_grad",
     "input_grad",
+    "search_params",
+    "optq_quantize",
     "bits_per_weight",
     "layer_bytes",
 ]
@@ -302,6 +310,123 @@ def matmul_rows(codes, scales, zeros, w_weak, idx, x, rows) -> np.ndarray:
     rows = np.asarray(rows, dtype=np.int64)
     W_hat = dequant(np.asarray(codes)[rows], np.asarray(scales)[rows], np.asarray(zeros)[rows])
     return matmul(W_hat, np.asarray(w_weak)[rows], idx, x)
+
+
+# ----------------------------------------------------------------------------------------
+# The paper's own dense quantiser: truncation-aware parameter search, then OPTQ with the weak
+# columns last
+# ----------------------------------------------------------------------------------------
+DEFAULT_ALPHAS = tuple(1.0 - 0.02 * i for i in range(26))   # range shrink factors 1.00 .. 0.50
+
+
+def _dequant_one(q: np.ndarray, s: np.float16, z: np.float16) -> np.ndarray:
+    return (np.float32(s) * (q.astype(F32) - np.float32(z))).astype(F16)
+
+
+def search_params(W: np.ndarray, bits: int, group: int, weak_idx=None, alphas=DEFAULT_ALPHAS):
+    """Truncation-aware 2-D grid search of (step size, zero point) per (row, group).
+
+    [PL] "Low-precision quantization" (paper "Quantization Configuration Search", pp.4-5):
+    before OPTQ, OWQ searches a 2-D grid over the step size and the zero point, with nearest
+    rounding and truncation (clamping), so that the range may shrink below min-max and the
+    reconstruction error drops.  Readings (the pages give no grid): the step sizes are the
+    min-max step of the range [min(0, min w), max(0, max w)] (the quantize_rtn rules) times a
+    shrink factor alpha in `alphas`, rounded to fp16; the zero points are every integer in
+    [0, 2^b - 1]; the error is sum_j (w_j - fp16_rn(s (q_j - z)))^2 in fp64 over the group's
+    dense columns, with q = clamp(rint(w / s) + z, 0, 2^b - 1) in fp32; the first minimum in
+    the order (alpha descending, z ascending) wins.  Weak columns are left out of the search.
+    Returns (scales fp16 N x G, zeros fp16 N x G).
+    """
+    W = np.asarray(W, dtype=F16)
+    N, K = W.shape
+    G = K // group
+    qmax = (1 << bits) - 1
+    dense = np.ones(K, dtype=bool)
+    if weak_idx is not None and len(weak_idx):
+        dense[np.asarray(weak_idx, dtype=np.int64)] = False
+    scales = np.zeros((N, G), dtype=F16)
+    zeros = np.zeros((N, G), dtype=F16)
+    for i in range(N):
+        for gi in range(G):
+            cols = np.arange(gi * group, (gi + 1) * group)
+            w = W[i, cols[dense[cols]]].astype(F32)
+            mn = min(F32(0), w.min()) if w.size else F32(0)
+            mx = max(F32(0), w.max()) if w.size else F32(0)
+            if mn == mx:
+                mn, mx = F32(-1), F32(1)
+            best = None
+            for a in alphas:
+                s16 = F16((mx - mn) * F32(a) / F32(qmax))
+                if s16 == 0:
+                    continue
+                s32 = F32(s16)
+                for z in range(qmax + 1):
+                    q = np.clip(np.rint(w / s32) + F32(z), F32(0), F32(qmax))
+                    e = w.astype(F64) - _dequant_one(q, s16, F16(z)).astype(F64)
+                    err = float((e * e).sum())
+                    if best is None or err < best[0]:
+                        best = (err, s16, z)
+            if best is None:   # a range below fp16 resolution: fall back to [-1, 1]
+                best = (0.0, F16(F32(2) / F32(qmax)), (qmax + 1) // 2)
+            scales[i, gi] = best[1]
+            zeros[i, gi] = F16(best[2])
+    return scales, zeros
+
+
+def optq_quantize(W: np.ndarray, X: np.ndarray, bits: int, group: int, weak_idx,
+                  scales: np.ndarray, zeros: np.ndarray, damp: float = 0.01) -> dict:
+    """OPTQ sequential column-wise quantisation with the weak columns moved to the end.
+
+    [PL] "Low-precision quantization" (paper p.4): the dense weights go through OPTQ's
+    column-by-column quantisation; the weak columns are moved to the end of the order, are
+    never quantised, and absorb the compensation of the columns before them, so the stored
+    fp16 weak block holds their compensated values.  [PL] "Layer-wise Quantization and
+    Hessian": each row's error is dW H dW^T with H built from the calibration inputs
+    (H = X^T X here; OPTQ's factor 2 cancels in every update).
+
+    Each step is the optimal-brain-surgeon update written from its definition: with F the
+    columns not yet quantised (the current column j first) and H_F^-1 the inverse of H
+    restricted to F (recomputed at every step; no Cholesky form, no blocking), quantise column
+    j with the given (scale, zero) of its group, then move the remaining columns of F by
+    -(w_j - w_hat_j) / [H_F^-1]_jj * [H_F^-1]_{j, F without j}, which keeps them at the minimum of
+    the row's error given the columns already fixed.  H gets damp * mean(diag H) added to its
+    diagonal (a reading: OPTQ's usual dampening; damp = 0 for an exact solve).  The code
+    decision is taken in fp32 on the current fp64 weight: q = clamp(rint(fp32(w) / s) + z).
+
+    Returns codes (uint8 N x K; z at the weak columns), the weak block fp16 N x k (compensated
+    values), and the compensated weak values in fp64 ("w_weak64") for checks.
+    """
+    W = np.asarray(W, dtype=F16)
+    N, K = W.shape
+    qmax = (1 << bits) - 1
+    weak = np.asarray(weak_idx if weak_idx is not None else [], dtype=np.int64)
+    is_weak = np.zeros(K, dtype=bool)
+    is_weak[weak] = True
+    order = np.concatenate([np.flatnonzero(~is_weak), np.sort(weak)])
+    X64 = np.asarray(X, dtype=F16).astype(F64)
+    H = X64.T @ X64
+    if damp:
+        H = H + damp * float(np.mean(np.diag(H))) * np.eye(K)
+    Wc = W.astype(F64)
+    codes = np.zeros((N, K), dtype=np.uint8)
+    n_dense = K - len(weak)
+    for step in range(n_dense):
+        j = order[step]
+        F = order[step:]
+        Hinv = np.linalg.inv(H[np.ix_(F, F)])
+        gi = j // group
+        s16, z16 = scales[:, gi], zeros[:, gi]
+        q = np.clip(np.rint(Wc[:, j].astype(F32) / s16.astype(F32)) + z16.astype(F32), F32(0), F32(qmax))
+        w_hat = (s16.astype(F32) * (q - z16.astype(F32))).astype(F16).astype(F64)
+        err = (Wc[:, j] - w_hat) / Hinv[0, 0]
+        Wc[:, F[1:]] -= err[:, None] * Hinv[0, 1:][None, :]
+        Wc[:, j] = w_hat
+        codes[:, j] = q.astype(np.uint8)
+    for t in weak:
+        codes[:, t] = zeros[:, t // group].astype(np.uint8)
+    w_weak64 = Wc[:, np.sort(weak)]
+    return {"codes": codes, "scales": np.asarray(scales, dtype=F16), "zeros": np.asarray(zeros, dtype=F16),
+            "idx": np.sort(weak).astype(np.int32), "w_weak": w_weak64.astype(F16), "w_weak64": w_weak64}
 
 
 # ----------------------------------------------------------------------------------------

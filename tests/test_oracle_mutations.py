@@ -160,3 +160,38 @@ def test_mutant_weak_grad_wrong_gather_is_caught(monkeypatch):
     _patch(monkeypatch, "weak_grad", bad)
     with pytest.raises(AssertionError):
         pins.test_weak_grad_is_directional_derivative_of_forward_product(5, 3)
+
+
+def test_mutant_optq_without_compensation_is_caught(monkeypatch):
+    orig = oo.optq_quantize
+
+    def bad(W, X, bits, group, weak_idx, scales, zeros, damp=0.01):
+        # an identity Hessian: every column is quantised on its own, nothing is compensated
+        K = np.asarray(W).shape[1]
+        return orig(W, np.eye(K, dtype=F16), bits, group, weak_idx, scales, zeros, damp=0.0)
+    _patch(monkeypatch, "optq_quantize", bad)
+    with pytest.raises(AssertionError):
+        pins.test_optq_weak_columns_are_least_squares_optimum(3, 32)
+
+
+def test_mutant_optq_weak_columns_first_is_caught(monkeypatch):
+    orig = oo.optq_quantize
+
+    def bad(W, X, bits, group, weak_idx, scales, zeros, damp=0.01):
+        # weak columns taken out of the compensation (their values never move)
+        r = orig(W, X, bits, group, weak_idx, scales, zeros, damp)
+        r["w_weak64"] = np.asarray(W, dtype=F16)[:, np.sort(weak_idx)].astype(F64)
+        return r
+    _patch(monkeypatch, "optq_quantize", bad)
+    with pytest.raises(AssertionError):
+        pins.test_optq_weak_columns_are_least_squares_optimum(4, 16)
+
+
+def test_mutant_search_without_truncation_is_caught(monkeypatch):
+    orig = oo.search_params
+
+    def bad(W, bits, group, weak_idx=None, alphas=None):
+        return orig(W, bits, group, weak_idx, alphas=(1.0,))
+    _patch(monkeypatch, "search_params", bad)
+    with pytest.raises(AssertionError):
+        pins.test_search_params_truncates_a_planted_outlier()

@@ -374,3 +374,81 @@ def test_weak_grad_is_directional_derivative_of_forward_product(k, M):
         V[i, t] = 1
         y = oracle.matmul(zero, V, r["idx"], d["x"])
         assert g[i, t] == pytest.approx(float((dy.astype(F64) * y).sum()), rel=1e-12, abs=1e-14)
+
+
+# ------------------------------------------------------------------ OPTQ and the parameter search
+def _rtn_error(w, s, z, bits):
+    """Squared reconstruction error of one group's weights under RTN with the given (s, z)
+    (test-side evaluation of a candidate; the oracle's RTN is pinned above)."""
+    s32, z32 = np.float32(s), np.float32(z)
+    q = np.clip(np.rint(w.astype(np.float32) / s32) + z32, 0, (1 << bits) - 1)
+    w_hat = (s32 * (q - z32)).astype(F16).astype(F64)
+    return float(((w.astype(F64) - w_hat) ** 2).sum())
+
+
+def test_optq_with_diagonal_hessian_is_rtn():
+    """With X^T X diagonal, H^-1 has no off-diagonal terms, so no column compensates another:
+    OPTQ gives exactly the RTN codes of the same parameters and keeps the weak columns."""
+    d = owq_synth.draw_small(6, 32, 1, 8, seed=120)
+    c = np.linspace(0.5, 3.0, 32).astype(F16)
+    X = np.diag(c).astype(F16)
+    weak = [3, 17, 30]
+    codes, s, z = oracle.quantize_rtn(d["W"], 3, 32, weak)
+    r = oracle.optq_quantize(d["W"], X, 3, 32, weak, s, z, damp=0.0)
+    assert np.array_equal(r["codes"], codes)
+    assert np.array_equal(r["w_weak"].view(np.uint16), d["W"][:, weak].view(np.uint16))
+
+
+@pytest.mark.parametrize("bits,group", [(3, 32), (4, 16)])
+def test_optq_weak_columns_are_least_squares_optimum(bits, group):
+    """The compensated weak columns minimise the row's output error ||X (w - w_hat)||^2 given the
+    quantised dense columns: checked against numpy's least-squares solve on X itself."""
+    rng = np.random.default_rng(130 + bits)
+    N, K, T = 5, 32, 96
+    W = (rng.standard_normal((N, K)) * 0.02).astype(F16)
+    X = rng.standard_normal((T, K)).astype(F16)
+    weak = [2, 9, 25]
+    s, z = oracle.search_params(W, bits, group, weak)
+    r = oracle.optq_quantize(W, X, bits, group, weak, s, z, damp=0.0)
+    W_hat = oracle.dequant(r["codes"], s, z).astype(F64)
+    dense = np.setdiff1d(np.arange(K), weak)
+    X64 = X.astype(F64)
+    for i in range(N):
+        target = X64 @ W[i].astype(F64) - X64[:, dense] @ W_hat[i, dense]
+        v, *_ = np.linalg.lstsq(X64[:, weak], target, rcond=None)
+        assert np.allclose(r["w_weak64"][i], v, rtol=1e-9, atol=1e-12)
+    # and the compensation is real: the optimum differs from the original weak values
+    assert not np.allclose(r["w_weak64"], W[:, weak].astype(F64), atol=1e-6)
+
+
+def test_search_params_never_worse_than_minmax_and_exact_on_grid_rows():
+    d = owq_synth.draw_small(8, 64, 1, 8, seed=140)
+    weak = [5]
+    s, z = oracle.search_params(d["W"], 3, 32, weak)
+    _, s0, z0 = oracle.quantize_rtn(d["W"], 3, 32, weak)
+    dense = np.ones(64, bool)
+    dense[weak] = False
+    for i in range(8):
+        for g in range(2):
+            cols = np.arange(32 * g, 32 * g + 32)
+            w = d["W"][i, cols[dense[cols]]]
+            assert _rtn_error(w, s[i, g], z[i, g], 3) <= _rtn_error(w, s0[i, g], z0[i, g], 3)
+    # a row that lies exactly on a 3-bit grid (codes 0..7, step 1/16, zero point 3) is
+    # reproduced with zero error by its own min-max parameters, which the search keeps
+    q = np.array([0, 7, 3, 1, 5, 2, 6, 4] * 4, dtype=np.float32)
+    row = ((q - 3) / 16).astype(F16)[None, :]
+    s1, z1 = oracle.search_params(row, 3, 32)
+    assert float(s1[0, 0]) == 1 / 16 and float(z1[0, 0]) == 3
+    assert _rtn_error(row[0], s1[0, 0], z1[0, 0], 3) == 0.0
+
+
+def test_search_params_truncates_a_planted_outlier():
+    """One large weight among small ones: clamping it lowers the total squared error, so the
+    search picks a step below the min-max step."""
+    rng = np.random.default_rng(150)
+    row = (rng.standard_normal(128) * 0.01).astype(F16)
+    row[77] = F16(0.5)
+    s, z = oracle.search_params(row[None, :], 3, 128)
+    _, s0, _ = oracle.quantize_rtn(row[None, :], 3, 128)
+    assert float(s[0, 0]) < float(s0[0, 0])
+    assert _rtn_error(row, s[0, 0], z[0, 0], 3) < _rtn_error(row, s0[0, 0], oracle.quantize_rtn(row[None, :], 3, 128)[2][0, 0], 3)
