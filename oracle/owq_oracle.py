@@ -40,6 +40,10 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
   weak_grad                   pinned: directional derivative of the pinned forward product
                               (the loss is linear in the weak block).
   input_grad                  pinned: adjoint identity against the pinned forward product.
+  pack_storage /
+  unpack_storage              pinned: the round trip gives the latency layout's codes (z at
+                              the weak columns); each code moves exactly its own bits; the
+                              layout's bytes reproduce the storage-favoured bits per weight.
   search_params               pinned: never worse than min-max RTN (whose parameters are a
                               grid point); exact rows reproduced with zero error; a planted
                               outlier is truncated.  The grid itself is a reading.
@@ -64,6 +68,8 @@ __all__ = [
     "matmul_rows",
     "weak_grad",
     "input_grad",
+    "pack_storage",
+    "unpack_storage",
     "search_params",
     "optq_quantize",
     "bits_per_weight",
@@ -280,6 +286,58 @@ def unpack(words: np.ndarray, K: int, bits: int) -> np.ndarray:
                 c[:, :, 4 * j + q, 0] = (w4[:, :, q, w] >> o) & mask
                 c[:, :, 4 * j + q, 1] = (w4[:, :, q, w] >> (16 + o)) & mask
     return c.reshape(N, K).astype(np.uint8)
+
+
+def pack_storage(codes: np.ndarray, idx, bits: int) -> np.ndarray:
+    """The storage-favoured dense stream: per row, only the codes of the K - k dense columns,
+    in column order, as one little-endian bit stream of `bits` bits per code (code p of the
+    stream at bits [p b, p b + b)), padded with zero bits to whole uint32 words.
+
+    [PL] "Storage Methods" (appendix §2, pp.10-11): the storage-favoured form drops the weak
+    columns from the low-precision matrix (b + (16 - b) k / K bits per weight) instead of
+    keeping them zero-filled (the latency-favoured form of ``pack``).  The bit order inside the
+    stream is not given on the pages; a plain LSB-first stream is the reading taken.
+    Returns uint32 N x ceil((K - k) b / 32).
+    """
+    codes = np.asarray(codes, dtype=np.uint8)
+    N, K = codes.shape
+    dense = np.ones(K, dtype=bool)
+    idx = np.asarray(idx if idx is not None else [], dtype=np.int64)
+    dense[idx] = False
+    nd = int(dense.sum())
+    W = (nd * bits + 31) // 32
+    out = np.zeros((N, W), dtype=np.uint64)
+    dc = codes[:, dense].astype(np.uint64)
+    for p in range(nd):
+        bit = p * bits
+        w, o = divmod(bit, 32)
+        v = dc[:, p] << np.uint64(o)
+        out[:, w] |= v & np.uint64(0xFFFFFFFF)
+        if o + bits > 32:
+            out[:, w + 1] |= v >> np.uint64(32)
+    return out.astype(np.uint32)
+
+
+def unpack_storage(words: np.ndarray, K: int, idx, bits: int, zeros: np.ndarray, group: int) -> np.ndarray:
+    """Inverse of ``pack_storage``, back to full N x K codes with the weak columns set to their
+    group's zero point (the latency-favoured, zero-filled codes)."""
+    words = np.asarray(words, dtype=np.uint32).astype(np.uint64)
+    N = words.shape[0]
+    dense = np.ones(K, dtype=bool)
+    idx = np.asarray(idx if idx is not None else [], dtype=np.int64)
+    dense[idx] = False
+    mask = np.uint64((1 << bits) - 1)
+    codes = np.zeros((N, K), dtype=np.uint8)
+    for p, j in enumerate(np.flatnonzero(dense)):
+        w, o = divmod(p * bits, 32)
+        v = words[:, w] >> np.uint64(o)
+        if o + bits > 32:
+            v |= words[:, w + 1] << np.uint64(32 - o)
+        codes[:, j] = (v & mask).astype(np.uint8)
+    z = np.asarray(zeros, dtype=F16).astype(np.uint8)
+    for j in idx:
+        codes[:, j] = z[:, j // group]
+    return codes
 
 
 # ----------------------------------------------------------------------------------------

@@ -195,3 +195,13 @@ def test_mutant_search_without_truncation_is_caught(monkeypatch):
     _patch(monkeypatch, "search_params", bad)
     with pytest.raises(AssertionError):
         pins.test_search_params_truncates_a_planted_outlier()
+
+
+def test_mutant_storage_stream_keeping_weak_columns_is_caught(monkeypatch):
+    orig = oo.pack_storage
+
+    def bad(codes, idx, bits):
+        return orig(codes, [], bits)
+    _patch(monkeypatch, "pack_storage", bad)
+    with pytest.raises(AssertionError):
+        pins.test_storage_layout_round_trip_matches_latency_layout(3, 128, 5)

@@ -452,3 +452,43 @@ def test_search_params_truncates_a_planted_outlier():
     _, s0, _ = oracle.quantize_rtn(row[None, :], 3, 128)
     assert float(s[0, 0]) < float(s0[0, 0])
     assert _rtn_error(row, s[0, 0], z[0, 0], 3) < _rtn_error(row, s0[0, 0], oracle.quantize_rtn(row[None, :], 3, 128)[2][0, 0], 3)
+
+
+# ------------------------------------------------------------------ storage-favoured layout
+@pytest.mark.parametrize("bits,group,k", [(3, 128, 5), (4, 256, 0), (3, 256, 11)])
+def test_storage_layout_round_trip_matches_latency_layout(bits, group, k):
+    """Both layouts hold the same quantised matrix: the storage-favoured stream, unpacked,
+    gives exactly the zero-filled codes the latency-favoured blocks hold."""
+    d = owq_synth.draw_small(7, 256, 1, 32, seed=160 + k)
+    r = oracle.owq_quantize(d["W"], d["X"], bits, group, k)
+    words = oracle.pack_storage(r["codes"], r["idx"], bits)
+    assert words.shape == (7, ((256 - k) * bits + 31) // 32)
+    back = oracle.unpack_storage(words, 256, r["idx"], bits, r["zeros"], group)
+    lat = oracle.unpack(oracle.pack(r["codes"], bits), 256, bits)
+    assert np.array_equal(back, lat)
+    assert np.array_equal(back, r["codes"])
+
+
+def test_storage_layout_single_code_moves_its_own_bits():
+    """A code of all ones at dense position p sets exactly bits [3p, 3p + 3) of the row's
+    stream, positions counted after the weak columns are removed (p = 10 starts at bit 30
+    and straddles words 0 and 1)."""
+    for p in (0, 5, 10, 11, 40):
+        codes = np.zeros((1, 128), dtype=np.uint8)
+        idx = [3, 64]
+        dense_cols = [j for j in range(128) if j not in idx]
+        codes[0, dense_cols[p]] = 7
+        words = oracle.pack_storage(codes, idx, 3)
+        bits = int(sum(int(w) << (32 * i) for i, w in enumerate(words[0])))
+        assert bits == 7 << (3 * p)
+
+
+def test_storage_layout_bytes_reproduce_storage_bits_per_weight():
+    """With (K - k) b a multiple of 32 there is no padding, and the layout's bits per weight
+    (stream + fp16 weak block) equal the pages' storage-favoured b + (16 - b) k / K."""
+    N, K, k, b = 4, 512, 32, 4
+    codes = np.zeros((N, K), dtype=np.uint8)
+    words = oracle.pack_storage(codes, np.arange(0, K, K // k)[:k], b)
+    bits = (words.size * 32 + N * k * 16) / (N * K)
+    assert bits == pytest.approx(oracle.bits_per_weight(K, b, k, layout="storage"), abs=1e-12)
+    assert bits < oracle.bits_per_weight(K, b, k, layout="latency")
