@@ -47,6 +47,9 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
   search_params               pinned: never worse than min-max RTN (whose parameters are a
                               grid point); exact rows reproduced with zero error; a planted
                               outlier is truncated.  The grid itself is a reading.
+  owq_quantize_optq           composition of pinned steps; pinned end to end: the planted
+                              outlier channels are selected and its weak columns are the
+                              least-squares optimum.
   optq_quantize               pinned: a diagonal Hessian reduces it to RTN; the compensated
                               weak columns equal the least-squares optimum given the
                               quantised dense columns (a different route: lstsq on X).
@@ -72,6 +75,7 @@ __all__ = [
     "unpack_storage",
     "search_params",
     "optq_quantize",
+    "owq_quantize_optq",
     "bits_per_weight",
     "layer_bytes",
 ]
@@ -485,6 +489,28 @@ def optq_quantize(W: np.ndarray, X: np.ndarray, bits: int, group: int, weak_idx,
     w_weak64 = Wc[:, np.sort(weak)]
     return {"codes": codes, "scales": np.asarray(scales, dtype=F16), "zeros": np.asarray(zeros, dtype=F16),
             "idx": np.sort(weak).astype(np.int32), "w_weak": w_weak64.astype(F16), "w_weak64": w_weak64}
+
+
+def owq_quantize_optq(W: np.ndarray, X: np.ndarray, bits: int, group: int, k: int,
+                      damp: float = 0.01, alphas=DEFAULT_ALPHAS) -> dict:
+    """The paper's full quantiser: weak-column selection, truncation-aware parameter search,
+    then OPTQ with the weak columns last ([PL] "Weak-column selection", "Low-precision
+    quantization").
+
+    1. lambda, the all-column RTN perturbation, the sensitivity and the top-k selection exactly
+       as in ``owq_quantize`` (steps 1-4);
+    2. (scale, zero) per (row, group) by ``search_params`` over the dense columns;
+    3. ``optq_quantize`` with those parameters; the weak block holds the compensated values.
+    """
+    W = np.asarray(W, dtype=F16)
+    lam = hessian_diag(X)
+    c0, s0, z0 = quantize_rtn(W, bits, group, None)
+    sens = sensitivity(W, dequant(c0, s0, z0), lam)
+    idx = select_weak(sens, k)
+    scales, zeros = search_params(W, bits, group, idx, alphas)
+    r = optq_quantize(W, X, bits, group, idx, scales, zeros, damp)
+    r["lam"], r["sens"] = lam, sens
+    return r
 
 
 # ----------------------------------------------------------------------------------------

@@ -492,3 +492,31 @@ def test_storage_layout_bytes_reproduce_storage_bits_per_weight():
     bits = (words.size * 32 + N * k * 16) / (N * K)
     assert bits == pytest.approx(oracle.bits_per_weight(K, b, k, layout="storage"), abs=1e-12)
     assert bits < oracle.bits_per_weight(K, b, k, layout="latency")
+
+
+def test_owq_quantize_optq_end_to_end():
+    """The full quantiser selects the planted outlier channels, and its stored weak columns
+    (before fp16 rounding) are the least-squares optimum given its quantised dense columns."""
+    rng = np.random.default_rng(170)
+    N, K, T = 6, 64, 160
+    W = (rng.standard_normal((N, K)) * 0.02).astype(F16)
+    X = rng.standard_normal((T, K)).astype(np.float32)
+    planted = [7, 40]
+    X[:, planted] *= 50
+    X = X.astype(F16)
+    r = oracle.owq_quantize_optq(W, X, 3, K, 2, damp=0.0)
+    assert r["idx"].tolist() == planted
+    W_hat = oracle.dequant(r["codes"], r["scales"], r["zeros"]).astype(F64)
+    dense = np.setdiff1d(np.arange(K), planted)
+    X64 = X.astype(F64)
+    for i in range(N):
+        target = X64 @ W[i].astype(F64) - X64[:, dense] @ W_hat[i, dense]
+        v, *_ = np.linalg.lstsq(X64[:, planted], target, rcond=None)
+        assert np.allclose(r["w_weak64"][i], v, rtol=1e-8, atol=1e-12)
+    # the output error of the full quantiser is below that of the RTN oracle quantiser
+    base = oracle.owq_quantize(W, X, 3, K, 2)
+    y_ref = X64 @ W.astype(F64).T
+    e_optq = np.linalg.norm(oracle.matmul(W_hat.astype(F16), r["w_weak"], r["idx"], X) - y_ref)
+    W_hat_b = oracle.dequant(base["codes"], base["scales"], base["zeros"])
+    e_rtn = np.linalg.norm(oracle.matmul(W_hat_b, base["w_weak"], base["idx"], X) - y_ref)
+    assert e_optq < e_rtn
