@@ -1,10 +1,28 @@
-"""Shared helpers of the GPU parity tests: the output tolerance and oracle caches."""
+"""Shared helpers of the GPU parity tests: the output tolerance, the report of the outputs
+that use the relaxed bound, and the oracle's product over all rows of a large layer."""
 import numpy as np
+
+import oracle
 
 F64 = np.float64
 
 REL_L2 = 1e-3
 MAX_ABS = 1e-2
+
+# one entry per check_output call that met an output with |y64| >= 32 (printed at the end of
+# the test session by tests/conftest.py)
+RELAXED_REPORT: list = []
+
+
+def oracle_rows_all(ref: dict, x: np.ndarray, slab: int = 1024) -> np.ndarray:
+    """The oracle's fp64 product y64 (M x N) over every output row, in row slabs so that a
+    large layer's fp64 copy of W_hat is never formed at once."""
+    N = ref["codes"].shape[0]
+    out = []
+    for r0 in range(0, N, slab):
+        rows = np.arange(r0, min(N, r0 + slab))
+        out.append(oracle.matmul_rows(ref["codes"], ref["scales"], ref["zeros"], ref["w_weak"], ref["idx"], x, rows))
+    return np.concatenate(out, axis=1)
 
 
 def check_output(y_gpu_fp16: np.ndarray, y64: np.ndarray, where: str = "") -> dict:
@@ -22,13 +40,25 @@ def check_output(y_gpu_fp16: np.ndarray, y64: np.ndarray, where: str = "") -> di
     err = np.abs(yg - y64)
     rel = float(np.linalg.norm(err) / max(np.linalg.norm(y64), 1e-300))
     big = np.abs(y64) >= 32.0
-    half_ulp = 0.5 * np.spacing(np.abs(y64).astype(np.float16)).astype(F64)
-    allowed = np.where(big, half_ulp + np.abs(y64) * 2.0 ** -13, MAX_ABS)
+    ulp = np.spacing(np.abs(y64).astype(np.float16)).astype(F64)
+    allowed = np.where(big, 0.5 * ulp + np.abs(y64) * 2.0 ** -13, MAX_ABS)
     worst = float(err.max()) if err.size else 0.0
     bad = err > allowed
+    # outputs over the 1e-2 target: allowed only where |y64| >= 32 (the fp16 grid there is
+    # coarser than the target); report their count and their error in fp16 spacings
+    over = err > MAX_ABS
+    n_over = int(over.sum())
+    info = {"rel_l2": rel, "max_abs": worst, "n_big": int(big.sum()), "n_relaxed": n_over,
+            "worst_relaxed_ulp": float((err[over] / ulp[over]).max()) if n_over else 0.0,
+            "max_abs_y": float(np.abs(y64).max()) if y64.size else 0.0}
+    if info["n_big"]:
+        RELAXED_REPORT.append((where, info))
     assert rel <= REL_L2, f"{where}: rel-L2 {rel:.3e} > {REL_L2}"
     assert not bad.any(), f"{where}: {int(bad.sum())} outputs over the bound, worst {worst:.4g}"
-    return {"rel_l2": rel, "max_abs": worst, "n_relaxed": int(big.sum())}
+    assert not (over & ~big).any(), f"{where}: an output with |y| < 32 is over {MAX_ABS}"
+    if info["max_abs_y"] < 32.0:
+        assert n_over == 0, where
+    return info
 
 
 def check_output_short(y_gpu_fp16: np.ndarray, W_hat: np.ndarray, w_weak: np.ndarray, idx: np.ndarray,
