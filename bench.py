@@ -231,148 +231,186 @@ def build_stack(owq, torch, spec, depth, M, dev):
     return sets, inputs, info
 
 
+class Stack:
+    """`depth` resident copies of one quantised layer set of a decode workload, and the timed
+    step over them: one token batch through every layer set, each launch group (layers that
+    share an input: q/k/v, gate/up) one launch, captured as CUDA graphs."""
+
+    def __init__(self, owq, torch, wl, depth, Mmax, dev):
+        self.owq, self.torch, self.wl, self.depth, self.dev = owq, torch, wl, depth, dev
+        self.spec = owq_synth.WORKLOADS[WID[wl]]
+        self.groups = GROUPS[wl]
+        self.sets, self.inputs, self.info = build_stack(owq, torch, self.spec, depth, Mmax, dev)
+
+    def launch_bytes(self, names, M):
+        info = self.info
+        return sum(layer_bytes(info[n].N, info[n].K, info[n].bits, info[n].group, info[n].k, M) for n in names)
+
+    def close(self):
+        for c in self.sets:
+            for L in c.values():
+                L.close()
+        self.sets = []
+
+    def measure(self, M, steps, warmup, world, local, e2e=True):
+        """Times `steps` replays of the step graph (after `warmup`); returns the figures of one
+        bench line (GB/s of the algorithmic bytes, per-launch diagnostics, e2e)."""
+        import torch
+
+        from cuda.bindings import runtime as rt
+        owq, dev, depth, groups, info = self.owq, self.dev, self.depth, self.groups, self.info
+        xs = {n: v["x"][:M].contiguous() for n, v in self.inputs.items()}
+        ys = {s: torch.empty((M, info[s].N), dtype=torch.float16, device=dev) for s in info}
+        step_bytes = depth * sum(self.launch_bytes(g, M) for g in groups)
+        step_wbytes = depth * sum(weight_bytes(info[n].N, info[n].K, info[n].bits, info[n].group, info[n].k)
+                                  for g in groups for n in g)
+        launches_per_step = depth * len(groups)
+        sets = self.sets
+
+        def issue(c, stream_ptr, ev=None):
+            """Enqueue one layer set (copy c); optional external event pairs around each launch."""
+            for gi, g in enumerate(groups):
+                if ev is not None:
+                    rt.cudaEventRecordWithFlags(ev[gi][0], stream_ptr, rt.cudaEventRecordExternal)
+                if len(g) == 1:
+                    st = owq.owq_gemv(sets[c][g[0]].handle, xs[g[0]], ys[g[0]], M, stream_ptr)
+                else:
+                    st = owq.owq_gemv_multi([sets[c][n].handle for n in g], [xs[n] for n in g],
+                                            [ys[n] for n in g], M, stream_ptr)
+                if st != 0:
+                    raise RuntimeError(f"launch failed: {owq.owq_status_string(st)}")
+                if ev is not None:
+                    rt.cudaEventRecordWithFlags(ev[gi][1], stream_ptr, rt.cudaEventRecordExternal)
+
+        stream = torch.cuda.Stream(device=dev)
+        sp = stream.cuda_stream
+        # eager warm-up of every copy (loads modules, sets kernel attributes)
+        for c in range(depth):
+            issue(c, sp)
+        torch.cuda.synchronize()
+
+        # the timed step: one CUDA graph of every launch, back to back, so that each kernel's
+        # prologue overlaps the previous kernel's tail (programmatic dependent launch)
+        NG = 2
+        graphs = []
+        for _ in range(NG):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                cs = torch.cuda.current_stream().cuda_stream
+                for c in range(depth):
+                    issue(c, cs)
+            graphs.append(g)
+        # diagnostic copy with an event pair around every launch (the events serialise the
+        # launches, so these per-launch times exclude the overlap the timed step gets)
+        ev_diag = [[[rt.cudaEventCreate()[1], rt.cudaEventCreate()[1]] for _ in groups] for _ in range(depth)]
+        g_diag = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_diag, stream=stream):
+            cs = torch.cuda.current_stream().cuda_stream
+            for c in range(depth):
+                issue(c, cs, ev_diag[c])
+
+        for i in range(warmup):
+            graphs[i % NG].replay()
+        torch.cuda.synchronize()
+
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            with torch.cuda.stream(stream):
+                t0.record(stream)
+                for i in range(steps):
+                    graphs[i % NG].replay()
+                t1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        ms_max = max_over_ranks(t0.elapsed_time(t1), world)
+
+        # per-launch diagnostics from the instrumented copy (after the timed region)
+        for _ in range(2):
+            g_diag.replay()
+        torch.cuda.synchronize()
+        durs = []
+        for c in range(depth):
+            for gi, g in enumerate(groups):
+                err, t = rt.cudaEventElapsedTime(ev_diag[c][gi][0], ev_diag[c][gi][1])
+                durs.append(t if err == rt.cudaError_t.cudaSuccess else float("nan"))
+        per_group = {}
+        for j, g in enumerate(groups):
+            sel = durs[j::len(groups)]
+            if sel:
+                us = 1e3 * sum(sel) / len(sel)
+                per_group["+".join(g)] = {"us": round(us, 3), "GBps": round(self.launch_bytes(g, M) / (us * 1e-6) / 1e9, 1)}
+        for pair in ev_diag:
+            for a, b in pair:
+                rt.cudaEventDestroy(a)
+                rt.cudaEventDestroy(b)
+        del g_diag
+
+        out = {"M": M, "ms_per_step": ms_max / steps, "ms_max": ms_max, "step_bytes": step_bytes,
+               "step_wbytes": step_wbytes, "launches_per_step": launches_per_step,
+               "per_group": per_group, "clocks": clk.summary()}
+        if e2e:
+            # e2e graph: pinned host activations in, outputs out, around the same step
+            host_x = {n: torch.empty_like(xs[n], device="cpu").pin_memory() for n in xs}
+            for n in xs:
+                host_x[n].copy_(xs[n].cpu())
+            host_y = {n: torch.empty_like(ys[n], device="cpu").pin_memory() for n in ys}
+            g_e2e = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_e2e, stream=stream):
+                for n in xs:
+                    xs[n].copy_(host_x[n], non_blocking=True)
+                cs = torch.cuda.current_stream().cuda_stream
+                for c in range(depth):
+                    issue(c, cs)
+                for n in ys:
+                    host_y[n].copy_(ys[n], non_blocking=True)
+            out["h2d"] = sum(v.numel() * v.element_size() for v in host_x.values())
+            out["d2h"] = sum(v.numel() * v.element_size() for v in host_y.values())
+            for _ in range(max(1, warmup)):
+                g_e2e.replay()
+            torch.cuda.synchronize()
+            barrier(world)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for i in range(steps):
+                    g_e2e.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            out["e2e_ms_max"] = max_over_ranks(e0.elapsed_time(e1), world)
+            del g_e2e
+        del graphs
+        torch.cuda.synchronize()
+        return out
+
+
 def run_owq(args, rank, world, local):
     import torch
 
     import weight_only_mixed_owq_b200 as owq
-    from cuda.bindings import runtime as rt
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     wl = args.workload
-    spec = owq_synth.WORKLOADS[WID[wl]]
     M = args.M
     depth = args.depth or DEPTH[wl]
-    groups = GROUPS[wl]
-    sets, inputs, info = build_stack(owq, torch, spec, depth, M, dev)
-    ys = {s: torch.empty((M, info[s].N), dtype=torch.float16, device=dev) for s in info}
-
-    # per-launch algorithmic bytes
-    def launch_bytes(names):
-        return sum(layer_bytes(info[n].N, info[n].K, info[n].bits, info[n].group, info[n].k, M) for n in names)
-
-    step_bytes = depth * sum(launch_bytes(g) for g in groups)
-    step_wbytes = depth * sum(weight_bytes(info[n].N, info[n].K, info[n].bits, info[n].group, info[n].k)
-                              for g in groups for n in g)
-    launches_per_step = depth * len(groups)
-
-    def issue(c, stream_ptr, ev=None):
-        """Enqueue one layer set (copy c); optional external event pairs around each launch."""
-        for gi, g in enumerate(groups):
-            if ev is not None:
-                rt.cudaEventRecordWithFlags(ev[gi][0], stream_ptr, rt.cudaEventRecordExternal)
-            if len(g) == 1:
-                st = owq.owq_gemv(sets[c][g[0]].handle, inputs[g[0]]["x"], ys[g[0]], M, stream_ptr)
-            else:
-                st = owq.owq_gemv_multi([sets[c][n].handle for n in g], [inputs[n]["x"] for n in g],
-                                        [ys[n] for n in g], M, stream_ptr)
-            if st != 0:
-                raise RuntimeError(f"launch failed: {owq.owq_status_string(st)}")
-            if ev is not None:
-                rt.cudaEventRecordWithFlags(ev[gi][1], stream_ptr, rt.cudaEventRecordExternal)
-
-    stream = torch.cuda.Stream(device=dev)
-    sp = stream.cuda_stream
-    # eager warm-up of every copy (loads modules, sets kernel attributes)
-    for c in range(depth):
-        issue(c, sp)
-    torch.cuda.synchronize()
-
-    # the timed step: one CUDA graph of every launch, back to back, so that each kernel's
-    # prologue overlaps the previous kernel's tail (programmatic dependent launch)
-    NG = 2
-    graphs = []
-    for gidx in range(NG):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            cs = torch.cuda.current_stream().cuda_stream
-            for c in range(depth):
-                issue(c, cs)
-        graphs.append(g)
-    # diagnostic copy with an event pair around every launch (the events serialise the
-    # launches, so these per-launch times exclude the overlap the timed step gets)
-    ev_diag = [[[rt.cudaEventCreate()[1], rt.cudaEventCreate()[1]] for _ in groups] for _ in range(depth)]
-    g_diag = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_diag, stream=stream):
-        cs = torch.cuda.current_stream().cuda_stream
-        for c in range(depth):
-            issue(c, cs, ev_diag[c])
-
-    # e2e graph: pinned host activations in, outputs out, around the same step
-    host_x = {n: torch.empty_like(inputs[n]["x"], device="cpu").pin_memory() for n in inputs}
-    for n in inputs:
-        host_x[n].copy_(inputs[n]["x"].cpu())
-    host_y = {n: torch.empty_like(ys[n], device="cpu").pin_memory() for n in ys}
-    g_e2e = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_e2e, stream=stream):
-        for n in inputs:
-            inputs[n]["x"].copy_(host_x[n], non_blocking=True)
-        cs = torch.cuda.current_stream().cuda_stream
-        for c in range(depth):
-            issue(c, cs)
-        for n in ys:
-            host_y[n].copy_(ys[n], non_blocking=True)
-    h2d = sum(v.numel() * v.element_size() for v in host_x.values())
-    d2h = sum(v.numel() * v.element_size() for v in host_y.values())
-
-    for i in range(args.warmup):
-        graphs[i % NG].replay()
-    torch.cuda.synchronize()
-
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            t0.record(stream)
-            for i in range(args.steps):
-                graphs[i % NG].replay()
-            t1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = t0.elapsed_time(t1)
-    ms_max = max_over_ranks(ms, world)
+    stack = Stack(owq, torch, wl, depth, M, dev)
+    spec, groups, info = stack.spec, stack.groups, stack.info
+    r = stack.measure(M, args.steps, args.warmup, world, local)
+    ms_max, step_bytes, step_wbytes = r["ms_max"], r["step_bytes"], r["step_wbytes"]
+    launches_per_step = r["launches_per_step"]
 
     # every launch of the timed region is the decode kernel: its average launch duration is
     # the timed region (CUDA events on the launching stream) over the launches in it
     launch_us = ms_max * 1e3 / (args.steps * launches_per_step)
     achieved = step_bytes * args.steps / (ms_max * 1e-3) / 1e9
 
-    # per-launch diagnostics from the instrumented copy (after the timed region)
-    for _ in range(2):
-        g_diag.replay()
-    torch.cuda.synchronize()
-    durs = []
-    for c in range(depth):
-        for gi, g in enumerate(groups):
-            err, t = rt.cudaEventElapsedTime(ev_diag[c][gi][0], ev_diag[c][gi][1])
-            durs.append(t if err == rt.cudaError_t.cudaSuccess else float("nan"))
-    per_group = {}
-    for j, g in enumerate(groups):
-        sel = durs[j::len(groups)]
-        if sel:
-            us = 1e3 * sum(sel) / len(sel)
-            per_group["+".join(g)] = {"us": round(us, 3), "GBps": round(launch_bytes(g) / (us * 1e-6) / 1e9, 1)}
-
-    # e2e
-    for _ in range(max(1, args.warmup)):
-        g_e2e.replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(args.steps):
-            g_e2e.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ems_max = max_over_ranks(e0.elapsed_time(e1), world)
-
     total_bytes = sum_over_ranks(step_bytes * args.steps, world)
     value = total_bytes / (ms_max * 1e-3) / 1e9
-    e2e_value = total_bytes / (ems_max * 1e-3) / 1e9
+    e2e_value = total_bytes / (r["e2e_ms_max"] * 1e-3) / 1e9
     peaks, peak_kind = measured_peaks()
     per_layer_us = ms_max * 1e3 / args.steps / (depth * sum(len(g) for g in groups))
 
@@ -400,7 +438,7 @@ def run_owq(args, rank, world, local):
             "weight_GBps": round(sum_over_ranks(step_wbytes * args.steps, world) / (ms_max * 1e-3) / 1e9, 2),
             "parallelism": f"replicas x{world}",
         },
-        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {
             "bound": "hbm",
@@ -414,14 +452,40 @@ def run_owq(args, rank, world, local):
             "traffic": ncu_traffic("k_gemv"),
             "launch_us": round(launch_us, 3),
             "basis": "algorithmic bytes of the timed launches / timed region (CUDA events); all launches are k_gemv",
-            "per_launch_group_serialised": per_group,
+            "per_launch_group_serialised": r["per_group"],
         },
-        "clocks": clk.summary(),
+        "clocks": r["clocks"],
     }
-    for c in sets:
-        for L in c.values():
-            L.close()
+    stack.close()
     return line
+
+
+def decode_sweep(args, wl, Ms, depth, steps, warmup, local):
+    """Further decode workloads measured in the same run (one GPU): the same step and timing as
+    the default line, for each token count in Ms.  Returns a dict keyed by M."""
+    import torch
+
+    import weight_only_mixed_owq_b200 as owq
+    dev = torch.device("cuda", local)
+    peaks, kind = measured_peaks()
+    stack = Stack(owq, torch, wl, depth, max(Ms), dev)
+    out = {}
+    for M in Ms:
+        r = stack.measure(M, steps, warmup, 1, local, e2e=False)
+        gbs = r["step_bytes"] * steps / (r["ms_max"] * 1e-3) / 1e9
+        out[str(M)] = {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                       "frac_of_8TBps_spec": round(gbs / 8000.0, 4),
+                       "ms_per_step": round(r["ms_per_step"], 4),
+                       "us_per_layer": round(r["ms_per_step"] * 1e3 / (depth * sum(len(g) for g in stack.groups)), 3),
+                       "per_launch_group_serialised": r["per_group"], "clocks": r["clocks"]}
+    layers = {n: [stack.info[n].N, stack.info[n].K] for n in stack.info}
+    stack.close()
+    torch.cuda.synchronize()
+    return {"workload": f"{wl}: {depth} resident layer sets per step", "layers": layers,
+            "bits": stack.spec.layers[0].bits,
+            "group": "per-channel" if stack.spec.layers[0].group == stack.spec.layers[0].K else stack.spec.layers[0].group,
+            "steps": steps, "warmup": warmup, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_kind": kind,
+            "timing": "CUDA graph of the whole step, CUDA events on the launching stream", "per_M": out}
 
 
 def prefill_measure(args, dev):
@@ -616,6 +680,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-wct", action="store_true", help="skip the weak column tuning kernels")
+    ap.add_argument("--no-sweeps", action="store_true", help="skip the LLaMA-7B and OPT-66B decode lines")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
@@ -629,6 +694,12 @@ def main(argv=None):
     line = run_owq(args, rank, world, local)
     if rank == 0 and world == 1:
         import torch
+        if not args.no_sweeps and args.workload == "opt-6.7b-decode":
+            # the LLaMA-7B token sweep and the whole 64-layer OPT-66B set (25.5 GB resident),
+            # each in the same step form as the default line
+            line["llama7b"] = decode_sweep(args, "llama-7b-decode", (1, 2, 4, 8, 16), DEPTH["llama-7b-decode"],
+                                           max(5, args.steps // 2), 3, local)
+            line["opt66b"] = decode_sweep(args, "opt-66b-decode", (1,), DEPTH["opt-66b-decode"], 3, 3, local)
         if not args.no_prefill:
             line["prefill"] = prefill_measure(args, torch.device("cuda", local))
         if not args.no_wct:

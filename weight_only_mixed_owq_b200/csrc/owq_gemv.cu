@@ -13,7 +13,8 @@
 //  * A warp streams its chunk through a private S-stage shared-memory ring filled by
 //    cp.async.bulk: the layer stores each 16-row tile block-major, so an item (16 rows x up to
 //    4 or 8 blocks of one tile) is one contiguous copy; the weak block, stored tile-major too,
-//    is streamed the same way at the start of each tile.
+//    is streamed the same way at the start of each tile.  Every weight copy carries an
+//    evict-first L2 hint: the weights are read once per call, the activations are not.
 //  * The contraction runs on the tensor cores (mma.sync m16n8k16, fp16 x fp16 -> fp32): with
 //    the packed layout of owq_format.cuh a lane's chunk of a block is exactly its A fragment,
 //    and one AND per code pair makes each A register (the codes as exact fp16 values
@@ -326,6 +327,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
   prod.init(hi, hi - lo, Kb, nsl, G_::kWs, SUB);
   cons.init(hi, hi - lo, Kb, nsl, G_::kWs, SUB);
   int issued = 0;
+  uint64_t pol;   // the weights are read once per call: evict them from L2 first
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   // lane 0 only: the next item of the chunk into the next stage (false once the chunk is exhausted)
   auto issue = [&]() -> bool {
     int kind, rt, first, cnt;
@@ -341,15 +344,15 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       bytes = (uint32_t)(cnt * G_::kTileBlk);
       if constexpr (PG) {
         mbar_arrive_expect_tx(&bars[st], bytes + (uint32_t)(cnt * 64));
-        bulk_load(ring + st * kStage + G_::kStageW, Pb.sz_t + ((size_t)rt * Kb + first) * 16, (uint32_t)(cnt * 64),
-                  &bars[st]);
-        bulk_load(ring + st * kStage, src, bytes, &bars[st]);
+        bulk_load_hint(ring + st * kStage + G_::kStageW, Pb.sz_t + ((size_t)rt * Kb + first) * 16, (uint32_t)(cnt * 64),
+                       &bars[st], pol);
+        bulk_load_hint(ring + st * kStage, src, bytes, &bars[st], pol);
         ++issued;
         return true;
       }
     }
     mbar_arrive_expect_tx(&bars[st], bytes);
-    bulk_load(ring + st * kStage, src, bytes, &bars[st]);
+    bulk_load_hint(ring + st * kStage, src, bytes, &bars[st], pol);
     ++issued;
     return true;
   };
