@@ -396,7 +396,9 @@ def search_params(W: np.ndarray, bits: int, group: int, weak_idx=None, alphas=DE
     shrink factor alpha in `alphas`, rounded to fp16; the zero points are every integer in
     [0, 2^b - 1]; the error is sum_j (w_j - fp16_rn(s (q_j - z)))^2 in fp64 over the group's
     dense columns, with q = clamp(rint(w / s) + z, 0, 2^b - 1) in fp32; the first minimum in
-    the order (alpha descending, z ascending) wins.  Weak columns are left out of the search.
+    the order (alpha descending, z ascending) wins; the error is a running fp64 sum in ascending
+    column order, each square rounded before it is added.  Weak columns are left out of the
+    search.
     Returns (scales fp16 N x G, zeros fp16 N x G).
     """
     W = np.asarray(W, dtype=F16)
@@ -425,7 +427,8 @@ def search_params(W: np.ndarray, bits: int, group: int, weak_idx=None, alphas=DE
                 for z in range(qmax + 1):
                     q = np.clip(np.rint(w / s32) + F32(z), F32(0), F32(qmax))
                     e = w.astype(F64) - _dequant_one(q, s16, F16(z)).astype(F64)
-                    err = float((e * e).sum())
+                    # fp64 sum of the squares in ascending column order (a running sum)
+                    err = float(np.cumsum(e * e)[-1]) if e.size else 0.0
                     if best is None or err < best[0]:
                         best = (err, s16, z)
             if best is None:   # a range below fp16 resolution: fall back to [-1, 1]
