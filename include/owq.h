@@ -110,6 +110,29 @@ owq_status_t owq_quantize_noalloc(const uint16_t* W, const uint16_t* X, int N, i
                                   int32_t* idx, uint16_t* w_weak, owq_stream_t stream);
 
 /*
+ * owq_search_params -- the truncation-aware 2-D grid search of the quantisation parameters
+ * that OWQ runs before OPTQ ("Low-precision quantization", paper "Quantization
+ * Configuration Search", pp.4-5: a search over step size and zero point with nearest rounding
+ * and truncation, which may shrink the range below min-max).  The pages give no grid; per
+ * (row, group), over the group's dense (non-idx) columns w (fp16 -> fp32):
+ *   mn = min(0, min w), mx = max(0, max w)  ([-1, 1] if mn == mx);
+ *   candidates: alpha in {1.00, 0.98, ..., 0.50} (alpha_i = fp32(1 - 0.02 i)) and every
+ *   integer z in [0, 2^bits - 1];  s = fp16_rn(fp32(fp32(mx - mn) * alpha) / (2^bits - 1))
+ *   (a candidate whose s is 0 is skipped);
+ *   error = sum over the dense columns in ascending order of (w - fp16_rn(s (q - z)))^2, fp64,
+ *   q = clamp(rint(w / s) + z, 0, 2^bits - 1) in fp32 (round half to even);
+ *   the first minimum in the order (alpha descending, z ascending) wins; if every s is 0,
+ *   s = fp16(2 / (2^bits - 1)) and z = 2^(bits-1).
+ * In:  W fp16 N x K; idx int32 k (device; strictly ascending in [0, K); may be NULL if k == 0).
+ * Out: scales, zeros fp16 N x (K / group) (fully overwritten; zeros integral).
+ * Synchronises `stream` once (idx validated on the host: OWQ_ERR_INDEX); one kernel, a CTA
+ * per (row, group) and a thread per candidate.  No scratch.  Deterministic.
+ */
+owq_status_t owq_search_params(const uint16_t* W, int N, int K, int bits, int group,
+                               const int32_t* idx, int k, uint16_t* scales, uint16_t* zeros,
+                               owq_stream_t stream);
+
+/*
  * owq_pack -- build a layer handle in the packed, latency-favoured layout ("Storage
  * Methods", appendix §2: a full low-precision matrix, zero-filled at the weak columns,
  * plus a separate fp16 block of the weak columns).
@@ -137,6 +160,54 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group,
                       const uint16_t* scales, const uint16_t* zeros,
                       const int32_t* idx, int k, const uint16_t* w_weak,
                       owq_stream_t stream, owq_layer_t* out);
+
+/*
+ * The storage-favoured form ("Storage Methods", appendix §2, pp.10-11: the low-precision
+ * matrix without the zero-filled weak columns, b + (16 - b) k / K bits per weight instead of
+ * b + 16 k / K; using it costs an index remap).  The pages give only the bit counts.  The
+ * stream used here: per row, the codes of the K - k dense (non-weak) columns in column order
+ * as one little-endian bit stream of `bits` bits per code -- code p of the row at bits
+ * [p*bits, p*bits + bits), bit b of the stream being bit b%32 of uint32 word b/32 -- padded
+ * with zero bits to W = ceil((K - k) * bits / 32) words per row; rows are consecutive
+ * (N x W uint32, row-major).  For a dense column j the stream position is p = j - #{t : idx[t]
+ * < j}.
+ */
+
+/* owq_storage_words -- W, the uint32 words per row of the storage-favoured stream (host
+ * call, no device work).  OWQ_ERR_SHAPE / OWQ_ERR_BITS for shapes outside the ranges above. */
+owq_status_t owq_storage_words(int K, int bits, int k, int* words_per_row);
+
+/*
+ * owq_storage_pack -- codes (uint8 N x K, values < 2^bits) -> the storage-favoured stream
+ * `words` (uint32 N x W, fully overwritten).  The codes of the idx columns are dropped.
+ * idx: int32 k (device; strictly ascending in [0, K); may be NULL when k == 0).
+ * Synchronises `stream` once (idx is copied to the host and validated: OWQ_ERR_INDEX), then
+ * launches one kernel (a thread per output word).
+ */
+owq_status_t owq_storage_pack(const uint8_t* codes, int N, int K, int bits,
+                              const int32_t* idx, int k, uint32_t* words, owq_stream_t stream);
+
+/*
+ * owq_storage_unpack -- the inverse: the storage-favoured stream `words` (uint32 N x W) ->
+ * codes (uint8 N x K, fully overwritten) with each weak column set to its group's zero point
+ * (the zero-filled codes the latency layout stores; zeros fp16 N x (K / group), integral).
+ * Synchronises `stream` once (idx validated on the host), then launches one kernel.
+ */
+owq_status_t owq_storage_unpack(const uint32_t* words, int N, int K, int bits, int group,
+                                const int32_t* idx, int k, const uint16_t* zeros,
+                                uint8_t* codes, owq_stream_t stream);
+
+/*
+ * owq_pack_storage -- build a layer handle from the storage-favoured stream: the stream is
+ * repacked on the GPU into the latency-favoured layout of owq_pack (same handle, same
+ * products, bit-identical to owq_pack of the unpacked codes).  Arguments as owq_pack, with
+ * `words` (uint32 N x W) in place of the codes.  Allocates an N x K byte code buffer for the
+ * duration of the call and frees it before returning; synchronises `stream`.
+ */
+owq_status_t owq_pack_storage(const uint32_t* words, int N, int K, int bits, int group,
+                              const uint16_t* scales, const uint16_t* zeros,
+                              const int32_t* idx, int k, const uint16_t* w_weak,
+                              owq_stream_t stream, owq_layer_t* out);
 
 /*
  * owq_gemv -- decode product for 1 <= M <= 16 tokens ("Real-device acceleration",

@@ -83,6 +83,23 @@ def test_host_validation_rejects_bad_arguments(owq):
     assert owq.owq_debug_inject(-1, 1000) == 12
     assert owq.owq_debug_inject(owq.OWQ_INJECT_GEMV_TAG, 0) == 12
     assert owq.owq_debug_inject(owq.OWQ_INJECT_NONE, 0) == 0
+    # parameter search
+    assert owq.owq_search_params(None, 16, 128, 3, 128, A, 1, A, A) == 1
+    assert owq.owq_search_params(A, 16, 128, 5, 128, A, 1, A, A) == 3
+    assert owq.owq_search_params(A, 16, 256, 3, 64, A, 1, A, A) == 4
+    assert owq.owq_search_params(A + 8, 16, 128, 3, 128, A, 1, A, A) == 6
+    # storage-favoured stream: host word count, NULL pointers, shapes, alignment
+    assert owq.owq_storage_words(4096, 3, 32) == (0, ((4096 - 32) * 3 + 31) // 32)
+    assert owq.owq_storage_words(11008, 4, 86) == (0, ((11008 - 86) * 4 + 31) // 32)
+    assert owq.owq_storage_words(4096, 5, 32)[0] == 3
+    assert owq.owq_storage_words(4096, 3, 1025)[0] == 2
+    assert owq.owq_storage_pack(None, 16, 128, 3, A, 1, A) == 1
+    assert owq.owq_storage_pack(A, 16, 100, 3, A, 1, A) == 2
+    assert owq.owq_storage_pack(A + 4, 16, 128, 3, A, 1, A) == 6
+    assert owq.owq_storage_unpack(A, 16, 256, 3, 64, A, 1, A, A) == 4
+    assert owq.owq_storage_unpack(A, 16, 128, 3, 128, None, 1, A, A) == 1
+    st, h = owq.owq_pack_storage(A, 16, 128, 4, 128, A, A, None, 1, A)
+    assert st == 1 and h is None
 
 
 @pytest.mark.skipif(_gpu_present(), reason="checks the no-device path; needs a machine without a GPU")

@@ -26,6 +26,11 @@ PROTOTYPES = [
     ("owq_quantize", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     ("owq_quantize_noalloc", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     ("owq_pack", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, ctypes.POINTER(_P)]),
+    ("owq_search_params", _I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
+    ("owq_storage_words", _I, [_I, _I, _I, ctypes.POINTER(_I)]),
+    ("owq_storage_pack", _I, [_P, _I, _I, _I, _P, _I, _P, _P]),
+    ("owq_storage_unpack", _I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
+    ("owq_pack_storage", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     ("owq_gemv", _I, [_P, _P, _P, _I, _P]),
     ("owq_gemv_multi", _I, [ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _I, _P]),
     ("owq_gemm", _I, [_P, _P, _P, _I, _P]),
@@ -106,6 +111,34 @@ def owq_pack(codes, N, K, bits, group, scales, zeros, idx, k, w_weak, stream=Non
     h = ctypes.c_void_p()
     st = LIB.owq_pack(_ptr(codes), N, K, bits, group, _ptr(scales), _ptr(zeros), _ptr(idx), k,
                       _ptr(w_weak), _stream(stream), ctypes.byref(h))
+    return st, h.value
+
+
+def owq_search_params(W, N, K, bits, group, idx, k, scales, zeros, stream=None) -> int:
+    return LIB.owq_search_params(_ptr(W), N, K, bits, group, _ptr(idx), k, _ptr(scales), _ptr(zeros), _stream(stream))
+
+
+def owq_storage_words(K, bits, k):
+    """Returns (status, uint32 words per row of the storage-favoured stream)."""
+    w = ctypes.c_int()
+    st = LIB.owq_storage_words(K, bits, k, ctypes.byref(w))
+    return st, w.value
+
+
+def owq_storage_pack(codes, N, K, bits, idx, k, words, stream=None) -> int:
+    return LIB.owq_storage_pack(_ptr(codes), N, K, bits, _ptr(idx), k, _ptr(words), _stream(stream))
+
+
+def owq_storage_unpack(words, N, K, bits, group, idx, k, zeros, codes, stream=None) -> int:
+    return LIB.owq_storage_unpack(_ptr(words), N, K, bits, group, _ptr(idx), k, _ptr(zeros), _ptr(codes),
+                                  _stream(stream))
+
+
+def owq_pack_storage(words, N, K, bits, group, scales, zeros, idx, k, w_weak, stream=None):
+    """Returns (status, handle)."""
+    h = ctypes.c_void_p()
+    st = LIB.owq_pack_storage(_ptr(words), N, K, bits, group, _ptr(scales), _ptr(zeros), _ptr(idx), k,
+                              _ptr(w_weak), _stream(stream), ctypes.byref(h))
     return st, h.value
 
 

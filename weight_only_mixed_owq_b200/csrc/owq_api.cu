@@ -53,6 +53,23 @@ owq_status_t check_shape(int N, int K, int bits, int group, int k) {
   return OWQ_OK;
 }
 
+// idx (k device ints) copied to the host on `s` (synchronised) and checked: strictly
+// ascending in [0, K)
+owq_status_t check_idx_on_host(const int32_t* idx, int k, int K, cudaStream_t s) {
+  if (k == 0) return OWQ_OK;
+  std::vector<int32_t> h(k);
+  if (cudaMemcpyAsync(h.data(), idx, sizeof(int32_t) * k, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return OWQ_ERR_CUDA;
+  }
+  for (int t = 0; t < k; ++t) {
+    if (h[t] < 0 || h[t] >= K) return OWQ_ERR_INDEX;
+    if (t > 0 && h[t] <= h[t - 1]) return OWQ_ERR_INDEX;
+  }
+  return OWQ_OK;
+}
+
 owq_status_t cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return OWQ_OK;
   cudaGetLastError();
@@ -216,6 +233,86 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   }
   *out = reinterpret_cast<owq_layer_t>(L);
   return OWQ_OK;
+}
+
+owq_status_t owq_search_params(const uint16_t* W, int N, int K, int bits, int group, const int32_t* idx, int k,
+                               uint16_t* scales, uint16_t* zeros, owq_stream_t stream) {
+  if (!W || !scales || !zeros || (k > 0 && !idx)) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, group, k);
+  if (st) return st;
+  if (!aligned16(W) || !aligned16(scales) || !aligned16(zeros) || (k > 0 && !aligned16(idx))) return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = check_idx_on_host(idx, k, K, s))) return st;
+  return cuda_status(launch_search_params(reinterpret_cast<const __half*>(W), N, K, bits, group, idx, k,
+                                          reinterpret_cast<__half*>(scales), reinterpret_cast<__half*>(zeros), s));
+}
+
+owq_status_t owq_storage_words(int K, int bits, int k, int* words_per_row) {
+  if (!words_per_row) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(1, K, bits, K, k);
+  if (st) return st;
+  *words_per_row = storage_words_per_row(K, bits, k);
+  return OWQ_OK;
+}
+
+owq_status_t owq_storage_pack(const uint8_t* codes, int N, int K, int bits, const int32_t* idx, int k,
+                              uint32_t* words, owq_stream_t stream) {
+  if (!codes || !words || (k > 0 && !idx)) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, K, k);
+  if (st) return st;
+  if (!aligned16(codes) || !aligned16(words) || (k > 0 && !aligned16(idx))) return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = check_idx_on_host(idx, k, K, s))) return st;
+  return cuda_status(launch_storage_pack(codes, N, K, bits, idx, k, words, s));
+}
+
+owq_status_t owq_storage_unpack(const uint32_t* words, int N, int K, int bits, int group, const int32_t* idx,
+                                int k, const uint16_t* zeros, uint8_t* codes, owq_stream_t stream) {
+  if (!words || !zeros || !codes || (k > 0 && !idx)) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, group, k);
+  if (st) return st;
+  if (!aligned16(words) || !aligned16(zeros) || !aligned16(codes) || (k > 0 && !aligned16(idx))) return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = check_idx_on_host(idx, k, K, s))) return st;
+  return cuda_status(launch_storage_unpack(words, N, K, bits, group, idx, k,
+                                           reinterpret_cast<const __half*>(zeros), codes, s));
+}
+
+owq_status_t owq_pack_storage(const uint32_t* words, int N, int K, int bits, int group, const uint16_t* scales,
+                              const uint16_t* zeros, const int32_t* idx, int k, const uint16_t* w_weak,
+                              owq_stream_t stream, owq_layer_t* out) {
+  if (!out) return OWQ_ERR_NULL;
+  *out = nullptr;
+  if (!words || !scales || !zeros || (k > 0 && (!idx || !w_weak))) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, group, k);
+  if (st) return st;
+  if (!aligned16(words) || !aligned16(scales) || !aligned16(zeros) ||
+      (k > 0 && (!aligned16(idx) || !aligned16(w_weak))))
+    return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = check_idx_on_host(idx, k, K, s))) return st;
+  // the full code matrix, for the time of the repack
+  uint8_t* codes = nullptr;
+  if (cudaMalloc(&codes, (size_t)N * K) != cudaSuccess) {
+    cudaGetLastError();
+    return OWQ_ERR_NOMEM;
+  }
+  cudaError_t e = launch_storage_unpack(words, N, K, bits, group, idx, k, reinterpret_cast<const __half*>(zeros),
+                                        codes, s);
+  st = e == cudaSuccess ? owq_pack(codes, N, K, bits, group, scales, zeros, idx, k, w_weak, stream, out)
+                        : cuda_status(e);
+  if (cudaStreamSynchronize(s) != cudaSuccess && st == OWQ_OK) st = OWQ_ERR_CUDA;
+  cudaGetLastError();
+  cudaFree(codes);
+  if (st != OWQ_OK && *out) {
+    owq_layer_free(*out);
+    *out = nullptr;
+  }
+  return st;
 }
 
 // one armed test failure (owq_debug_inject), taken by the next call of its kind

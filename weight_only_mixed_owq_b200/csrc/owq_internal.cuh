@@ -109,6 +109,17 @@ cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int 
                             int group, int k, uint8_t* codes, __half* scales, __half* zeros,
                             int32_t* idx, __half* w_weak, cudaStream_t s);
 
+// truncation-aware (step, zero) grid search per (row, group) over the dense columns
+cudaError_t launch_search_params(const __half* W, int N, int K, int bits, int group, const int32_t* idx, int k,
+                                 __half* scales, __half* zeros, cudaStream_t s);
+
+// storage-favoured dense stream (words per row = ceil((K - k) bits / 32)) <-> full code matrix
+int storage_words_per_row(int K, int bits, int k);
+cudaError_t launch_storage_pack(const uint8_t* codes, int N, int K, int bits, const int32_t* idx, int k,
+                                uint32_t* words, cudaStream_t s);
+cudaError_t launch_storage_unpack(const uint32_t* words, int N, int K, int bits, int group, const int32_t* idx,
+                                  int k, const __half* zeros, uint8_t* codes, cudaStream_t s);
+
 // weak column tuning: dW_weak = dY^T x[:, idx] (fp32 N x k) and dX = dY W_eff (fp16 M x K)
 cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, float* dw, int M,
                              cudaStream_t s);
