@@ -96,9 +96,12 @@ owq_status_t owq_quantize(const uint16_t* W, const uint16_t* X, int N, int K, in
  * outputs and results (bit-identical) as owq_quantize, but its scratch lives in a static
  * device array sized for K <= OWQ_NOALLOC_MAX_K columns (25 bytes per column, 1 MB), which
  * every GPU that loads this library keeps until the process exits.  K above that limit
- * returns OWQ_ERR_SHAPE and launches nothing.  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) and caches it, so make that first call
- * outside any stream capture.  All calls share the one array: calls that can overlap on the
+ * returns OWQ_ERR_SHAPE and launches nothing.  Every call made outside a stream capture
+ * looks up the array's device address in the current context (cudaGetSymbolAddress) and
+ * caches it per device; a call inside a capture uses that cache, so the first call on a
+ * device must come before any stream capture (a capture before it returns OWQ_ERR_CUDA).
+ * The address belongs to the context current at the lookup: after cudaDeviceReset, or in
+ * another context on the same device, make one call outside a capture first.  All calls share the one array: calls that can overlap on the
  * GPU (unordered streams) race on it and must be serialised by the caller.  No state carries
  * over between calls (each kernel fully writes what it later reads).  Calls no cudaMalloc,
  * cudaFree or other allocating routine.
@@ -154,7 +157,9 @@ owq_status_t owq_search_params(const uint16_t* W, int N, int K, int bits, int gr
  *   to a multiple of 16 with zero words) and, for the decode kernel, tile-major copies of
  *   the weak block and of the (scale, zero) pairs plus a split-tile workspace (2 KB per
  *   16-row tile and per extra CTA that may share it: one for most layers, N/16 * 2 KB).
- * Synchronises `stream` once (idx is copied to the host and validated: OWQ_ERR_INDEX).
+ * Synchronises `stream` twice: once to copy idx to the host and validate it (OWQ_ERR_INDEX,
+ * before anything is allocated), and once at the end, so that the host-side tables it uploads
+ * outlive their copies.
  */
 owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group,
                       const uint16_t* scales, const uint16_t* zeros,
@@ -239,8 +244,8 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
 
 /*
  * owq_gemm -- prefill product for any M >= 1 (tuned for M >= 64): TMA-staged packed tiles,
- * dequantised into shared memory and fed to tcgen05 MMA with fp32 accumulators in tensor
- * memory; the weak block and the weak activations (gathered by a small kernel into the
+ * dequantised in registers into tensor memory (the A operand of tcgen05 MMA, B = the
+ * activations in shared memory) with fp32 accumulators in tensor memory; the weak block and the weak activations (gathered by a small kernel into the
  * handle's scratch) run as extra K-steps into the same accumulator.  Same semantics and
  * layouts as owq_gemv; M <= 65536.  Bounded device waits: on a timeout the kernel abandons
  * its tile, sets the device status word and this call's later owq_device_status returns
@@ -308,8 +313,12 @@ owq_status_t owq_layer_bytes(owq_layer_t layer, size_t* packed, size_t* scales_z
 /* Release a layer (stream-ordered on the stream given to owq_pack). NULL is a no-op. */
 owq_status_t owq_layer_free(owq_layer_t layer);
 
-/* Synchronises the device, then returns and clears the device status word that bounded
- * waits set (OWQ_OK, or OWQ_ERR_TIMEOUT). */
+/* Synchronises the current device (cudaDeviceSynchronize), then returns and clears its device
+ * status word (OWQ_OK, or OWQ_ERR_TIMEOUT if a bounded wait of any call on this device gave up
+ * since the last query).  The word is per device, not per handle: a bounded wait gives up
+ * inside a kernel, which has no way to name the handle of the call that launched it, and the
+ * kernels of every handle on a device write the same word.  The whole device is synchronised
+ * because the failed call may sit on any stream; call this between steps, not on a hot path. */
 owq_status_t owq_device_status(void);
 
 /*

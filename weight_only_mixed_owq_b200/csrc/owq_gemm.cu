@@ -440,8 +440,8 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   const int nK = L.K / kStepCodes;
   const long long tiles = (long long)((L.N + kBM - 1) / kBM) * ((M + BN - 1) / BN);
   int splits = 1;
-  static int sms = 0;
-  if (!sms && (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, L.device) != cudaSuccess || sms <= 0)) {
+  int sms = 0;   // SM count of the layer's device
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, L.device) != cudaSuccess || sms <= 0) {
     cudaGetLastError();
     sms = 148;
   }

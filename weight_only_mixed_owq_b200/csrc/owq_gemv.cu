@@ -765,17 +765,24 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
       mbar_wait(&bars[j % S], (uint32_t)((j / S) & 1), args.status, args.wait_limit);
 }
 
+// SM count of the current device (cached per device ordinal)
 int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      n = 148;
-    }
+  constexpr int kMaxDev = 64;
+  static int n[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return 148;
   }
-  return n;
+  if (!n[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      v = 148;
+    }
+    n[dev] = v;
+  }
+  return n[dev];
 }
 
 // Exact per-pair dequantisation (see the kernel) for two token tiles, and for per-group layers

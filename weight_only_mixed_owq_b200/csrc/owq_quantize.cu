@@ -244,19 +244,28 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 unsigned char* g_noalloc_addr[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device (looked up once per device;
-// in host code the array's name is only a host-side stand-in, never a device address).
-cudaError_t noalloc_scratch(unsigned char** out) {
+// Device address of the static scratch on the current device.  In host code the array's name
+// is only a host-side stand-in, never a device address, so the address is looked up with the
+// device current: on every call made outside a stream capture (so a context created anew, e.g.
+// after cudaDeviceReset, gets its own address), and taken from the per-device cache during a
+// capture (a lookup there could load the module, which a capture does not allow; the first
+// call on a device must therefore come before any capture).
+cudaError_t noalloc_scratch(cudaStream_t s, unsigned char** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> g(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, owq_noalloc_scratch);
     if (e != cudaSuccess) return e;
     g_noalloc_addr[dev] = static_cast<unsigned char*>(p);
+  } else if (!g_noalloc_addr[dev]) {
+    return cudaErrorStreamCaptureUnsupported;
   }
   *out = g_noalloc_addr[dev];
   return cudaSuccess;
@@ -266,7 +275,7 @@ cudaError_t launch_quantize_static(const __half* W, const __half* X, int N, int 
                                    int group, int k, uint8_t* codes, __half* scales, __half* zeros,
                                    int32_t* idx, __half* w_weak, cudaStream_t s) {
   unsigned char* buf = nullptr;
-  cudaError_t e = noalloc_scratch(&buf);
+  cudaError_t e = noalloc_scratch(s, &buf);
   if (e != cudaSuccess) return e;
   double* lam = reinterpret_cast<double*>(buf);
   double* colsum = lam + K;

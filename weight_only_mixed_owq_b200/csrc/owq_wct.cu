@@ -275,13 +275,20 @@ k_input_grad(const IgArgs a) {
   if (tid == 0) a.count[b] = 0u;   // ready for the next call on this stream
 }
 
+// SM count of device `dev` (cached per device ordinal)
 int wct_sm_count(int dev) {
-  static int n = 0;
-  if (!n && (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)) {
-    cudaGetLastError();
-    n = 148;
+  constexpr int kMaxDev = 64;
+  static int n[kMaxDev] = {};
+  if (dev < 0 || dev >= kMaxDev) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      v = 148;
+    }
+    n[dev] = v;
   }
-  return n;
+  return n[dev];
 }
 
 template <int BITS, int TOK>
