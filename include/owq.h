@@ -136,6 +136,46 @@ owq_status_t owq_search_params(const uint16_t* W, int N, int K, int bits, int gr
                                owq_stream_t stream);
 
 /*
+ * owq_optq -- OPTQ with the weak columns moved last, the dense quantiser the paper runs after
+ * the parameter search ("Low-precision quantization", paper p.4: column-by-column quantisation
+ * whose error each step compensates on the columns not yet quantised; the weak columns come
+ * last, are never quantised, and keep their compensated fp16 values; "Layer-wise Quantization
+ * and Hessian", p.3: each row's error is dW H dW^T).
+ *   H = X^T X + damp * mean(diag(X^T X)) * I                 (fp64; damp = 0.01 is OPTQ's usual)
+ *   order = the dense (non-idx) columns ascending, then the idx columns ascending;
+ *   for each dense column j in that order, with F the columns from j on and M = (H over F)^-1:
+ *     q = clamp(rint(fp32(w_j) / s) + z, 0, 2^bits - 1)  (the (s, z) of j's group, given);
+ *     w_hat = fp16_rn(s (q - z));  w_F\j -= (w_j - w_hat) / M[j][j] * M[j][F\j];  w_j = w_hat.
+ *   M is kept exact from step to step by the Schur-complement identity of the inverse of a
+ *   principal submatrix (one fp64 Gauss-Jordan inversion of H first); all arithmetic is fp64.
+ * In:  W fp16 N x K; X fp16 T x K (calibration tokens; 1 <= T <= 2^20); idx int32 k (device,
+ *      strictly ascending); scales, zeros fp16 N x (K / group) (e.g. from owq_search_params);
+ *      0 <= damp (H must be positive definite: with damp = 0, T >= K is needed).
+ * Out: codes uint8 N x K (the weak columns get their group's zero point, so the result can
+ *      go straight to owq_pack); w_weak fp16 N x k (the compensated weak columns).
+ * Allocates K*K + N*K doubles (+ small) of stream-ordered scratch, freed before it returns;
+ * synchronises `stream` once (idx is validated on the host).  Offline: 2 K + 2 (K - k) kernel
+ * launches; about 0.5 s for a 4096 x 4096 layer.  Deterministic.
+ */
+owq_status_t owq_optq(const uint16_t* W, const uint16_t* X, int N, int K, int T, int bits,
+                      int group, const int32_t* idx, int k, const uint16_t* scales,
+                      const uint16_t* zeros, double damp, uint8_t* codes, uint16_t* w_weak,
+                      owq_stream_t stream);
+
+/*
+ * owq_quantize_optq -- the paper's dense quantiser, end to end ("Weak-column selection",
+ * "Low-precision quantization", pp.4-5): the weak columns of owq_quantize (lambda, all-column
+ * RTN perturbation, sensitivity, top k), then owq_search_params over the dense columns, then
+ * owq_optq with those parameters.  Same arguments and outputs as owq_quantize plus damp;
+ * scales/zeros are the searched ones, codes and w_weak those of OPTQ (w_weak holds the
+ * compensated weak columns).  Synchronises `stream` (idx validation of the two later steps).
+ */
+owq_status_t owq_quantize_optq(const uint16_t* W, const uint16_t* X, int N, int K, int T,
+                               int bits, int group, int k, double damp,
+                               uint8_t* codes, uint16_t* scales, uint16_t* zeros,
+                               int32_t* idx, uint16_t* w_weak, owq_stream_t stream);
+
+/*
  * owq_pack -- build a layer handle in the packed, latency-favoured layout ("Storage
  * Methods", appendix §2: a full low-precision matrix, zero-filled at the weak columns,
  * plus a separate fp16 block of the weak columns).

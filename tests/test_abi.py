@@ -88,6 +88,14 @@ def test_host_validation_rejects_bad_arguments(owq):
     assert owq.owq_search_params(A, 16, 128, 5, 128, A, 1, A, A) == 3
     assert owq.owq_search_params(A, 16, 256, 3, 64, A, 1, A, A) == 4
     assert owq.owq_search_params(A + 8, 16, 128, 3, 128, A, 1, A, A) == 6
+    # OPTQ
+    assert owq.owq_optq(None, A, 16, 128, 8, 3, 128, A, 1, A, A, 0.01, A, A) == 1
+    assert owq.owq_optq(A, A, 16, 128, 0, 3, 128, A, 1, A, A, 0.01, A, A) == 2
+    assert owq.owq_optq(A, A, 16, 128, 8, 3, 128, A, 1, A, A, -1.0, A, A) == 12
+    assert owq.owq_optq(A, A, 16, 128, 8, 3, 128, A, 1, A, A, float("nan"), A, A) == 12
+    assert owq.owq_optq(A, A + 2, 16, 128, 8, 3, 128, A, 1, A, A, 0.01, A, A) == 6
+    assert owq.owq_quantize_optq(A, A, 16, 128, 8, 3, 128, 1, -0.5, A, A, A, A, A) == 12
+    assert owq.owq_quantize_optq(None, A, 16, 128, 8, 3, 128, 1, 0.01, A, A, A, A, A) == 1
     # storage-favoured stream: host word count, NULL pointers, shapes, alignment
     assert owq.owq_storage_words(4096, 3, 32) == (0, ((4096 - 32) * 3 + 31) // 32)
     assert owq.owq_storage_words(11008, 4, 86) == (0, ((11008 - 86) * 4 + 31) // 32)

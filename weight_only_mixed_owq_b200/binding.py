@@ -27,6 +27,8 @@ PROTOTYPES = [
     ("owq_quantize_noalloc", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     ("owq_pack", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, ctypes.POINTER(_P)]),
     ("owq_search_params", _I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
+    ("owq_optq", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, ctypes.c_double, _P, _P, _P]),
+    ("owq_quantize_optq", _I, [_P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_double, _P, _P, _P, _P, _P, _P]),
     ("owq_storage_words", _I, [_I, _I, _I, ctypes.POINTER(_I)]),
     ("owq_storage_pack", _I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     ("owq_storage_unpack", _I, [_P, _I, _I, _I, _I, _P, _I, _P, _P, _P]),
@@ -116,6 +118,16 @@ def owq_pack(codes, N, K, bits, group, scales, zeros, idx, k, w_weak, stream=Non
 
 def owq_search_params(W, N, K, bits, group, idx, k, scales, zeros, stream=None) -> int:
     return LIB.owq_search_params(_ptr(W), N, K, bits, group, _ptr(idx), k, _ptr(scales), _ptr(zeros), _stream(stream))
+
+
+def owq_optq(W, X, N, K, T, bits, group, idx, k, scales, zeros, damp, codes, w_weak, stream=None) -> int:
+    return LIB.owq_optq(_ptr(W), _ptr(X), N, K, T, bits, group, _ptr(idx), k, _ptr(scales), _ptr(zeros),
+                        float(damp), _ptr(codes), _ptr(w_weak), _stream(stream))
+
+
+def owq_quantize_optq(W, X, N, K, T, bits, group, k, damp, codes, scales, zeros, idx, w_weak, stream=None) -> int:
+    return LIB.owq_quantize_optq(_ptr(W), _ptr(X), N, K, T, bits, group, k, float(damp), _ptr(codes), _ptr(scales),
+                                 _ptr(zeros), _ptr(idx), _ptr(w_weak), _stream(stream))
 
 
 def owq_storage_words(K, bits, k):
@@ -290,6 +302,25 @@ class OwqLayer:
             self.close()
         except Exception:
             pass
+
+
+def quantize_optq(W, X, bits: int, group: int, k: int, damp: float = 0.01, stream=None) -> dict:
+    """Run owq_quantize_optq (selection, parameter search, OPTQ with the weak columns last) on
+    fp16 CUDA tensors W (N x K) and X (T x K); allocates the outputs."""
+    import torch
+    N, K = W.shape
+    T = X.shape[0]
+    dev = W.device
+    out = {
+        "codes": torch.empty((N, K), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((N, K // group), dtype=torch.float16, device=dev),
+        "zeros": torch.empty((N, K // group), dtype=torch.float16, device=dev),
+        "idx": torch.empty((k,), dtype=torch.int32, device=dev),
+        "w_weak": torch.empty((N, k), dtype=torch.float16, device=dev),
+    }
+    _check(owq_quantize_optq(W, X, N, K, T, bits, group, k, damp, out["codes"], out["scales"], out["zeros"],
+                             out["idx"] if k else None, out["w_weak"] if k else None, stream), "owq_quantize_optq")
+    return out
 
 
 def quantize_pack(W, X, bits: int, group: int, k: int, stream=None) -> tuple[OwqLayer, dict]:

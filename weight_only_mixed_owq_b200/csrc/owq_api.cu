@@ -248,6 +248,59 @@ owq_status_t owq_search_params(const uint16_t* W, int N, int K, int bits, int gr
                                           reinterpret_cast<__half*>(scales), reinterpret_cast<__half*>(zeros), s));
 }
 
+owq_status_t owq_optq(const uint16_t* W, const uint16_t* X, int N, int K, int T, int bits, int group,
+                      const int32_t* idx, int k, const uint16_t* scales, const uint16_t* zeros, double damp,
+                      uint8_t* codes, uint16_t* w_weak, owq_stream_t stream) {
+  if (!W || !X || !scales || !zeros || !codes || (k > 0 && (!idx || !w_weak))) return OWQ_ERR_NULL;
+  owq_status_t st = check_shape(N, K, bits, group, k);
+  if (st) return st;
+  if (T < 1 || T > (1 << 20)) return OWQ_ERR_SHAPE;
+  if (!(damp >= 0.0) || !(damp <= 1e6)) return OWQ_ERR_ARG;
+  if (!aligned16(W) || !aligned16(X) || !aligned16(scales) || !aligned16(zeros) || !aligned16(codes) ||
+      (k > 0 && (!aligned16(idx) || !aligned16(w_weak))))
+    return OWQ_ERR_ALIGN;
+  if ((st = check_device())) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<int32_t> h(k);
+  if (k > 0) {
+    if (cudaMemcpyAsync(h.data(), idx, sizeof(int32_t) * k, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return OWQ_ERR_CUDA;
+    }
+    for (int t = 0; t < k; ++t) {
+      if (h[t] < 0 || h[t] >= K) return OWQ_ERR_INDEX;
+      if (t > 0 && h[t] <= h[t - 1]) return OWQ_ERR_INDEX;
+    }
+  }
+  // the order of the columns: the dense ones ascending, then the weak ones ascending
+  std::vector<int> perm;
+  perm.reserve(K);
+  std::vector<char> weak(K, 0);
+  for (int t = 0; t < k; ++t) weak[h[t]] = 1;
+  for (int j = 0; j < K; ++j)
+    if (!weak[j]) perm.push_back(j);
+  for (int t = 0; t < k; ++t) perm.push_back(h[t]);
+  return cuda_status(launch_optq(reinterpret_cast<const __half*>(W), reinterpret_cast<const __half*>(X), N, K, T,
+                                 bits, group, perm.data(), k, reinterpret_cast<const __half*>(scales),
+                                 reinterpret_cast<const __half*>(zeros), damp, codes,
+                                 reinterpret_cast<__half*>(w_weak), s));
+}
+
+owq_status_t owq_quantize_optq(const uint16_t* W, const uint16_t* X, int N, int K, int T, int bits, int group,
+                               int k, double damp, uint8_t* codes, uint16_t* scales, uint16_t* zeros, int32_t* idx,
+                               uint16_t* w_weak, owq_stream_t stream) {
+  if (!(damp >= 0.0) || !(damp <= 1e6)) return OWQ_ERR_ARG;
+  // 1. the weak columns (the selection of owq_quantize; its RTN outputs are overwritten below)
+  owq_status_t st = owq_quantize(W, X, N, K, T, bits, group, k, codes, scales, zeros, idx, w_weak, stream);
+  if (st) return st;
+  // 2. the (step, zero) search over the dense columns, 3. OPTQ with the weak columns last
+  st = owq_search_params(W, N, K, bits, group, k > 0 ? idx : nullptr, k, scales, zeros, stream);
+  if (st) return st;
+  return owq_optq(W, X, N, K, T, bits, group, k > 0 ? idx : nullptr, k, scales, zeros, damp, codes,
+                  k > 0 ? w_weak : nullptr, stream);
+}
+
 owq_status_t owq_storage_words(int K, int bits, int k, int* words_per_row) {
   if (!words_per_row) return OWQ_ERR_NULL;
   owq_status_t st = check_shape(1, K, bits, K, k);

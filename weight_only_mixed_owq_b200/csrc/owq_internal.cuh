@@ -113,6 +113,13 @@ cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int 
 cudaError_t launch_search_params(const __half* W, int N, int K, int bits, int group, const int32_t* idx, int k,
                                  __half* scales, __half* zeros, cudaStream_t s);
 
+// OPTQ with the weak columns last: perm (host, K entries) = dense columns ascending, then the
+// weak columns ascending; scratch K*K + N*K doubles (stream-ordered)
+size_t optq_scratch_bytes(int N, int K);
+cudaError_t launch_optq(const __half* W, const __half* X, int N, int K, int T, int bits, int group,
+                        const int* perm_host, int k, const __half* scales, const __half* zeros, double damp,
+                        uint8_t* codes, __half* w_weak, cudaStream_t s);
+
 // storage-favoured dense stream (words per row = ceil((K - k) bits / 32)) <-> full code matrix
 int storage_words_per_row(int K, int bits, int k);
 cudaError_t launch_storage_pack(const uint8_t* codes, int N, int K, int bits, const int32_t* idx, int k,
