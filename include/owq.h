@@ -308,7 +308,15 @@ owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
  * In:  x fp16 M x K row-major (the layer's forward input), dy fp16 M x N row-major (the
  *      gradient of its output); 1 <= M <= 65536.
  * Out: dw_weak fp32 N x k row-major (fully overwritten; may be NULL when k == 0, and then
- *      nothing is launched).  fp32 accumulation in token order.  No scratch, no waits.
+ *      nothing is launched).  A dense N x k x M contraction on the tensor cores (mma.sync
+ *      m16n8k16, fp16 products exact in fp32, fp32 accumulation): a small kernel gathers
+ *      x[:, idx] into the handle's scratch, the product kernel splits the tokens over CTAs when
+ *      the output alone would not fill the GPU, and a last kernel adds the splits in split
+ *      order, so repeated calls give identical bits.  The scratch (M * k rounded up to 32 fp16,
+ *      plus splits * N * k fp32) grows on the first call that needs more, which must be outside
+ *      a stream capture; inside one, or when N is not a multiple of 8, a CUDA-core kernel that
+ *      needs no scratch runs instead (same result up to fp32 rounding).  Calls on one handle
+ *      must be ordered (they share the scratch).  No waits.
  * Device pointers, 16-byte aligned (OWQ_ERR_ALIGN); asynchronous on `stream`.
  */
 owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t* dy,

@@ -28,6 +28,7 @@ CASES = [
     ("k0", 96, 384, 3, 128, 0, (4,), None),
     ("many-slices", 1000, 1280, 3, 128, 13, (16,), None),
     ("edges-pair-weak", 130, 1024, 4, 1024, 6, (8,), (0, 1023, 2, 3, 511, 512)),
+    ("token-splits", 256, 512, 3, 128, 40, (1000,), None),
 ]
 
 

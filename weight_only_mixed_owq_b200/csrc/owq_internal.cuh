@@ -43,6 +43,8 @@ struct Layer {
   size_t gemm_xw_bytes;
   void* ig_ws;          // input-gradient workspace: arrival counters per column block (zero
   size_t ig_ws_bytes;   // between calls), then per-slice partial sums (grown on first need)
+  void* wg_ws;          // weak-gradient scratch: gathered weak activations [M][k rounded up to
+  size_t wg_ws_bytes;   // 32] fp16, then per-token-split fp32 partials (grown on first need)
   // tcgen05 GEMM tensor maps, encoded lazily on first use
   bool maps_ready;
   alignas(64) CUtensorMap map_packed;

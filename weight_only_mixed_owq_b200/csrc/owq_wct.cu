@@ -57,6 +57,124 @@ k_weak_grad(const __half* __restrict__ x, const __half* __restrict__ dy,
   }
 }
 
+// ---------------------------------------------------------------- weak-block gradient on the tensor cores
+// dW_weak = dY^T xw as mma.sync m16n8k16 (fp16 x fp16 -> fp32): MMA rows = output rows i, MMA K =
+// tokens, MMA N = weak columns t.  A CTA of 4 warps computes a 64-row x 32-column tile of one
+// token split; tokens stream 32 at a time through a 4-stage cp.async ring holding the dY tile
+// [32 tokens][64 rows] (rows contiguous, as dY stores them) and the gathered activations
+// [32 tokens][32 columns].  Both operands reach their fragments through ldmatrix.trans, so dY
+// is never transposed in memory.  Rows are padded by 16 bytes against bank conflicts.  Each split
+// writes its fp32 tile (to dW directly when there is one split); the splits are then added in
+// split order, so repeated calls give the same bits.
+constexpr int kWmRows = 64, kWmCols = 32, kWmTok = 32, kWmThreads = 128, kWmStages = 4;
+constexpr int kWmDyLd = kWmRows + 8, kWmXLd = kWmCols + 8;   // padded row strides (halves)
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  const int n = valid ? 16 : 0;   // 0: the 16 bytes are filled with zeros
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(d), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+               "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// xw[m][t] = x[m][idx[t]] for t < k, 0 for k <= t < kp
+__global__ void k_wg_gather(const __half* __restrict__ x, int M, int K, const int32_t* __restrict__ idx, int k,
+                            int kp, __half* __restrict__ xw) {
+  const size_t n = (size_t)M * kp;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t m = e / kp;
+    const int t = (int)(e % kp);
+    xw[e] = t < k ? x[m * K + idx[t]] : __float2half_rn(0.f);
+  }
+}
+
+// grid (N / 64, kp / 32, token splits); out = dW (one split) or the split's partial [N][k]
+__global__ void __launch_bounds__(kWmThreads)
+k_weak_grad_mma(const __half* __restrict__ dy, const __half* __restrict__ xw, float* __restrict__ out, int N,
+                int k, int kp, int M, int per) {
+  __shared__ __align__(128) __half s_dy[kWmStages][kWmTok][kWmDyLd];
+  __shared__ __align__(128) __half s_x[kWmStages][kWmTok][kWmXLd];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i0 = blockIdx.x * kWmRows, t0 = blockIdx.y * kWmCols;
+  const int m_lo = blockIdx.z * per, m_hi = min(M, m_lo + per);
+  const int nchunk = (m_hi - m_lo + kWmTok - 1) / kWmTok;
+  auto load = [&](int c, int st) {   // chunk c of this split into stage st
+    const int mb = m_lo + c * kWmTok;
+    #pragma unroll
+    for (int u = 0; u < 2; ++u) {    // dY: 32 tokens x 8 pieces of 8 rows
+      const int e = tid + u * kWmThreads, m = e >> 3, pc = e & 7;
+      const int mm = mb + m, row = i0 + pc * 8;
+      const bool ok = mm < m_hi && row < N;
+      cp_async16(&s_dy[st][m][pc * 8], dy + (ok ? (size_t)mm * N + row : 0), ok);
+    }
+    {                                // xw: 32 tokens x 4 pieces of 8 columns
+      const int m = tid >> 2, pc = tid & 3, mm = mb + m;
+      const bool ok = mm < m_hi;
+      cp_async16(&s_x[st][m][pc * 8], xw + (ok ? (size_t)mm * kp + t0 + pc * 8 : 0), ok);
+    }
+  };
+  float d[4][4];
+  #pragma unroll
+  for (int n = 0; n < 4; ++n)
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) d[n][i] = 0.f;
+  #pragma unroll
+  for (int st = 0; st < kWmStages - 1; ++st) {
+    if (st < nchunk) load(st, st);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  const int q = lane >> 3, r8 = lane & 7;   // ldmatrix: matrix q, row r8
+  for (int c = 0; c < nchunk; ++c) {
+    asm volatile("cp.async.wait_group %0;" :: "n"(kWmStages - 2) : "memory");
+    __syncthreads();   // chunk c landed for every thread; the stage refilled below is free
+    if (c + kWmStages - 1 < nchunk) load(c + kWmStages - 1, (c + kWmStages - 1) % kWmStages);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const int st = c % kWmStages;
+    #pragma unroll
+    for (int ks = 0; ks < kWmTok / 16; ++ks) {
+      const int mk = ks * 16;
+      uint32_t a[4];
+      // A = dY^T rows 16 warp + 0..15, tokens mk..mk+15: matrices (m 0-7, i 0-7), (m 0-7, i 8-15),
+      // (m 8-15, i 0-7), (m 8-15, i 8-15), each read transposed
+      ldsm_x4_t(a, &s_dy[st][mk + (q >> 1) * 8 + r8][warp * 16 + (q & 1) * 8]);
+      #pragma unroll
+      for (int nh = 0; nh < 2; ++nh) {
+        uint32_t b[4];   // B = xw, tokens mk..mk+15 x columns 16 nh .. 16 nh + 15 (two n8 tiles)
+        ldsm_x4_t(b, &s_x[st][mk + (q & 1) * 8 + r8][nh * 16 + (q >> 1) * 8]);
+        mma_16816(d[2 * nh], a, b[0], b[1]);
+        mma_16816(d[2 * nh + 1], a, b[2], b[3]);
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  const int g = lane >> 2, c4 = lane & 3;
+  #pragma unroll
+  for (int n = 0; n < 4; ++n)
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = i0 + warp * 16 + g + 8 * (i >> 1), t = t0 + n * 8 + 2 * c4 + (i & 1);
+      if (row < N && t < k) out[((size_t)blockIdx.z * N + row) * k + t] = d[n][i];
+    }
+}
+
+// dW = sum of the splits' partials in split order
+__global__ void k_wg_reduce(const float* __restrict__ part, int splits, size_t n, float* __restrict__ dw) {
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    float v = part[e];
+    for (int z = 1; z < splits; ++z) v += part[(size_t)z * n + e];
+    dw[e] = v;
+  }
+}
+
 // ---------------------------------------------------------------- input gradient
 // Grid: (K / 128 column blocks) x (row slices).  A CTA walks its slice of one column block in
 // stages of 64 rows (four 16-row tiles, whose blocks are contiguous in the tiled storage); each
@@ -311,8 +429,52 @@ cudaError_t launch_ig_tok(const IgArgs& a, int slices, cudaStream_t s) {
 cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, float* dw, int M,
                              cudaStream_t s) {
   if (L.k == 0) return cudaSuccess;
-  const dim3 grid((L.N + kWgRows - 1) / kWgRows, (L.k + kWgCols - 1) / kWgCols);
-  k_weak_grad<<<grid, kWgThreads, 0, s>>>(x, dy, L.idx, dw, L.N, L.K, L.k, M);
+  // tensor-core kernel: needs 16-byte rows of dY (N % 8 == 0) and the gathered activations
+  // (and, with several token splits, the partials) in the handle's scratch, which grows only
+  // outside a stream capture; otherwise the CUDA-core kernel, which needs no scratch
+  const int kp = (L.k + kWmCols - 1) / kWmCols * kWmCols;
+  const int R = (L.N + kWmRows - 1) / kWmRows, C = kp / kWmCols;
+  const int sms = wct_sm_count(L.device);
+  int splits = std::max(1, std::min((2 * sms + R * C - 1) / (R * C), (M + 255) / 256));
+  int per = (M + splits - 1) / splits;
+  per = (per + kWmTok - 1) / kWmTok * kWmTok;
+  splits = (M + per - 1) / per;
+  const size_t xw_bytes = ((size_t)M * kp * sizeof(__half) + 255) / 256 * 256;
+  const size_t need = xw_bytes + (splits > 1 ? (size_t)splits * L.N * L.k * sizeof(float) : 0);
+  Layer& Lm = const_cast<Layer&>(L);
+  bool mma = L.N % 8 == 0;
+  if (mma && need > L.wg_ws_bytes) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+      cudaGetLastError();
+      mma = false;
+    } else {
+      cudaFree(Lm.wg_ws);
+      Lm.wg_ws = nullptr;
+      Lm.wg_ws_bytes = 0;
+      if (cudaMalloc(&Lm.wg_ws, need) != cudaSuccess) {
+        cudaGetLastError();
+        Lm.wg_ws = nullptr;
+        mma = false;
+      } else {
+        Lm.wg_ws_bytes = need;
+      }
+    }
+  }
+  if (!mma) {
+    const dim3 grid((L.N + kWgRows - 1) / kWgRows, (L.k + kWgCols - 1) / kWgCols);
+    k_weak_grad<<<grid, kWgThreads, 0, s>>>(x, dy, L.idx, dw, L.N, L.K, L.k, M);
+    return cudaGetLastError();
+  }
+  __half* xw = reinterpret_cast<__half*>(L.wg_ws);
+  float* part = splits > 1 ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(L.wg_ws) + xw_bytes) : nullptr;
+  const size_t nxw = (size_t)M * kp;
+  k_wg_gather<<<(unsigned)std::min<size_t>((nxw + 255) / 256, 4096), 256, 0, s>>>(x, M, L.K, L.idx, L.k, kp, xw);
+  k_weak_grad_mma<<<dim3(R, C, splits), kWmThreads, 0, s>>>(dy, xw, splits > 1 ? part : dw, L.N, L.k, kp, M, per);
+  if (splits > 1) {
+    const size_t n = (size_t)L.N * L.k;
+    k_wg_reduce<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, s>>>(part, splits, n, dw);
+  }
   return cudaGetLastError();
 }
 
