@@ -133,3 +133,73 @@ def test_a_rank_that_never_joins_ends_set_up_with_an_error(tmp_path):
     o, e = procs[0].communicate(timeout=120)
     assert procs[0].returncode != 0
     assert "no error" not in o
+
+
+def test_row_ranges_cover_whole_tiles():
+    from weight_only_mixed_owq_b200 import shard
+    for N in (1, 15, 16, 17, 100, 4096, 4100, 36864):
+        for world in (1, 2, 3, 4, 8):
+            rs = [shard.row_range(N, world, r) for r in range(world)]
+            assert rs[0][0] == 0 and rs[-1][1] == N
+            for (a, b), (c, d) in zip(rs, rs[1:]):
+                assert b == c and a <= b
+            for lo, hi in rs:
+                if hi < N:     # every shard but the one that ends the layer is whole tiles
+                    assert lo % 16 == 0 and (hi - lo) % 16 == 0
+                else:          # that one, and any empty ones after it, start on a tile boundary
+                    assert lo % 16 == 0 or lo == N
+            tiles = [-(-(hi - lo) // 16) for lo, hi in rs]
+            assert max(tiles) - min(tiles) <= 1
+
+
+SHARD_CHILD = textwrap.dedent(
+    """
+    import os, sys, json
+    import numpy as np
+    sys.path.insert(0, {root!r})
+    import torch, torch.distributed as dist
+    import oracle, owq_synth
+    from weight_only_mixed_owq_b200 import shard
+    import bench
+    rank, world, local = bench.dist_setup()
+    N, K, bits, group, k, M = {N}, 512, 3, 128, 5, 3
+    d = owq_synth.draw_small(N, K, M, 64, seed=55, n_outliers=3)
+    q = oracle.owq_quantize(d["W"], d["X"], bits, group, k)     # same on every rank (seeded)
+    lo, hi = shard.row_range(N, world, rank)
+    part = shard.shard_operands(q, lo, hi)
+    # this rank's product over its rows (the library's kernel on a GPU; the oracle here)
+    W_hat = oracle.dequant(part["codes"], part["scales"], part["zeros"])
+    y_local = torch.from_numpy(oracle.matmul(W_hat, part["w_weak"], part["idx"], d["x"]))
+    y = shard.all_gather_rows(y_local, N, world).numpy()
+    full = oracle.matmul(oracle.dequant(q["codes"], q["scales"], q["zeros"]), q["w_weak"], q["idx"], d["x"])
+    out = {{"rank": rank, "lo": lo, "hi": hi, "equal": bool(np.array_equal(y, full)), "shape": list(y.shape)}}
+    bench.teardown(world)
+    print(json.dumps(out))
+    """
+)
+
+
+@pytest.mark.parametrize("N", [96, 100])
+def test_row_sharded_product_all_gathers_to_the_single_rank_result(tmp_path, N):
+    """Two gloo ranks each own a block of whole 16-row tiles of one layer, compute their rows
+    and all-gather y: the result equals the single-rank product exactly (rows are independent,
+    so nothing is re-associated).  Not measured on GPU hardware: every call there has one GPU."""
+    script = tmp_path / "shard_child.py"
+    script.write_text(SHARD_CHILD.format(root=ROOT, N=N))
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2",
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen([sys.executable, str(script)], env=env,
+                                      stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
+    import json
+    res = []
+    for p in procs:
+        o, e = p.communicate(timeout=180)
+        assert p.returncode == 0, e
+        res.append(json.loads(o.strip().splitlines()[-1]))
+    res.sort(key=lambda d: d["rank"])
+    assert res[0]["lo"] == 0 and res[0]["hi"] == res[1]["lo"] and res[1]["hi"] == N
+    for d in res:
+        assert d["equal"] and d["shape"] == [3, N]
