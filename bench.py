@@ -488,9 +488,10 @@ def decode_sweep(args, wl, Ms, depth, steps, warmup, local):
             "timing": "CUDA graph of the whole step, CUDA events on the launching stream", "per_M": out}
 
 
-def prefill_measure(args, dev):
+def prefill_measure(args, dev, Ms=None, reps=10):
     """TFLOP/s of owq_gemm on the LLaMA-13B-shaped prefill layers (13824x5120, 5120x13824,
-    3-bit, g = 128, k = 40 / 108) for the token counts of that workload."""
+    3-bit, g = 128, k = 40 / 108) for the token counts of that workload (or `Ms`), median of
+    `reps` single launches with L2 flushed before each."""
     import torch
 
     import weight_only_mixed_owq_b200 as owq
@@ -504,7 +505,7 @@ def prefill_measure(args, dev):
         lay, _ = owq.quantize_pack(W, X, L.bits, L.group, L.k)
         layers.append((L, lay, torch.from_numpy(d["x"]).to(dev)))
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    for M in spec.Ms:
+    for M in (Ms or spec.Ms):
         tot_flop, tot_ms = 0.0, 0.0
         for L, lay, x in layers:
             xm = x[:M].contiguous()
@@ -512,7 +513,7 @@ def prefill_measure(args, dev):
             for _ in range(3):
                 lay.gemm(xm, y)
             times = []
-            for _ in range(10):
+            for _ in range(reps):
                 flush.zero_()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
@@ -530,7 +531,7 @@ def prefill_measure(args, dev):
         lay.close()
     return {"layers": "13824x5120 + 5120x13824, 3-bit g128, k=40/108", "per_M": out,
             "peak_tflops": peaks["bf16_tflops"], "peak_kind": kind,
-            "timing": "median of 10 single launches, L2 flushed between launches"}
+            "timing": f"median of {reps} single launches, L2 flushed between launches"}
 
 
 def wct_measure(args, dev):
@@ -681,10 +682,19 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-wct", action="store_true", help="skip the weak column tuning kernels")
     ap.add_argument("--no-sweeps", action="store_true", help="skip the LLaMA-7B and OPT-66B decode lines")
+    ap.add_argument("--prefill-only", default="", help="comma-separated token counts: time only owq_gemm on "
+                    "the LLaMA-13B-shaped layers at those counts (3 launches each) and print that line")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
     rank, world, local = dist_setup()
+    if args.prefill_only:
+        import torch
+        if rank == 0:
+            Ms = [int(v) for v in args.prefill_only.split(",")]
+            print(json.dumps({"prefill": prefill_measure(args, torch.device("cuda", local), Ms, reps=3)}), flush=True)
+        teardown(world)
+        return 0
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
