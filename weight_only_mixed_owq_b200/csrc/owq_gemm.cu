@@ -178,21 +178,26 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
+      // This one thread paces the CTA at small M, so its loop is kept short: the shared-memory
+      // descriptor is linear in its 16-byte-granular start address (shared addresses stay below
+      // 2^18, so the 14-bit field never carries), hence one base descriptor plus per-stage and
+      // per-slice constants; and it waits only for the A stage: the dequantisation threads
+      // arrive there after waiting for the same stage's TMA barrier, so the activation tile
+      // the MMA reads has landed too.
       constexpr uint32_t idesc = idesc_f16_f32(kBM, BN);
+      const uint64_t dbase = desc_sw128_kmajor(smem_u32(smem));
       bool ok = true;
       for (int i = 0; i < nK && ok; ++i) {
         const int s = i % S, u = i / S;
-        ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit) &&
-             mbar_wait(&afull[s], u & 1, p.status, p.wait_limit);
+        ok = mbar_wait(&afull[s], u & 1, p.status, p.wait_limit);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t xa = smem_u32(smem + s * L::kStage);
+        const uint64_t ds = dbase + (uint64_t)((s * L::kStage) >> 4);
         const uint32_t at = tmem + BN + 64 * s;
+        mma_f16_ts(tmem, at, ds, idesc, i != 0);
         #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = desc_sw128_kmajor(xa + (kk >> 2) * BN * 128 + (kk & 3) * 32);
-          mma_f16_ts(tmem, at + 8 * kk, bd, idesc, (i | kk) != 0);
-        }
+        for (int kk = 1; kk < 8; ++kk)
+          mma_f16_ts(tmem, at + 8 * kk, ds + (uint64_t)((((kk >> 2) * BN * 128) + (kk & 3) * 32) >> 4), idesc, 1u);
         mma_commit(&empty[s]);
       }
       mma_commit(accf);
