@@ -538,56 +538,80 @@ def wct_measure(args, dev):
     """Weak column tuning kernels on the OPT-6.7B-shaped layers (3-bit per channel, k = K/128):
     owq_input_grad (dX = dY W_eff from the packed layout; HBM-bound, GB/s of its algorithmic
     bytes: packed + scales/zeros + weak block + idx + dY + dX) and owq_weak_grad
-    (dW_weak = dY^T x[:, idx]; bytes dY + the gathered x columns + fp32 dW_weak)."""
+    (dW_weak = dY^T x[:, idx]; bytes dY + the gathered x columns + fp32 dW_weak).
+
+    Timing: one CUDA graph of R calls over R distinct operand sets (R packed copies of the layer
+    for the input gradient, R (x, dY) pairs for the weak-block gradient) that together hold more
+    than twice the L2, so every call reads its operands from HBM; device time of the replay / R,
+    median of 5 replays after 3."""
     import torch
 
     import weight_only_mixed_owq_b200 as owq
     spec = owq_synth.WORKLOADS[1]
     peaks, kind = measured_peaks()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    l2 = 126 * 2**20
 
-    def timed(fn):
+    def copies(per_call_bytes, cap=64):
+        return int(max(2, min(cap, -(-2 * l2 // max(1, per_call_bytes)))))
+
+    def graph_time(calls):
+        for c in calls:   # grows the handles' scratch outside the capture
+            c()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in calls:
+                c()
         for _ in range(3):
-            fn()
+            g.replay()
+        torch.cuda.synchronize()
         times = []
-        for _ in range(10):
-            flush.zero_()
+        for _ in range(5):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fn()
+            g.replay()
             b.record()
             torch.cuda.synchronize()
             times.append(a.elapsed_time(b))
-        return statistics.median(times) * 1e-3
+        del g
+        return statistics.median(times) * 1e-3 / len(calls)
 
     out = {}
     for li in (0, 4, 5):   # q (4096 x 4096), fc1 (16384 x 4096), fc2 (4096 x 16384)
         L = spec.layers[li]
         d = owq_synth.draw_layer(L, spec, 16, owq_synth.seed_for(1, li))
         W, X = torch.from_numpy(d["W"]).to(dev), torch.from_numpy(d["X"]).to(dev)
-        lay, _ = owq.quantize_pack(W, X, L.bits, L.group, L.k)
+        q = owq.quantize(W, X, L.bits, L.group, L.k)
         del W, X
         wbytes = L.N * L.K * L.bits // 8 + L.N * (L.K // L.group) * 4 + L.N * L.k * 2 + 4 * L.k
+        R = copies(wbytes)
+        lays = [owq.OwqLayer(q["codes"], q["scales"], q["zeros"], q["idx"], q["w_weak"], L.bits, L.group)
+                for _ in range(R)]
         row = {}
         for M in (1, 16):
             dy = torch.randn((M, L.N), device=dev).half()
             dx = torch.empty((M, L.K), dtype=torch.float16, device=dev)
-            t = timed(lambda: lay.input_grad(dy, dx))
+            t = graph_time([lambda lay=lay: lay.input_grad(dy, dx) for lay in lays])
             B = wbytes + 2 * M * L.N + 2 * M * L.K
             row[f"input_grad_M{M}"] = {"us": round(t * 1e6, 2), "GBps": round(B / t / 1e9, 1),
-                                       "frac_hbm": round(B / t / 1e9 / peaks["hbm_gbs"], 4)}
+                                       "frac_hbm": round(B / t / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
+        for lay in lays[1:]:
+            lay.close()
+        lay = lays[0]
         for M in (16, 2048):
-            x = torch.randn((M, L.K), device=dev).half()
-            dy = torch.randn((M, L.N), device=dev).half()
-            dw = torch.empty((L.N, L.k), dtype=torch.float32, device=dev)
-            t = timed(lambda: lay.weak_grad(x, dy, dw))
             B = 2 * M * L.N + 2 * M * L.k + 4 * L.N * L.k
+            Rw = copies(2 * M * (L.N + L.K), cap=16)
+            xs = [torch.randn((M, L.K), device=dev).half() for _ in range(Rw)]
+            dys = [torch.randn((M, L.N), device=dev).half() for _ in range(Rw)]
+            dw = torch.empty((L.N, L.k), dtype=torch.float32, device=dev)
+            t = graph_time([lambda x=x, dy=dy: lay.weak_grad(x, dy, dw) for x, dy in zip(xs, dys)])
             row[f"weak_grad_M{M}"] = {"us": round(t * 1e6, 2), "GBps": round(B / t / 1e9, 1),
-                                      "TFLOPs": round(2.0 * M * L.N * L.k / t / 1e12, 2)}
+                                      "TFLOPs": round(2.0 * M * L.N * L.k / t / 1e12, 2), "copies": Rw}
+            del xs, dys
         out[f"{L.name} {L.N}x{L.K} k={L.k}"] = row
         lay.close()
     return {"layers": out, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_kind": kind,
-            "timing": "median of 10 single launches, L2 flushed between launches"}
+            "timing": "CUDA graph of R calls over R operand sets holding > 2x L2; device time / R"}
 
 
 # ---------------------------------------------------------------------------------- oracle arm

@@ -326,18 +326,20 @@ owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t*
  * owq_input_grad -- weak column tuning: the gradient the frozen layer passes to its input
  * (same pages; earlier layers' weak columns need it), the transposed product
  *   dx[m][j] = sum_i dy[m][i] * W_eff[i][j],
- * W_eff = W_hat = fp16_rn(s * (q - z)) except at the weak columns, which take their fp16
- * values from the weak block.  Read straight from the packed layout (no W_hat in memory),
- * fp32 accumulation, one fp16 rounding of each output.
+ * W_eff = s * (q - z) except at the weak columns, which take their fp16 values from the weak
+ * block.  Read straight from the packed layout (no W_hat in memory) on the tensor cores
+ * (mma.sync m16n8k16): the exact integers q - z times dy * s carried as an fp16 pair (high
+ * part + residual), fp32 accumulation, one fp16 rounding of each output.  Like the decode
+ * product this multiplies the unrounded s (q - z) rather than W_hat = fp16_rn(s (q - z)): each
+ * weight differs by at most half an fp16 spacing; with a single nonzero dy (1.0) per token the
+ * output row is W_eff's row bit for bit.
  * In:  dy fp16 M x N row-major; 1 <= M <= 65536 (one pass over the packed weights per 16
  *      tokens).  Out: dx fp16 M x K row-major (fully overwritten).
- * The rows are split over CTAs; their fp32 partial sums go to a workspace the handle owns
- * (slices x 16 tokens x K x 4 bytes, with at most 2 x SMs / (K / 128) slices so that the
- * grid is one wave: 2.1 MB at K = 4096 on 148 SMs), allocated on the first call that needs it; that first call must not be inside a stream capture (inside one, a
- * handle without the workspace runs one slice per column block: slower, same result).
- * The last CTA of each column block adds the slices in a fixed order: repeated calls give
- * identical bits.  Calls on one handle must be ordered (one stream, or events between
- * streams): they share that workspace.  Device pointers, 16-byte aligned; asynchronous.
+ * The rows are split over up to 8 CTAs per 128-column block, one thread-block cluster; the
+ * CTAs' fp32 sums are added in a fixed order through distributed shared memory, so repeated
+ * calls give identical bits.  No workspace and no allocation: allowed inside a stream capture.
+ * Copy waits are bounded (OWQ_ERR_TIMEOUT through owq_device_status).  Device pointers,
+ * 16-byte aligned; asynchronous on `stream`.
  */
 owq_status_t owq_input_grad(owq_layer_t layer, const uint16_t* dy, uint16_t* dx, int M,
                             owq_stream_t stream);

@@ -29,6 +29,9 @@ CASES = [
     ("many-slices", 1000, 1280, 3, 128, 13, (16,), None),
     ("edges-pair-weak", 130, 1024, 4, 1024, 6, (8,), (0, 1023, 2, 3, 511, 512)),
     ("token-splits", 256, 512, 3, 128, 40, (1000,), None),
+    ("cluster-of-3", 300, 384, 3, 384, 5, (1, 9), None),
+    # 40 weak columns in one block over 512-row slices: too many to stage in shared memory
+    ("weak-heavy-block", 4096, 256, 4, 128, 40, (2, 16), tuple(range(0, 80, 2))),
 ]
 
 
@@ -54,6 +57,24 @@ def _check_weak_grad(got, x, dy, idx, where):
     bound = dy.shape[0] * 2.0 ** -24 * terms + 1e-30
     err = np.abs(got - want)
     assert np.all(err <= bound), f"{where}: weak grad error {float(err.max()):.3g}"
+
+
+def _check_input_grad_bound(got, W_hat, w_weak, idx, dy, where):
+    """Per output: the kernel multiplies dY by the unrounded s (q - z) (dY s carried as an fp16
+    pair to 2^-22), the oracle by W_hat = fp16_rn(s (q - z)); each weight differs by at most half
+    an fp16 spacing, 2^-11 of its magnitude (2^-25 absolute below the normal range).  So
+    |dx - dx64| <= 2^-11 sum_i |dY_i W_eff_ij| + 2^-25 sum_i |dY_i| + half an fp16 spacing of
+    dx64 + 2^-20 sum_i |dY_i W_eff_ij| (fp32 accumulation)."""
+    want = oracle.input_grad(W_hat, w_weak, idx, dy)
+    w_eff = np.abs(W_hat.astype(F64))
+    if len(idx):
+        w_eff[:, idx] = np.abs(w_weak.astype(F64))
+    ady = np.abs(dy.astype(F64))
+    terms = ady @ w_eff
+    bound = ((2.0 ** -11 + 2.0 ** -20) * terms + 2.0 ** -25 * ady.sum(axis=1, keepdims=True)
+             + 0.5 * np.spacing(np.abs(want).astype(np.float16)).astype(F64))
+    err = np.abs(np.asarray(got, dtype=np.float16).astype(F64) - want)
+    assert np.all(err <= bound), f"{where}: input grad error {float((err - bound).max()):.3g} over the bound"
 
 
 def _case(case):
@@ -85,6 +106,7 @@ def test_wct_gradients_match_oracle(case):
         torch.cuda.synchronize()
         check_output(dx.cpu().numpy(), oracle.input_grad(W_hat, ref["w_weak"], ref["idx"], dy),
                      f"{name} input_grad M={M}")
+        _check_input_grad_bound(dx.cpu().numpy(), W_hat, ref["w_weak"], ref["idx"], dy, f"{name} M={M}")
         assert torch.equal(dx.view(torch.int16), dx2.view(torch.int16)), "repeat differs"
         if k:
             _check_weak_grad(dw.cpu().numpy(), x, dy, ref["idx"], f"{name} M={M}")
@@ -110,6 +132,32 @@ def test_wct_gradients_fullsize_opt67b_attention_layer():
         check_output(dx.cpu().numpy(), oracle.input_grad(W_hat, ref["w_weak"], ref["idx"], dy),
                      f"{L.name} input_grad M={M}")
         _check_weak_grad(dw.cpu().numpy(), x, dy, ref["idx"], f"{L.name} M={M}")
+    layer.close()
+
+
+@pytest.mark.parametrize("case", [CASES[1], CASES[2], CASES[5], CASES[7], CASES[8]], ids=lambda c: c[0])
+def test_input_grad_one_hot_rows_are_w_eff(case):
+    """One nonzero dY (1.0) per token: dX's row is row i of W_eff (W_hat with the weak columns'
+    fp16 values) bit for bit, since the kernel's only rounding is then the final fp16 one
+    (-0 weak values give +0: +0 (dense) + (-0) (weak) = +0)."""
+    import weight_only_mixed_owq_b200 as owq
+    name, N, K, bits, group, k, Ms, forced = case
+    d, ref = _case(case)
+    w = oracle.dequant(ref["codes"], ref["scales"], ref["zeros"]).copy()
+    if k:
+        assert np.all(w[:, ref["idx"]] == 0)
+        w[:, ref["idx"]] = ref["w_weak"]
+    want = w.view(np.uint16).copy()
+    want[want == 0x8000] = 0
+    layer = _layer(owq, ref, bits, group)
+    rows = np.unique(np.concatenate([[0, N - 1, N // 2], np.arange(0, N, max(1, N // 29))]))
+    for r0 in range(0, len(rows), 16):
+        rr = rows[r0:r0 + 16]
+        dy = np.zeros((len(rr), N), dtype=np.float16)
+        dy[np.arange(len(rr)), rr] = 1.0
+        got = layer.input_grad(_gpu(dy)).cpu().numpy().view(np.uint16)
+        bad = np.argwhere(got != want[rr])
+        assert bad.size == 0, f"{name}: row {rr[bad[0][0]]} column {bad[0][1]}: {got[tuple(bad[0])]:#06x} != {want[rr][tuple(bad[0])]:#06x}"
     layer.close()
 
 

@@ -88,7 +88,6 @@ void release(Layer* L) {
   cudaFree(L->xfrag);
   cudaFree(L->gemm_ws);
   cudaFree(L->gemm_xw);
-  cudaFree(L->ig_ws);
   cudaFree(L->wg_ws);
   cudaFree(L->part);
   L->magic = 0;

@@ -41,8 +41,6 @@ struct Layer {
   size_t gemm_ws_bytes;
   __half* gemm_xw;      // prefill weak activations [M][k_ld] (grown on first need, outside capture)
   size_t gemm_xw_bytes;
-  void* ig_ws;          // input-gradient workspace: arrival counters per column block (zero
-  size_t ig_ws_bytes;   // between calls), then per-slice partial sums (grown on first need)
   void* wg_ws;          // weak-gradient scratch: gathered weak activations [M][k rounded up to
   size_t wg_ws_bytes;   // 32] fp16, then per-token-split fp32 partials (grown on first need)
   // tcgen05 GEMM tensor maps, encoded lazily on first use

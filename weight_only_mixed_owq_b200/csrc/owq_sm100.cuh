@@ -1,5 +1,6 @@
-// Thin inline-PTX wrappers for the sm_100a features the prefill kernel uses: mbarriers,
-// TMA tile loads (no cluster multicast anywhere in this library), tcgen05 MMA / TMEM.
+// Thin inline-PTX wrappers for the sm_100a features the library's kernels use: mbarriers, bulk
+// and TMA tile loads (no cluster multicast anywhere in this library), thread-block clusters and
+// distributed shared memory, tcgen05 MMA / TMEM.
 #pragma once
 #include <cstdint>
 
@@ -76,6 +77,25 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- thread-block clusters ----
+// Every thread of every CTA of the cluster must call this (a hardware barrier, not a spin).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// fp32 load from the shared memory of CTA `rank` of this cluster, at the offset `p` has here.
+__device__ __forceinline__ float ld_dsmem_f32(const void* p, uint32_t rank) {
+  uint32_t ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
 }
 
 // ---- tcgen05 ----

@@ -9,9 +9,11 @@
 // in place of their zero-filled codes.  Both accumulate in fp32.
 #include "owq_internal.cuh"
 #include "owq_format.cuh"
+#include "owq_sm100.cuh"
 
 namespace owq {
 namespace {
+using namespace sm100;
 
 // ---------------------------------------------------------------- weak-block gradient
 // A CTA computes a 32-row x 32-weak-column tile of dW_weak; its 256 threads own one weak column
@@ -176,221 +178,417 @@ __global__ void k_wg_reduce(const float* __restrict__ part, int splits, size_t n
 }
 
 // ---------------------------------------------------------------- input gradient
-// Grid: (K / 128 column blocks) x (row slices).  A CTA walks its slice of one column block in
-// stages of 64 rows (four 16-row tiles, whose blocks are contiguous in the tiled storage); each
-// of its 256 threads owns one code pair (two adjacent columns) and 16 rows of every stage.
-//
-// Dequantisation in fp16x2: the pair's two codes sit at the same bit offset of the two halves
-// of one word, so one shift-and-mask gives (q_even, q_odd) as 16-bit integers; OR-ing 0x6400
-// (1024.0) into each half makes the exact halves 1024 + q, subtracting (1024 + z) leaves q - z
-// exactly, and one fp16x2 multiply by the scale rounds s (q - z) once, i.e. fp16_rn(s (q - z)).
-//
-// The four row quarters of a pair are summed in shared memory in a fixed order.  With more
-// than one slice, each CTA stores its fp32 partial sums to the layer's workspace; the last CTA
-// of a column block to finish (a counter per block) adds the slices in slice order and writes
-// the fp16 result, so repeated calls give identical bits.  Nothing waits on another CTA.
-constexpr int kIgThreads = 256, kIgStageRows = 64, kIgMaxTok = 16;
+constexpr int kIgThreads = 256, kIgMaxTok = 16, kIgStages = 4, kIgMaxSlices = 8;
+constexpr int kIgWeakBytes = 32 * 1024;   // shared memory for a column block's weak values
 
 struct IgArgs {
   const uint32_t* packed;
-  const __half* scales;
-  const __half* zeros;
-  const __half* w_weak;
-  const int32_t* idx;
-  const __half* dy;   // M x N (this pass's first token)
-  __half* dx;         // M x K
-  float* part;        // [slices][16 tokens][K] (slices > 1)
-  unsigned int* count;  // [K / 128], zero between calls
-  int N, K, G, group, k, k_ld, M, stages_per_slice;
+  const __half2* sz_t;    // (scale, zero) pairs, tile-major [N/16][G][16]
+  const __half* w_weak;   // N x k_ld
+  const int32_t* idx;     // k, strictly increasing
+  const __half* dy;       // M x N (this pass's first token)
+  __half* dx;             // M x K
+  int* status;            // device status word (bounded waits)
+  long long wait_limit;
+  int N, K, G, group, k, k_ld, M, tiles_per_slice;
 };
 
-template <int BITS>
-__device__ __forceinline__ uint32_t pair_codes(const uint32_t* w, int word, int shift, bool spread) {
-  if (BITS == 3 && spread)   // bit e of the even / odd code is bit 15 / 31 of word e
-    return ((w[word] >> 15) & 0x00010001u) | ((w[word + 1] >> 14) & 0x00020002u) |
-           ((w[word + 2] >> 13) & 0x00040004u);
-  return (w[word] >> shift) & (((1u << BITS) - 1u) * 0x00010001u);
+// ---------------------------------------------------------------- input gradient on the tensor cores
+// dX^T = W_eff^T dY^T per (16-row tile, 128-code block) unit as mma.sync m16n8k16: MMA rows =
+// 16 input columns j, MMA K = the tile's 16 rows i, MMA N = 8 tokens.  Grid: (K / 128 column
+// blocks) x (row slices); a CTA of 8 warps covers one column block and one slice of the row
+// tiles, warp w taking tiles w, w + 8, ... of the slice.  Each warp streams its tiles' packed
+// block (one contiguous 16 x 16 * bits byte run of the tiled storage) and the tile's (scale,
+// zero) pairs through a private 4-stage ring of bulk copies; the block's weak values over the
+// slice's rows are staged in shared memory once (their slots are consecutive, the index list
+// being increasing).
+//
+// The scale varies along the contraction here (row i), so it goes with dY: the A operand is the
+// exact integer q - z, the B operand dY s split into an fp16 high part and the fp16 residual
+// (dY s - hi, exact in fp16 unless it falls below the normal range), both multiplied by the same
+// A; every product is exact and the sums are fp32.  This evaluates dY (s (q - z)) with the unrounded dequantised weights, like the
+// decode product, instead of fp16_rn(s (q - z)): each weight differs by at most half an fp16
+// spacing; with one nonzero dY per token the output is fp16_rn(s (q - z)) exactly.
+//
+// The transposed operand is built straight from the staged block.  Lane (g, t) holds, for MMA
+// row g (column 16 s + g of slice s) and g + 8, the rows 2t, 2t + 1 and 2t + 8, 2t + 9; all its
+// codes lie in chunk g / 2 of those four rows (pairs 2 s and 2 s + 1, the even code for even g,
+// the odd one for odd g).  One byte permute puts the same half of two rows' words side by side
+// (shifted down a byte where the code sits at bit 8 or above), an AND with OR leaves
+// 1024 + q 2^o in each fp16 half and one fp16x2 fma with the row pair's constants leaves q - z
+// exactly.  The weak columns' codes give exactly 0 (they hold the integral zero point); their
+// fp16 values enter through one more product with the unscaled dY per 16-column slice that
+// holds any.  The warps' partial sums meet in shared memory in a fixed tree.  The slices of a
+// column block form one thread-block cluster: each CTA then adds, for its share of the block's
+// outputs, the CTAs' sums in slice order through distributed shared memory, so repeated calls
+// give identical bits and no workspace is needed.  Every ring wait is bounded (on expiry: the
+// status word, no further products, the copies in flight waited for).
+__device__ __forceinline__ uint32_t ig_h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ __half2 u32_h2(uint32_t u) { return *reinterpret_cast<const __half2*>(&u); }
+__device__ __forceinline__ uint32_t h2_u32(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+__device__ __forceinline__ uint32_t ig_h2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-template <int BITS, int TOK>
-__global__ void __launch_bounds__(kIgThreads)
-k_input_grad(const IgArgs a) {
-  constexpr int kStageWords4 = 4 * 16 * BITS;   // uint4 per stage: 4 tiles x 16 blocks x BITS
-  __shared__ uint4 s_words[2][kStageWords4];
-  __shared__ __half2 s_scale[2][kIgStageRows];
-  __shared__ __half2 s_zb[2][kIgStageRows];       // (1024 + z, 1024 + z)
-  __shared__ __align__(16) float s_dy[2][kIgStageRows][TOK];
-  __shared__ float2 s_red[3][TOK][64];
-  __shared__ int s_last;
-  __shared__ int s_slot[kBlockCodes];
+// Bit offset of pair j's codes in each half after extraction (codes at bit 8 or above are
+// moved down a byte by the permute), and the classes of those offsets.
+template <int BITS>
+__host__ __device__ constexpr int ig_off(int j) {
+  if (BITS == 3 && j == 11) return 6;   // the spread pair, rebuilt at offset 6
+  const int o = BITS == 3 ? slot3(j).off : slot4(j).off;
+  return o >= 8 ? o - 8 : o;
+}
+template <int BITS>
+__host__ __device__ constexpr int ig_ncls() { return BITS == 3 ? 5 : 2; }
+template <int BITS>
+__host__ __device__ constexpr int ig_cls_off(int c) {   // 3-bit: 0, 3, 6, 1, 4; 4-bit: 0, 4
+  return BITS == 3 ? (c == 0 ? 0 : c == 1 ? 3 : c == 2 ? 6 : c == 3 ? 1 : 4) : 4 * c;
+}
+template <int BITS>
+__host__ __device__ constexpr int ig_cls(int off) {
+  return BITS == 3 ? (off == 0 ? 0 : off == 3 ? 1 : off == 6 ? 2 : off == 1 ? 3 : 4) : off / 4;
+}
 
-  const int tid = threadIdx.x, p = tid & 63, h = tid >> 6;
+// Codes of pair j (the half `sel` picks) of rows a (low fp16 half) and b (high half), as
+// 1024 + q 2^o in each half (the bits 0x6400 with the code at offset o = ig_off(j)).
+template <int BITS>
+__device__ __forceinline__ uint32_t ig_tpair(const uint32_t* wa, const uint32_t* wb, int j, uint32_t sel,
+                                             uint32_t sel8) {
+  constexpr uint32_t kMagic = 0x64006400u;
+  if constexpr (BITS == 3) {
+    if (j == 11) {   // bit e of each code at bit 15 of word e: to bits 6, 7, 8
+      const uint32_t t0 = __byte_perm(wa[0], wb[0], sel), t1 = __byte_perm(wa[1], wb[1], sel);
+      const uint32_t t2 = __byte_perm(wa[2], wb[2], sel);
+      return ((t0 >> 9) & 0x00400040u) | ((t1 >> 8) & 0x00800080u) | ((t2 >> 7) & 0x01000100u) | kMagic;
+    }
+    const Slot sl = slot3(j);
+    const uint32_t v = __byte_perm(wa[sl.word], wb[sl.word], sl.off >= 8 ? sel8 : sel);
+    return (v & (0x00070007u << ig_off<3>(j))) | kMagic;
+  } else {
+    const Slot sl = slot4(j);
+    const uint32_t v = __byte_perm(wa[sl.word], wb[sl.word], sl.off >= 8 ? sel8 : sel);
+    return (v & (0x000F000Fu << ig_off<4>(j))) | kMagic;
+  }
+}
+
+template <int BITS>
+__host__ __device__ constexpr int ig_stage_bytes() { return 256 * BITS + 64; }   // one tile's block + its 16 (s, z) pairs
+template <int BITS>
+__host__ __device__ constexpr int ig_smem_bytes() {   // the warps' rings, their barriers, the staged weak values
+  return (kIgThreads / 32) * kIgStages * (ig_stage_bytes<BITS>() + 8) + kIgWeakBytes;
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(kIgThreads, 2)
+k_input_grad_mma(const __grid_constant__ IgArgs a) {
+  constexpr int NCL = ig_ncls<BITS>();
+  constexpr int kBlkB = 16 * BITS;                 // one row's block, bytes
+  constexpr int kTileBlkB = 16 * kBlkB;            // one tile's block, bytes
+  constexpr int kStage = ig_stage_bytes<BITS>();
+  constexpr int kTok = 8 * NT;
+  extern __shared__ __align__(128) unsigned char ig_smem[];
+  __shared__ float s_red[4][kTok][kBlockCodes];
+  __shared__ int s_slot[kBlockCodes];              // weak slot of column c of the block, or -1
+  __shared__ int s_t0, s_nweak, s_wsl;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tg = lane & 3;
   const int b = blockIdx.x, slice = blockIdx.y, S = gridDim.y;
   const int Kb = a.K / kBlockCodes, tiles = (a.N + 15) / 16;
-  const int g = (b * kBlockCodes) / a.group;
-  const int col = b * kBlockCodes + 2 * p;
+  const int grp = (b * kBlockCodes) / a.group;   // the block's group (per-channel: 0)
+  unsigned char* ring = ig_smem + warp * kIgStages * kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ig_smem + (kIgThreads / 32) * kIgStages * kStage) + warp * kIgStages;
+  __half* s_wv = reinterpret_cast<__half*>(ig_smem + (kIgThreads / 32) * kIgStages * (kStage + 8));
 
-  // the pair's slot in a block: chunk p % 4, pair p / 4 of the chunk
-  const int chunk = p & 3, jj = p >> 2;
-  const Slot sl = BITS == 3 ? slot3(jj) : slot4(jj);
-  const bool spread = sl.word < 0;
-  const int word = chunk * BITS + (spread ? 0 : sl.word);
-  const int shift = spread ? 0 : sl.off;
+  const int t_lo = slice * a.tiles_per_slice, t_hi = min(tiles, t_lo + a.tiles_per_slice);
+  const int rows = max(0, t_hi - t_lo) * 16;
+  const int nmine = t_hi > t_lo + warp ? (t_hi - t_lo - warp + 7) / 8 : 0;   // this warp's tiles
+  int issued = 0;
+  // lane 0: the warp's next tile (block b of 16 rows, then its (scale, zero) pairs) into its stage
+  const unsigned char* src_blk = reinterpret_cast<const unsigned char*>(a.packed) + ((size_t)(t_lo + warp) * Kb + b) * kTileBlkB;
+  const __half2* src_sz = a.sz_t + ((size_t)(t_lo + warp) * a.G + grp) * 16;
+  auto issue = [&]() {
+    const int st = issued % kIgStages;
+    mbar_arrive_expect_tx(&bars[st], (uint32_t)kStage);
+    bulk_load(ring + st * kStage, src_blk, (uint32_t)kTileBlkB, &bars[st]);
+    bulk_load(ring + st * kStage + kTileBlkB, src_sz, 64u, &bars[st]);
+    src_blk += (size_t)8 * Kb * kTileBlkB;
+    src_sz += (size_t)8 * a.G * 16;
+    ++issued;
+  };
+  if (lane == 0) {
+    for (int st = 0; st < kIgStages; ++st) mbar_init(&bars[st], 1);
+    fence_mbar_init();
+    while (issued < min(nmine, kIgStages)) issue();
+  }
 
-  // weak slots of the block's columns: one parallel pass over idx into a shared table
   if (tid < kBlockCodes) s_slot[tid] = -1;
+  if (tid == 0) { s_t0 = 0x7fffffff; s_nweak = 0; s_wsl = 0; }
   __syncthreads();
   for (int t = tid; t < a.k; t += kIgThreads) {
     const int c = a.idx[t] - b * kBlockCodes;
-    if (c >= 0 && c < kBlockCodes) s_slot[c] = t;
+    if (c >= 0 && c < kBlockCodes) {
+      s_slot[c] = t;
+      atomicMin(&s_t0, t);
+      atomicAdd(&s_nweak, 1);
+      atomicOr(&s_wsl, 1 << (c >> 4));
+    }
   }
   __syncthreads();
-  const int tw0 = s_slot[2 * p], tw1 = s_slot[2 * p + 1];
-  const bool weak = tw0 >= 0 || tw1 >= 0;
-
-  const int nstages = (tiles + 3) / 4;
-  const int st0 = slice * a.stages_per_slice;
-  const int st1 = min(nstages, st0 + a.stages_per_slice);
-
-  // staged loads of one stage into registers
-  uint4 r_words = make_uint4(0, 0, 0, 0);
-  __half r_s = __float2half(0.f), r_z = __float2half(0.f);
-  __half r_dy[(TOK * kIgStageRows + kIgThreads - 1) / kIgThreads];
-  // weak values of this thread's rows, one stage ahead (threads with a weak column only)
-  __half2 wk_next[16], wk_cur[16];
-  auto load = [&](int st) {
-    if (weak) {
+  const int nweak = s_nweak, t0 = s_t0;
+  // the block's weak values over the slice's rows: s_wv[(slot - t0) * rows + r] (rows >= N: 0),
+  // staged for up to 8 weak columns, 4 rows x 8 columns of loads in flight per thread
+  const int wsl = s_wsl;   // slices (16 columns) of the block holding weak columns
+  const bool staged = nweak > 0 && nweak <= 8 && nweak * rows * (int)sizeof(__half) <= kIgWeakBytes;
+  if (staged) {
+    for (int r0 = tid; r0 < rows; r0 += 4 * kIgThreads) {
+      uint16_t v[4][8];
       #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        const int row = st * kIgStageRows + h * 16 + rr;
-        const __half* wr = a.w_weak + (size_t)row * a.k_ld;
-        wk_next[rr] = __halves2half2(tw0 >= 0 && row < a.N ? wr[tw0] : __float2half(0.f),
-                                     tw1 >= 0 && row < a.N ? wr[tw1] : __float2half(0.f));
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * kIgThreads, row = t_lo * 16 + r;
+        const __half* src = a.w_weak + (size_t)row * a.k_ld + t0;
+        #pragma unroll
+        for (int wi = 0; wi < 8; ++wi)
+          v[u][wi] = wi < nweak && r < rows && row < a.N ? __half_as_ushort(src[wi]) : (uint16_t)0;
+      }
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * kIgThreads;
+        #pragma unroll
+        for (int wi = 0; wi < 8; ++wi)
+          if (wi < nweak && r < rows) s_wv[wi * rows + r] = __ushort_as_half(v[u][wi]);
       }
     }
-    if (tid < kStageWords4) {
-      const int tile = st * 4 + tid / (16 * BITS);
-      r_words = make_uint4(0, 0, 0, 0);
-      if (tile < tiles)
-        r_words = reinterpret_cast<const uint4*>(a.packed + ((size_t)tile * Kb + b) * 16 * 4 * BITS)[tid % (16 * BITS)];
-    }
-    if (tid < kIgStageRows) {
-      const int row = st * kIgStageRows + tid;
-      r_s = row < a.N ? a.scales[(size_t)row * a.G + g] : __float2half(0.f);
-      r_z = row < a.N ? a.zeros[(size_t)row * a.G + g] : __float2half(0.f);
-    }
-    #pragma unroll
-    for (int u = 0; u < (int)(sizeof(r_dy) / sizeof(r_dy[0])); ++u) {
-      const int e = tid + u * kIgThreads, m = e / kIgStageRows, rr = e % kIgStageRows;
-      const int row = st * kIgStageRows + rr;
-      r_dy[u] = (e < TOK * kIgStageRows && m < a.M && row < a.N) ? a.dy[(size_t)m * a.N + row] : __float2half(0.f);
-    }
-  };
-  auto store = [&](int buf) {
-    if (weak) {
-      #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) wk_cur[rr] = wk_next[rr];
-    }
-    if (tid < kStageWords4) s_words[buf][tid] = r_words;
-    if (tid < kIgStageRows) {
-      s_scale[buf][tid] = __halves2half2(r_s, r_s);
-      const __half zb = __hadd(r_z, __float2half(1024.f));   // exact: z is a small integer
-      s_zb[buf][tid] = __halves2half2(zb, zb);
-    }
-    #pragma unroll
-    for (int u = 0; u < (int)(sizeof(r_dy) / sizeof(r_dy[0])); ++u) {
-      const int e = tid + u * kIgThreads;
-      if (e < TOK * kIgStageRows) s_dy[buf][e % kIgStageRows][e / kIgStageRows] = __half2float(r_dy[u]);
-    }
-  };
-
-  float2 acc[TOK];
-  #pragma unroll
-  for (int m = 0; m < TOK; ++m) acc[m] = make_float2(0.f, 0.f);
-
-  if (st0 < st1) {
-    load(st0);
-    store(0);
-  }
-  __syncthreads();
-  for (int st = st0; st < st1; ++st) {
-    const int buf = (st - st0) & 1;
-    if (st + 1 < st1) load(st + 1);
-    const uint32_t* sw = reinterpret_cast<const uint32_t*>(s_words[buf]);
-    #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int r = h * 16 + rr;               // row within the stage
-      // row r of the stage is row r % 16 of tile r / 16: block (r / 16) * 16 + r % 16 = r
-      const uint32_t v = pair_codes<BITS>(sw + r * 4 * BITS, word, shift, spread) | 0x64006400u;
-      const __half2 qz = __hsub2(*reinterpret_cast<const __half2*>(&v), s_zb[buf][r]);
-      float2 wv = __half22float2(__hmul2(s_scale[buf][r], qz));
-      if (weak) {
-        const float2 wk = __half22float2(wk_cur[rr]);
-        if (tw0 >= 0) wv.x = wk.x;
-        if (tw1 >= 0) wv.y = wk.y;
-      }
-      const float* d = s_dy[buf][r];
-      #pragma unroll
-      for (int m = 0; m < TOK; ++m) {
-        acc[m].x = fmaf(wv.x, d[m], acc[m].x);
-        acc[m].y = fmaf(wv.y, d[m], acc[m].y);
-      }
-    }
-    if (st + 1 < st1) store(buf ^ 1);
     __syncthreads();
   }
-
-  // the four row quarters, summed in the order 0, 1, 2, 3
-  if (h > 0) {
+  // the lane's weak columns: bit 2 s for column 16 s + g, bit 2 s + 1 for column 16 s + g + 8
+  uint32_t wmask = 0;
+  if (nweak > 0) {
     #pragma unroll
-    for (int m = 0; m < TOK; ++m) s_red[h - 1][m][p] = acc[m];
+    for (int sl = 0; sl < 8; ++sl) {
+      wmask |= (s_slot[16 * sl + g] >= 0 ? 1u : 0u) << (2 * sl);
+      wmask |= (s_slot[16 * sl + g + 8] >= 0 ? 2u : 0u) << (2 * sl);
+    }
   }
-  __syncthreads();
-  if (h == 0) {
+
+  // byte permutes taking half g % 2 of two words (sel), the same one byte lower (sel8)
+  const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u, sel8 = (g & 1) ? 0x7733u : 0x5511u;
+
+  float D[8][NT][4];
+  #pragma unroll
+  for (int sl = 0; sl < 8; ++sl)
     #pragma unroll
-    for (int m = 0; m < TOK; ++m) {
+    for (int nt = 0; nt < NT; ++nt)
       #pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        acc[m].x += s_red[q][m][p].x;
-        acc[m].y += s_red[q][m][p].y;
+      for (int i = 0; i < 4; ++i) D[sl][nt][i] = 0.f;
+
+  // dY fragments of a tile (rows 16 tile + 2 tg (+1, +8, +9), token 8 nt + g), loaded two tiles
+  // ahead (one with two token blocks): two 32-bit loads per token block where the tile is whole and N even, else by halves
+  const bool n_even = (a.N & 1) == 0;
+  auto load_dy = [&](int tile, uint32_t (&yy)[NT][2]) {
+    const int i0 = tile * 16 + 2 * tg;
+    const bool whole = n_even && tile * 16 + 16 <= a.N;
+    #pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int m = 8 * nt + g;
+      yy[nt][0] = yy[nt][1] = 0u;
+      if (m >= a.M) continue;
+      const __half* p = a.dy + (size_t)m * a.N + i0;
+      if (whole) {
+        yy[nt][0] = *reinterpret_cast<const uint32_t*>(p);
+        yy[nt][1] = *reinterpret_cast<const uint32_t*>(p + 8);
+      } else {
+        uint16_t v[4];
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int du = (u & 1) + 8 * (u >> 1);
+          v[u] = i0 + du < a.N ? __half_as_ushort(p[du]) : (uint16_t)0;
+        }
+        yy[nt][0] = (uint32_t)v[0] | ((uint32_t)v[1] << 16);
+        yy[nt][1] = (uint32_t)v[2] | ((uint32_t)v[3] << 16);
       }
     }
-    if (S == 1) {
+  };
+  constexpr int PD = NT == 1 ? 2 : 1;   // prefetch distance, in the warp's tiles
+  uint32_t yq[PD + 1][NT][2];           // dY of the warp's tiles j .. j + PD
+  #pragma unroll
+  for (int p = 0; p < PD; ++p)
+    if (p < nmine) load_dy(t_lo + warp + 8 * p, yq[p]);
+  bool ok = true;
+  int failed_at = -1;
+  for (int j = 0; j < nmine; ++j) {
+    const int tile = t_lo + warp + 8 * j, st = j % kIgStages;
+    if (j + PD < nmine) load_dy(tile + 8 * PD, yq[PD]);
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars[st], (uint32_t)((j / kIgStages) & 1), a.status, a.wait_limit));
+      if (!ok) failed_at = j;
+    }
+    if (ok) {
+      const unsigned char* stg = ring + st * kStage;
+      // chunk g / 2 of rows 2 tg, 2 tg + 1, 2 tg + 8, 2 tg + 9, and their (scale, zero) pairs
+      uint32_t w0[BITS], w1[BITS], w2[BITS], w3[BITS];
       #pragma unroll
-      for (int m = 0; m < TOK; ++m)
-        if (m < a.M)
-          *reinterpret_cast<__half2*>(a.dx + (size_t)m * a.K + col) = __floats2half2_rn(acc[m].x, acc[m].y);
-    } else {
+      for (int jj = 0; jj < BITS; ++jj) {
+        const unsigned char* c0 = stg + (g >> 1) * 4 * BITS + 4 * jj;
+        w0[jj] = *reinterpret_cast<const uint32_t*>(c0 + (2 * tg) * kBlkB);
+        w1[jj] = *reinterpret_cast<const uint32_t*>(c0 + (2 * tg + 1) * kBlkB);
+        w2[jj] = *reinterpret_cast<const uint32_t*>(c0 + (2 * tg + 8) * kBlkB);
+        w3[jj] = *reinterpret_cast<const uint32_t*>(c0 + (2 * tg + 9) * kBlkB);
+      }
+      const uint32_t* szs = reinterpret_cast<const uint32_t*>(stg + kTileBlkB);
+      const uint32_t sz0 = szs[2 * tg], sz1 = szs[2 * tg + 1], sz2 = szs[2 * tg + 8], sz3 = szs[2 * tg + 9];
+      __syncwarp();   // every lane has read the stage
+      if (lane == 0 && issued < nmine) {
+        fence_proxy_async_smem();
+        issue();      // into the stage just read
+      }
+      // row pairs (2 tg, 2 tg + 1) and (2 tg + 8, 2 tg + 9): scales, and -(1024 2^-o + z) per class
+      const uint32_t S2[2] = {__byte_perm(sz0, sz1, 0x5410), __byte_perm(sz2, sz3, 0x5410)};
+      const uint32_t Z2[2] = {__byte_perm(sz0, sz1, 0x7632), __byte_perm(sz2, sz3, 0x7632)};
+      uint32_t NZ[2][NCL];
       #pragma unroll
-      for (int m = 0; m < TOK; ++m)
-        *reinterpret_cast<float2*>(a.part + ((size_t)slice * kIgMaxTok + m) * a.K + col) = acc[m];
+      for (int c = 0; c < NCL; ++c) {
+        const uint32_t neg_o = 0x8000u | ((uint32_t)(25 - ig_cls_off<BITS>(c)) << 10);   // -2^(10 - o)
+        NZ[0][c] = ig_h2_sub(neg_o | (neg_o << 16), Z2[0]);
+        NZ[1][c] = ig_h2_sub(neg_o | (neg_o << 16), Z2[1]);
+      }
+      // B operands: dY s as fp16 hi + lo, rows (2 tg, 2 tg + 1) and (2 tg + 8, 2 tg + 9)
+      uint32_t bh[NT][2], bl[NT][2];
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const __half2 y = u32_h2(yq[0][nt][h]), sc2 = u32_h2(S2[h]);
+          const __half2 hi = __hmul2(y, sc2);
+          bh[nt][h] = h2_u32(hi);
+          bl[nt][h] = h2_u32(__hfma2(y, sc2, __hneg2(hi)));
+        }
+      const int ra = (tile - t_lo) * 16 + 2 * tg;   // row 2 tg of the tile, within the slice
+      #pragma unroll
+      for (int sl = 0; sl < 8; ++sl) {
+        uint32_t at[4];
+        #pragma unroll
+        for (int r = 0; r < 4; ++r) {   // r: (rows 2 tg.. | 2 tg + 8..) x (column g | g + 8)
+          const int jp = 2 * sl + (r & 1), rp = r >> 1;
+          const int cls = ig_cls<BITS>(ig_off<BITS>(jp));
+          const uint32_t sc = (uint32_t)(15 - ig_cls_off<BITS>(cls)) << 10;   // 2^-o
+          const uint32_t v = rp == 0 ? ig_tpair<BITS>(w0, w1, jp, sel, sel8) : ig_tpair<BITS>(w2, w3, jp, sel, sel8);
+          at[r] = ig_h2_fma(v, sc | (sc << 16), NZ[rp][cls]);   // q - z, exact
+        }
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816(D[sl][nt], at, bh[nt][0], bh[nt][1]);
+          mma_16816(D[sl][nt], at, bl[nt][0], bl[nt][1]);
+        }
+      }
+      // the weak columns (their codes gave exactly 0): one more product per slice holding any,
+      // with their fp16 values for this lane's columns and zeros elsewhere
+      if (wsl) {
+        #pragma unroll
+        for (int sl = 0; sl < 8; ++sl) {
+          if (!((wsl >> sl) & 1)) continue;
+          uint32_t aw[4] = {0u, 0u, 0u, 0u};
+          #pragma unroll
+          for (int u = 0; u < 2; ++u) {   // u: column 16 sl + g (+ 8 u) -> registers u, u + 2
+            if (!((wmask >> (2 * sl + u)) & 1u)) continue;
+            const int wi = s_slot[16 * sl + g + 8 * u] - t0;
+            if (staged) {
+              aw[u] = *reinterpret_cast<const uint32_t*>(s_wv + wi * rows + ra);
+              aw[u + 2] = *reinterpret_cast<const uint32_t*>(s_wv + wi * rows + ra + 8);
+            } else {
+              uint16_t v[4];
+              #pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int gr = t_lo * 16 + ra + (e & 1) + 8 * (e >> 1);
+                v[e] = gr < a.N ? __half_as_ushort(a.w_weak[(size_t)gr * a.k_ld + t0 + wi]) : (uint16_t)0;
+              }
+              aw[u] = (uint32_t)v[0] | ((uint32_t)v[1] << 16);
+              aw[u + 2] = (uint32_t)v[2] | ((uint32_t)v[3] << 16);
+            }
+          }
+          #pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816(D[sl][nt], aw, yq[0][nt][0], yq[0][nt][1]);
+        }
+      }
+    }
+    #pragma unroll
+    for (int p = 0; p < PD; ++p)
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt) { yq[p][nt][0] = yq[p + 1][nt][0]; yq[p][nt][1] = yq[p + 1][nt][1]; }
+  }
+  // after a timeout: never leave with bulk copies still writing into this CTA's memory
+  if (failed_at >= 0 && lane == 0)
+    for (int j = failed_at; j < issued; ++j)
+      mbar_wait(&bars[j % kIgStages], (uint32_t)((j / kIgStages) & 1), a.status, a.wait_limit);
+
+  // the 8 warps' sums in a fixed tree: (w, w + 4), then (w, w + 2), then (0, 1)
+  // D[sl][nt][i]: column 16 sl + g + 8 (i >> 1), token 8 nt + 2 tg + (i & 1)
+  #pragma unroll
+  for (int half = 4; half >= 1; half >>= 1) {
+    if (warp >= half && warp < 2 * half) {
+      #pragma unroll
+      for (int sl = 0; sl < 8; ++sl)
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i)
+            s_red[warp - half][8 * nt + 2 * tg + (i & 1)][16 * sl + g + 8 * (i >> 1)] = D[sl][nt][i];
+    }
+    __syncthreads();
+    if (warp < half) {
+      #pragma unroll
+      for (int sl = 0; sl < 8; ++sl)
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i)
+            D[sl][nt][i] += s_red[warp][8 * nt + 2 * tg + (i & 1)][16 * sl + g + 8 * (i >> 1)];
+    }
+    __syncthreads();
+  }
+  if (S == 1) {   // one slice: the CTA's sums are the outputs
+    if (warp == 0) {
+      #pragma unroll
+      for (int sl = 0; sl < 8; ++sl)
+        #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int m = 8 * nt + 2 * tg + (i & 1), c = b * kBlockCodes + 16 * sl + g + 8 * (i >> 1);
+            if (m < a.M) a.dx[(size_t)m * a.K + c] = __float2half_rn(D[sl][nt][i]);
+          }
+    }
+    return;
+  }
+  // the cluster of the column block's S slices: publish, then add in slice order
+  if (warp == 0) {
+    #pragma unroll
+    for (int sl = 0; sl < 8; ++sl)
+      #pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          s_red[0][8 * nt + 2 * tg + (i & 1)][16 * sl + g + 8 * (i >> 1)] = D[sl][nt][i];
+  }
+  cluster_sync();
+  {
+    constexpr int ne = kTok * kBlockCodes;
+    const int share = (ne + S - 1) / S, rank = (int)cluster_ctarank();
+    const int e_hi = min(ne, (rank + 1) * share);
+    for (int e = rank * share + tid; e < e_hi; e += kIgThreads) {
+      const int m = e / kBlockCodes, c = e % kBlockCodes;
+      if (m >= a.M) continue;
+      float sum = 0.f;
+      for (int r = 0; r < S; ++r) sum += ld_dsmem_f32(&s_red[0][m][c], (uint32_t)r);
+      a.dx[(size_t)m * a.K + b * kBlockCodes + c] = __float2half_rn(sum);
     }
   }
-  if (S == 1) return;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(a.count + b, 1u) == (unsigned)(S - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int e = tid; e < TOK * kBlockCodes; e += kIgThreads) {
-    const int m = e / kBlockCodes, c = b * kBlockCodes + e % kBlockCodes;
-    const float* src = a.part + (size_t)m * a.K + c;
-    const size_t step = (size_t)kIgMaxTok * a.K;
-    float sum = 0.f;
-    int s = 0;
-    for (; s + 4 <= S; s += 4) {   // four loads in flight, added in slice order
-      const float v0 = __ldcg(src + s * step), v1 = __ldcg(src + (s + 1) * step);
-      const float v2 = __ldcg(src + (s + 2) * step), v3 = __ldcg(src + (s + 3) * step);
-      sum += v0;
-      sum += v1;
-      sum += v2;
-      sum += v3;
-    }
-    for (; s < S; ++s) sum += __ldcg(src + s * step);
-    if (m < a.M) a.dx[(size_t)m * a.K + c] = __float2half_rn(sum);
-  }
-  if (tid == 0) a.count[b] = 0u;   // ready for the next call on this stream
+  cluster_sync();   // no CTA leaves while its sums may still be read
 }
 
 // SM count of device `dev` (cached per device ordinal)
@@ -409,19 +607,29 @@ int wct_sm_count(int dev) {
   return n[dev];
 }
 
-template <int BITS, int TOK>
-cudaError_t launch_ig(const IgArgs& a, int slices, cudaStream_t s) {
-  k_input_grad<BITS, TOK><<<dim3(a.K / kBlockCodes, slices), kIgThreads, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-template <int BITS>
-cudaError_t launch_ig_tok(const IgArgs& a, int slices, cudaStream_t s) {
-  if (a.M <= 1) return launch_ig<BITS, 1>(a, slices, s);
-  if (a.M <= 2) return launch_ig<BITS, 2>(a, slices, s);
-  if (a.M <= 4) return launch_ig<BITS, 4>(a, slices, s);
-  if (a.M <= 8) return launch_ig<BITS, 8>(a, slices, s);
-  return launch_ig<BITS, 16>(a, slices, s);
+template <int BITS, int NT>
+cudaError_t launch_ig(const IgArgs& a, int dev, int Kb, int slices, cudaStream_t s) {
+  constexpr int smem = ig_smem_bytes<BITS>();
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_input_grad_mma<BITS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)Kb, (unsigned)slices, 1);
+  cfg.blockDim = dim3(kIgThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = (unsigned)slices;   // the slices of a column block: one cluster
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_input_grad_mma<BITS, NT>, a);
 }
 
 }  // namespace
@@ -480,58 +688,34 @@ cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, 
 
 cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s) {
   const int Kb = L.K / kBlockCodes;
-  const int nstages = ((L.N + 15) / 16 + 3) / 4;
-  // two CTAs per SM (what the registers allow) over the column blocks and row slices, rounded
-  // down so that the grid is one wave
-  int slices = std::max(1, std::min(nstages, (2 * wct_sm_count(L.device)) / Kb));
-  int per = (nstages + slices - 1) / slices;
-  slices = (nstages + per - 1) / per;
-  // workspace: one arrival counter per column block (zero between calls), then the partial sums
-  const size_t cnt_bytes = ((size_t)Kb * sizeof(unsigned int) + 255) / 256 * 256;
-  if (slices > 1) {
-    const size_t need = cnt_bytes + (size_t)slices * kIgMaxTok * L.K * sizeof(float);
-    if (need > L.ig_ws_bytes) {
-      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-      if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
-        cudaGetLastError();
-        slices = 1;   // no allocation inside a capture: one slice needs no workspace
-      } else {
-        cudaFree(L.ig_ws);
-        L.ig_ws = nullptr;
-        L.ig_ws_bytes = 0;
-        if (cudaMalloc(&L.ig_ws, need) != cudaSuccess) {
-          cudaGetLastError();
-          L.ig_ws = nullptr;
-          slices = 1;
-        } else if (cudaMemsetAsync(L.ig_ws, 0, cnt_bytes, s) != cudaSuccess) {
-          return cudaGetLastError();
-        } else {
-          L.ig_ws_bytes = need;
-        }
-      }
-    }
-  }
-  if (slices == 1) per = nstages;
+  const int tiles = (L.N + 15) / 16;
+  // two CTAs per SM over the column blocks and row slices (about one wave), each slice at least
+  // one tile per warp, the slices of a column block one cluster (at most 8 CTAs)
+  int slices = std::max(1, std::min({(tiles + 7) / 8, (2 * wct_sm_count(L.device)) / Kb, kIgMaxSlices}));
+  const int per = (tiles + slices - 1) / slices;
+  slices = (tiles + per - 1) / per;
   IgArgs a;
   a.packed = L.packed;
-  a.scales = L.scales;
-  a.zeros = L.zeros;
+  a.sz_t = L.sz_t;
   a.w_weak = L.w_weak;
   a.idx = L.idx;
-  a.count = slices > 1 ? reinterpret_cast<unsigned int*>(L.ig_ws) : nullptr;
-  a.part = slices > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(L.ig_ws) + cnt_bytes) : nullptr;
+  a.status = device_status_ptr();
+  a.wait_limit = kDefaultWaitLimit;
   a.N = L.N;
   a.K = L.K;
   a.G = L.G;
   a.group = L.group;
   a.k = L.k;
   a.k_ld = L.k_ld;
-  a.stages_per_slice = per;
+  a.tiles_per_slice = per;
+  if (!a.status) return cudaErrorInvalidDevicePointer;
   for (int m0 = 0; m0 < M; m0 += kIgMaxTok) {
     a.dy = dy + (size_t)m0 * L.N;
     a.dx = dx + (size_t)m0 * L.K;
     a.M = std::min(kIgMaxTok, M - m0);
-    const cudaError_t e = L.bits == 3 ? launch_ig_tok<3>(a, slices, s) : launch_ig_tok<4>(a, slices, s);
+    const cudaError_t e =
+        L.bits == 3 ? (a.M <= 8 ? launch_ig<3, 1>(a, L.device, Kb, slices, s) : launch_ig<3, 2>(a, L.device, Kb, slices, s))
+                    : (a.M <= 8 ? launch_ig<4, 1>(a, L.device, Kb, slices, s) : launch_ig<4, 2>(a, L.device, Kb, slices, s));
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
