@@ -536,8 +536,9 @@ def prefill_measure(args, dev, Ms=None, reps=10):
 
 def wct_measure(args, dev):
     """Weak column tuning kernels on the OPT-6.7B-shaped layers (3-bit per channel, k = K/128):
-    owq_input_grad (dX = dY W_eff from the packed layout; HBM-bound, GB/s of its algorithmic
-    bytes: packed + scales/zeros + weak block + idx + dY + dX) and owq_weak_grad
+    owq_input_grad (dX = dY W_eff from the packed layout; GB/s of its algorithmic bytes: packed +
+    scales/zeros + weak block + idx + dY + dX, against the HBM roofline at 1 and 16 tokens, and
+    TFLOP/s of 2 M N K against the bf16 tensor roofline at 256 and 2048) and owq_weak_grad
     (dW_weak = dY^T x[:, idx]; bytes dY + the gathered x columns + fp32 dW_weak).
 
     Timing: one CUDA graph of R calls over R distinct operand sets (R packed copies of the layer
@@ -588,13 +589,16 @@ def wct_measure(args, dev):
         lays = [owq.OwqLayer(q["codes"], q["scales"], q["zeros"], q["idx"], q["w_weak"], L.bits, L.group)
                 for _ in range(R)]
         row = {}
-        for M in (1, 16):
+        for M in (1, 16, 256, 2048):
             dy = torch.randn((M, L.N), device=dev).half()
             dx = torch.empty((M, L.K), dtype=torch.float16, device=dev)
             t = graph_time([lambda lay=lay: lay.input_grad(dy, dx) for lay in lays])
             B = wbytes + 2 * M * L.N + 2 * M * L.K
+            F = 2.0 * M * L.N * L.K
             row[f"input_grad_M{M}"] = {"us": round(t * 1e6, 2), "GBps": round(B / t / 1e9, 1),
-                                       "frac_hbm": round(B / t / 1e9 / peaks["hbm_gbs"], 4), "copies": R}
+                                       "frac_hbm": round(B / t / 1e9 / peaks["hbm_gbs"], 4),
+                                       "TFLOPs": round(F / t / 1e12, 1),
+                                       "frac_bf16": round(F / t / 1e12 / peaks["bf16_tflops"], 4), "copies": R}
         for lay in lays[1:]:
             lay.close()
         lay = lays[0]

@@ -326,20 +326,28 @@ owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t*
  * owq_input_grad -- weak column tuning: the gradient the frozen layer passes to its input
  * (same pages; earlier layers' weak columns need it), the transposed product
  *   dx[m][j] = sum_i dy[m][i] * W_eff[i][j],
- * W_eff = s * (q - z) except at the weak columns, which take their fp16 values from the weak
- * block.  Read straight from the packed layout (no W_hat in memory) on the tensor cores
- * (mma.sync m16n8k16): the exact integers q - z times dy * s carried as an fp16 pair (high
- * part + residual), fp32 accumulation, one fp16 rounding of each output.  Like the decode
- * product this multiplies the unrounded s (q - z) rather than W_hat = fp16_rn(s (q - z)): each
- * weight differs by at most half an fp16 spacing; with a single nonzero dy (1.0) per token the
- * output row is W_eff's row bit for bit.
- * In:  dy fp16 M x N row-major; 1 <= M <= 65536 (one pass over the packed weights per 16
- *      tokens).  Out: dx fp16 M x K row-major (fully overwritten).
- * The rows are split over up to 8 CTAs per 128-column block, one thread-block cluster; the
- * CTAs' fp32 sums are added in a fixed order through distributed shared memory, so repeated
- * calls give identical bits.  No workspace and no allocation: allowed inside a stream capture.
- * Copy waits are bounded (OWQ_ERR_TIMEOUT through owq_device_status).  Device pointers,
- * 16-byte aligned; asynchronous on `stream`.
+ * W_eff = the dequantised matrix except at the weak columns, which take their fp16 values from
+ * the weak block.  Read straight from the packed layout (no W_hat in memory), fp32
+ * accumulation, one fp16 rounding of each output.  Two paths:
+ *  - M <= 32, or N not a multiple of 8: 16 tokens per pass (mma.sync m16n8k16); the exact
+ *    integers q - z times dy * s carried as an fp16 pair (high part + residual), i.e. the
+ *    unrounded s (q - z) like the decode product (each weight within half an fp16 spacing of
+ *    W_hat = fp16_rn(s (q - z))).  The rows of a 128-column block are split over up to 8 CTAs
+ *    of one thread-block cluster whose fp32 sums are added in a fixed order through distributed
+ *    shared memory: no workspace, allowed inside a stream capture.
+ *  - M > 32 and N % 8 == 0: the 5th-generation tensor cores (tcgen05.mma, accumulator and the
+ *    A operand W_hat^T in tensor memory, dy by TMA) multiply W_hat = fp16_rn(s (q - z)) itself,
+ *    bit-exact per weight; the weak columns come out exactly 0 there (their codes hold q = z)
+ *    and a second kernel then writes dx[:, idx] = dy W_weak (mma.sync).  With fewer output
+ *    tiles than SMs the rows are split over CTAs: fp32 partials in the handle's prefill
+ *    workspace (and the weak pass's in the weak-gradient scratch), grown on the first call that
+ *    needs more, which must be outside a stream capture (inside one: a single split, slower,
+ *    same result); the splits are added in split order.  Calls on one handle must be ordered.
+ * Both paths: with a single nonzero dy (1.0) per token the output row is W_eff's row bit for
+ * bit; repeated calls give identical bits.  Waits are bounded (OWQ_ERR_TIMEOUT through
+ * owq_device_status).
+ * In:  dy fp16 M x N row-major; 1 <= M <= 65536.  Out: dx fp16 M x K row-major (fully
+ *      overwritten).  Device pointers, 16-byte aligned; asynchronous on `stream`.
  */
 owq_status_t owq_input_grad(owq_layer_t layer, const uint16_t* dy, uint16_t* dx, int M,
                             owq_stream_t stream);

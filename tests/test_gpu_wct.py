@@ -32,6 +32,14 @@ CASES = [
     ("cluster-of-3", 300, 384, 3, 384, 5, (1, 9), None),
     # 40 weak columns in one block over 512-row slices: too many to stage in shared memory
     ("weak-heavy-block", 4096, 256, 4, 128, 40, (2, 16), tuple(range(0, 80, 2))),
+    # from 33 tokens (N % 8 == 0): the tensor-memory pipeline, token tiles of 64 / 128 / 256,
+    # ragged 128-row steps, then the weak-column pass
+    ("many-tokens-3b", 520, 640, 3, 640, 7, (33, 100, 300), None),
+    ("many-tokens-4b-g128", 384, 512, 4, 128, 13, (64, 257), None),
+    ("many-tokens-k0", 256, 384, 4, 128, 0, (40,), None),
+    ("many-tokens-weak-heavy", 1024, 256, 3, 128, 40, (48,), tuple(range(0, 80, 2))),
+    # N % 8 != 0: many tokens run through the 16-token kernel
+    ("many-tokens-n-odd", 130, 512, 3, 128, 6, (40,), None),
 ]
 
 
@@ -135,7 +143,10 @@ def test_wct_gradients_fullsize_opt67b_attention_layer():
     layer.close()
 
 
-@pytest.mark.parametrize("case", [CASES[1], CASES[2], CASES[5], CASES[7], CASES[8]], ids=lambda c: c[0])
+ONE_HOT = [CASES[1], CASES[2], CASES[5], CASES[7], CASES[8], CASES[9], CASES[10], CASES[12]]
+
+
+@pytest.mark.parametrize("case", ONE_HOT, ids=lambda c: c[0])
 def test_input_grad_one_hot_rows_are_w_eff(case):
     """One nonzero dY (1.0) per token: dX's row is row i of W_eff (W_hat with the weak columns'
     fp16 values) bit for bit, since the kernel's only rounding is then the final fp16 one
@@ -151,8 +162,12 @@ def test_input_grad_one_hot_rows_are_w_eff(case):
     want[want == 0x8000] = 0
     layer = _layer(owq, ref, bits, group)
     rows = np.unique(np.concatenate([[0, N - 1, N // 2], np.arange(0, N, max(1, N // 29))]))
-    for r0 in range(0, len(rows), 16):
-        rr = rows[r0:r0 + 16]
+    # 16 tokens per call (the 16-token kernel); with M >= 33 in a case, all rows in one call too
+    # (the tensor-memory pipeline when N % 8 == 0; rows repeated up to 40 tokens)
+    groups = [rows[r0:r0 + 16] for r0 in range(0, len(rows), 16)]
+    if max(Ms) >= 33:
+        groups.append(np.resize(rows, max(40, len(rows))))
+    for rr in groups:
         dy = np.zeros((len(rr), N), dtype=np.float16)
         dy[np.arange(len(rr)), rr] = 1.0
         got = layer.input_grad(_gpu(dy)).cpu().numpy().view(np.uint16)

@@ -473,9 +473,15 @@ owq_status_t owq_input_grad(owq_layer_t layer, const uint16_t* dy, uint16_t* dx,
   if (M < 1 || M > 65536) return OWQ_ERR_SHAPE;
   if (!dy || !dx) return OWQ_ERR_NULL;
   if (!aligned16(dy) || !aligned16(dx)) return OWQ_ERR_ALIGN;
-  return cuda_status(launch_input_grad(*L, reinterpret_cast<const __half*>(dy),
-                                       reinterpret_cast<__half*>(dx), M,
-                                       reinterpret_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const __half* dyh = reinterpret_cast<const __half*>(dy);
+  __half* dxh = reinterpret_cast<__half*>(dx);
+  if (M > kIgGemmMinM && L->N % 8 == 0) {   // dY rows must be 16-byte strided for its tensor map
+    const owq_status_t st = igemm_sm100(*L, dyh, dxh, M, kDefaultWaitLimit, s);
+    if (st) return st;
+    return cuda_status(launch_input_grad_weak(*L, dyh, dxh, M, s));
+  }
+  return cuda_status(launch_input_grad(*L, dyh, dxh, M, s));
 }
 
 owq_status_t owq_dequant(owq_layer_t layer, uint16_t* w_hat, uint8_t* codes, owq_stream_t stream) {

@@ -83,6 +83,11 @@ __device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 __device__ __forceinline__ uint32_t h2_splat(float v) {
   __half h = __float2half_rn(v);
   uint32_t u = __half_as_ushort(h);
@@ -324,6 +329,244 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   }
 }
 
+// ---------------------------------------------------------------- input gradient, many tokens
+// dX = dY W_hat on the same pipeline, transposed: one CTA computes a 128-column x BN-token tile
+// of dX^T (MMA M = the 128 columns of one packed block, MMA N = tokens), looping over the rows
+// (the contraction) in 128-row steps.
+//   warp 0      TMA producer: the step's packed block of 8 16-row tiles (the prefill's box, at
+//               block b and the step's tiles), their (scale, zero) pairs for block b's group, and
+//               two 128B-swizzled BN x 64 fp16 boxes of dY (tokens x rows).
+//   warp 1      TMEM allocation and the MMA-issuing thread (unchanged).
+//   warps 2..   the A operand W_hat^T: thread (lane quarter, lane) owns column j = TMEM lane and a
+//               slab of the step's rows; tensor memory packs two K values (rows 2c, 2c + 1) per
+//               32-bit column.  Column j's code sits in the same word of every row (chunk
+//               (j / 2) % 4, pair (j / 2) / 4, half j % 2), so one byte permute of two rows'
+//               words gives the row pair (moved down a byte where the code sits at bit 8 or
+//               above), AND/OR 0x6400 gives 1024 + q 2^o, and fp16x2 fma, subtract and multiply
+//               with the row pair's (s, z) give fp16_rn(s (q - z)) bit-exactly.  The weak
+//               columns hold q = z, so they come out exactly 0 here; a separate pass writes
+//               them.  The same warps run the epilogue.
+//   last warp   prep: per step, each row pair's scales and zero points side by side, and (3-bit)
+//               the pair whose bits are spread over a chunk's three words rebuilt as an ordinary
+//               word, so every A thread runs the same eight instructions per row pair.
+// Every mbarrier wait is bounded, as in the prefill kernel.
+// Stage layout: the prefill's (dY boxes, packed block, (s, z) pairs), then what the prep warp
+// derives from them: the 3-bit spread pair of every (row, chunk) rebuilt as an ordinary word
+// (even code at bits 6-8, odd at 22-24) and each row pair's scales and zero points side by side.
+template <int BITS, int BN>
+struct IgSmem {
+  static constexpr int kX = Smem<BITS, BN>::kX, kP = Smem<BITS, BN>::kP, kSZ = Smem<BITS, BN>::kSZ;
+  static constexpr int kTma = kX + kP + kSZ;
+  static constexpr int kAuxD = BITS == 3 ? kBM * 4 * 4 : 0;   // [128 rows][4 chunks] words
+  static constexpr int kAuxS = 64 * 8;                        // [64 row pairs] {s2, z2}
+  static constexpr int kStage = ((kTma + kAuxD + kAuxS) + 1023) & ~1023;
+};
+template <int BITS, int BN, int S>
+constexpr int ig_smem_bytes() { return S * IgSmem<BITS, BN>::kStage + 1024 /*barriers*/ + 1024 /*align slack*/; }
+
+struct IgGemmParams {
+  __half* dx;
+  float* ws;        // split-K partial sums [split][M][K] (NULL: one split, fp16 dx directly)
+  int* status;
+  int N, K, M, group;
+  int rsteps;       // 128-row steps per split (blockIdx.z)
+  long long wait_limit;
+};
+
+template <int BITS, int BN, int S, int DW>
+__global__ void __launch_bounds__(32 * (3 + DW), 1)
+k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant__ CUtensorMap map_p,
+              const __grid_constant__ CUtensorMap map_sz, const __grid_constant__ IgGemmParams p) {
+  using L = IgSmem<BITS, BN>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage);
+  uint64_t* full = bars;            // [S] TMA landed
+  uint64_t* empty = bars + S;       // [S] MMAs of the stage done
+  uint64_t* afull = bars + 2 * S;   // [S] A tile written to tensor memory
+  uint64_t* accf = bars + 3 * S;    // accumulator complete
+  uint64_t* pfull = bars + 3 * S + 1;   // [S] prep warp's words written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * S + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x;             // column block (128 columns)
+  const int m0 = blockIdx.y * BN;       // first token
+  const int nR = (p.N + 127) / 128;
+  const int rb0 = blockIdx.z * p.rsteps;                 // first row step of this split
+  const int nK = max(0, min(p.rsteps, nR - rb0));
+  const int grp = (b * kStepCodes) / p.group;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&afull[s], 32 * DW);
+      mbar_init(&pfull[s], 32);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+    prefetch_tmap(&map_dy);
+    prefetch_tmap(&map_p);
+    prefetch_tmap(&map_sz);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, tmem_cols<BN, S>());
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      const uint32_t kBytes = L::kTma;
+      bool ok = true;
+      int issued = 0;
+      for (int i = 0; i < nK && ok; ++i) {
+        const int s = i % S, u = i / S;
+        if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, p.status, p.wait_limit);
+        if (!ok) break;
+        unsigned char* st = smem + s * L::kStage;
+        const int rb = rb0 + i;
+        mbar_arrive_expect_tx(&full[s], kBytes);
+        tma_load_3d(st + L::kX, &map_p, &full[s], 0, b, rb * 8);
+        tma_load_3d(st + L::kX + L::kP, &map_sz, &full[s], 0, grp, rb * 8);
+        tma_load_2d(st, &map_dy, &full[s], rb * 128, m0);
+        tma_load_2d(st + BN * 128, &map_dy, &full[s], rb * 128 + 64, m0);
+        issued = i + 1;
+      }
+      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait(&full[i % S], (i / S) & 1, p.status, p.wait_limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_f16_f32(kBM, BN);
+      const uint64_t dbase = desc_sw128_kmajor(smem_u32(smem));
+      bool ok = true;
+      for (int i = 0; i < nK && ok; ++i) {
+        const int s = i % S, u = i / S;
+        ok = mbar_wait(&afull[s], u & 1, p.status, p.wait_limit);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t ds = dbase + (uint64_t)((s * L::kStage) >> 4);
+        const uint32_t at = tmem + BN + 64 * s;
+        mma_f16_ts(tmem, at, ds, idesc, i != 0);
+        #pragma unroll
+        for (int kk = 1; kk < 8; ++kk)
+          mma_f16_ts(tmem, at + 8 * kk, ds + (uint64_t)((((kk >> 2) * BN * 128) + (kk & 3) * 32) >> 4), idesc, 1u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accf);
+    }
+  } else if (warp == 2 + DW) {
+    // ---------------- prep warp ----------------
+    bool ok = true;
+    for (int i = 0; i < nK && ok; ++i) {
+      const int s = i % S, u = i / S;
+      ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);
+      if (!ok) break;
+      unsigned char* st = smem + s * L::kStage;
+      const uint2* sz = reinterpret_cast<const uint2*>(st + L::kX + L::kP);
+      uint2* aux_s = reinterpret_cast<uint2*>(st + L::kTma + L::kAuxD);
+      #pragma unroll
+      for (int pp = lane; pp < 64; pp += 32) {
+        const uint2 v = sz[pp];
+        aux_s[pp] = make_uint2(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.x, v.y, 0x7632));
+      }
+      if constexpr (BITS == 3) {   // bit e of the spread pair: bit 15 / 31 of word e -> 6 + e / 22 + e
+        uint32_t* aux_d = reinterpret_cast<uint32_t*>(st + L::kTma);
+        #pragma unroll 4
+        for (int e = lane; e < kBM * 4; e += 32) {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(st + L::kX + (e >> 2) * 48 + (e & 3) * 12);
+          aux_d[e] = ((w[0] >> 9) & 0x00400040u) | ((w[1] >> 8) & 0x00800080u) | ((w[2] >> 7) & 0x01000100u);
+        }
+      }
+      mbar_arrive(&pfull[s]);
+    }
+  } else {
+    // ---------------- A operand: W_hat^T ----------------
+    // NSL = DW / 4 warps per lane quarter; warp w takes lane quarter w % 4 and row slab
+    // (w - 2) / 4, RP row pairs of each step (tensor-memory columns RP jh .. RP jh + RP - 1).
+    constexpr int NSL = DW / 4, RP = 64 / NSL;
+    const int quarter = warp & 3, jh = (warp - 2) >> 2;
+    const int j = 32 * quarter + lane;             // column of the block
+    const int pj = j >> 1, q = pj & 3, jj = pj >> 2, h = j & 1;
+    const bool spread = BITS == 3 && jj == 11;
+    // the slot of pair jj (the 3-bit table of owq_format.cuh as packed fields: word, offset / 3)
+    const Slot sl = spread ? Slot{0, 6}
+                  : BITS == 3 ? Slot{(int)((0xaa244444u >> (2 * jj)) & 3u), 3 * (int)((0x3041024433221100ull >> (4 * jj)) & 15u)}
+                              : Slot{2 * (jj / 8) + (jj % 2), 4 * ((jj % 8) / 2)};
+    const bool hi8 = !spread && sl.off >= 8;
+    const int o2 = hi8 ? sl.off - 8 : sl.off;
+    const uint32_t sel = h ? (hi8 ? 0x7733u : 0x7632u) : (hi8 ? 0x5511u : 0x5410u);
+    const uint32_t m1 = ((1u << BITS) - 1u) << o2, mask = m1 | (m1 << 16);
+    const uint32_t sc = ((uint32_t)(15 - o2) << 10) * 0x00010001u;                // 2^-o
+    const uint32_t nego = (0x8000u | ((uint32_t)(25 - o2) << 10)) * 0x00010001u;  // -2^(10 - o)
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+    // the word holding column j's code in each row: the packed block, or for the spread pair the
+    // prep warp's rebuilt word (then at offset 6, the unshifted half)
+    const int woff = spread ? L::kTma + 4 * q : L::kX + q * 4 * BITS + 4 * sl.word;
+    const int rstride = spread ? 16 : 16 * BITS;
+    bool ok = true;
+    for (int i = 0; i < nK && ok; ++i) {
+      const int s = i % S, u = i / S;
+      ok = mbar_wait(&pfull[s], u & 1, p.status, p.wait_limit);   // (implies the TMA landed)
+      if (!ok) break;
+      tc_fence_after();
+      const unsigned char* st = smem + s * L::kStage;
+      const unsigned char* pk = st + woff + (2 * RP * jh) * rstride;
+      const uint2* szp = reinterpret_cast<const uint2*>(st + L::kTma + L::kAuxD) + RP * jh;
+      uint32_t d[RP];
+      #pragma unroll
+      for (int pr = 0; pr < RP; ++pr) {
+        const uint32_t wa = *reinterpret_cast<const uint32_t*>(pk + (2 * pr) * rstride);
+        const uint32_t wb = *reinterpret_cast<const uint32_t*>(pk + (2 * pr + 1) * rstride);
+        const uint32_t v = (__byte_perm(wa, wb, sel) & mask) | 0x64006400u;
+        const uint2 sz = szp[pr];   // {s2, z2} of rows 2 pr, 2 pr + 1 of the slab
+        d[pr] = h2_mul(h2_sub(h2_fma(v, sc, nego), sz.y), sz.x);   // fp16_rn(s (q - z))
+      }
+      const uint32_t at = tmem + lane_base + BN + 64 * s + RP * jh;
+      #pragma unroll
+      for (int c = 0; c < RP / 16; ++c)
+        tmem_st16(at + 16 * c, *reinterpret_cast<const uint32_t(*)[16]>(d + 16 * c));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&afull[s]);
+    }
+
+    // ---------------- epilogue ----------------
+    const bool acc_ok = mbar_wait(accf, 0, p.status, p.wait_limit);
+    tc_fence_after();
+    const int col = b * kStepCodes + j;
+    #pragma unroll 1
+    for (int c0 = jh * (BN / NSL); c0 < (jh + 1) * (BN / NSL); c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
+      tmem_ld_wait();
+      if (acc_ok) {
+        if (p.ws) {
+          float* w = p.ws + (size_t)blockIdx.z * p.M * p.K;
+          #pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (m0 + c0 + t < p.M) w[(size_t)(m0 + c0 + t) * p.K + col] = __uint_as_float(v[t]);
+        } else {
+          #pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (m0 + c0 + t < p.M) p.dx[(size_t)(m0 + c0 + t) * p.K + col] = __float2half_rn(__uint_as_float(v[t]));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols<BN, S>());
+    tmem_relinquish();
+  }
+}
+
 // Weak activations of every token, in the weak block's column order: xw[m][t] = x[m][idx[t]]
 // (t < k), 0 for t in [k, k_ld).
 __global__ void k_gather_weak_x(const __half* __restrict__ x, int M, int K, const int32_t* __restrict__ idx,
@@ -426,7 +669,7 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
                  cudaStream_t s) {
   if (!L.maps_ready) {
     if (!encode_packed_3d(&L.map_packed, L.packed, L.K, L.N, BITS)) return OWQ_ERR_CUDA;
-    if (L.G > 1 && !encode_sz_3d(&L.map_sz, L.sz_t, L.G, L.N)) return OWQ_ERR_CUDA;
+    if (!encode_sz_3d(&L.map_sz, L.sz_t, L.G, L.N)) return OWQ_ERR_CUDA;   // (used by per-group prefill and the input gradient)
     L.maps_ready = true;
   }
   CUtensorMap mx;
@@ -523,12 +766,81 @@ owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, long long wl,
   return run<BITS, 256, 3, 16>(L, x, y, M, wl, skip, s);
 }
 
+template <int BITS, int BN, int S, int DW>
+owq_status_t ig_run(Layer& L, const __half* dy, __half* dx, int M, long long wait_limit, cudaStream_t s) {
+  if (!L.maps_ready) {
+    if (!encode_packed_3d(&L.map_packed, L.packed, L.K, L.N, BITS)) return OWQ_ERR_CUDA;
+    if (!encode_sz_3d(&L.map_sz, L.sz_t, L.G, L.N)) return OWQ_ERR_CUDA;
+    L.maps_ready = true;
+  }
+  CUtensorMap mdy;
+  if (!encode_2d(&mdy, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dy, (uint64_t)L.N, (uint64_t)M, (uint64_t)L.N * 2, 64, BN,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return OWQ_ERR_CUDA;
+  IgGemmParams prm;
+  prm.dx = dx;
+  prm.status = device_status_ptr();
+  prm.N = L.N; prm.K = L.K; prm.M = M; prm.group = L.group;
+  prm.wait_limit = wait_limit;
+  if (!prm.status) return OWQ_ERR_CUDA;
+  // fewer tiles than SMs: split the rows over CTAs (at least 4 steps each), fp32 partials in the
+  // layer's prefill workspace, then the split-order reduction; never grown during stream capture
+  const int nR = (L.N + 127) / 128, Kb = L.K / kStepCodes;
+  const long long tiles = (long long)Kb * ((M + BN - 1) / BN);
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, L.device) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  int splits = tiles < sms ? (int)std::max<long long>(1, std::min<long long>(sms / tiles, nR / 4)) : 1;
+  if (splits > 1) {
+    prm.rsteps = (nR + splits - 1) / splits;
+    splits = (nR + prm.rsteps - 1) / prm.rsteps;
+    if (!ensure_scratch(reinterpret_cast<void**>(&L.gemm_ws), &L.gemm_ws_bytes, (size_t)splits * M * L.K * sizeof(float), s))
+      splits = 1;
+  }
+  if (splits == 1) {
+    prm.rsteps = nR;
+    prm.ws = nullptr;
+  } else {
+    prm.ws = L.gemm_ws;
+  }
+  auto kern = k_igemm_sm100<BITS, BN, S, DW>;
+  constexpr int smem = ig_smem_bytes<BITS, BN, S>();
+  static_assert(smem <= 232448, "shared memory budget");
+  static_assert((232448 / smem) * tmem_cols<BN, S>() <= 512, "tensor memory per SM");
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return OWQ_ERR_CUDA;
+  }
+  dim3 grid(Kb, (M + BN - 1) / BN, splits);
+  kern<<<grid, 32 * (3 + DW), smem, s>>>(mdy, L.map_packed, L.map_sz, prm);
+  if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
+  if (splits > 1) {
+    const size_t MK = (size_t)M * L.K;
+    k_splitk_reduce<<<(unsigned)std::min<size_t>((MK + 255) / 256, 4096), 256, 0, s>>>(prm.ws, splits, MK, dx);
+    if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
+  }
+  return OWQ_OK;
+}
+
+template <int BITS>
+owq_status_t ig_dispatch(Layer& L, const __half* dy, __half* dx, int M, long long wl, cudaStream_t s) {
+  if (M <= 64) return ig_run<BITS, 64, 6, 8>(L, dy, dx, M, wl, s);
+  if (M <= 256) return ig_run<BITS, 128, 4, 8>(L, dy, dx, M, wl, s);
+  return ig_run<BITS, 256, 3, 16>(L, dy, dx, M, wl, s);
+}
+
 }  // namespace
 
 owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, long long wait_limit,
                         bool skip_arrive, cudaStream_t s) {
   return L.bits == 3 ? dispatch<3>(L, x, y, M, wait_limit, skip_arrive, s)
                      : dispatch<4>(L, x, y, M, wait_limit, skip_arrive, s);
+}
+
+owq_status_t igemm_sm100(Layer& L, const __half* dy, __half* dx, int M, long long wait_limit, cudaStream_t s) {
+  return L.bits == 3 ? ig_dispatch<3>(L, dy, dx, M, wait_limit, s) : ig_dispatch<4>(L, dy, dx, M, wait_limit, s);
 }
 
 }  // namespace owq

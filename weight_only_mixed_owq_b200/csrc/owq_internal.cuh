@@ -131,6 +131,11 @@ cudaError_t launch_storage_unpack(const uint32_t* words, int N, int K, int bits,
 cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, float* dw, int M,
                              cudaStream_t s);
 cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s);
+// many tokens: the packed product on the 5th-generation tensor cores (weak columns left at
+// exactly 0), then the weak columns dx[:, idx] = dY W_weak (overwritten)
+constexpr int kIgGemmMinM = 32;   // the tensor-memory pipeline from this many tokens (N % 8 == 0)
+owq_status_t igemm_sm100(Layer& L, const __half* dy, __half* dx, int M, long long wait_limit, cudaStream_t s);
+cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s);
 
 // skip_arrive: a test-injected lost arrival (one dequantisation thread per CTA skips its first
 // arrival), so that the bounded waits run out

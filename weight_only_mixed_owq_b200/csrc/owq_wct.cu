@@ -177,6 +177,104 @@ __global__ void k_wg_reduce(const float* __restrict__ part, int splits, size_t n
   }
 }
 
+// ---------------------------------------------------------------- input gradient, weak columns
+// dx[m][idx[t]] = fp16_rn(sum_i dY[m][i] W_weak[i][t]) for many tokens.  The packed product runs
+// first and leaves exactly 0 in the weak columns (their codes hold q = z), so this pass simply
+// writes them.  mma.sync m16n8k16: MMA rows = tokens, MMA K = rows i, MMA N = weak slots.  A CTA
+// of 4 warps computes 64 tokens x 32 slots over one split of the rows, 32 rows at a time
+// through a 4-stage cp.async ring ([64 tokens][32 rows] of dY, [32 rows][32 slots] of the weak
+// block); A through ldmatrix, B through ldmatrix.trans.  One split writes dx directly; several
+// write fp32 partials that a second kernel adds in split order (repeat calls: identical bits).
+constexpr int kIwTok = 64, kIwCols = 32, kIwRows = 32, kIwThreads = 128, kIwStages = 4;
+constexpr int kIwDyLd = kIwRows + 8, kIwWLd = kIwCols + 8;   // padded row strides (halves)
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+
+// grid (M / 64, k_ld / 32, row splits of `per` rows, a multiple of 32); N % 8 == 0
+__global__ void __launch_bounds__(kIwThreads)
+k_igw_mma(const __half* __restrict__ dy, const __half* __restrict__ w, const int32_t* __restrict__ idx,
+          __half* __restrict__ dx, float* __restrict__ part, int N, int K, int M, int k, int k_ld, int per) {
+  __shared__ __align__(128) __half s_dy[kIwStages][kIwTok][kIwDyLd];
+  __shared__ __align__(128) __half s_w[kIwStages][kIwRows][kIwWLd];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mb = blockIdx.x * kIwTok, t0 = blockIdx.y * kIwCols;
+  const int i_lo = blockIdx.z * per, i_hi = min(N, i_lo + per);
+  const int nchunk = (i_hi - i_lo + kIwRows - 1) / kIwRows;
+  auto load = [&](int c, int st) {   // rows i_lo + 32 c .. of this split into stage st
+    const int ib = i_lo + c * kIwRows;
+    #pragma unroll
+    for (int u = 0; u < 2; ++u) {    // dY: 64 tokens x 4 pieces of 8 rows
+      const int e = tid + u * kIwThreads, m = e >> 2, pc = e & 3;
+      const int mm = mb + m, row = ib + pc * 8;
+      const bool ok = mm < M && row < i_hi;
+      cp_async16(&s_dy[st][m][pc * 8], dy + (ok ? (size_t)mm * N + row : 0), ok);
+    }
+    {                                // weak block: 32 rows x 4 pieces of 8 slots
+      const int r = tid >> 2, pc = tid & 3, row = ib + r, col = t0 + pc * 8;
+      const bool ok = row < i_hi && col < k_ld;
+      cp_async16(&s_w[st][r][pc * 8], w + (ok ? (size_t)row * k_ld + col : 0), ok);
+    }
+  };
+  float d[4][4];
+  #pragma unroll
+  for (int n = 0; n < 4; ++n)
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) d[n][i] = 0.f;
+  #pragma unroll
+  for (int st = 0; st < kIwStages - 1; ++st) {
+    if (st < nchunk) load(st, st);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  const int q = lane >> 3, r8 = lane & 7;   // ldmatrix: matrix q, row r8
+  for (int c = 0; c < nchunk; ++c) {
+    asm volatile("cp.async.wait_group %0;" :: "n"(kIwStages - 2) : "memory");
+    __syncthreads();   // chunk c landed for every thread; the stage refilled below is free
+    if (c + kIwStages - 1 < nchunk) load(c + kIwStages - 1, (c + kIwStages - 1) % kIwStages);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const int st = c % kIwStages;
+    #pragma unroll
+    for (int ks = 0; ks < kIwRows / 16; ++ks) {
+      const int mk = ks * 16;
+      uint32_t a[4];   // tokens 16 warp + 0..15 x rows mk..mk+15: (t 0-7, i 0-7), (t 8-15, i 0-7), (t 0-7, i 8-15), (t 8-15, i 8-15)
+      ldsm_x4(a, &s_dy[st][warp * 16 + (q & 1) * 8 + r8][mk + (q >> 1) * 8]);
+      #pragma unroll
+      for (int nh = 0; nh < 2; ++nh) {
+        uint32_t bb[4];   // rows mk..mk+15 x slots 16 nh..16 nh+15, read transposed (two n8 tiles)
+        ldsm_x4_t(bb, &s_w[st][mk + (q & 1) * 8 + r8][nh * 16 + (q >> 1) * 8]);
+        mma_16816(d[2 * nh], a, bb[0], bb[1]);
+        mma_16816(d[2 * nh + 1], a, bb[2], bb[3]);
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  const int g = lane >> 2, c4 = lane & 3;
+  #pragma unroll
+  for (int n = 0; n < 4; ++n)
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = mb + warp * 16 + g + 8 * (i >> 1), t = t0 + n * 8 + 2 * c4 + (i & 1);
+      if (m < M && t < k) {
+        if (part) part[((size_t)blockIdx.z * M + m) * k + t] = d[n][i];
+        else dx[(size_t)m * K + idx[t]] = __float2half_rn(d[n][i]);
+      }
+    }
+}
+
+// dx[m][idx[t]] = fp16 of the sum of the splits' partials, in split order
+__global__ void k_igw_reduce(const float* __restrict__ part, int splits, int M, int k, int K,
+                             const int32_t* __restrict__ idx, __half* __restrict__ dx) {
+  const size_t n = (size_t)M * k;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    float v = part[e];
+    for (int z = 1; z < splits; ++z) v += part[(size_t)z * n + e];
+    dx[(e / k) * K + idx[e % k]] = __float2half_rn(v);
+  }
+}
+
 // ---------------------------------------------------------------- input gradient
 constexpr int kIgThreads = 256, kIgMaxTok = 16, kIgStages = 4, kIgMaxSlices = 8;
 constexpr int kIgWeakBytes = 32 * 1024;   // shared memory for a column block's weak values
@@ -719,6 +817,47 @@ cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cud
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s) {
+  if (L.k == 0) return cudaSuccess;
+  const int R = (M + kIwTok - 1) / kIwTok, C = (L.k + kIwCols - 1) / kIwCols;
+  const int nch = (L.N + kIwRows - 1) / kIwRows;
+  // split the rows so that about two CTAs per SM run, at least 4 chunks each
+  int splits = std::max(1, std::min((2 * wct_sm_count(L.device) + R * C - 1) / (R * C), nch / 4));
+  int per = (nch + splits - 1) / splits;
+  splits = (nch + per - 1) / per;
+  per *= kIwRows;
+  float* part = nullptr;
+  if (splits > 1) {
+    const size_t need = (size_t)splits * M * L.k * sizeof(float);
+    bool have = need <= L.wg_ws_bytes;
+    if (!have) {
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone) {
+        cudaFree(L.wg_ws);
+        L.wg_ws = nullptr;
+        L.wg_ws_bytes = 0;
+        if (cudaMalloc(&L.wg_ws, need) == cudaSuccess) {
+          L.wg_ws_bytes = need;
+          have = true;
+        }
+      }
+      cudaGetLastError();
+    }
+    if (have) {
+      part = reinterpret_cast<float*>(L.wg_ws);
+    } else {   // inside a capture without scratch: one split
+      splits = 1;
+      per = nch * kIwRows;
+    }
+  }
+  k_igw_mma<<<dim3(R, C, splits), kIwThreads, 0, s>>>(dy, L.w_weak, L.idx, dx, part, L.N, L.K, M, L.k, L.k_ld, per);
+  if (splits > 1) {
+    const size_t n = (size_t)M * L.k;
+    k_igw_reduce<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, s>>>(part, splits, M, L.k, L.K, L.idx, dx);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace owq
