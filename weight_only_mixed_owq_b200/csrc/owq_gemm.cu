@@ -348,19 +348,32 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
 //               them.  The same warps run the epilogue.
 //   last warp   prep: per step, each row pair's scales and zero points side by side, and (3-bit)
 //               the pair whose bits are spread over a chunk's three words rebuilt as an ordinary
-//               word, so every A thread runs the same eight instructions per row pair.
+//               word, so every A thread runs the same six instructions per row pair.
 // Every mbarrier wait is bounded, as in the prefill kernel.
 // Stage layout: the prefill's (dY boxes, packed block, (s, z) pairs), then what the prep warp
-// derives from them: the 3-bit spread pair of every (row, chunk) rebuilt as an ordinary word
-// (even code at bits 6-8, odd at 22-24) and each row pair's scales and zero points side by side.
+// derives from them.  The prep warp rewrites the packed block in place with the two rows of
+// each row pair interleaved word by word ([64 pairs][4 bits words] of {row 2P, row 2P + 1}),
+// rebuilds the 3-bit pair whose bits are spread over a chunk's three words as an ordinary word
+// pair ([64 pairs][4 chunks], even code at bits 6-8, odd at 22-24) and writes per row pair and
+// offset class {s2, -(1024 2^-o + z2)}.
 template <int BITS, int BN>
 struct IgSmem {
   static constexpr int kX = Smem<BITS, BN>::kX, kP = Smem<BITS, BN>::kP, kSZ = Smem<BITS, BN>::kSZ;
   static constexpr int kTma = kX + kP + kSZ;
-  static constexpr int kAuxD = BITS == 3 ? kBM * 4 * 4 : 0;   // [128 rows][4 chunks] words
-  static constexpr int kAuxS = 64 * 8;                        // [64 row pairs] {s2, z2}
+  static constexpr int kCls = BITS == 3 ? 5 : 2;              // code offsets 0, 3, 6, 1, 4 / 0, 4
+  static constexpr int kAuxD = BITS == 3 ? 64 * 4 * 8 : 0;    // [64 pairs][4 chunks] uint2
+  static constexpr int kAuxS = 64 * kCls * 8;                 // [64 pairs][classes] {s2, nz2}
   static constexpr int kStage = ((kTma + kAuxD + kAuxS) + 1023) & ~1023;
 };
+// class of a code offset (after the byte shift): 3-bit 0, 3, 6, 1, 4 -> 0..4; 4-bit 0, 4 -> 0, 1
+template <int BITS>
+__host__ __device__ constexpr int ig_off_cls(int o) {
+  return BITS == 3 ? (o == 0 ? 0 : o == 3 ? 1 : o == 6 ? 2 : o == 1 ? 3 : 4) : o / 4;
+}
+template <int BITS>
+__host__ __device__ constexpr int ig_cls_off(int c) {
+  return BITS == 3 ? (c == 0 ? 0 : c == 1 ? 3 : c == 2 ? 6 : c == 3 ? 1 : 4) : 4 * c;
+}
 template <int BITS, int BN, int S>
 constexpr int ig_smem_bytes() { return S * IgSmem<BITS, BN>::kStage + 1024 /*barriers*/ + 1024 /*align slack*/; }
 
@@ -376,7 +389,8 @@ struct IgGemmParams {
 template <int BITS, int BN, int S, int DW>
 __global__ void __launch_bounds__(32 * (3 + DW), 1)
 k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant__ CUtensorMap map_p,
-              const __grid_constant__ CUtensorMap map_sz, const __grid_constant__ IgGemmParams p) {
+              const __grid_constant__ CUtensorMap map_sz, const __grid_constant__ CUtensorMap map_dx,
+              const __grid_constant__ IgGemmParams p) {
   using L = IgSmem<BITS, BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -466,21 +480,40 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
       ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);
       if (!ok) break;
       unsigned char* st = smem + s * L::kStage;
-      const uint2* sz = reinterpret_cast<const uint2*>(st + L::kX + L::kP);
-      uint2* aux_s = reinterpret_cast<uint2*>(st + L::kTma + L::kAuxD);
-      #pragma unroll
-      for (int pp = lane; pp < 64; pp += 32) {
-        const uint2 v = sz[pp];
-        aux_s[pp] = make_uint2(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.x, v.y, 0x7632));
-      }
-      if constexpr (BITS == 3) {   // bit e of the spread pair: bit 15 / 31 of word e -> 6 + e / 22 + e
-        uint32_t* aux_d = reinterpret_cast<uint32_t*>(st + L::kTma);
-        #pragma unroll 4
-        for (int e = lane; e < kBM * 4; e += 32) {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(st + L::kX + (e >> 2) * 48 + (e & 3) * 12);
-          aux_d[e] = ((w[0] >> 9) & 0x00400040u) | ((w[1] >> 8) & 0x00800080u) | ((w[2] >> 7) & 0x01000100u);
+      constexpr int W = 4 * BITS;   // words of a row's block
+      #pragma unroll 1
+      for (int P = lane; P < 64; P += 32) {   // one row pair per lane and pass
+        uint32_t a[W], c[W];
+        const uint4* ra = reinterpret_cast<const uint4*>(st + L::kX + (2 * P) * 16 * BITS);
+        #pragma unroll
+        for (int v = 0; v < BITS; ++v) {
+          const uint4 x = ra[v], y = ra[BITS + v];
+          a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
+          c[4 * v] = y.x; c[4 * v + 1] = y.y; c[4 * v + 2] = y.z; c[4 * v + 3] = y.w;
+        }
+        if constexpr (BITS == 3) {   // bit e of the spread pair: bit 15 / 31 of word e -> 6 + e / 22 + e
+          uint2* aux_d = reinterpret_cast<uint2*>(st + L::kTma) + 4 * P;
+          #pragma unroll
+          for (int qc = 0; qc < 4; ++qc) {
+            const uint32_t* x = a + 3 * qc;
+            const uint32_t* y = c + 3 * qc;
+            aux_d[qc] = make_uint2(((x[0] >> 9) & 0x00400040u) | ((x[1] >> 8) & 0x00800080u) | ((x[2] >> 7) & 0x01000100u),
+                                   ((y[0] >> 9) & 0x00400040u) | ((y[1] >> 8) & 0x00800080u) | ((y[2] >> 7) & 0x01000100u));
+          }
+        }
+        uint4* out = reinterpret_cast<uint4*>(st + L::kX + (2 * P) * 16 * BITS);   // the pair's own bytes
+        #pragma unroll
+        for (int v = 0; v < W / 2; ++v) out[v] = make_uint4(a[2 * v], c[2 * v], a[2 * v + 1], c[2 * v + 1]);
+        const uint2 z = reinterpret_cast<const uint2*>(st + L::kX + L::kP)[P];   // (s, z) of rows 2P, 2P + 1
+        const uint32_t s2 = __byte_perm(z.x, z.y, 0x5410), z2 = __byte_perm(z.x, z.y, 0x7632);
+        uint2* aux_s = reinterpret_cast<uint2*>(st + L::kTma + L::kAuxD) + L::kCls * P;
+        #pragma unroll
+        for (int cl = 0; cl < L::kCls; ++cl) {
+          const uint32_t nego = (0x8000u | ((uint32_t)(25 - ig_cls_off<BITS>(cl)) << 10)) * 0x00010001u;   // -2^(10 - o)
+          aux_s[cl] = make_uint2(s2, h2_sub(nego, z2));
         }
       }
+      __syncwarp();
       mbar_arrive(&pfull[s]);
     }
   } else {
@@ -501,12 +534,12 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
     const uint32_t sel = h ? (hi8 ? 0x7733u : 0x7632u) : (hi8 ? 0x5511u : 0x5410u);
     const uint32_t m1 = ((1u << BITS) - 1u) << o2, mask = m1 | (m1 << 16);
     const uint32_t sc = ((uint32_t)(15 - o2) << 10) * 0x00010001u;                // 2^-o
-    const uint32_t nego = (0x8000u | ((uint32_t)(25 - o2) << 10)) * 0x00010001u;  // -2^(10 - o)
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-    // the word holding column j's code in each row: the packed block, or for the spread pair the
-    // prep warp's rebuilt word (then at offset 6, the unshifted half)
-    const int woff = spread ? L::kTma + 4 * q : L::kX + q * 4 * BITS + 4 * sl.word;
-    const int rstride = spread ? 16 : 16 * BITS;
+    // column j's word pair (rows 2P, 2P + 1) in each row pair: the interleaved packed block, or
+    // for the spread pair the prep warp's rebuilt pair (then at offset 6, the unshifted half)
+    const int woff = spread ? L::kTma + 8 * q : L::kX + 8 * (q * BITS + sl.word);
+    const int pstride = spread ? 32 : 32 * BITS;
+    const int cls = ig_off_cls<BITS>(o2);
     bool ok = true;
     for (int i = 0; i < nK && ok; ++i) {
       const int s = i % S, u = i / S;
@@ -514,16 +547,15 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
       if (!ok) break;
       tc_fence_after();
       const unsigned char* st = smem + s * L::kStage;
-      const unsigned char* pk = st + woff + (2 * RP * jh) * rstride;
-      const uint2* szp = reinterpret_cast<const uint2*>(st + L::kTma + L::kAuxD) + RP * jh;
+      const unsigned char* pk = st + woff + (RP * jh) * pstride;
+      const uint2* snp = reinterpret_cast<const uint2*>(st + L::kTma + L::kAuxD) + L::kCls * RP * jh + cls;
       uint32_t d[RP];
       #pragma unroll
       for (int pr = 0; pr < RP; ++pr) {
-        const uint32_t wa = *reinterpret_cast<const uint32_t*>(pk + (2 * pr) * rstride);
-        const uint32_t wb = *reinterpret_cast<const uint32_t*>(pk + (2 * pr + 1) * rstride);
-        const uint32_t v = (__byte_perm(wa, wb, sel) & mask) | 0x64006400u;
-        const uint2 sz = szp[pr];   // {s2, z2} of rows 2 pr, 2 pr + 1 of the slab
-        d[pr] = h2_mul(h2_sub(h2_fma(v, sc, nego), sz.y), sz.x);   // fp16_rn(s (q - z))
+        const uint2 w = *reinterpret_cast<const uint2*>(pk + pr * pstride);
+        const uint32_t v = (__byte_perm(w.x, w.y, sel) & mask) | 0x64006400u;
+        const uint2 sn = snp[L::kCls * pr];   // {s2, -(1024 2^-o + z2)} of the pair
+        d[pr] = h2_mul(h2_fma(v, sc, sn.y), sn.x);   // fp16_rn(s (q - z))
       }
       const uint32_t at = tmem + lane_base + BN + 64 * s + RP * jh;
       #pragma unroll
@@ -535,25 +567,38 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
     }
 
     // ---------------- epilogue ----------------
+    // One split: the fp16 tile goes to shared memory as [BN tokens][128 columns] (the stages are
+    // idle once the accumulator is complete: every load was consumed by an MMA) and out with one
+    // TMA store, which drops the rows past M.  Several splits: fp32 partials straight to the
+    // workspace.
     const bool acc_ok = mbar_wait(accf, 0, p.status, p.wait_limit);
     tc_fence_after();
     const int col = b * kStepCodes + j;
+    __half* s_out = reinterpret_cast<__half*>(smem);
     #pragma unroll 1
     for (int c0 = jh * (BN / NSL); c0 < (jh + 1) * (BN / NSL); c0 += 16) {
       uint32_t v[16];
       tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
       tmem_ld_wait();
-      if (acc_ok) {
-        if (p.ws) {
+      if (p.ws) {
+        if (acc_ok) {
           float* w = p.ws + (size_t)blockIdx.z * p.M * p.K;
           #pragma unroll
           for (int t = 0; t < 16; ++t)
             if (m0 + c0 + t < p.M) w[(size_t)(m0 + c0 + t) * p.K + col] = __uint_as_float(v[t]);
-        } else {
-          #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (m0 + c0 + t < p.M) p.dx[(size_t)(m0 + c0 + t) * p.K + col] = __float2half_rn(__uint_as_float(v[t]));
         }
+      } else {
+        #pragma unroll
+        for (int t = 0; t < 16; ++t) s_out[(c0 + t) * kStepCodes + j] = __float2half_rn(__uint_as_float(v[t]));
+      }
+    }
+    if (!p.ws) {
+      fence_proxy_async_smem();          // the tile, written by the generic proxy, to the TMA
+      named_bar_sync(1, 32 * DW);        // every A thread's part of the tile is written
+      if (warp == 2 && lane == 0 && acc_ok) {
+        tma_store_2d(&map_dx, s_out, b * kStepCodes, m0);
+        bulk_commit();
+        bulk_wait_read0();               // shared memory read out before the CTA may exit
       }
     }
   }
@@ -773,9 +818,11 @@ owq_status_t ig_run(Layer& L, const __half* dy, __half* dx, int M, long long wai
     if (!encode_sz_3d(&L.map_sz, L.sz_t, L.G, L.N)) return OWQ_ERR_CUDA;
     L.maps_ready = true;
   }
-  CUtensorMap mdy;
+  CUtensorMap mdy, mdx;
   if (!encode_2d(&mdy, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dy, (uint64_t)L.N, (uint64_t)M, (uint64_t)L.N * 2, 64, BN,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&mdx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, dx, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, kStepCodes, BN,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return OWQ_ERR_CUDA;
   IgGemmParams prm;
   prm.dx = dx;
@@ -814,7 +861,8 @@ owq_status_t ig_run(Layer& L, const __half* dy, __half* dx, int M, long long wai
     return OWQ_ERR_CUDA;
   }
   dim3 grid(Kb, (M + BN - 1) / BN, splits);
-  kern<<<grid, 32 * (3 + DW), smem, s>>>(mdy, L.map_packed, L.map_sz, prm);
+  static_assert(BN * kStepCodes * 2 <= IgSmem<BITS, BN>::kStage, "output tile in the first stage");
+  kern<<<grid, 32 * (3 + DW), smem, s>>>(mdy, L.map_packed, L.map_sz, mdx, prm);
   if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
   if (splits > 1) {
     const size_t MK = (size_t)M * L.K;
