@@ -488,53 +488,75 @@ def decode_sweep(args, wl, Ms, depth, steps, warmup, local):
             "timing": "CUDA graph of the whole step, CUDA events on the launching stream", "per_M": out}
 
 
-def prefill_measure(args, dev, Ms=None, reps=10):
+def graph_time(calls, replays=5):
+    """Device seconds per call: one CUDA graph of `calls` (zero-argument callables, one library
+    call each, over distinct operand sets), 3 warm-up replays, median of `replays` timed ones."""
+    import torch
+    for c in calls:   # grows the handles' scratch outside the capture
+        c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(replays):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    del g
+    return statistics.median(times) * 1e-3 / len(calls)
+
+
+def cold_copies(per_call_bytes, cap=64):
+    """Operand sets needed so that one pass over them holds more than twice the 126 MB L2."""
+    return int(max(2, min(cap, -(-2 * 126 * 2**20 // max(1, per_call_bytes)))))
+
+
+def prefill_measure(args, dev, Ms=None, reps=5):
     """TFLOP/s of owq_gemm on the LLaMA-13B-shaped prefill layers (13824x5120, 5120x13824,
-    3-bit, g = 128, k = 40 / 108) for the token counts of that workload (or `Ms`), median of
-    `reps` single launches with L2 flushed before each."""
+    3-bit, g = 128, k = 40 / 108) for the token counts of that workload (or `Ms`): one CUDA
+    graph over R packed copies of the pair (more than twice the L2 in all), device time / R."""
     import torch
 
     import weight_only_mixed_owq_b200 as owq
     spec = owq_synth.WORKLOADS[4]
     out = {}
     peaks, kind = measured_peaks()
-    layers = []
+    pair, xs = [], []
     for li, L in enumerate(spec.layers):
         d = owq_synth.draw_layer(L, spec, max(spec.Ms), owq_synth.seed_for(4, li))
         W, X = torch.from_numpy(d["W"]).to(dev), torch.from_numpy(d["X"]).to(dev)
-        lay, _ = owq.quantize_pack(W, X, L.bits, L.group, L.k)
-        layers.append((L, lay, torch.from_numpy(d["x"]).to(dev)))
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        pair.append((L, owq.quantize(W, X, L.bits, L.group, L.k)))
+        xs.append(torch.from_numpy(d["x"]).to(dev))
+        del W, X
+    pair_bytes = sum(L.N * L.K * L.bits // 8 for L, _ in pair)
+    R = cold_copies(pair_bytes, cap=8)
+    layers = [(L, owq.OwqLayer(q["codes"], q["scales"], q["zeros"], q["idx"], q["w_weak"], L.bits, L.group), li)
+              for _ in range(R) for li, (L, q) in enumerate(pair)]
     for M in (Ms or spec.Ms):
-        tot_flop, tot_ms = 0.0, 0.0
-        for L, lay, x in layers:
-            xm = x[:M].contiguous()
-            y = torch.empty((M, L.N), dtype=torch.float16, device=dev)
-            for _ in range(3):
-                lay.gemm(xm, y)
-            times = []
-            for _ in range(reps):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                lay.gemm(xm, y)
-                b.record()
-                torch.cuda.synchronize()
-                times.append(a.elapsed_time(b))
-            t = statistics.median(times)
-            tot_flop += 2.0 * M * L.N * L.K
-            tot_ms += t
-        tf = tot_flop / (tot_ms * 1e-3) / 1e12
+        ys = [torch.empty((M, L.N), dtype=torch.float16, device=dev) for L, _ in pair]
+        xm = [x[:M].contiguous() for x in xs]
+        t = graph_time([lambda lay=lay, li=li: lay.gemm(xm[li], ys[li]) for L, lay, li in layers], replays=reps)
+        t_pair = t * 2   # seconds per call x two layers
+        flop = sum(2.0 * M * L.N * L.K for L, _ in pair)
+        tf = flop / t_pair / 1e12
         out[str(M)] = {"tflops": round(tf, 2), "frac_burst": round(tf / peaks["bf16_tflops"], 4),
-                       "us_per_pair": round(tot_ms * 1e3, 2)}
+                       "us_per_pair": round(t_pair * 1e6, 2)}
     for _, lay, _ in layers:
         lay.close()
     return {"layers": "13824x5120 + 5120x13824, 3-bit g128, k=40/108", "per_M": out,
-            "peak_tflops": peaks["bf16_tflops"], "peak_kind": kind,
-            "timing": f"median of {reps} single launches, L2 flushed between launches"}
+            "peak_tflops": peaks["bf16_tflops"], "peak_kind": kind, "copies": R,
+            "timing": "CUDA graph over R copies of the layer pair (> 2x L2), device time per pair"}
 
 
-def wct_measure(args, dev):
+def wct_measure(args, dev, layers=(0, 4, 5), Ms=(1, 16, 256, 2048), weak=True):
     """Weak column tuning kernels on the OPT-6.7B-shaped layers (3-bit per channel, k = K/128):
     owq_input_grad (dX = dY W_eff from the packed layout; GB/s of its algorithmic bytes: packed +
     scales/zeros + weak block + idx + dY + dX, against the HBM roofline at 1 and 16 tokens, and
@@ -550,46 +572,20 @@ def wct_measure(args, dev):
     import weight_only_mixed_owq_b200 as owq
     spec = owq_synth.WORKLOADS[1]
     peaks, kind = measured_peaks()
-    l2 = 126 * 2**20
-
-    def copies(per_call_bytes, cap=64):
-        return int(max(2, min(cap, -(-2 * l2 // max(1, per_call_bytes)))))
-
-    def graph_time(calls):
-        for c in calls:   # grows the handles' scratch outside the capture
-            c()
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for c in calls:
-                c()
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        times = []
-        for _ in range(5):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            g.replay()
-            b.record()
-            torch.cuda.synchronize()
-            times.append(a.elapsed_time(b))
-        del g
-        return statistics.median(times) * 1e-3 / len(calls)
 
     out = {}
-    for li in (0, 4, 5):   # q (4096 x 4096), fc1 (16384 x 4096), fc2 (4096 x 16384)
+    for li in layers:   # 0: q (4096 x 4096), 4: fc1 (16384 x 4096), 5: fc2 (4096 x 16384)
         L = spec.layers[li]
         d = owq_synth.draw_layer(L, spec, 16, owq_synth.seed_for(1, li))
         W, X = torch.from_numpy(d["W"]).to(dev), torch.from_numpy(d["X"]).to(dev)
         q = owq.quantize(W, X, L.bits, L.group, L.k)
         del W, X
         wbytes = L.N * L.K * L.bits // 8 + L.N * (L.K // L.group) * 4 + L.N * L.k * 2 + 4 * L.k
-        R = copies(wbytes)
+        R = cold_copies(wbytes)
         lays = [owq.OwqLayer(q["codes"], q["scales"], q["zeros"], q["idx"], q["w_weak"], L.bits, L.group)
                 for _ in range(R)]
         row = {}
-        for M in (1, 16, 256, 2048):
+        for M in Ms:
             dy = torch.randn((M, L.N), device=dev).half()
             dx = torch.empty((M, L.K), dtype=torch.float16, device=dev)
             t = graph_time([lambda lay=lay: lay.input_grad(dy, dx) for lay in lays])
@@ -602,9 +598,9 @@ def wct_measure(args, dev):
         for lay in lays[1:]:
             lay.close()
         lay = lays[0]
-        for M in (16, 2048):
+        for M in ((16, 2048) if weak else ()):
             B = 2 * M * L.N + 2 * M * L.k + 4 * L.N * L.k
-            Rw = copies(2 * M * (L.N + L.K), cap=16)
+            Rw = cold_copies(2 * M * (L.N + L.K), cap=16)
             xs = [torch.randn((M, L.K), device=dev).half() for _ in range(Rw)]
             dys = [torch.randn((M, L.N), device=dev).half() for _ in range(Rw)]
             dw = torch.empty((L.N, L.k), dtype=torch.float32, device=dev)
@@ -712,6 +708,8 @@ def main(argv=None):
     ap.add_argument("--no-sweeps", action="store_true", help="skip the LLaMA-7B and OPT-66B decode lines")
     ap.add_argument("--prefill-only", default="", help="comma-separated token counts: time only owq_gemm on "
                     "the LLaMA-13B-shaped layers at those counts (3 launches each) and print that line")
+    ap.add_argument("--input-grad-only", default="", help="comma-separated token counts: time only "
+                    "owq_input_grad on the OPT-6.7B-shaped q layer (4096x4096, 3-bit) and print that line")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
@@ -721,6 +719,14 @@ def main(argv=None):
         if rank == 0:
             Ms = [int(v) for v in args.prefill_only.split(",")]
             print(json.dumps({"prefill": prefill_measure(args, torch.device("cuda", local), Ms, reps=3)}), flush=True)
+        teardown(world)
+        return 0
+    if args.input_grad_only:
+        import torch
+        if rank == 0:
+            Ms = [int(v) for v in args.input_grad_only.split(",")]
+            print(json.dumps({"wct": wct_measure(args, torch.device("cuda", local), layers=(0,), Ms=Ms, weak=False)}),
+                  flush=True)
         teardown(world)
         return 0
     if args.impl == "reference":

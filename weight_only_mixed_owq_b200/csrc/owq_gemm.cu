@@ -242,15 +242,16 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       const uint32_t at = tmem + lane_base + BN + 64 * s + 4 * U * jh;
       uint32_t d[U / 4][16];
       if (i < nD) {
+        const uint32_t sst = smem_u32(st);   // shared address of the stage
         if (per_group) {   // this step's pair, staged with the packed tile ([8 tiles][16 rows])
-          const __half2 sz = *reinterpret_cast<const __half2*>(st + L::kX + L::kP + r * 4);
-          set_sz(__low2half(sz), __high2half(sz));
+          uint32_t szw;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(szw) : "r"(sst + L::kX + L::kP + r * 4) : "memory");
+          set_sz(__ushort_as_half((uint16_t)(szw & 0xFFFFu)), __ushort_as_half((uint16_t)(szw >> 16)));
         }
-        const uint4* pw = reinterpret_cast<const uint4*>(st + L::kX + r * 16 * BITS);
         uint32_t w[4 * BITS];
         #pragma unroll
         for (int v = 0; v < BITS; ++v) {
-          const uint4 q = pw[v];
+          const uint4 q = lds_u4(sst + L::kX + r * 16 * BITS + 16 * v);
           w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
         }
         // the slab is uniform per warp: each branch sees compile-time pair indices.  The weak
@@ -479,38 +480,39 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
       const int s = i % S, u = i / S;
       ok = mbar_wait(&full[s], u & 1, p.status, p.wait_limit);
       if (!ok) break;
-      unsigned char* st = smem + s * L::kStage;
+      const uint32_t st = smem_u32(smem) + s * L::kStage;   // shared address of the stage
       constexpr int W = 4 * BITS;   // words of a row's block
       #pragma unroll 1
       for (int P = lane; P < 64; P += 32) {   // one row pair per lane and pass
         uint32_t a[W], c[W];
-        const uint4* ra = reinterpret_cast<const uint4*>(st + L::kX + (2 * P) * 16 * BITS);
+        const uint32_t ra = st + L::kX + (2 * P) * 16 * BITS;
         #pragma unroll
         for (int v = 0; v < BITS; ++v) {
-          const uint4 x = ra[v], y = ra[BITS + v];
+          const uint4 x = lds_u4(ra + 16 * v), y = lds_u4(ra + 16 * (BITS + v));
           a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
           c[4 * v] = y.x; c[4 * v + 1] = y.y; c[4 * v + 2] = y.z; c[4 * v + 3] = y.w;
         }
         if constexpr (BITS == 3) {   // bit e of the spread pair: bit 15 / 31 of word e -> 6 + e / 22 + e
-          uint2* aux_d = reinterpret_cast<uint2*>(st + L::kTma) + 4 * P;
+          const uint32_t aux_d = st + L::kTma + 32 * P;
           #pragma unroll
           for (int qc = 0; qc < 4; ++qc) {
             const uint32_t* x = a + 3 * qc;
             const uint32_t* y = c + 3 * qc;
-            aux_d[qc] = make_uint2(((x[0] >> 9) & 0x00400040u) | ((x[1] >> 8) & 0x00800080u) | ((x[2] >> 7) & 0x01000100u),
-                                   ((y[0] >> 9) & 0x00400040u) | ((y[1] >> 8) & 0x00800080u) | ((y[2] >> 7) & 0x01000100u));
+            sts_u2(aux_d + 8 * qc,
+                   make_uint2(((x[0] >> 9) & 0x00400040u) | ((x[1] >> 8) & 0x00800080u) | ((x[2] >> 7) & 0x01000100u),
+                              ((y[0] >> 9) & 0x00400040u) | ((y[1] >> 8) & 0x00800080u) | ((y[2] >> 7) & 0x01000100u)));
           }
         }
-        uint4* out = reinterpret_cast<uint4*>(st + L::kX + (2 * P) * 16 * BITS);   // the pair's own bytes
         #pragma unroll
-        for (int v = 0; v < W / 2; ++v) out[v] = make_uint4(a[2 * v], c[2 * v], a[2 * v + 1], c[2 * v + 1]);
-        const uint2 z = reinterpret_cast<const uint2*>(st + L::kX + L::kP)[P];   // (s, z) of rows 2P, 2P + 1
+        for (int v = 0; v < W / 2; ++v)   // the pair's own bytes, rows interleaved word by word
+          sts_u4(ra + 16 * v, make_uint4(a[2 * v], c[2 * v], a[2 * v + 1], c[2 * v + 1]));
+        const uint2 z = lds_u2(st + L::kX + L::kP + 8 * P);   // (s, z) of rows 2P, 2P + 1
         const uint32_t s2 = __byte_perm(z.x, z.y, 0x5410), z2 = __byte_perm(z.x, z.y, 0x7632);
-        uint2* aux_s = reinterpret_cast<uint2*>(st + L::kTma + L::kAuxD) + L::kCls * P;
+        const uint32_t aux_s = st + L::kTma + L::kAuxD + 8 * L::kCls * P;
         #pragma unroll
         for (int cl = 0; cl < L::kCls; ++cl) {
           const uint32_t nego = (0x8000u | ((uint32_t)(25 - ig_cls_off<BITS>(cl)) << 10)) * 0x00010001u;   // -2^(10 - o)
-          aux_s[cl] = make_uint2(s2, h2_sub(nego, z2));
+          sts_u2(aux_s + 8 * cl, make_uint2(s2, h2_sub(nego, z2)));
         }
       }
       __syncwarp();
@@ -546,15 +548,15 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
       ok = mbar_wait(&pfull[s], u & 1, p.status, p.wait_limit);   // (implies the TMA landed)
       if (!ok) break;
       tc_fence_after();
-      const unsigned char* st = smem + s * L::kStage;
-      const unsigned char* pk = st + woff + (RP * jh) * pstride;
-      const uint2* snp = reinterpret_cast<const uint2*>(st + L::kTma + L::kAuxD) + L::kCls * RP * jh + cls;
+      const uint32_t st = smem_u32(smem) + s * L::kStage;   // shared address of the stage
+      const uint32_t pk = st + woff + (RP * jh) * pstride;
+      const uint32_t snp = st + L::kTma + L::kAuxD + 8 * (L::kCls * RP * jh + cls);
       uint32_t d[RP];
       #pragma unroll
       for (int pr = 0; pr < RP; ++pr) {
-        const uint2 w = *reinterpret_cast<const uint2*>(pk + pr * pstride);
+        const uint2 w = lds_u2(pk + pr * pstride);
         const uint32_t v = (__byte_perm(w.x, w.y, sel) & mask) | 0x64006400u;
-        const uint2 sn = snp[L::kCls * pr];   // {s2, -(1024 2^-o + z2)} of the pair
+        const uint2 sn = lds_u2(snp + 8 * L::kCls * pr);   // {s2, -(1024 2^-o + z2)} of the pair
         d[pr] = h2_mul(h2_fma(v, sc, sn.y), sn.x);   // fp16_rn(s (q - z))
       }
       const uint32_t at = tmem + lane_base + BN + 64 * s + RP * jh;
@@ -589,7 +591,8 @@ k_igemm_sm100(const __grid_constant__ CUtensorMap map_dy, const __grid_constant_
         }
       } else {
         #pragma unroll
-        for (int t = 0; t < 16; ++t) s_out[(c0 + t) * kStepCodes + j] = __float2half_rn(__uint_as_float(v[t]));
+        for (int t = 0; t < 16; ++t)
+          sts_u16(smem_u32(s_out) + 2 * ((c0 + t) * kStepCodes + j), __half_as_ushort(__float2half_rn(__uint_as_float(v[t]))));
       }
     }
     if (!p.ws) {
