@@ -52,11 +52,13 @@ typedef int owq_status_t;
 #define OWQ_ERR_HANDLE    10  /* the layer handle is NULL or not one this library made         */
 #define OWQ_ERR_DEVICE    11  /* no CUDA device, or the device is not sm_100                   */
 #define OWQ_ERR_ARG       12  /* an argument outside its documented set (owq_debug_inject)      */
+#define OWQ_ERR_BOUNDS    13  /* debug-bounds build: a device index check failed (owq_device_status) */
 
 /* Failures owq_debug_inject can arm. */
 #define OWQ_INJECT_NONE         0
 #define OWQ_INJECT_GEMV_TAG     1
 #define OWQ_INJECT_GEMM_ARRIVE  2
+#define OWQ_INJECT_BOUNDS       3
 
 /* Opaque handle of one packed layer; owns the device buffers owq_pack allocated. */
 typedef struct owq_layer_s* owq_layer_t;
@@ -373,7 +375,12 @@ owq_status_t owq_layer_free(owq_layer_t layer);
 
 /* Synchronises the current device (cudaDeviceSynchronize), then returns and clears its device
  * status word (OWQ_OK, or OWQ_ERR_TIMEOUT if a bounded wait of any call on this device gave up
- * since the last query).  The word is per device, not per handle: a bounded wait gives up
+ * since the last query, or OWQ_ERR_BOUNDS, first, if a check of the debug-bounds build failed).
+ * The debug-bounds build (libowq_b200_bounds.so, compiled with -DOWQ_DEBUG_BOUNDS; owq_version
+ * ends in "+debug-bounds") checks the kernels' data-dependent indices before each access -- the
+ * weak index list in every gather and scatter, the storage stream positions -- and skips an
+ * access that fails (writing 0 or nothing), so an indexing fault reports here instead of
+ * faulting the GPU.  The default build compiles the checks out.  The word is per device, not per handle: a bounded wait gives up
  * inside a kernel, which has no way to name the handle of the call that launched it, and the
  * kernels of every handle on a device write the same word.  The whole device is synchronised
  * because the failed call may sit on any stream; call this between steps, not on a hot path. */
@@ -393,6 +400,12 @@ owq_status_t owq_device_status(void);
  * bound is 4e9 cycles, about 2 s).  The kernel records the timeout in the device status
  * word, leaves y undefined, lets its own bulk copies land, frees its tensor memory and
  * returns: the next owq_device_status returns OWQ_ERR_TIMEOUT and the context stays usable.
+ *   OWQ_INJECT_BOUNDS       debug-bounds build only (OWQ_ERR_ARG otherwise; wait_cycles ignored):
+ *                           the next owq_input_grad that takes the many-token path on a handle
+ *                           with weak columns stores token 0 of weak slot 0 one row of K past
+ *                           its column; the bounds check skips that store and the next
+ *                           owq_device_status returns OWQ_ERR_BOUNDS (dx[0][idx[0]] is then
+ *                           undefined, every other output as without the injection).
  * OWQ_INJECT_NONE disarms (wait_cycles ignored).  Errors: OWQ_ERR_ARG for an unknown `what`
  * or wait_cycles < 1.
  */

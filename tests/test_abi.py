@@ -44,6 +44,21 @@ def test_library_exports_every_declared_symbol(owq):
     assert {p[0] for p in owq.PROTOTYPES} == set(_declared_functions())
 
 
+def test_debug_bounds_variant_exports_every_declared_symbol(owq):
+    """The debug-bounds build (built by __graft_entry__.build()) exports the same boundary and
+    names itself in owq_version; OWQ_INJECT_BOUNDS is refused by the default build."""
+    from weight_only_mixed_owq_b200 import build
+    path = build.LIB_BOUNDS
+    if not os.path.exists(path):
+        pytest.skip("debug-bounds variant not built (python -m weight_only_mixed_owq_b200.build --debug-bounds)")
+    lib = ctypes.CDLL(path)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    lib.owq_version.restype = ctypes.c_char_p
+    assert lib.owq_version().decode().endswith("+debug-bounds")
+    assert owq.owq_debug_inject(owq.OWQ_INJECT_BOUNDS, 1) == 12   # OWQ_ERR_ARG in the default build
+
+
 def test_status_strings_and_version(owq):
     for code, name in owq.STATUS_NAMES.items():
         assert owq.owq_status_string(code).startswith(name)

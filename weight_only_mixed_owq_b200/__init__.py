@@ -8,7 +8,7 @@ script, `weight_only_mixed_owq_b200.build`, imports without the library.
 import importlib
 
 _EXPORTS = (
-    "LIB", "LIB_PATH", "OWQ_OK", "OWQ_INJECT_NONE", "OWQ_INJECT_GEMV_TAG", "OWQ_INJECT_GEMM_ARRIVE",
+    "LIB", "LIB_PATH", "OWQ_OK", "OWQ_INJECT_NONE", "OWQ_INJECT_GEMV_TAG", "OWQ_INJECT_GEMM_ARRIVE", "OWQ_INJECT_BOUNDS",
     "OwqError", "OwqLayer", "PROTOTYPES", "STATUS_NAMES",
     "owq_debug_inject", "owq_dequant", "owq_device_status", "owq_gemm", "owq_gemv", "owq_gemv_multi", "owq_input_grad", "owq_layer_bytes",
     "owq_layer_free", "owq_layer_info", "owq_pack", "owq_pack_storage", "owq_quantize", "owq_quantize_noalloc", "owq_quantize_optq",

@@ -10,15 +10,20 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libowq_b200.so")
+# OWQ_LIB_VARIANT=bounds loads the debug-bounds build (libowq_b200_bounds.so) built beside it
+VARIANTS = {"": "libowq_b200.so", "bounds": "libowq_b200_bounds.so"}
+_variant = os.environ.get("OWQ_LIB_VARIANT", "")
+if _variant not in VARIANTS:
+    raise ImportError(f"OWQ_LIB_VARIANT={_variant!r}: expected one of {sorted(VARIANTS)}")
+LIB_PATH = os.path.join(PKG, VARIANTS[_variant])
 
 OWQ_OK = 0
 STATUS_NAMES = {
     0: "OWQ_OK", 1: "OWQ_ERR_NULL", 2: "OWQ_ERR_SHAPE", 3: "OWQ_ERR_BITS", 4: "OWQ_ERR_GROUP",
     5: "OWQ_ERR_INDEX", 6: "OWQ_ERR_ALIGN", 7: "OWQ_ERR_CUDA", 8: "OWQ_ERR_TIMEOUT",
-    9: "OWQ_ERR_NOMEM", 10: "OWQ_ERR_HANDLE", 11: "OWQ_ERR_DEVICE", 12: "OWQ_ERR_ARG",
+    9: "OWQ_ERR_NOMEM", 10: "OWQ_ERR_HANDLE", 11: "OWQ_ERR_DEVICE", 12: "OWQ_ERR_ARG", 13: "OWQ_ERR_BOUNDS",
 }
-OWQ_INJECT_NONE, OWQ_INJECT_GEMV_TAG, OWQ_INJECT_GEMM_ARRIVE = 0, 1, 2
+OWQ_INJECT_NONE, OWQ_INJECT_GEMV_TAG, OWQ_INJECT_GEMM_ARRIVE, OWQ_INJECT_BOUNDS = 0, 1, 2, 3
 
 # (name, restype, argtypes) of every exported symbol of include/owq.h
 _P, _I, _SZ, _S = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t), ctypes.c_char_p

@@ -116,11 +116,12 @@ const char* owq_status_string(owq_status_t s) {
     case OWQ_ERR_HANDLE: return "OWQ_ERR_HANDLE: not a live layer handle";
     case OWQ_ERR_DEVICE: return "OWQ_ERR_DEVICE: no sm_100 CUDA device";
     case OWQ_ERR_ARG: return "OWQ_ERR_ARG: argument outside its documented set";
+    case OWQ_ERR_BOUNDS: return "OWQ_ERR_BOUNDS: a debug-bounds index check failed on the device";
     default: return "OWQ: unknown status";
   }
 }
 
-const char* owq_version(void) { return "0.1.0"; }
+const char* owq_version(void) { return kDebugBounds ? "0.1.0+debug-bounds" : "0.1.0"; }
 
 owq_status_t owq_quantize(const uint16_t* W, const uint16_t* X, int N, int K, int T, int bits,
                           int group, int k, uint8_t* codes, uint16_t* scales, uint16_t* zeros,
@@ -383,6 +384,11 @@ static bool take_inject(int what, long long* wait_limit) {
 
 owq_status_t owq_debug_inject(int what, long long wait_cycles) {
   if (what == OWQ_INJECT_NONE) { g_inject = what; return OWQ_OK; }
+  if (what == OWQ_INJECT_BOUNDS) {   // the debug-bounds build only
+    if (!kDebugBounds) return OWQ_ERR_ARG;
+    g_inject = what;
+    return OWQ_OK;
+  }
   if ((what != OWQ_INJECT_GEMV_TAG && what != OWQ_INJECT_GEMM_ARRIVE) || wait_cycles < 1) return OWQ_ERR_ARG;
   g_inject = what;
   g_inject_wait = wait_cycles;
@@ -479,7 +485,9 @@ owq_status_t owq_input_grad(owq_layer_t layer, const uint16_t* dy, uint16_t* dx,
   if (M > kIgGemmMinM && L->N % 8 == 0) {   // dY rows must be 16-byte strided for its tensor map
     const owq_status_t st = igemm_sm100(*L, dyh, dxh, M, kDefaultWaitLimit, s);
     if (st) return st;
-    return cuda_status(launch_input_grad_weak(*L, dyh, dxh, M, s));
+    long long wl;
+    const bool inject = L->k > 0 && take_inject(OWQ_INJECT_BOUNDS, &wl);
+    return cuda_status(launch_input_grad_weak(*L, dyh, dxh, M, inject, s));
   }
   return cuda_status(launch_input_grad(*L, dyh, dxh, M, s));
 }
@@ -534,7 +542,7 @@ owq_status_t owq_device_status(void) {
   if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_CUDA; }
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return OWQ_ERR_CUDA; }
-  return v ? OWQ_ERR_TIMEOUT : OWQ_OK;
+  return (v & kStatusBounds) ? OWQ_ERR_BOUNDS : v ? OWQ_ERR_TIMEOUT : OWQ_OK;
 }
 
 }  // extern "C"

@@ -404,7 +404,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
         #pragma unroll
         for (int it = 0; it < 2; ++it) {
           const int e = it * blockDim.x + threadIdx.x;
-          gx[it] = gidx[it] >= 0 ? Pb.x[(size_t)(e / k_ld) * K + gidx[it]] : __float2half_rn(0.f);
+          gx[it] = gidx[it] >= 0 && in_range(gidx[it], K, args.status) ? Pb.x[(size_t)(e / k_ld) * K + gidx[it]]
+                                                                         : __float2half_rn(0.f);
         }
         if (lane == 0)
           for (int j = 1; j < ahead; ++j)
@@ -448,7 +449,8 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     #pragma unroll 1
     for (int e = 2 * blockDim.x + threadIdx.x; e < MT * k_ld; e += blockDim.x) {
       const int m = e / k_ld, t = e - m * k_ld;
-      xw[e] = (m < M && t < k) ? Pb.x[(size_t)m * K + Pb.idx[t]] : __float2half_rn(0.f);
+      xw[e] = (m < M && t < k && in_range(Pb.idx[t], K, args.status)) ? Pb.x[(size_t)m * K + Pb.idx[t]]
+                                                                       : __float2half_rn(0.f);
     }
   } else {
     // activations stay in global memory (fragment-ordered by k_x_frag): per-block sums (for
@@ -486,7 +488,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
     for (int e = threadIdx.x; e < MT * k_ld; e += blockDim.x) {
       const int m = e / k_ld, t = e - m * k_ld;
       const int col = e < (int)blockDim.x ? gidx[0] : e < 2 * (int)blockDim.x ? gidx[1] : ((m < M && t < k) ? Pb.idx[t] : -1);
-      xw[e] = col >= 0 ? Pb.x[(size_t)m * K + col] : __float2half_rn(0.f);
+      xw[e] = col >= 0 && in_range(col, K, args.status) ? Pb.x[(size_t)m * K + col] : __float2half_rn(0.f);
     }
   }
   __syncthreads();
@@ -731,7 +733,7 @@ k_gemv_mma(const __grid_constant__ GemvArgs args) {
                 for (int i = 0; i < 4; ++i) {
                   while ((uint32_t)(w[nt][i] >> 32) != Pb.epoch) {
                     if (clock64() - t_start > args.wait_limit) {
-                      atomicExch(args.status, 1);
+                      atomicOr(args.status, 1);
                       good = false;
                       break;
                     }

@@ -51,8 +51,30 @@ struct Layer {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Device status word set by bounded waits (owq_device_status reads and clears it).
+// Device status word (owq_device_status reads and clears it): bit 0 a bounded wait gave up,
+// bit 1 a debug-bounds check failed.
 int* device_status_ptr();
+constexpr int kStatusTimeout = 1, kStatusBounds = 2;
+
+// Debug-bounds build (-DOWQ_DEBUG_BOUNDS): the kernels check their data-dependent indices (the
+// weak index list and the positions derived from it) before an access; a failed check sets
+// kStatusBounds in the status word and the access is skipped, so an indexing fault reports as
+// OWQ_ERR_BOUNDS instead of faulting.  In the default build in_range is constant true.
+#ifdef OWQ_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool in_range(long long i, long long n, int* status) {
+  if constexpr (kDebugBounds) {
+    if (i >= 0 && i < n) return true;
+    if (status) atomicOr(status, kStatusBounds);
+    return false;
+  } else {
+    (void)i; (void)n; (void)status;
+    return true;
+  }
+}
 // Bound of a device wait when no test shortens it: about 2 s at the B200's clock.
 constexpr long long kDefaultWaitLimit = 4000000000LL;
 
@@ -135,7 +157,9 @@ cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cud
 // exactly 0), then the weak columns dx[:, idx] = dY W_weak (overwritten)
 constexpr int kIgGemmMinM = 32;   // the tensor-memory pipeline from this many tokens (N % 8 == 0)
 owq_status_t igemm_sm100(Layer& L, const __half* dy, __half* dx, int M, long long wait_limit, cudaStream_t s);
-cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s);
+// inject (debug-bounds build tests): token 0 of slot 0 is stored one row of K too far, which
+// the bounds check must catch
+cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, bool inject, cudaStream_t s);
 
 // skip_arrive: a test-injected lost arrival (one dequantisation thread per CTA skips its first
 // arrival), so that the bounded waits run out

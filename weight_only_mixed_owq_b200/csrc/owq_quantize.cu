@@ -179,11 +179,11 @@ __global__ void k_codes(const __half* __restrict__ W, int N, int K, int group, i
 }
 
 __global__ void k_gather_weak(const __half* __restrict__ W, int N, int K,
-                              const int32_t* __restrict__ idx, int k, __half* __restrict__ w_weak) {
+                              const int32_t* __restrict__ idx, int k, __half* __restrict__ w_weak, int* status) {
   size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= (size_t)N * k) return;
   int i = (int)(e / k), t = (int)(e % k);
-  w_weak[e] = W[(size_t)i * K + idx[t]];
+  w_weak[e] = in_range(idx[t], K, status) ? W[(size_t)i * K + idx[t]] : __float2half_rn(0.f);
 }
 
 }  // namespace
@@ -212,7 +212,7 @@ cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int 
   k_codes<<<(unsigned)((NK + 255) / 256), 256, 0, s>>>(W, N, K, group, bits, scales, zeros, mask, codes);
   if (k > 0) {
     const size_t Nk = (size_t)N * k;
-    k_gather_weak<<<(unsigned)((Nk + 255) / 256), 256, 0, s>>>(W, N, K, idx, k, w_weak);
+    k_gather_weak<<<(unsigned)((Nk + 255) / 256), 256, 0, s>>>(W, N, K, idx, k, w_weak, device_status_ptr());
   }
   e = cudaGetLastError();
   cudaError_t e2 = cudaFreeAsync(buf, s);
@@ -292,7 +292,7 @@ cudaError_t launch_quantize_static(const __half* W, const __half* X, int N, int 
   k_codes<<<(unsigned)((NK + 255) / 256), 256, 0, s>>>(W, N, K, group, bits, scales, zeros, mask, codes);
   if (k > 0) {
     const size_t Nk = (size_t)N * k;
-    k_gather_weak<<<(unsigned)((Nk + 255) / 256), 256, 0, s>>>(W, N, K, idx, k, w_weak);
+    k_gather_weak<<<(unsigned)((Nk + 255) / 256), 256, 0, s>>>(W, N, K, idx, k, w_weak, device_status_ptr());
   }
   return cudaGetLastError();
 }

@@ -40,7 +40,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (clock64() - t0 > limit) {
-      atomicExch(status, 1);
+      atomicOr(status, 1);   // bit 0: a bounded wait gave up
       return false;
     }
   }

@@ -52,7 +52,8 @@ __device__ __forceinline__ bool is_weak(const int* idx, int k, int j) {
 // grid (ceil(Ws / 256), rows): thread = one word w of the stream, for rows blockIdx.y,
 // blockIdx.y + gridDim.y, ...
 __global__ void k_storage_pack(const uint8_t* __restrict__ codes, int N, int K, int bits,
-                               const int32_t* __restrict__ idx_g, int k, int Ws, uint32_t* __restrict__ words) {
+                               const int32_t* __restrict__ idx_g, int k, int Ws, uint32_t* __restrict__ words,
+                               int* status) {
   __shared__ int idx[kMaxWeak];
   for (int t = threadIdx.x; t < k; t += blockDim.x) idx[t] = idx_g[t];
   __syncthreads();
@@ -68,7 +69,7 @@ __global__ void k_storage_pack(const uint8_t* __restrict__ codes, int N, int K, 
     uint32_t out = 0u;
     int j = j0;
     for (int p = p0; p < p_end; ++p) {
-      const uint32_t v = c[j];
+      const uint32_t v = in_range(j, K, status) ? c[j] : 0u;   // the p-th dense column
       const long long o = (long long)p * bits - b0;   // bit offset of code p in this word (may be < 0)
       out |= o >= 0 ? (v << o) : (v >> -o);
       ++j;                                            // the next dense column
@@ -82,7 +83,7 @@ __global__ void k_storage_pack(const uint8_t* __restrict__ codes, int N, int K, 
 // gridDim.y, ...
 __global__ void k_storage_unpack(const uint32_t* __restrict__ words, int N, int K, int bits, int group,
                                  const int32_t* __restrict__ idx_g, int k, int Ws,
-                                 const __half* __restrict__ zeros, uint8_t* __restrict__ codes) {
+                                 const __half* __restrict__ zeros, uint8_t* __restrict__ codes, int* status) {
   __shared__ int idx[kMaxWeak];
   for (int t = threadIdx.x; t < k; t += blockDim.x) idx[t] = idx_g[t];
   __syncthreads();
@@ -100,8 +101,8 @@ __global__ void k_storage_unpack(const uint32_t* __restrict__ words, int N, int 
       v = (uint32_t)__half2float(zeros[(size_t)row * G + j / group]);
     } else {
       const uint32_t* r = words + (size_t)row * Ws;
-      v = r[w] >> o;
-      if (o + bits > 32) v |= r[w + 1] << (32 - o);
+      v = in_range(w, Ws, status) ? r[w] >> o : 0u;   // the column's position in the dense stream
+      if (o + bits > 32 && in_range(w + 1, Ws, status)) v |= r[w + 1] << (32 - o);
       v &= (1u << bits) - 1u;
     }
     codes[(size_t)row * K + j] = (uint8_t)v;
@@ -117,7 +118,7 @@ cudaError_t launch_storage_pack(const uint8_t* codes, int N, int K, int bits, co
   const int Ws = storage_words_per_row(K, bits, k);
   if (Ws == 0) return cudaSuccess;
   dim3 grid((Ws + kStoreThreads - 1) / kStoreThreads, std::min(N, 65535));
-  k_storage_pack<<<grid, kStoreThreads, 0, s>>>(codes, N, K, bits, idx, k, Ws, words);
+  k_storage_pack<<<grid, kStoreThreads, 0, s>>>(codes, N, K, bits, idx, k, Ws, words, device_status_ptr());
   return cudaGetLastError();
 }
 
@@ -125,7 +126,8 @@ cudaError_t launch_storage_unpack(const uint32_t* words, int N, int K, int bits,
                                   int k, const __half* zeros, uint8_t* codes, cudaStream_t s) {
   const int Ws = storage_words_per_row(K, bits, k);
   dim3 grid((K + kStoreThreads - 1) / kStoreThreads, std::min(N, 65535));
-  k_storage_unpack<<<grid, kStoreThreads, 0, s>>>(words, N, K, bits, group, idx, k, Ws, zeros, codes);
+  k_storage_unpack<<<grid, kStoreThreads, 0, s>>>(words, N, K, bits, group, idx, k, Ws, zeros, codes,
+                                                 device_status_ptr());
   return cudaGetLastError();
 }
 

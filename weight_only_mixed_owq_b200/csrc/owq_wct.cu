@@ -23,7 +23,7 @@ constexpr int kWgRows = 32, kWgCols = 32, kWgTok = 32, kWgThreads = 256;
 
 __global__ void __launch_bounds__(kWgThreads)
 k_weak_grad(const __half* __restrict__ x, const __half* __restrict__ dy,
-            const int32_t* __restrict__ idx, float* __restrict__ dw, int N, int K, int k, int M) {
+            const int32_t* __restrict__ idx, float* __restrict__ dw, int N, int K, int k, int M, int* status) {
   __shared__ float s_dy[kWgTok][kWgRows];
   __shared__ float s_xw[kWgTok][kWgCols];
   __shared__ int s_idx[kWgCols];
@@ -39,7 +39,7 @@ k_weak_grad(const __half* __restrict__ x, const __half* __restrict__ dy,
       const int mm = m0 + m, row = i0 + r;
       s_dy[m][r] = (mm < M && row < N) ? __half2float(dy[(size_t)mm * N + row]) : 0.f;
       const int col = s_idx[r];   // r doubles as the weak-column slot (kWgRows == kWgCols)
-      s_xw[m][r] = (mm < M && col >= 0) ? __half2float(x[(size_t)mm * K + col]) : 0.f;
+      s_xw[m][r] = (mm < M && col >= 0 && in_range(col, K, status)) ? __half2float(x[(size_t)mm * K + col]) : 0.f;
     }
     __syncthreads();
     #pragma unroll 8
@@ -90,12 +90,12 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 
 // xw[m][t] = x[m][idx[t]] for t < k, 0 for k <= t < kp
 __global__ void k_wg_gather(const __half* __restrict__ x, int M, int K, const int32_t* __restrict__ idx, int k,
-                            int kp, __half* __restrict__ xw) {
+                            int kp, __half* __restrict__ xw, int* status) {
   const size_t n = (size_t)M * kp;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
     const size_t m = e / kp;
     const int t = (int)(e % kp);
-    xw[e] = t < k ? x[m * K + idx[t]] : __float2half_rn(0.f);
+    xw[e] = t < k && in_range(idx[t], K, status) ? x[m * K + idx[t]] : __float2half_rn(0.f);
   }
 }
 
@@ -197,7 +197,8 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
 // grid (M / 64, k_ld / 32, row splits of `per` rows, a multiple of 32); N % 8 == 0
 __global__ void __launch_bounds__(kIwThreads)
 k_igw_mma(const __half* __restrict__ dy, const __half* __restrict__ w, const int32_t* __restrict__ idx,
-          __half* __restrict__ dx, float* __restrict__ part, int N, int K, int M, int k, int k_ld, int per) {
+          __half* __restrict__ dx, float* __restrict__ part, int N, int K, int M, int k, int k_ld, int per,
+          int* status, int inject) {
   __shared__ __align__(128) __half s_dy[kIwStages][kIwTok][kIwDyLd];
   __shared__ __align__(128) __half s_w[kIwStages][kIwRows][kIwWLd];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -258,20 +259,26 @@ k_igw_mma(const __half* __restrict__ dy, const __half* __restrict__ w, const int
     for (int i = 0; i < 4; ++i) {
       const int m = mb + warp * 16 + g + 8 * (i >> 1), t = t0 + n * 8 + 2 * c4 + (i & 1);
       if (m < M && t < k) {
-        if (part) part[((size_t)blockIdx.z * M + m) * k + t] = d[n][i];
-        else dx[(size_t)m * K + idx[t]] = __float2half_rn(d[n][i]);
+        if (part) {
+          part[((size_t)blockIdx.z * M + m) * k + t] = d[n][i];
+        } else {
+          // (inject: the debug-bounds test's planted index, token 0 of slot 0 one row of K too far)
+          const int col = idx[t] + (kDebugBounds && inject && m == 0 && t == 0 ? K : 0);
+          if (in_range(col, K, status)) dx[(size_t)m * K + col] = __float2half_rn(d[n][i]);
+        }
       }
     }
 }
 
 // dx[m][idx[t]] = fp16 of the sum of the splits' partials, in split order
 __global__ void k_igw_reduce(const float* __restrict__ part, int splits, int M, int k, int K,
-                             const int32_t* __restrict__ idx, __half* __restrict__ dx) {
+                             const int32_t* __restrict__ idx, __half* __restrict__ dx, int* status, int inject) {
   const size_t n = (size_t)M * k;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
     float v = part[e];
     for (int z = 1; z < splits; ++z) v += part[(size_t)z * n + e];
-    dx[(e / k) * K + idx[e % k]] = __float2half_rn(v);
+    const int col = idx[e % k] + (kDebugBounds && inject && e == 0 ? K : 0);
+    if (in_range(col, K, status)) dx[(e / k) * K + col] = __float2half_rn(v);
   }
 }
 
@@ -769,13 +776,14 @@ cudaError_t launch_weak_grad(const Layer& L, const __half* x, const __half* dy, 
   }
   if (!mma) {
     const dim3 grid((L.N + kWgRows - 1) / kWgRows, (L.k + kWgCols - 1) / kWgCols);
-    k_weak_grad<<<grid, kWgThreads, 0, s>>>(x, dy, L.idx, dw, L.N, L.K, L.k, M);
+    k_weak_grad<<<grid, kWgThreads, 0, s>>>(x, dy, L.idx, dw, L.N, L.K, L.k, M, device_status_ptr());
     return cudaGetLastError();
   }
   __half* xw = reinterpret_cast<__half*>(L.wg_ws);
   float* part = splits > 1 ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(L.wg_ws) + xw_bytes) : nullptr;
   const size_t nxw = (size_t)M * kp;
-  k_wg_gather<<<(unsigned)std::min<size_t>((nxw + 255) / 256, 4096), 256, 0, s>>>(x, M, L.K, L.idx, L.k, kp, xw);
+  k_wg_gather<<<(unsigned)std::min<size_t>((nxw + 255) / 256, 4096), 256, 0, s>>>(x, M, L.K, L.idx, L.k, kp, xw,
+                                                                                       device_status_ptr());
   k_weak_grad_mma<<<dim3(R, C, splits), kWmThreads, 0, s>>>(dy, xw, splits > 1 ? part : dw, L.N, L.k, kp, M, per);
   if (splits > 1) {
     const size_t n = (size_t)L.N * L.k;
@@ -819,7 +827,7 @@ cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cud
   return cudaSuccess;
 }
 
-cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, cudaStream_t s) {
+cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, bool inject, cudaStream_t s) {
   if (L.k == 0) return cudaSuccess;
   const int R = (M + kIwTok - 1) / kIwTok, C = (L.k + kIwCols - 1) / kIwCols;
   const int nch = (L.N + kIwRows - 1) / kIwRows;
@@ -852,10 +860,13 @@ cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M
       per = nch * kIwRows;
     }
   }
-  k_igw_mma<<<dim3(R, C, splits), kIwThreads, 0, s>>>(dy, L.w_weak, L.idx, dx, part, L.N, L.K, M, L.k, L.k_ld, per);
+  int* status = device_status_ptr();
+  k_igw_mma<<<dim3(R, C, splits), kIwThreads, 0, s>>>(dy, L.w_weak, L.idx, dx, part, L.N, L.K, M, L.k, L.k_ld, per,
+                                                      status, inject ? 1 : 0);
   if (splits > 1) {
     const size_t n = (size_t)M * L.k;
-    k_igw_reduce<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, s>>>(part, splits, M, L.k, L.K, L.idx, dx);
+    k_igw_reduce<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, s>>>(part, splits, M, L.k, L.K, L.idx, dx,
+                                                                                          status, inject ? 1 : 0);
   }
   return cudaGetLastError();
 }
