@@ -331,13 +331,13 @@ owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t*
  * W_eff = the dequantised matrix except at the weak columns, which take their fp16 values from
  * the weak block.  Read straight from the packed layout (no W_hat in memory), fp32
  * accumulation, one fp16 rounding of each output.  Two paths:
- *  - M <= 32, or N not a multiple of 8: 16 tokens per pass (mma.sync m16n8k16); the exact
+ *  - M <= 16, or N not a multiple of 8: 16 tokens per pass (mma.sync m16n8k16); the exact
  *    integers q - z times dy * s carried as an fp16 pair (high part + residual), i.e. the
  *    unrounded s (q - z) like the decode product (each weight within half an fp16 spacing of
  *    W_hat = fp16_rn(s (q - z))).  The rows of a 128-column block are split over up to 8 CTAs
  *    of one thread-block cluster whose fp32 sums are added in a fixed order through distributed
  *    shared memory: no workspace, allowed inside a stream capture.
- *  - M > 32 and N % 8 == 0: the 5th-generation tensor cores (tcgen05.mma, accumulator and the
+ *  - M > 16 and N % 8 == 0: the 5th-generation tensor cores (tcgen05.mma, accumulator and the
  *    A operand W_hat^T in tensor memory, dy by TMA) multiply W_hat = fp16_rn(s (q - z)) itself,
  *    bit-exact per weight; the weak columns come out exactly 0 there (their codes hold q = z)
  *    and a second kernel then writes dx[:, idx] = dy W_weak (mma.sync).  With fewer output

@@ -32,9 +32,9 @@ CASES = [
     ("cluster-of-3", 300, 384, 3, 384, 5, (1, 9), None),
     # 40 weak columns in one block over 512-row slices: too many to stage in shared memory
     ("weak-heavy-block", 4096, 256, 4, 128, 40, (2, 16), tuple(range(0, 80, 2))),
-    # from 33 tokens (N % 8 == 0): the tensor-memory pipeline, token tiles of 64 / 128 / 256,
+    # from 17 tokens (N % 8 == 0): the tensor-memory pipeline, token tiles of 64 / 128 / 256,
     # ragged 128-row steps, then the weak-column pass
-    ("many-tokens-3b", 520, 640, 3, 640, 7, (33, 100, 300), None),
+    ("many-tokens-3b", 520, 640, 3, 640, 7, (17, 33, 100, 300), None),
     ("many-tokens-4b-g128", 384, 512, 4, 128, 13, (64, 257), None),
     ("many-tokens-k0", 256, 384, 4, 128, 0, (40,), None),
     ("many-tokens-weak-heavy", 1024, 256, 3, 128, 40, (48,), tuple(range(0, 80, 2))),
@@ -162,10 +162,10 @@ def test_input_grad_one_hot_rows_are_w_eff(case):
     want[want == 0x8000] = 0
     layer = _layer(owq, ref, bits, group)
     rows = np.unique(np.concatenate([[0, N - 1, N // 2], np.arange(0, N, max(1, N // 29))]))
-    # 16 tokens per call (the 16-token kernel); with M >= 33 in a case, all rows in one call too
+    # 16 tokens per call (the 16-token kernel); with M >= 17 in a case, all rows in one call too
     # (the tensor-memory pipeline when N % 8 == 0; rows repeated up to 40 tokens)
     groups = [rows[r0:r0 + 16] for r0 in range(0, len(rows), 16)]
-    if max(Ms) >= 33:
+    if max(Ms) >= 17:
         groups.append(np.resize(rows, max(40, len(rows))))
     for rr in groups:
         dy = np.zeros((len(rr), N), dtype=np.float16)
