@@ -192,3 +192,38 @@ def test_wct_error_paths():
     assert owq.owq_weak_grad(h, buf, buf, f32, 0) == 2
     assert owq.owq_weak_grad(None, buf, buf, f32, 1) == owq.owq_input_grad(None, buf, buf, 1)
     layer.close()
+
+
+@pytest.mark.parametrize("M", [8, 300])
+def test_wct_products_captured_in_a_graph_on_a_fresh_handle(M):
+    """Both products inside a CUDA graph capture on a handle that has never run them, so no
+    scratch can be grown: the input gradient (16-token kernel at M = 8, tcgen05 path with the
+    weak-column pass at M = 300) and the weak-block gradient take their one-split forms; the
+    replayed results meet the same bounds as uncaptured calls."""
+    import weight_only_mixed_owq_b200 as owq
+    case = CASES[9]   # 520 x 640, 3-bit, 7 weak columns
+    name, N, K, bits, group, k, Ms, forced = case
+    d, ref = _case(case)
+    W_hat = oracle.dequant(ref["codes"], ref["scales"], ref["zeros"])
+    layer = _layer(owq, ref, bits, group)
+    dy = _dy(M, N, 123)
+    x = d["x"][:M] if d["x"].shape[0] >= M else np.resize(d["x"], (M, K)).astype(np.float16)
+    dy_g, x_g = _gpu(dy), _gpu(x)
+    dx = torch.empty((M, K), dtype=torch.float16, device=DEV)
+    dw = torch.empty((N, k), dtype=torch.float32, device=DEV)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.input_grad(dy_g, dx)
+        layer.weak_grad(x_g, dy_g, dw)
+    dx.zero_()
+    dw.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    want = oracle.input_grad(W_hat, ref["w_weak"], ref["idx"], dy)
+    check_output(dx.cpu().numpy(), want, f"captured input_grad M={M}")
+    _check_input_grad_bound(dx.cpu().numpy(), W_hat, ref["w_weak"], ref["idx"], dy, f"captured M={M}")
+    _check_weak_grad(dw.cpu().numpy(), x, dy, ref["idx"], f"captured weak_grad M={M}")
+    assert owq.owq_device_status() == owq.OWQ_OK
+    del g
+    layer.close()
