@@ -85,25 +85,56 @@ __global__ void k_rtn_params(const __half* __restrict__ W, int N, int K, int gro
 }
 
 // colsum_j = sum_i (W[i,j] - W_hat0[i,j])^2, i ascending; W_hat0 = fp16_rn(s (q - z)) of the
-// all-column RTN (scales/zeros hold that quantisation here).  One thread per column.
-__global__ void k_colsum_dw2(const __half* __restrict__ W, int N, int K, int group, int bits,
-                             const __half* __restrict__ scales, const __half* __restrict__ zeros,
-                             double* __restrict__ colsum) {
-  int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= K) return;
-  const int G = K / group, g = j / group, qmax = (1 << bits) - 1;
-  double acc = 0.0;
-  #pragma unroll 4
-  for (int i = 0; i < N; ++i) {
-    float w = __half2float(W[(size_t)i * K + j]);
-    float s32 = __half2float(scales[(size_t)i * G + g]);
-    float z32 = __half2float(zeros[(size_t)i * G + g]);
-    float q = rtn_code(w, s32, z32, qmax);
-    float wh = __half2float(__float2half_rn(__fmul_rn(s32, __fsub_rn(q, z32))));
-    double d = __dsub_rn((double)w, (double)wh);
-    acc = __dadd_rn(acc, __dmul_rn(d, d));
+// all-column RTN (scales/zeros hold that quantisation here).  The squares are independent, only
+// each column's sum is ordered: a CTA owns 32 columns; its 256 threads form the squared
+// differences of a 64-row chunk into shared memory (the next chunk's weights and (scale, zero)
+// pairs already in registers), then warp 0 adds each column's 64 values in row order to its
+// running fp64 sum -- the same __dmul_rn / __dadd_rn sequence as one thread walking the column.
+constexpr int kCsCols = 32, kCsRows = 64, kCsThreads = 256, kCsPer = kCsRows * kCsCols / kCsThreads;
+__global__ void __launch_bounds__(kCsThreads) k_colsum_dw2(const __half* __restrict__ W, int N, int K, int group,
+                                                            int bits, const __half* __restrict__ scales,
+                                                            const __half* __restrict__ zeros,
+                                                            double* __restrict__ colsum) {
+  __shared__ double s_d2[2][kCsRows][kCsCols];
+  const int tid = threadIdx.x, j0 = blockIdx.x * kCsCols;
+  const int G = K / group, qmax = (1 << bits) - 1;
+  const int nch = (N + kCsRows - 1) / kCsRows;
+  // this thread's elements of a chunk: row (tid + u 256) / 32, column (tid % 32)
+  const int c = tid % kCsCols, j = j0 + c, g = j / group;
+  __half wv[kCsPer], sv[kCsPer], zv[kCsPer];
+  auto load = [&](int ch) {
+    #pragma unroll
+    for (int u = 0; u < kCsPer; ++u) {
+      const int i = ch * kCsRows + (tid + u * kCsThreads) / kCsCols;
+      const bool ok = i < N && j < K;
+      wv[u] = ok ? W[(size_t)i * K + j] : __float2half_rn(0.f);
+      sv[u] = ok ? scales[(size_t)i * G + g] : __float2half_rn(0.f);
+      zv[u] = ok ? zeros[(size_t)i * G + g] : __float2half_rn(0.f);
+    }
+  };
+  double acc = 0.0;   // warp 0, lane c: column j0 + c
+  if (nch > 0) load(0);
+  for (int ch = 0; ch < nch; ++ch) {
+    const int buf = ch & 1;
+    double d2[kCsPer];
+    #pragma unroll
+    for (int u = 0; u < kCsPer; ++u) {
+      const float w = __half2float(wv[u]), s32 = __half2float(sv[u]), z32 = __half2float(zv[u]);
+      const float q = rtn_code(w, s32, z32, qmax);
+      const float wh = __half2float(__float2half_rn(__fmul_rn(s32, __fsub_rn(q, z32))));
+      const double d = __dsub_rn((double)w, (double)wh);
+      d2[u] = __dmul_rn(d, d);
+    }
+    if (ch + 1 < nch) load(ch + 1);   // in flight while the sums below run
+    #pragma unroll
+    for (int u = 0; u < kCsPer; ++u) s_d2[buf][(tid + u * kCsThreads) / kCsCols][c] = d2[u];
+    __syncthreads();   // (also: warp 0 finished the sums of chunk ch - 1, which used the other buffer)
+    if (tid < kCsCols) {
+      const int rows = min(kCsRows, N - ch * kCsRows);
+      for (int r = 0; r < rows; ++r) acc = __dadd_rn(acc, s_d2[buf][r][tid]);
+    }
   }
-  colsum[j] = acc;
+  if (tid < kCsCols && j0 + tid < K) colsum[j0 + tid] = acc;
 }
 
 struct Cand { double v; int j; };
@@ -205,7 +236,7 @@ cudaError_t launch_quantize(const __half* W, const __half* X, int N, int K, int 
   k_hessian_diag<<<(K + 255) / 256, 256, 0, s>>>(X, T, K, lam);
   // all-column RTN into the output scale/zero buffers (overwritten below)
   k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, nullptr, scales, zeros);
-  k_colsum_dw2<<<(K + 127) / 128, 128, 0, s>>>(W, N, K, group, bits, scales, zeros, colsum);
+  k_colsum_dw2<<<(K + kCsCols - 1) / kCsCols, kCsThreads, 0, s>>>(W, N, K, group, bits, scales, zeros, colsum);
   k_topk<<<1, 1024, 0, s>>>(lam, colsum, sens, K, k, idx, mask);
   k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, mask, scales, zeros);
   const size_t NK = (size_t)N * K;
@@ -285,7 +316,7 @@ cudaError_t launch_quantize_static(const __half* W, const __half* X, int N, int 
   const long long items = (long long)N * G;
   k_hessian_diag<<<(K + 255) / 256, 256, 0, s>>>(X, T, K, lam);
   k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, nullptr, scales, zeros);
-  k_colsum_dw2<<<(K + 127) / 128, 128, 0, s>>>(W, N, K, group, bits, scales, zeros, colsum);
+  k_colsum_dw2<<<(K + kCsCols - 1) / kCsCols, kCsThreads, 0, s>>>(W, N, K, group, bits, scales, zeros, colsum);
   k_topk<<<1, 1024, 0, s>>>(lam, colsum, sens, K, k, idx, mask);
   k_rtn_params<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(W, N, K, group, bits, mask, scales, zeros);
   const size_t NK = (size_t)N * K;
