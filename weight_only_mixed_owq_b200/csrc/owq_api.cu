@@ -207,9 +207,14 @@ owq_status_t owq_pack(const uint8_t* codes, int N, int K, int bits, int group, c
   alloc((void**)&mask_dev, sizeof(uint32_t) * (K / 32));
   if (e != cudaSuccess) { cudaFree(mask_dev); release(L); return cuda_status(e); }
 
-  // host-side table: weak bitmask per 32-code chunk
+  // host-side tables: weak bitmask per 32-code chunk; first weak slot and count per block
   std::vector<uint32_t> mask(K / 32, 0u);
   for (int t = 0; t < k; ++t) mask[hidx[t] / 32] |= 1u << (hidx[t] % 32);
+  for (int b = 0; b < K / kBlockCodes; ++b) L->blk_weak[b] = 0u;
+  for (int t = k - 1; t >= 0; --t) {   // descending: the first slot of each block wins
+    const int b = hidx[t] / kBlockCodes;
+    L->blk_weak[b] = ((uint32_t)t << 16) | ((L->blk_weak[b] & 0xFFFFu) + 1u);
+  }
 
   if (e == cudaSuccess) e = cudaMemsetAsync(L->packed, 0, packed_bytes, s);   // padding rows of the last tile
   if (e == cudaSuccess) e = cudaMemcpyAsync(L->scales, scales, sz_bytes, cudaMemcpyDeviceToDevice, s);

@@ -16,6 +16,7 @@ constexpr uint32_t kLayerMagic = 0x4f575131u;  // "OWQ1"
 constexpr int kBlockCodes = 128;               // codes per packed block (16 * bits bytes)
 constexpr int kChunkCodes = 32;                // codes per chunk (bits words)
 constexpr int kMaxWeak = 1024;
+constexpr int kMaxBlocks = 512;                // K <= 65536
 constexpr int kMaxGemvM = 16;
 
 struct Layer {
@@ -34,6 +35,9 @@ struct Layer {
   // [N/16 tiles][cta_slots][16 rows][16 tokens], each a 64-bit word (fp32 value | call epoch
   // << 32); zero at pack time
   unsigned long long* part;
+  // per 128-column block: its first weak slot << 16 | its weak-column count (the slots of a
+  // block are consecutive, the index list being increasing); host copy, made at pack time
+  uint32_t blk_weak[kMaxBlocks];
   int cta_slots;        // most CTAs below the one finishing a row tile in the decode product
   uint32_t epoch;       // decode calls made on this handle (tags the partial sums of each call)
   cudaStream_t stream;  // stream of owq_pack (used to order the release)

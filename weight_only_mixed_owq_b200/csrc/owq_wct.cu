@@ -296,6 +296,7 @@ struct IgArgs {
   int* status;            // device status word (bounded waits)
   long long wait_limit;
   int N, K, G, group, k, k_ld, M, tiles_per_slice;
+  uint32_t blk[kMaxBlocks];   // per column block: first weak slot << 16 | weak-column count
 };
 
 // ---------------------------------------------------------------- input gradient on the tensor cores
@@ -400,7 +401,7 @@ k_input_grad_mma(const __grid_constant__ IgArgs a) {
   extern __shared__ __align__(128) unsigned char ig_smem[];
   __shared__ float s_red[4][kTok][kBlockCodes];
   __shared__ int s_slot[kBlockCodes];              // weak slot of column c of the block, or -1
-  __shared__ int s_t0, s_nweak, s_wsl;
+  __shared__ int s_wsl;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tg = lane & 3;
   const int b = blockIdx.x, slice = blockIdx.y, S = gridDim.y;
@@ -432,45 +433,52 @@ k_input_grad_mma(const __grid_constant__ IgArgs a) {
     while (issued < min(nmine, kIgStages)) issue();
   }
 
+  // the block's weak slots t0 .. t0 + nweak - 1 (from the pack-time table): their columns and,
+  // staged, their values over the slice's rows are loaded in one round trip
+  const int t0 = (int)(a.blk[b] >> 16), nweak = (int)(a.blk[b] & 0xFFFFu);
   if (tid < kBlockCodes) s_slot[tid] = -1;
-  if (tid == 0) { s_t0 = 0x7fffffff; s_nweak = 0; s_wsl = 0; }
-  __syncthreads();
-  for (int t = tid; t < a.k; t += kIgThreads) {
-    const int c = a.idx[t] - b * kBlockCodes;
-    if (c >= 0 && c < kBlockCodes) {
-      s_slot[c] = t;
-      atomicMin(&s_t0, t);
-      atomicAdd(&s_nweak, 1);
-      atomicOr(&s_wsl, 1 << (c >> 4));
-    }
-  }
-  __syncthreads();
-  const int nweak = s_nweak, t0 = s_t0;
-  // the block's weak values over the slice's rows: s_wv[(slot - t0) * rows + r] (rows >= N: 0),
-  // staged for up to 8 weak columns, 4 rows x 8 columns of loads in flight per thread
-  const int wsl = s_wsl;   // slices (16 columns) of the block holding weak columns
+  if (tid == 0) s_wsl = 0;
+  const int my_t = tid < nweak ? t0 + tid : -1;
+  const int my_col = my_t >= 0 ? a.idx[my_t] - b * kBlockCodes : -1;
+  // s_wv[(slot - t0) * rows + r] (rows >= N: 0), staged for up to 8 weak columns, 4 rows x 8
+  // columns of loads in flight per thread per pass
   const bool staged = nweak > 0 && nweak <= 8 && nweak * rows * (int)sizeof(__half) <= kIgWeakBytes;
-  if (staged) {
-    for (int r0 = tid; r0 < rows; r0 += 4 * kIgThreads) {
-      uint16_t v[4][8];
+  const int passes = staged ? (rows + 4 * kIgThreads - 1) / (4 * kIgThreads) : 0;
+  uint16_t v[4][8];
+  auto stage_load = [&](int r0) {
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = r0 + u * kIgThreads, row = t_lo * 16 + r;
+      const __half* src = a.w_weak + (size_t)row * a.k_ld + t0;
       #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + u * kIgThreads, row = t_lo * 16 + r;
-        const __half* src = a.w_weak + (size_t)row * a.k_ld + t0;
-        #pragma unroll
-        for (int wi = 0; wi < 8; ++wi)
-          v[u][wi] = wi < nweak && r < rows && row < a.N ? __half_as_ushort(src[wi]) : (uint16_t)0;
-      }
-      #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + u * kIgThreads;
-        #pragma unroll
-        for (int wi = 0; wi < 8; ++wi)
-          if (wi < nweak && r < rows) s_wv[wi * rows + r] = __ushort_as_half(v[u][wi]);
-      }
+      for (int wi = 0; wi < 8; ++wi)
+        v[u][wi] = wi < nweak && r < rows && row < a.N ? __half_as_ushort(src[wi]) : (uint16_t)0;
     }
-    __syncthreads();
+  };
+  auto stage_store = [&](int r0) {
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = r0 + u * kIgThreads;
+      #pragma unroll
+      for (int wi = 0; wi < 8; ++wi)
+        if (wi < nweak && r < rows) s_wv[wi * rows + r] = __ushort_as_half(v[u][wi]);
+    }
+  };
+  if (passes > 0) stage_load(tid);
+  __syncthreads();   // s_slot cleared
+  if (my_col >= 0 && my_col < kBlockCodes) {
+    s_slot[my_col] = my_t;
+    atomicOr(&s_wsl, 1 << (my_col >> 4));
   }
+  if (passes > 0) {
+    stage_store(tid);
+    for (int pz = 1; pz < passes; ++pz) {
+      stage_load(tid + pz * 4 * kIgThreads);
+      stage_store(tid + pz * 4 * kIgThreads);
+    }
+  }
+  __syncthreads();
+  const int wsl = s_wsl;   // slices (16 columns) of the block holding weak columns
   // the lane's weak columns: bit 2 s for column 16 s + g, bit 2 s + 1 for column 16 s + g + 8
   uint32_t wmask = 0;
   if (nweak > 0) {
@@ -814,6 +822,7 @@ cudaError_t launch_input_grad(Layer& L, const __half* dy, __half* dx, int M, cud
   a.k = L.k;
   a.k_ld = L.k_ld;
   a.tiles_per_slice = per;
+  for (int i = 0; i < Kb; ++i) a.blk[i] = L.blk_weak[i];
   if (!a.status) return cudaErrorInvalidDevicePointer;
   for (int m0 = 0; m0 < M; m0 += kIgMaxTok) {
     a.dy = dy + (size_t)m0 * L.N;
