@@ -127,11 +127,11 @@ def test_wct_gradients_fullsize_opt67b_attention_layer():
     import weight_only_mixed_owq_b200 as owq
     spec = owq_synth.WORKLOADS[1]
     L = spec.layers[0]
-    d = owq_synth.draw_layer(L, spec, 16, owq_synth.seed_for(1, 0))
+    d = owq_synth.draw_layer(L, spec, 2048, owq_synth.seed_for(1, 0))
     ref = oracle.owq_quantize(d["W"], d["X"], L.bits, L.group, L.k)
     W_hat = oracle.dequant(ref["codes"], ref["scales"], ref["zeros"])
     layer = _layer(owq, ref, L.bits, L.group)
-    for M in (1, 16):
+    for M in (1, 16, 256, 2048):   # the 16-token kernel, then the tcgen05 path (128- / 256-token tiles)
         dy = _dy(M, L.N, 77 + M)
         x = d["x"][:M]
         dx = layer.input_grad(_gpu(dy))
@@ -139,6 +139,7 @@ def test_wct_gradients_fullsize_opt67b_attention_layer():
         torch.cuda.synchronize()
         check_output(dx.cpu().numpy(), oracle.input_grad(W_hat, ref["w_weak"], ref["idx"], dy),
                      f"{L.name} input_grad M={M}")
+        _check_input_grad_bound(dx.cpu().numpy(), W_hat, ref["w_weak"], ref["idx"], dy, f"{L.name} M={M}")
         _check_weak_grad(dw.cpu().numpy(), x, dy, ref["idx"], f"{L.name} M={M}")
     layer.close()
 
