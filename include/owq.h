@@ -293,14 +293,30 @@ owq_status_t owq_gemv_multi(const owq_layer_t* layers, const uint16_t* const* xs
  * its tile, sets the device status word and this call's later owq_device_status returns
  * OWQ_ERR_TIMEOUT (y is then undefined).  The first call on a handle builds its tensor
  * maps on the host: first calls from several host threads on one handle must be
- * serialised.  The handle's scratch (M * k_ld * 2 bytes of weak activations; for few row
- * tiles also a split-K workspace) grows on the first call that needs more, which must not
- * be inside a stream capture: there a too-small weak-activation scratch gives OWQ_ERR_NOMEM
- * (the split-K workspace falls back to one split).  Calls on one handle must be ordered
- * (same stream, or synchronised): they share that scratch.
+ * serialised.  The handle's scratch (M * k_ld * 2 bytes of weak activations; when
+ * owq_gemm_plan splits K, also a workspace of fp32 partial sums) grows on the first call that
+ * needs more, which must not be inside a stream capture: there a too-small weak-activation
+ * scratch gives OWQ_ERR_NOMEM (a too-small partial-sum workspace: the call runs unsplit).
+ * Split outputs are the fp32 partials added in split order, then rounded once: repeated calls
+ * give identical bits.  Calls on one handle must be ordered (same stream, or synchronised):
+ * they share that scratch.
  */
 owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M,
                       owq_stream_t stream);
+
+/*
+ * owq_gemm_plan -- the launch shape owq_gemm takes for an N x K layer, M tokens, on a device
+ * with `sms` SMs (host only; no device, no handle).  Tiles are 128 weight rows x `tile_tokens`
+ * tokens (64 for M <= 64, 128 for M <= 256, else 256).  With fewer tiles than SMs every tile
+ * is split over K; with a short last wave the row tiles of the last few token tiles are split
+ * over K instead (the "tail"), to run on the SMs the whole tiles leave idle.  Either way a
+ * reduction kernel adds the fp32 partials in split order.
+ * Out: plan[0] tile_tokens, plan[1] K splits of every tile (1: none), plan[2] token tiles in
+ *      the tail (0: none), plan[3] K splits of each tail tile (1: none).
+ * Errors: OWQ_ERR_NULL (plan NULL), OWQ_ERR_SHAPE (N, K outside owq_pack's ranges, M outside
+ * 1..65536), OWQ_ERR_ARG (sms < 1).
+ */
+owq_status_t owq_gemm_plan(int N, int K, int M, int sms, int plan[4]);
 
 /*
  * owq_weak_grad -- weak column tuning: gradient of a loss with respect to the layer's fp16

@@ -26,7 +26,7 @@ CASES = [
     (2, 6, (1, 2, 4, 8, 16), ()),  # LLaMA-7B down 4096 x 11008, 4-bit g128, k = 86
     (3, 5, (1,), ()),              # OPT-66B fc2 9216 x 36864, 3-bit per channel, k = 288
     (4, 0, (), (64, 2048)),        # LLaMA-13B up 13824 x 5120, 3-bit g128, k = 40
-    (4, 1, (), (128,)),            # LLaMA-13B down 5120 x 13824, k = 108
+    (4, 1, (), (128, 2048)),       # LLaMA-13B down 5120 x 13824, k = 108 (2048: split tail)
 ]
 
 

@@ -41,6 +41,7 @@ PROTOTYPES = [
     ("owq_gemv", _I, [_P, _P, _P, _I, _P]),
     ("owq_gemv_multi", _I, [ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _I, _P]),
     ("owq_gemm", _I, [_P, _P, _P, _I, _P]),
+    ("owq_gemm_plan", _I, [_I, _I, _I, _I, ctypes.POINTER(_I)]),
     ("owq_weak_grad", _I, [_P, _P, _P, _P, _I, _P]),
     ("owq_input_grad", _I, [_P, _P, _P, _I, _P]),
     ("owq_dequant", _I, [_P, _P, _P, _P]),
@@ -173,6 +174,13 @@ def owq_gemv_multi(layers, xs, ys, M, stream=None) -> int:
 
 def owq_gemm(layer, x, y, M, stream=None) -> int:
     return LIB.owq_gemm(layer, _ptr(x), _ptr(y), M, _stream(stream))
+
+
+def owq_gemm_plan(N, K, M, sms):
+    """Returns (status, {tile_tokens, splits, tail_tiles, tail_splits}): owq_gemm's launch shape."""
+    out = (ctypes.c_int * 4)()
+    st = LIB.owq_gemm_plan(N, K, M, sms, out)
+    return st, dict(zip(("tile_tokens", "splits", "tail_tiles", "tail_splits"), out))
 
 
 def owq_weak_grad(layer, x, dy, dw_weak, M, stream=None) -> int:

@@ -465,6 +465,19 @@ owq_status_t owq_gemm(owq_layer_t layer, const uint16_t* x, uint16_t* y, int M, 
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+owq_status_t owq_gemm_plan(int N, int K, int M, int sms, int plan[4]) {
+  if (!plan) return OWQ_ERR_NULL;
+  if (N < 1 || N > (1 << 20) || K < kBlockCodes || K > 65536 || K % kBlockCodes || M < 1 || M > 65536)
+    return OWQ_ERR_SHAPE;
+  if (sms < 1) return OWQ_ERR_ARG;
+  const GemmPlan g = gemm_plan(N, K, M, sms);
+  plan[0] = g.tile_tokens;
+  plan[1] = g.splits;
+  plan[2] = g.tail_tt;
+  plan[3] = g.tail_sp;
+  return OWQ_OK;
+}
+
 owq_status_t owq_weak_grad(owq_layer_t layer, const uint16_t* x, const uint16_t* dy, float* dw_weak,
                            int M, owq_stream_t stream) {
   Layer* L = lookup(layer);

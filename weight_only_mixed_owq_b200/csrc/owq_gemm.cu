@@ -63,10 +63,15 @@ struct GemmParams {
   const __half* w_weak;   // the weak block [N][k_ld] (read by the A-operand warps in weak steps)
   int k_ld;
   __half* y;
-  float* ws;        // split-K partial sums [split][M][N] (NULL: one split, fp16 y directly)
+  float* ws;        // split-K partial sums: split sp, token t, row n at sp * ws_stride + (t - ws_t0) N + n
+  size_t ws_stride;
+  int ws_t0;
   int* status;
   int N, K, M, G;
   int ksteps;       // dense 128-code steps per split (blockIdx.z)
+  // short last wave: grid.y = tail_y0 whole token tiles, then tail_sp CTAs (K splits of
+  // tail_ksteps steps) for each further token tile (tail_y0 = grid.y: no tail)
+  int tail_y0, tail_sp, tail_ksteps;
   int nw;           // weak steps: 128 columns of the weak block each (run by the last split)
   long long wait_limit;   // bound of every mbarrier wait, in SM clock cycles
   int skip_arrive;  // test-injected lost arrival: dequantisation thread 0 skips its first one
@@ -121,11 +126,20 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // (row tile, token tile, K split) of this CTA
+  int ty = blockIdx.y, sp = blockIdx.z, nsp = gridDim.z, ksteps = p.ksteps;
+  if (ty >= p.tail_y0) {
+    const int u = ty - p.tail_y0;
+    ty = p.tail_y0 + u / p.tail_sp;
+    sp = u % p.tail_sp;
+    nsp = p.tail_sp;
+    ksteps = p.tail_ksteps;
+  }
   const int n0 = blockIdx.x * kBM;      // first weight row
-  const int m0 = blockIdx.y * BN;       // first token
-  const int kb0 = blockIdx.z * p.ksteps;                          // first dense step of this split
-  const int nD = max(0, min(p.ksteps, p.K / kStepCodes - kb0));   // dense steps of this split
-  const int nK = nD + (blockIdx.z == gridDim.z - 1 ? p.nw : 0);   // + the weak steps (last split)
+  const int m0 = ty * BN;               // first token
+  const int kb0 = sp * ksteps;                                  // first dense step of this split
+  const int nD = max(0, min(ksteps, p.K / kStepCodes - kb0));   // dense steps of this split
+  const int nK = nD + (sp == nsp - 1 ? p.nw : 0);               // + the weak steps (last split)
   const bool per_group = p.G > 1;
 
   if (threadIdx.x == 0) {
@@ -304,12 +318,12 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
       tmem_ld_wait();
       if (acc_ok && orow < p.N) {
-        if (p.ws) {   // split-K: fp32 partial of this split
-          float* w = p.ws + (size_t)blockIdx.z * p.M * p.N;
+        if (nsp > 1) {   // split-K: fp32 partial of this split
+          float* w = p.ws + (size_t)sp * p.ws_stride;
           #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = m0 + c0 + j;
-            if (t < p.M) w[(size_t)t * p.N + orow] = __uint_as_float(v[j]);
+            if (t < p.M) w[(size_t)(t - p.ws_t0) * p.N + orow] = __uint_as_float(v[j]);
           }
         } else {
           #pragma unroll
@@ -627,7 +641,8 @@ __global__ void k_gather_weak_x(const __half* __restrict__ x, int M, int K, cons
   }
 }
 
-// Split-K: y = fp16_rn(sum of the splits' fp32 partials, in split order).
+// Split-K: y = fp16_rn(sum of the splits' fp32 partials, in split order); MN outputs, the
+// splits' partials MN floats apart.
 __global__ void k_splitk_reduce(const float* __restrict__ ws, int splits, size_t MN, __half* __restrict__ y) {
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < MN; e += (size_t)gridDim.x * blockDim.x) {
     float v = ws[e];
@@ -713,6 +728,68 @@ bool ensure_scratch(void** buf, size_t* have, size_t need, cudaStream_t s) {
   return true;
 }
 
+}  // namespace
+
+// Token tile width: wider tiles dequantise each weight tile once for more tokens (the
+// dequantisation, not the MMA, bounds the narrower tiles); the widest one fits three stages.
+int gemm_tile_tokens(int M) { return M <= 64 ? 64 : M <= 256 ? 128 : 256; }
+
+// The launch shape of one product (see GemmPlan).  Two cases leave SMs idle:
+//  * fewer tiles than SMs: every tile is split over K (at least 4 steps per split);
+//  * a short last wave: the CTAs are dispatched in order, so the last ceil(T / P) - T / P of a
+//    wave of whole tiles holds few of them.  The row tiles of the last tt token tiles are then
+//    split S ways over K instead; these short CTAs go to the SMs the whole tiles leave free.
+//    The choice is a model in units of one whole tile's time: whole tiles end at w (or w + 1
+//    with a partial wave of r); a short CTA takes its share of the steps plus a fixed cost
+//    (start-up, pipeline fill, fp32 epilogue); the reduction's traffic (partials written and
+//    read, the fp16 result) and its launch are charged at the end.  The tail is taken only
+//    when the model saves at least kMinGain of a tile's time.
+GemmPlan gemm_plan(int N, int K, int M, int sms) {
+  constexpr double kSmFlops = 11e12;   // measured per-SM rate of whole 256-token tiles
+  constexpr double kHbm = 6e12;        // bytes/s the reduction streams at
+  constexpr double kCtaFixed = 3e-6;   // seconds of fixed cost per short CTA
+  constexpr double kLaunch = 3e-6;     // seconds for the reduction's launch
+  constexpr double kMinGain = 0.15;
+  GemmPlan g;
+  g.tile_tokens = gemm_tile_tokens(M);
+  const int nK = K / kStepCodes;
+  g.splits = 1; g.ksteps = nK;
+  g.tail_tt = 0; g.tail_sp = 1; g.tail_ksteps = nK;
+  if (sms < 1 || nK < 1 || N < 1 || M < 1) return g;
+  const long long RT = (N + kBM - 1) / kBM, TT = (M + g.tile_tokens - 1) / g.tile_tokens, T = RT * TT;
+  if (T < sms) {
+    const int sp = (int)std::max<long long>(1, std::min<long long>(sms / T, nK / 4));
+    if (sp > 1) {
+      g.ksteps = (nK + sp - 1) / sp;
+      g.splits = (nK + g.ksteps - 1) / g.ksteps;
+    }
+    return g;
+  }
+  const double tile_s = 2.0 * kBM * g.tile_tokens * (double)K / kSmFlops;
+  const double fixed = kCtaFixed / tile_s;
+  double best = (double)((T + sms - 1) / sms) - kMinGain;
+  for (int tt = 1; tt <= 2 && tt < TT; ++tt) {
+    const long long Tm = RT * (TT - tt), w = Tm / sms, r = Tm % sms, f = sms - r;
+    for (int S = 2; S <= 8 && nK / S >= 4; ++S) {
+      const int ks = (nK + S - 1) / S, se = (nK + ks - 1) / ks;   // the splits actually formed
+      const double d = (double)ks / nK + fixed;
+      const long long n = RT * tt * se, per = (long long)(1.0 / d);
+      double end;
+      if (r == 0) end = w + (double)((n + sms - 1) / sms) * d;
+      else if (n <= f * per) end = w + 1.0;
+      else end = w + 1.0 + (double)((n - f * per + sms - 1) / sms) * d;
+      end += ((8.0 * se + 2.0) * tt * g.tile_tokens * (double)N / kHbm + kLaunch) / tile_s;
+      if (end < best) {
+        best = end;
+        g.tail_tt = tt; g.tail_sp = se; g.tail_ksteps = ks;
+      }
+    }
+  }
+  return g;
+}
+
+namespace {
+
 template <int BITS, int BN, int S, int DW>
 owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_limit, bool skip_arrive,
                  cudaStream_t s) {
@@ -732,46 +809,30 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   prm.nw = L.k > 0 ? (L.k_ld + kStepCodes - 1) / kStepCodes : 0;
   prm.wait_limit = wait_limit; prm.skip_arrive = skip_arrive ? 1 : 0;
   if (!prm.status) return OWQ_ERR_CUDA;
-  // fewer tiles than SMs: split K over CTAs (at least 4 steps each), fp32 partials in the
-  // layer's workspace, then one reduction kernel; never grown during stream capture
-  const int nK = L.K / kStepCodes;
-  const long long tiles = (long long)((L.N + kBM - 1) / kBM) * ((M + BN - 1) / BN);
-  int splits = 1;
   int sms = 0;   // SM count of the layer's device
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, L.device) != cudaSuccess || sms <= 0) {
     cudaGetLastError();
     sms = 148;
   }
-  if (tiles < sms) splits = (int)std::max<long long>(1, std::min<long long>(sms / tiles, nK / 4));
-  if (splits > 1) {
-    prm.ksteps = (nK + splits - 1) / splits;
-    splits = (nK + prm.ksteps - 1) / prm.ksteps;
-    const size_t need = (size_t)splits * M * L.N * sizeof(float);
-    if (need > L.gemm_ws_bytes) {
-      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-      if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
-        cudaGetLastError();
-        splits = 1;
-      } else {
-        cudaFree(L.gemm_ws);
-        L.gemm_ws = nullptr;
-        L.gemm_ws_bytes = 0;
-        if (cudaMalloc(&L.gemm_ws, need) != cudaSuccess) {
-          cudaGetLastError();
-          L.gemm_ws = nullptr;
-          splits = 1;
-        } else {
-          L.gemm_ws_bytes = need;
-        }
-      }
-    }
+  GemmPlan g = gemm_plan(L.N, L.K, M, sms);
+  const int RT = (L.N + kBM - 1) / kBM, TT = (M + BN - 1) / BN;
+  // the split partials live in the layer's workspace, never grown during stream capture (the
+  // call then runs unsplit)
+  const int t0 = g.tail_sp > 1 ? (TT - g.tail_tt) * BN : 0;   // first token with split partials
+  const int nsp = g.tail_sp > 1 ? g.tail_sp : g.splits;
+  if (nsp > 1 && !ensure_scratch(reinterpret_cast<void**>(&L.gemm_ws), &L.gemm_ws_bytes,
+                                 (size_t)nsp * (M - t0) * L.N * sizeof(float), s)) {
+    g.splits = 1; g.ksteps = L.K / kStepCodes;
+    g.tail_tt = 0; g.tail_sp = 1;
   }
-  if (splits == 1) {
-    prm.ksteps = nK;
-    prm.ws = nullptr;
-  } else {
-    prm.ws = L.gemm_ws;
-  }
+  prm.ksteps = g.ksteps;
+  prm.tail_y0 = TT - g.tail_tt;
+  prm.tail_sp = g.tail_sp;
+  prm.tail_ksteps = g.tail_ksteps;
+  const bool split = g.splits > 1 || g.tail_sp > 1;
+  prm.ws = split ? L.gemm_ws : nullptr;
+  prm.ws_t0 = g.tail_sp > 1 ? t0 : 0;
+  prm.ws_stride = (size_t)(M - prm.ws_t0) * L.N;
   auto kern = k_gemm_sm100<BITS, BN, S, DW>;
   constexpr int smem = smem_bytes<BITS, BN, S>();
   static_assert(smem <= 232448, "shared memory budget");
@@ -783,7 +844,7 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
     cudaGetLastError();
     return OWQ_ERR_CUDA;
   }
-  dim3 grid((L.N + kBM - 1) / kBM, (M + BN - 1) / BN, splits);
+  dim3 grid(RT, prm.tail_y0 + g.tail_tt * g.tail_sp, g.splits);
   // the weak activations, gathered once per call into the layer's scratch (grown outside capture)
   CUtensorMap mxw = mx;
   if (L.k > 0) {
@@ -799,9 +860,10 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   }
   kern<<<grid, 32 * (2 + DW), smem, s>>>(mx, L.map_packed, mxw, L.G > 1 ? L.map_sz : mx, prm);
   if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
-  if (splits > 1) {
-    const size_t MN = (size_t)M * L.N;
-    k_splitk_reduce<<<(unsigned)std::min<size_t>((MN + 255) / 256, 4096), 256, 0, s>>>(prm.ws, splits, MN, y);
+  if (split) {   // the split outputs: every token (K split over all tiles) or the tail's tokens
+    const size_t MN = prm.ws_stride;
+    k_splitk_reduce<<<(unsigned)std::min<size_t>((MN + 255) / 256, 4096), 256, 0, s>>>(prm.ws, nsp, MN,
+                                                                                        y + (size_t)prm.ws_t0 * L.N);
     if (cudaGetLastError() != cudaSuccess) return OWQ_ERR_CUDA;
   }
   return OWQ_OK;
@@ -809,11 +871,11 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
 
 template <int BITS>
 owq_status_t dispatch(Layer& L, const __half* x, __half* y, int M, long long wl, bool skip, cudaStream_t s) {
-  // wider token tiles dequantise each weight tile once for more tokens (the dequantisation,
-  // not the MMA, bounds the narrower tiles); the widest one fits two stages
-  if (M <= 64) return run<BITS, 64, 6, 8>(L, x, y, M, wl, skip, s);
-  if (M <= 256) return run<BITS, 128, 4, 8>(L, x, y, M, wl, skip, s);
-  return run<BITS, 256, 3, 16>(L, x, y, M, wl, skip, s);
+  switch (gemm_tile_tokens(M)) {
+    case 64: return run<BITS, 64, 6, 8>(L, x, y, M, wl, skip, s);
+    case 128: return run<BITS, 128, 4, 8>(L, x, y, M, wl, skip, s);
+    default: return run<BITS, 256, 3, 16>(L, x, y, M, wl, skip, s);
+  }
 }
 
 template <int BITS, int BN, int S, int DW>

@@ -167,6 +167,15 @@ owq_status_t igemm_sm100(Layer& L, const __half* dy, __half* dx, int M, long lon
 // the bounds check must catch
 cudaError_t launch_input_grad_weak(Layer& L, const __half* dy, __half* dx, int M, bool inject, cudaStream_t s);
 
+// Launch shape of one prefill product: tile width in tokens; K splits of every tile (fewer
+// tiles than SMs; `ksteps` 128-code steps each); or a split tail: the row tiles of the last
+// tail_tt token tiles split tail_sp ways over K (tail_ksteps steps each).  Host only.
+struct GemmPlan {
+  int tile_tokens, splits, ksteps, tail_tt, tail_sp, tail_ksteps;
+};
+int gemm_tile_tokens(int M);
+GemmPlan gemm_plan(int N, int K, int M, int sms);
+
 // skip_arrive: a test-injected lost arrival (one dequantisation thread per CTA skips its first
 // arrival), so that the bounded waits run out
 owq_status_t gemm_sm100(Layer& L, const __half* x, __half* y, int M, long long wait_limit,
