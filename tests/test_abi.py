@@ -51,6 +51,8 @@ def test_debug_bounds_variant_exports_every_declared_symbol(owq):
     path = build.LIB_BOUNDS
     if not os.path.exists(path):
         pytest.skip("debug-bounds variant not built (python -m weight_only_mixed_owq_b200.build --debug-bounds)")
+    if not build.up_to_date(path):   # built from older sources: rebuild it first
+        build.build(debug_bounds=True)
     lib = ctypes.CDLL(path)
     for name in _declared_functions():
         assert hasattr(lib, name), name
