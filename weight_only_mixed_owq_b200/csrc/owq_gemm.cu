@@ -110,7 +110,10 @@ __device__ __forceinline__ uint32_t dequant_pair(const uint32_t* w, int j, uint3
   return h2_mul(h2_fma(pair_bits<BITS>(w, j) | kMagic, scl[c], nz[c]), s2);
 }
 
-template <int BITS, int BN, int S, int DW>
+// TAIL: the grid holds a split tail (GemmParams::tail_*); without it the CTA's token tile and
+// K split are blockIdx.y and blockIdx.z, and none of the tail arithmetic is compiled in (it
+// cost the 64-token tiles 5% where it was always present)
+template <int BITS, int BN, int S, int DW, bool TAIL>
 __global__ void __launch_bounds__(32 * (2 + DW), 1)
 k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_p,
              const __grid_constant__ CUtensorMap map_xw, const __grid_constant__ CUtensorMap map_sz,
@@ -127,19 +130,22 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // (row tile, token tile, K split) of this CTA
-  int ty = blockIdx.y, sp = blockIdx.z, nsp = gridDim.z, ksteps = p.ksteps;
-  if (ty >= p.tail_y0) {
-    const int u = ty - p.tail_y0;
-    ty = p.tail_y0 + u / p.tail_sp;
-    sp = u % p.tail_sp;
-    nsp = p.tail_sp;
-    ksteps = p.tail_ksteps;
+  int ty = 0, sp = 0, nsp = 1, ksteps = 0;
+  if constexpr (TAIL) {
+    ty = blockIdx.y; sp = blockIdx.z; nsp = gridDim.z; ksteps = p.ksteps;
+    if (ty >= p.tail_y0) {
+      const int u = ty - p.tail_y0;
+      ty = p.tail_y0 + u / p.tail_sp;
+      sp = u % p.tail_sp;
+      nsp = p.tail_sp;
+      ksteps = p.tail_ksteps;
+    }
   }
-  const int n0 = blockIdx.x * kBM;      // first weight row
-  const int m0 = ty * BN;               // first token
-  const int kb0 = sp * ksteps;                                  // first dense step of this split
-  const int nD = max(0, min(ksteps, p.K / kStepCodes - kb0));   // dense steps of this split
-  const int nK = nD + (sp == nsp - 1 ? p.nw : 0);               // + the weak steps (last split)
+  const int n0 = blockIdx.x * kBM;                     // first weight row
+  const int m0 = (TAIL ? ty : (int)blockIdx.y) * BN;   // first token
+  const int kb0 = TAIL ? sp * ksteps : (int)blockIdx.z * p.ksteps;                  // first dense step of this split
+  const int nD = max(0, min(TAIL ? ksteps : p.ksteps, p.K / kStepCodes - kb0));     // dense steps of this split
+  const int nK = nD + ((TAIL ? sp == nsp - 1 : blockIdx.z == gridDim.z - 1) ? p.nw : 0);   // + the weak steps (last split)
   const bool per_group = p.G > 1;
 
   if (threadIdx.x == 0) {
@@ -318,12 +324,13 @@ k_gemm_sm100(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ 
       tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
       tmem_ld_wait();
       if (acc_ok && orow < p.N) {
-        if (nsp > 1) {   // split-K: fp32 partial of this split
-          float* w = p.ws + (size_t)sp * p.ws_stride;
+        if (TAIL ? nsp > 1 : p.ws != nullptr) {   // split-K: fp32 partial of this split
+          // without a tail the partials are [split][M][N] (ws_stride = M N, ws_t0 = 0)
+          float* w = TAIL ? p.ws + (size_t)sp * p.ws_stride : p.ws + (size_t)blockIdx.z * p.M * p.N;
           #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int t = m0 + c0 + j;
-            if (t < p.M) w[(size_t)(t - p.ws_t0) * p.N + orow] = __uint_as_float(v[j]);
+            if (t < p.M) w[(size_t)(TAIL ? t - p.ws_t0 : t) * p.N + orow] = __uint_as_float(v[j]);
           }
         } else {
           #pragma unroll
@@ -833,7 +840,12 @@ owq_status_t run(Layer& L, const __half* x, __half* y, int M, long long wait_lim
   prm.ws = split ? L.gemm_ws : nullptr;
   prm.ws_t0 = g.tail_sp > 1 ? t0 : 0;
   prm.ws_stride = (size_t)(M - prm.ws_t0) * L.N;
-  auto kern = k_gemm_sm100<BITS, BN, S, DW>;
+  // the tail variant only where a tail can occur (64-token tiles: one token tile per call)
+  auto kern = k_gemm_sm100<BITS, BN, S, DW, false>;
+  if (g.tail_sp > 1) {
+    if constexpr (BN > 64) kern = k_gemm_sm100<BITS, BN, S, DW, true>;
+    else return OWQ_ERR_CUDA;   // never planned: a tail needs two token tiles
+  }
   constexpr int smem = smem_bytes<BITS, BN, S>();
   static_assert(smem <= 232448, "shared memory budget");
   // the CTAs an SM can hold (by shared memory) never need more than its 512 tensor-memory
